@@ -1,0 +1,223 @@
+"""fp64 CPU oracle for the ParaRNN / DEER Newton solve (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It wraps ``oracle.c`` (plain C, fp64,
+threads across independent channels only) through ctypes and shares no code with the
+CUDA library in ``nonlinear_rnn_solve_newton_b200``.
+
+What each function computes, and the passage it follows:
+
+* ``scan_diag`` / ``scan_block2``: the block bi-diagonal linear system
+  h_t = A_t h_{t-1} + b_t solved sequentially in t (ParaRNN TL;DR: the Newton
+  step is a block bi-diagonal system; Figure 2 caption: diagonal and 2x2
+  block-diagonal variants).
+* ``rollout_gru`` / ``rollout_lstm``: the sequential application of the cell,
+  the plain definition of the result that Newton must reproduce (ParaRNN
+  abstract, "naive sequential application"; DEER summary: outputs agree with
+  sequential evaluation).
+* ``newton_gru`` / ``newton_lstm``: Newton's method on the stacked system,
+  serial, with the max-abs residual over the whole batch as the stopping
+  test (ParaRNN abstract and Figure 4 caption; DEER summary: tolerance 1e-4).
+* ``gru_cell`` / ``lstm_cell``: one cell step and its Jacobian.
+
+Parity status: every function above is pinned in ``tests/test_oracle_pins.py``
+against closed forms, brute force, PyTorch's fp64 ``GRUCell``/``LSTMCell`` and
+autograd, and Newton's own invariants.  The iteration count has no printed
+value to pin against (Figure 4 survived only as a caption): parity unpinned for
+the count itself; it is checked only through the invariants (one iteration for
+an affine recurrence, two for an LSTM with no recurrence, at most L).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_intp = ctypes.POINTER(ctypes.c_int)
+_i64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, -O2, pthreads)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fPIC", "-shared", "-fno-fast-math",
+               "-ffp-contract=off", "-std=c11", _SRC, "-o", _LIB + ".tmp", "-lm", "-lpthread"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_scan_diag.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+            lib.oracle_scan_block2.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+            lib.oracle_gru_cell.argtypes = [_f64p, _f64p, ctypes.c_double, _f64p, _f64p]
+            lib.oracle_lstm_cell.argtypes = [_f64p, _f64p, ctypes.c_double, ctypes.c_double,
+                                             _f64p, _f64p, _f64p]
+            lib.oracle_rollout_gru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+            lib.oracle_rollout_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
+                                                _i64, _i64, _i64]
+            lib.oracle_newton_gru.argtypes = [_f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_int,
+                                              _i64, _i64, _i64, _f64p, _f64p, _i32p, _intp, _intp]
+            lib.oracle_newton_gru.restype = ctypes.c_int
+            lib.oracle_newton_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, ctypes.c_double,
+                                               ctypes.c_int, _i64, _i64, _i64, _f64p, _f64p,
+                                               _f64p, _i32p, _intp, _intp]
+            lib.oracle_newton_lstm.restype = ctypes.c_int
+            lib.oracle_residual_gru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+            lib.oracle_residual_gru.restype = ctypes.c_double
+            lib.oracle_set_threads.argtypes = [ctypes.c_int]
+            lib.oracle_get_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def set_threads(n: int) -> None:
+    """Number of host threads the oracle uses (0 = every CPU in the affinity mask)."""
+    _load().oracle_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(_load().oracle_get_threads())
+
+
+def _d(x):
+    """Contiguous fp64 copy (widening is exact for fp32 and bf16-valued inputs)."""
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(x):
+    return None if x is None else x.ctypes.data_as(_f64p)
+
+
+def scan_diag(A, b, h0=None):
+    """h[b,t,d] = A[b,t,d] * h[b,t-1,d] + b[b,t,d]; A, b: [B,L,D]; h0: [B,D] or None (= 0)."""
+    A, b = _d(A), _d(b)
+    B, L, D = A.shape
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    h = np.empty_like(A)
+    _load().oracle_scan_diag(_p(A), _p(b), _p(h0), _p(h), B, L, D)
+    return h
+
+
+def scan_block2(A, b, x0=None):
+    """x_t = A_t x_{t-1} + b_t; A: [B,L,D,2,2] row-major, b: [B,L,D,2], x0: [B,D,2] or None."""
+    A, b = _d(A), _d(b)
+    B, L, D = A.shape[:3]
+    x0 = None if x0 is None else _d(x0).reshape(B, D, 2)
+    x = np.empty_like(b)
+    _load().oracle_scan_block2(_p(A), _p(b), _p(x0), _p(x), B, L, D)
+    return x
+
+
+def gru_cell(p, w, h):
+    """One ParaGRU step: p = (Pz, Pr, Pc), w = (az, ar, ac) -> (h', dh'/dh)."""
+    p, w = _d(p), _d(w)
+    f = ctypes.c_double()
+    J = ctypes.c_double()
+    _load().oracle_gru_cell(_p(p), _p(w), float(h), ctypes.byref(f), ctypes.byref(J))
+    return f.value, J.value
+
+
+def lstm_cell(p, w, c, h):
+    """One ParaLSTM step: p = (Pi, Pf, Pg, Po) -> (c', h', J 2x2 d(c',h')/d(c,h))."""
+    p, w = _d(p), _d(w)
+    fc = ctypes.c_double()
+    fh = ctypes.c_double()
+    J = np.zeros(4)
+    _load().oracle_lstm_cell(_p(p), _p(w), float(c), float(h), ctypes.byref(fc),
+                             ctypes.byref(fh), _p(J))
+    return fc.value, fh.value, J.reshape(2, 2)
+
+
+def rollout_gru(P, a, h0=None):
+    """Sequential ParaGRU rollout. P: [B,L,3,D], a: [3,D], h0: [B,D] or None -> h [B,L,D]."""
+    P, a = _d(P), _d(a)
+    B, L, G, D = P.shape
+    assert G == 3
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    h = np.empty((B, L, D))
+    _load().oracle_rollout_gru(_p(P), _p(a), _p(h0), _p(h), B, L, D)
+    return h
+
+
+def rollout_lstm(P, a, c0=None, h0=None):
+    """Sequential ParaLSTM rollout. P: [B,L,4,D], a: [4,D] -> (c, h) each [B,L,D]."""
+    P, a = _d(P), _d(a)
+    B, L, G, D = P.shape
+    assert G == 4
+    c0 = None if c0 is None else _d(c0).reshape(B, D)
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    c = np.empty((B, L, D))
+    h = np.empty((B, L, D))
+    _load().oracle_rollout_lstm(_p(P), _p(a), _p(c0), _p(h0), _p(c), _p(h), B, L, D)
+    return c, h
+
+
+class NewtonResult:
+    def __init__(self, iterations, converged, nonfinite, rho, chan_iters, **states):
+        self.iterations = iterations
+        self.converged = bool(converged)
+        self.nonfinite = bool(nonfinite)
+        self.rho = rho                  # rho_0 .. rho_iterations
+        self.chan_iters = chan_iters    # per channel [B, D]
+        for k, v in states.items():
+            setattr(self, k, v)
+
+
+def newton_gru(P, a, h0=None, tol=1e-4, max_iters=32):
+    """Serial Newton for the ParaGRU system from h^0 = 0 (see oracle.c)."""
+    P, a = _d(P), _d(a)
+    B, L, G, D = P.shape
+    assert G == 3
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    h = np.empty((B, L, D))
+    rho = np.full(max_iters + 1, np.nan)
+    ci = np.empty((B, D), dtype=np.int32)
+    conv = ctypes.c_int()
+    nf = ctypes.c_int()
+    k = _load().oracle_newton_gru(_p(P), _p(a), _p(h0), float(tol), int(max_iters), B, L, D,
+                                  _p(h), _p(rho), ci.ctypes.data_as(_i32p), ctypes.byref(conv),
+                                  ctypes.byref(nf))
+    return NewtonResult(k, conv.value, nf.value, rho[: k + 1], ci, h=h)
+
+
+def newton_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32):
+    """Serial Newton for the ParaLSTM system from (c, h)^0 = 0 (see oracle.c)."""
+    P, a = _d(P), _d(a)
+    B, L, G, D = P.shape
+    assert G == 4
+    c0 = None if c0 is None else _d(c0).reshape(B, D)
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    c = np.empty((B, L, D))
+    h = np.empty((B, L, D))
+    rho = np.full(max_iters + 1, np.nan)
+    ci = np.empty((B, D), dtype=np.int32)
+    conv = ctypes.c_int()
+    nf = ctypes.c_int()
+    k = _load().oracle_newton_lstm(_p(P), _p(a), _p(c0), _p(h0), float(tol), int(max_iters),
+                                   B, L, D, _p(c), _p(h), _p(rho), ci.ctypes.data_as(_i32p),
+                                   ctypes.byref(conv), ctypes.byref(nf))
+    return NewtonResult(k, conv.value, nf.value, rho[: k + 1], ci, c=c, h=h)
+
+
+def residual_gru(P, a, h, h0=None):
+    """fp64 max_t |f(h_{t-1}, P_t) - h_t| of a given trajectory h [B,L,D]."""
+    P, a, h = _d(P), _d(a), _d(h)
+    B, L, G, D = P.shape
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    return _load().oracle_residual_gru(_p(P), _p(a), _p(h0), _p(h), B, L, D)

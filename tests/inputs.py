@@ -1,0 +1,135 @@
+"""Seeded synthetic inputs shared by the oracle side and the CUDA side.
+
+This module holds no arithmetic of the method: it only draws random numbers
+(numpy PCG64 ``default_rng``) in a fixed order and, for bf16 workloads, rounds
+the fp32 draws to bf16 once (round to nearest even).  Both sides receive the
+same bytes: the CUDA library reads the bf16 bits, the oracle reads the same
+values widened exactly to fp64.
+
+The pages measure on evaluation datasets and language-model corpora (ParaRNN
+Figure 4 caption; DEER summary's task table).  None of those is used here:
+these synthetic draws stand in for them, with the shapes of the workloads:
+
+=======  =====================================  ==========================
+name     operation                              shape (B, L, D)
+=======  =====================================  ==========================
+gru_s    ParaGRU solve, fp32                    2, 512, 16
+scan     diagonal affine scan, fp32             8, 4096, 1024
+gru_l    ParaGRU solve, fp32, L sweep 2^6..2^14 8, L, 1024
+lstm     ParaLSTM solve, fp32 (+ block scan)    8, 4096, 1024
+deer     ParaGRU solve, fp32, DEER shape        16, 2^20, 1
+lm       ParaGRU solve, bf16 P, fp32 state      8, 8192, 4096
+=======  =====================================  ==========================
+
+Distributions: projected gate inputs P ~ N(0, 1); diagonal recurrence weights
+a ~ U(-0.5, 0.5); h0 = c0 = 0 for the solves.  Diagonal scan: A ~ U(0, 1),
+b ~ N(0, 1), h0 ~ N(0, 1).  Block scan: A entries ~ U(-0.5, 0.5), b ~ N(0, 1),
+x0 ~ N(0, 1).  Draw order: P (or A) first, then a (or b), then h0 (or x0).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+WORKLOADS = {
+    "gru_s": dict(op="gru", B=2, L=512, D=16, seed=1, bf16=False),
+    "scan": dict(op="scan_diag", B=8, L=4096, D=1024, seed=2, bf16=False),
+    "gru_l": dict(op="gru", B=8, L=4096, D=1024, seed=2, bf16=False),
+    "lstm": dict(op="lstm", B=8, L=4096, D=1024, seed=3, bf16=False),
+    "block2": dict(op="scan_block2", B=8, L=4096, D=1024, seed=3, bf16=False),
+    "deer": dict(op="gru", B=16, L=1 << 20, D=1, seed=4, bf16=False),
+    "lm": dict(op="gru", B=8, L=8192, D=4096, seed=5, bf16=True),
+}
+
+L_SWEEP = [1 << e for e in range(6, 15)]
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def round_to_bf16(x32: np.ndarray):
+    """Round fp32 values to bf16 (nearest even).  Returns (bits uint16, values fp32)."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32)
+    bias = np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    bits = ((u + bias) >> np.uint32(16)).astype(np.uint16)
+    vals = (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    return bits, vals
+
+
+def _normal(rng, shape):
+    return rng.standard_normal(size=shape, dtype=np.float32)
+
+
+def _uniform(rng, lo, hi, shape):
+    return (rng.random(size=shape, dtype=np.float32) * np.float32(hi - lo) + np.float32(lo)).astype(
+        np.float32)
+
+
+def gate_inputs(G, B, L, D, seed, bf16=False, h0_normal=False):
+    """Projected pre-activations P [B,L,G,D], weights a [G,D], initial state.
+
+    Returns a dict with ``P`` (fp32 values, already bf16-rounded if ``bf16``),
+    ``P_bits`` (uint16 bf16 bits or None), ``a`` [G,D] fp32 and ``h0`` [B,D]
+    (and ``c0`` for G == 4) fp32, zeros unless ``h0_normal``.
+    """
+    rng = _rng(seed)
+    P = _normal(rng, (B, L, G, D))
+    a = _uniform(rng, -0.5, 0.5, (G, D))
+    out = {}
+    if h0_normal:
+        out["h0"] = _normal(rng, (B, D))
+        if G == 4:
+            out["c0"] = _normal(rng, (B, D))
+    else:
+        out["h0"] = np.zeros((B, D), np.float32)
+        if G == 4:
+            out["c0"] = np.zeros((B, D), np.float32)
+    bits = None
+    if bf16:
+        bits, P = round_to_bf16(P)
+    out.update(P=P, P_bits=bits, a=a)
+    return out
+
+
+def gru_inputs(B, L, D, seed, bf16=False, h0_normal=False):
+    return gate_inputs(3, B, L, D, seed, bf16, h0_normal)
+
+
+def lstm_inputs(B, L, D, seed, bf16=False, h0_normal=False):
+    return gate_inputs(4, B, L, D, seed, bf16, h0_normal)
+
+
+def scan_diag_inputs(B, L, D, seed, a_lo=0.0, a_hi=1.0):
+    rng = _rng(seed)
+    A = _uniform(rng, a_lo, a_hi, (B, L, D))
+    b = _normal(rng, (B, L, D))
+    h0 = _normal(rng, (B, D))
+    return dict(A=A, b=b, h0=h0)
+
+
+def scan_block2_inputs(B, L, D, seed, a_lo=-0.5, a_hi=0.5):
+    rng = _rng(seed)
+    A = _uniform(rng, a_lo, a_hi, (B, L, D, 2, 2))
+    b = _normal(rng, (B, L, D, 2))
+    x0 = _normal(rng, (B, D, 2))
+    return dict(A=A, b=b, x0=x0)
+
+
+def workload_inputs(name, L=None):
+    """Inputs of a named workload (``L`` overrides the length for the sweep)."""
+    w = dict(WORKLOADS[name])
+    if L is not None:
+        w["L"] = L
+        seed = [w["seed"], L]
+    else:
+        seed = w["seed"]
+    op = w["op"]
+    if op == "gru":
+        return gru_inputs(w["B"], w["L"], w["D"], seed, w["bf16"])
+    if op == "lstm":
+        return lstm_inputs(w["B"], w["L"], w["D"], seed, w["bf16"])
+    if op == "scan_diag":
+        return scan_diag_inputs(w["B"], w["L"], w["D"], seed)
+    if op == "scan_block2":
+        return scan_block2_inputs(w["B"], w["L"], w["D"], seed)
+    raise KeyError(op)
