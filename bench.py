@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the ParaGRU Newton solve (and the diagonal affine scan) on B200.
+
+One step = one complete Newton solve, all iterations, of the ParaGRU layer
+B=8, L=4096, D=1024 in fp32 (P ~ N(0,1), a ~ U(-0.5,0.5), h0 = 0, tol 1e-4,
+max 32 iterations) -- the workload shape of the diagonal-scan configuration,
+whose Newton solve is its headline metric.  The same run times the diagonal
+affine scan at that shape (the scan HBM GB/s half of the metric).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gru_l|lm|deer|gru_s|lstm]
+
+Under torchrun (N > 1) every rank solves its own independent batch (weak
+scaling, no data-path collective); the time is the max over ranks.  Rank 0
+prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from tests import inputs  # noqa: E402  (seeded synthetic inputs only)
+
+METRIC = "Newton-solve channel-steps/sec (B*L*D) and scan HBM GB/s, % of B200 HBM peak"
+UNIT = "channel-steps/s"
+MUFU_PER_SM_PER_CLK = 16        # ex2 / rcp issue rate per SM per clock
+SMS = 148
+MUFU_PER_STEP = {"gru": 6, "lstm": 10}   # (ex2 + rcp) per sigmoid/tanh, per channel-step
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured", j
+    except Exception:
+        return 6650.0, "fallback", {}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (weak scaling: one independent batch per rank)
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def maybe_init_pg(world, backend):
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(val, world, device):
+    if world == 1:
+        return val
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([val], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# sweep accounting (mirrors the kernel's schedule: m_first then m_next per sweep)
+# ---------------------------------------------------------------------------
+def evaluated_iterations(passes, max_iters, m_first=4, m_next=2):
+    k0, total = 0, 0
+    for q in range(passes):
+        m = m_first if q == 0 else m_next
+        m = min(m, max_iters + 1 - k0)
+        total += m
+        k0 += m
+    return total
+
+
+def algorithmic_bytes(op, bf16, B, L, D, passes):
+    """Bytes a launch must move: each sweep reads P once, reads the iterate
+    (not in the first sweep: h^0 = 0) and writes the new iterate."""
+    G = 3 if op == "gru" else 4
+    ns = 1 if op == "gru" else 2
+    pbytes = G * (2 if bf16 else 4)
+    first = pbytes + 4 * ns
+    later = pbytes + 8 * ns
+    return B * L * D * (first + later * (passes - 1))
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    import torch
+
+    import nonlinear_rnn_solve_newton_b200 as pr
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    maybe_init_pg(world, "nccl")
+    pr.load()
+    w = dict(inputs.WORKLOADS[args.workload])
+    op, B, L, D, bf16 = w["op"], w["B"], w["L"], w["D"], w["bf16"]
+    seed = w["seed"] if rank == 0 else [w["seed"], 1000 + rank]
+    if op == "gru":
+        x = inputs.gru_inputs(B, L, D, seed, bf16)
+    else:
+        x = inputs.lstm_inputs(B, L, D, seed, bf16)
+    if bf16:
+        P_host = torch.from_numpy(x["P_bits"].view(np.int16)).view(torch.bfloat16)
+    else:
+        P_host = torch.from_numpy(x["P"])
+    P = P_host.to(device)
+    a = torch.from_numpy(x["a"]).to(device)
+    h0 = torch.from_numpy(x["h0"]).to(device)
+    c0 = torch.from_numpy(x["c0"]).to(device) if op == "lstm" else None
+    tol, max_iters = 1e-4, 32
+    N = B * L * D
+    stream = torch.cuda.current_stream()
+
+    h = torch.empty((B, L, D), dtype=torch.float32, device=device)
+    c = torch.empty_like(h) if op == "lstm" else None
+    info_t = torch.empty(pr.INFO_BYTES // 4, dtype=torch.int32, device=device)
+
+    def step():
+        if op == "gru":
+            pr.solve_gru(P, a, h0, tol, max_iters, out=h, info=info_t)
+        else:
+            pr.solve_lstm(P, a, c0, h0, tol, max_iters, out=(c, h), info=info_t)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    info = pr.SolveInfo(info_t)
+    if info.status != 0 or not info.converged:
+        raise SystemExit(f"solve did not converge: {info.as_dict()}")
+    iters, passes = info.iterations, info.passes
+
+    # ---- timed region: exactly K solves --------------------------------------
+    K = args.steps
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        evs[0].record(stream)
+        for i in range(K):
+            step()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
+    ms_local = evs[0].elapsed_time(evs[K]) / K
+    ms = max_over_ranks(ms_local, world, device)
+    value = world * N / (ms * 1e-3)
+    clocks = clk.summary()
+
+    # dominant kernel: the fused Newton kernel, one launch per solve.  Its
+    # per-launch time is bracketed by events on the launching stream; the
+    # bracket also holds the 1-2 us zeroing of the look-back flags.
+    launch_ms = statistics.mean(per_step)
+    hbm_peak, peak_kind, pk = peaks()
+    bytes_launch = algorithmic_bytes(op, bf16, B, L, D, passes)
+    achieved_gbs = bytes_launch / (launch_ms * 1e-3) / 1e9
+    ev_iters = evaluated_iterations(passes, max_iters)
+    mufu_ops = N * ev_iters * MUFU_PER_STEP[op]
+    sm_mhz = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
+    mufu_peak = SMS * MUFU_PER_SM_PER_CLK * sm_mhz * 1e6
+    mufu_frac = mufu_ops / (launch_ms * 1e-3) / mufu_peak
+    hbm_frac = achieved_gbs / hbm_peak
+    if mufu_frac > hbm_frac:
+        roofline = {"bound": "alu", "achieved": mufu_ops / (launch_ms * 1e-3) / 1e12,
+                    "peak": mufu_peak / 1e12, "unit": "Tops/s (MUFU ex2+rcp)",
+                    "frac": mufu_frac, "traffic": None,
+                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": hbm_frac, "peak_kind": peak_kind}}
+    else:
+        roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": hbm_frac, "traffic": None, "peak_kind": peak_kind,
+                    "alu": {"achieved": mufu_ops / (launch_ms * 1e-3) / 1e12,
+                            "peak": mufu_peak / 1e12, "unit": "Tops/s (MUFU ex2+rcp)",
+                            "frac": mufu_frac}}
+    roofline["kernel"] = "pararnn_kernel<GRU>" if op == "gru" else "pararnn_kernel<LSTM>"
+    roofline["algorithmic_bytes_per_launch"] = bytes_launch
+    roofline["launch_ms"] = launch_ms
+
+    # ---- the diagonal scan at the same shape (the scan half of the metric) ---
+    scan = None
+    if args.workload == "gru_l" and not args.no_scan:
+        xs = inputs.scan_diag_inputs(B, L, D, inputs.WORKLOADS["scan"]["seed"])
+        A_s = torch.from_numpy(xs["A"]).to(device)
+        b_s = torch.from_numpy(xs["b"]).to(device)
+        h0_s = torch.from_numpy(xs["h0"]).to(device)
+        hs = torch.empty_like(A_s)
+        for _ in range(max(args.warmup, 3)):
+            pr.scan_diag(A_s, b_s, h0_s, out=hs)
+        torch.cuda.synchronize()
+        sev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        barrier(world)
+        sev[0].record(stream)
+        for _ in range(K):
+            pr.scan_diag(A_s, b_s, h0_s, out=hs)
+        sev[1].record(stream)
+        torch.cuda.synchronize()
+        sms = max_over_ranks(sev[0].elapsed_time(sev[1]) / K, world, device)
+        sbytes = 12 * B * L * D
+        sgbs = sbytes / (sms * 1e-3) / 1e9
+        scan = {"workload": f"diagonal scan fp32 B={B} L={L} D={D}", "ms": sms,
+                "channel_steps_per_s": world * B * L * D / (sms * 1e-3),
+                "achieved_gbs": sgbs, "algorithmic_bytes": sbytes,
+                "frac_of_measured_hbm": sgbs / hbm_peak, "frac_of_8tbs": sgbs / 8000.0}
+        del A_s, b_s, h0_s, hs
+
+    # ---- end to end through the public API with pinned host buffers ---------
+    P_pin = P_host.pin_memory()
+    a_pin = torch.from_numpy(x["a"]).pin_memory()
+    h0_pin = torch.from_numpy(x["h0"]).pin_memory()
+    out_pin = torch.empty((B, L, D), dtype=torch.float32).pin_memory()
+    out2_pin = torch.empty((B, L, D), dtype=torch.float32).pin_memory() if op == "lstm" else None
+
+    def e2e_step():
+        Pd = P_pin.to(device, non_blocking=True)
+        ad = a_pin.to(device, non_blocking=True)
+        h0d = h0_pin.to(device, non_blocking=True)
+        if op == "gru":
+            hd, _ = pr.solve_gru(Pd, ad, h0d, tol, max_iters, out=h, info=info_t)
+            out_pin.copy_(hd, non_blocking=True)
+        else:
+            cd, hd, _ = pr.solve_lstm(Pd, ad, None, h0d, tol, max_iters, out=(c, h), info=info_t)
+            out_pin.copy_(hd, non_blocking=True)
+            out2_pin.copy_(cd, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    Ke = min(K, 5)
+    barrier(world)
+    ee[0].record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    ee[1].record(stream)
+    torch.cuda.synchronize()
+    ems = max_over_ranks(ee[0].elapsed_time(ee[1]) / Ke, world, device)
+    h2d = P_host.numel() * P_host.element_size() + 4 * a_pin.numel() + 4 * h0_pin.numel()
+    d2h = 4 * N * (2 if op == "lstm" else 1)
+    e2e = {"value": world * N / (ems * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+
+    # ---- the oracle on the host cores (rank 0, N = 1 only) -------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(x, op, B, L, D, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        wl = {"gru_l": "ParaGRU Newton solve fp32",
+              "lm": "ParaGRU Newton solve, bf16 P, fp32 state",
+              "deer": "ParaGRU Newton solve fp32 (DEER shape)",
+              "gru_s": "ParaGRU Newton solve fp32 (small)",
+              "lstm": "ParaLSTM Newton solve fp32"}[args.workload]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32" if not bf16 else "bf16-in/f32",
+            "data": "synthetic (seeded numpy: P~N(0,1), a~U(-0.5,0.5), h0=0)",
+            "config": {"workload": f"{wl} B={B} L={L} D={D}", "B": B, "L": L, "D": D,
+                       "tol": tol, "max_iters": max_iters, "newton_iterations": iters,
+                       "sweeps": passes, "evaluated_iterations": ev_iters,
+                       "parallelism": f"replicas x{world} (independent batches)",
+                       "l2": "inputs larger than L2 (P alone is %.0f MB)" % (
+                           P_host.numel() * P_host.element_size() / 1e6)},
+            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "gpu_launches": K, "scan": scan, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def cpu_baseline(x, op, B, L, D, budget_s=15.0):
+    """The oracle's serial Newton (and its sequential rollout) on the host cores,
+    on a bounded sample of the workload: the first batch rows, as many channels
+    as fit the time budget (estimated from a short calibration run)."""
+    import oracle
+
+    oracle.build()
+    cores = oracle.get_threads()
+    # calibrate on 64 channels
+    nd = min(D, 64)
+    Pc = x["P"][:1, :, :, :nd]
+    ac = x["a"][:, :nd]
+    t0 = time.perf_counter()
+    if op == "gru":
+        oracle.newton_gru(Pc, ac, tol=1e-4, max_iters=32)
+    else:
+        oracle.newton_lstm(Pc, ac, tol=1e-4, max_iters=32)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    per_chan = dt / nd
+    nchan = int(max(1, min(B * D, budget_s / per_chan)))
+    nb = max(1, min(B, nchan // D)) if nchan >= D else 1
+    ndd = D if nchan >= D else nchan
+    Ps = x["P"][:nb, :, :, :ndd]
+    as_ = x["a"][:, :ndd]
+    t0 = time.perf_counter()
+    if op == "gru":
+        res = oracle.newton_gru(Ps, as_, tol=1e-4, max_iters=32)
+    else:
+        res = oracle.newton_lstm(Ps, as_, tol=1e-4, max_iters=32)
+    dt = time.perf_counter() - t0
+    steps = nb * L * ndd
+    t1 = time.perf_counter()
+    if op == "gru":
+        oracle.rollout_gru(Ps, as_)
+    else:
+        oracle.rollout_lstm(Ps, as_)
+    dtr = time.perf_counter() - t1
+    return {"value": steps / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"serial fp64 Newton on B={nb} x D={ndd} channels x L={L} "
+                      f"({steps} channel-steps, {res.iterations} iterations, {dt:.1f} s)",
+            "rollout_channel_steps_per_s": steps / dtr}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle, as it stands, on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, world, rank, local):
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    w = dict(inputs.WORKLOADS[args.workload])
+    op, B, L, D, bf16 = w["op"], w["B"], w["L"], w["D"], w["bf16"]
+    x = (inputs.gru_inputs if op == "gru" else inputs.lstm_inputs)(B, L, D, w["seed"], bf16)
+    cores = oracle.get_threads()
+    # each step: the serial Newton on one batch row's first channels (bounded)
+    nd = min(D, 256)
+    Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
+    as_ = np.ascontiguousarray(x["a"][:, :nd])
+    fn = oracle.newton_gru if op == "gru" else oracle.newton_lstm
+
+    def step():
+        return fn(Ps, as_, tol=1e-4, max_iters=32)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    steps = L * nd
+    value = steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 1), "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded numpy)",
+            "config": {"workload": f"oracle serial Newton, sample of B=1 x D={nd} x L={L} "
+                                   f"from the {args.workload} workload (B={B}, D={D})"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"B=1, D={nd}, L={L} per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gru_l", choices=["gru_l", "lm", "deer", "gru_s", "lstm"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-scan", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

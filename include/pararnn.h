@@ -1,0 +1,175 @@
+/*
+ * pararnn.h -- C ABI of libpararnn.so: parallel-in-time Newton solves of
+ * nonlinear RNN recurrences on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed (page titles and passages):
+ *  - "ParaRNN: Unlocking Parallel Training of Nonlinear RNNs for Large Language
+ *    Models", TL;DR and Abstract: the recurrence h_t = f(h_{t-1}, x_t) over a
+ *    whole sequence is one nonlinear system, solved by Newton's iterations; each
+ *    iteration solves a block bi-diagonal linear system by a parallel reduction.
+ *    Figure 2 caption: diagonal Jacobians (ParaGRU) and 2x2 block-diagonal ones
+ *    (ParaLSTM).  Figure 4 caption: the residual is the max over the batch.
+ *  - DEER summary ("Recasting nonlinear recurrences as quadratically convergent
+ *    fixed-point iterations with parallel scans"): the converged result equals
+ *    sequential evaluation; a tolerance of 1e-4 suffices in float32; Newton may
+ *    diverge far from the solution (no damping here: that is reported, not fixed).
+ *
+ * Conventions shared by every entry point
+ *  - Every array pointer is a DEVICE pointer owned by the caller.  The library
+ *    never allocates, frees or synchronises; each call only enqueues work on
+ *    `stream` (a cudaStream_t passed as void*, NULL = legacy default stream)
+ *    and returns.
+ *  - Layouts are C order with the channel axis D innermost.  A "channel" is
+ *    one (b, d) pair; channels are independent problems.
+ *  - Outputs must not alias inputs.  Arrays must be naturally aligned for their
+ *    element type (4 B for float, 2 B for bf16); the 2x2 scan additionally needs
+ *    A 16-byte aligned and b, x, x0 8-byte aligned.
+ *  - `ws` is caller-owned device scratch of at least pararnn_workspace_size()
+ *    bytes, 256-byte aligned.  Its contents need no initialisation and are
+ *    meaningless after the call.  Concurrent calls need distinct workspaces.
+ *  - The return value reports host-side validation and launch errors only.
+ *    What happens on the device (iteration count, convergence, a timed-out
+ *    wait, a non-finite residual) is written to a caller-owned device struct
+ *    that is valid once `stream` has been synchronised.
+ *  - Every device-side wait (look-back between time chunks, the grid barrier
+ *    between sweeps) is bounded; on expiry the kernel stops, reports
+ *    PARARNN_ERR_DEVICE_TIMEOUT and leaves the CUDA context usable.
+ */
+#ifndef PARARNN_H_
+#define PARARNN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PARARNN_VERSION 1
+/* Largest max_iters a solve accepts (the info struct keeps every residual). */
+#define PARARNN_MAX_ITERS 127
+
+typedef enum {
+  PARARNN_OK = 0,
+  PARARNN_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misalignment, bad dtype */
+  PARARNN_ERR_UNSUPPORTED = 2,      /* no kernel for this device (needs sm_100a) */
+  PARARNN_ERR_CUDA = 3,             /* a CUDA runtime call failed (launch, memset) */
+  PARARNN_ERR_DEVICE_TIMEOUT = 4,   /* device side: a bounded wait expired */
+  PARARNN_ERR_NONFINITE = 5,        /* device side: a residual was NaN or Inf */
+  PARARNN_ERR_WORKSPACE = 6         /* ws is NULL, too small or misaligned */
+} pararnn_status_t;
+
+typedef enum { PARARNN_F32 = 0, PARARNN_BF16 = 1 } pararnn_dtype_t;
+
+typedef enum {
+  PARARNN_OP_SCAN_DIAG = 0,
+  PARARNN_OP_SCAN_BLOCK2 = 1,
+  PARARNN_OP_GRU = 2,
+  PARARNN_OP_LSTM = 3
+} pararnn_op_t;
+
+/* Device-side outcome of a solve (caller-owned DEVICE memory, written by the
+ * kernel; read it after synchronising the stream).
+ *  iterations   : Newton semantics -- the first k with rho_k <= tol, or
+ *                 max_iters if none (then converged = 0).
+ *  converged    : 1 if some rho_k <= tol.
+ *  status       : a pararnn_status_t for the device side (OK, DEVICE_TIMEOUT,
+ *                 NONFINITE).
+ *  updates      : Newton updates contained in the returned trajectory.  The
+ *                 kernel evaluates m iterations per sweep over memory, so a
+ *                 converged solve may return h^{k+j} (j >= 1 further updates
+ *                 after the certified iterate h^k); an unconverged one returns
+ *                 exactly h^{max_iters}.
+ *  passes       : sweeps over the inputs in HBM.
+ *  max_residual : rho at `iterations`.
+ *  rho[k]       : rho_k = max over (b, t, d, component) of |f(h^k_{t-1}) - h^k_t|
+ *                 for every k evaluated (k <= iterations at least); others 0. */
+typedef struct {
+  int32_t iterations;
+  int32_t converged;
+  int32_t status;
+  int32_t updates;
+  int32_t passes;
+  int32_t reserved;
+  float max_residual;
+  float rho[PARARNN_MAX_ITERS + 1];
+} pararnn_solve_info_t;
+
+/* Optional tuning and test hooks (host struct; pass NULL for defaults).
+ *  iters_first : Newton iterations evaluated in the first sweep (0 = 4).
+ *  iters_next  : Newton iterations per later sweep (0 = 2).
+ *  wait_timeout_ns : bound on every device-side wait (0 = 1e9, i.e. 1 s).
+ *  debug_stall_unit: test hook, -1 = off.  The work unit with this index
+ *                 never publishes its look-back status, so the units after it
+ *                 run their bounded waits out; the call must then report
+ *                 PARARNN_ERR_DEVICE_TIMEOUT. */
+typedef struct {
+  int32_t iters_first;
+  int32_t iters_next;
+  int64_t wait_timeout_ns;
+  int64_t debug_stall_unit;
+} pararnn_options_t;
+
+/* Bytes of workspace the call with the same arguments needs. 0 on bad sizes. */
+size_t pararnn_workspace_size(pararnn_op_t op, int64_t B, int64_t L, int64_t D,
+                              int32_t max_iters, const pararnn_options_t* opts);
+
+/* Diagonal affine scan (the linear solve of one Newton step, diagonal case;
+ * ParaRNN Figure 2 left):  h_t = A_t * h_{t-1} + b_t  for t = 1..L.
+ *  A, b : [B, L, D] fp32.      h0 : [B, D] fp32 or NULL (= 0).
+ *  h    : [B, L, D] fp32 output (t = 1..L; h0 is not repeated).
+ *  status_dev : optional device int32 receiving the device-side status. */
+pararnn_status_t pararnn_scan_diag(const float* A, const float* b, const float* h0, float* h,
+                                   int64_t B, int64_t L, int64_t D, void* ws, size_t ws_bytes,
+                                   int32_t* status_dev, const pararnn_options_t* opts,
+                                   void* stream);
+
+/* 2x2 block affine scan (ParaLSTM's linear solve; ParaRNN Figure 2 left):
+ *  x_t = A_t x_{t-1} + b_t,  A : [B, L, D, 2, 2] row-major ((0,0),(0,1),(1,0),(1,1)),
+ *  b : [B, L, D, 2],  x0 : [B, D, 2] or NULL,  x : [B, L, D, 2] output. */
+pararnn_status_t pararnn_scan_block2(const float* A, const float* b, const float* x0, float* x,
+                                     int64_t B, int64_t L, int64_t D, void* ws, size_t ws_bytes,
+                                     int32_t* status_dev, const pararnn_options_t* opts,
+                                     void* stream);
+
+/* ParaGRU Newton solve (ParaRNN Abstract; Figure 2 right, Figure 5 left).
+ * Cell, per channel, with diagonal recurrence weights:
+ *   z = sig(Pz + az h), r = sig(Pr + ar h), c = tanh(Pc + ac (r h)),
+ *   h' = (1 - z) h + z c.
+ *  P  : [B, L, 3, D] projected pre-activations, gate order (z, r, c); fp32 or
+ *       bf16 (p_dtype); state, Jacobians and scan are fp32 either way.
+ *  a  : [3, D] fp32 (az, ar, ac).     h0 : [B, D] fp32 or NULL (= 0).
+ *  h  : [B, L, D] fp32 output trajectory, t = 1..L.
+ *  tol: stop at the first k with rho_k <= tol (1e-4 per the DEER summary).
+ *  max_iters : 0..PARARNN_MAX_ITERS.   info : device struct (required).
+ * Newton starts from h^0 = 0 and applies no damping. */
+pararnn_status_t pararnn_solve_gru(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                   const float* h0, float* h, int64_t B, int64_t L, int64_t D,
+                                   float tol, int32_t max_iters, void* ws, size_t ws_bytes,
+                                   pararnn_solve_info_t* info, const pararnn_options_t* opts,
+                                   void* stream);
+
+/* ParaLSTM Newton solve with per-channel state (c, h) and a 2x2 Jacobian
+ * (ParaRNN Figure 2 caption; Figure 5 right).  Cell (diagonal recurrence on h):
+ *   i = sig(Pi + ai h), f = sig(Pf + af h), g = tanh(Pg + ag h),
+ *   o = sig(Po + ao h), c' = f c + i g, h' = o tanh(c').
+ *  P : [B, L, 4, D] gate order (i, f, g, o), fp32 or bf16.   a : [4, D] fp32.
+ *  c0, h0 : [B, D] fp32 or NULL (= 0).   c, h : [B, L, D] fp32 outputs.
+ *  The residual max runs over both components.  Other arguments as for GRU. */
+pararnn_status_t pararnn_solve_lstm(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                    const float* c0, const float* h0, float* c, float* h,
+                                    int64_t B, int64_t L, int64_t D, float tol, int32_t max_iters,
+                                    void* ws, size_t ws_bytes, pararnn_solve_info_t* info,
+                                    const pararnn_options_t* opts, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* pararnn_status_string(pararnn_status_t status);
+
+/* PARARNN_VERSION of the loaded library. */
+int32_t pararnn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARARNN_H_ */

@@ -1,0 +1,300 @@
+"""Python binding of libpararnn.so: Newton solves of nonlinear RNNs on a B200.
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+kernels of ``libpararnn.so`` (C ABI in ``include/pararnn.h``); torch provides
+device memory (outputs, workspace, the info struct) and the current stream.
+There is no CPU fallback: if the library is missing or the tensors are not on a
+CUDA device, the calls raise.
+
+Entry points (same names as the C ABI, without the ``pararnn_`` prefix):
+
+* ``scan_diag(A, b, h0=None)``      h_t = A_t h_{t-1} + b_t           [B, L, D]
+* ``scan_block2(A, b, x0=None)``    x_t = A_t x_{t-1} + b_t, 2x2 blocks  [B, L, D, 2]
+* ``solve_gru(P, a, h0=None, tol=1e-4, max_iters=32)``   ParaGRU Newton solve
+* ``solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32)``  ParaLSTM Newton solve
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+__all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "workspace_size",
+           "SolveInfo", "Options", "PararnnError", "library_path", "load", "MAX_ITERS"]
+
+MAX_ITERS = 127
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libpararnn.so")
+
+OP_SCAN_DIAG, OP_SCAN_BLOCK2, OP_GRU, OP_LSTM = 0, 1, 2, 3
+F32, BF16 = 0, 1
+
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA runtime error",
+           4: "device-side wait timed out", 5: "non-finite residual",
+           6: "workspace missing, too small or misaligned"}
+
+
+class PararnnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {_STATUS.get(self.status, 'unknown status')} ({self.status})")
+
+
+class _Info(ctypes.Structure):
+    _fields_ = [("iterations", ctypes.c_int32), ("converged", ctypes.c_int32),
+                ("status", ctypes.c_int32), ("updates", ctypes.c_int32),
+                ("passes", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("max_residual", ctypes.c_float), ("rho", ctypes.c_float * (MAX_ITERS + 1))]
+
+
+class Options(ctypes.Structure):
+    """Tuning and test hooks (see pararnn_options_t)."""
+    _fields_ = [("iters_first", ctypes.c_int32), ("iters_next", ctypes.c_int32),
+                ("wait_timeout_ns", ctypes.c_int64), ("debug_stall_unit", ctypes.c_int64)]
+
+    def __init__(self, iters_first=0, iters_next=0, wait_timeout_ns=0, debug_stall_unit=-1):
+        super().__init__(iters_first, iters_next, wait_timeout_ns, debug_stall_unit)
+
+
+INFO_BYTES = ctypes.sizeof(_Info)
+
+_lock = threading.Lock()
+_lib = None
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+def load(build_if_missing: bool = True):
+    """Load libpararnn.so (building it in-tree with nvcc if it is missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if build_if_missing and _build.needs_build():
+                _build.build()
+            if not os.path.exists(library_path):
+                raise RuntimeError(f"libpararnn.so not found at {library_path}")
+            lib = ctypes.CDLL(library_path)
+            lib.pararnn_workspace_size.argtypes = [ctypes.c_int, _i64, _i64, _i64, ctypes.c_int32,
+                                                   _vp]
+            lib.pararnn_workspace_size.restype = ctypes.c_size_t
+            for name in ("pararnn_scan_diag", "pararnn_scan_block2"):
+                f = getattr(lib, name)
+                f.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp, _vp,
+                              _vp]
+                f.restype = ctypes.c_int
+            lib.pararnn_solve_gru.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64,
+                                              ctypes.c_float, ctypes.c_int32, _vp, ctypes.c_size_t,
+                                              _vp, _vp, _vp]
+            lib.pararnn_solve_gru.restype = ctypes.c_int
+            lib.pararnn_solve_lstm.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i64,
+                                               _i64, _i64, ctypes.c_float, ctypes.c_int32, _vp,
+                                               ctypes.c_size_t, _vp, _vp, _vp]
+            lib.pararnn_solve_lstm.restype = ctypes.c_int
+            lib.pararnn_status_string.argtypes = [ctypes.c_int]
+            lib.pararnn_status_string.restype = ctypes.c_char_p
+            lib.pararnn_version.restype = ctypes.c_int32
+            _lib = lib
+    return _lib
+
+
+def workspace_size(op: int, B: int, L: int, D: int, max_iters: int = 0, opts: Options | None = None):
+    n = load().pararnn_workspace_size(int(op), int(B), int(L), int(D), int(max_iters),
+                                      ctypes.byref(opts) if opts is not None else None)
+    if n == 0:
+        raise PararnnError(1, "workspace_size")
+    return int(n)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_dev(name, t, dtype, shape):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_handle(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+_ws_cache = threading.local()
+
+
+def _workspace(nbytes, device):
+    """Workspace from torch's allocator, reused between calls on the same thread and device."""
+    cache = getattr(_ws_cache, "bufs", None)
+    if cache is None:
+        cache = _ws_cache.bufs = {}
+    key = (device.index if device.index is not None else torch.cuda.current_device())
+    buf = cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        cache[key] = buf
+    return buf
+
+
+class SolveInfo:
+    """Device-side outcome of a solve; fields are read (one device->host copy) on first access."""
+
+    def __init__(self, dev_tensor: torch.Tensor):
+        self.tensor = dev_tensor
+        self._host = None
+
+    def _get(self):
+        if self._host is None:
+            raw = self.tensor.cpu().numpy().tobytes()
+            self._host = _Info.from_buffer_copy(raw)
+        return self._host
+
+    @property
+    def iterations(self):
+        return int(self._get().iterations)
+
+    @property
+    def converged(self):
+        return bool(self._get().converged)
+
+    @property
+    def status(self):
+        return int(self._get().status)
+
+    @property
+    def updates(self):
+        return int(self._get().updates)
+
+    @property
+    def passes(self):
+        return int(self._get().passes)
+
+    @property
+    def max_residual(self):
+        return float(self._get().max_residual)
+
+    @property
+    def rho(self):
+        h = self._get()
+        return [float(h.rho[k]) for k in range(MAX_ITERS + 1)]
+
+    def as_dict(self):
+        return dict(iterations=self.iterations, converged=self.converged, status=self.status,
+                    updates=self.updates, passes=self.passes, max_residual=self.max_residual)
+
+
+def _raise(st, where):
+    if st != 0:
+        raise PararnnError(st, where)
+
+
+def scan_diag(A, b, h0=None, out=None, status=None, opts: Options | None = None, stream=None):
+    """h[b, t, d] = A[b, t, d] * h[b, t-1, d] + b[b, t, d] (fp32, [B, L, D])."""
+    lib = load()
+    B, L, D = A.shape
+    _check_dev("A", A, torch.float32, (B, L, D))
+    _check_dev("b", b, torch.float32, (B, L, D))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    h = torch.empty_like(A) if out is None else out
+    _check_dev("out", h, torch.float32, (B, L, D))
+    n = workspace_size(OP_SCAN_DIAG, B, L, D, 0, opts)
+    ws = _workspace(n, A.device)
+    st = lib.pararnn_scan_diag(_ptr(A), _ptr(b), _ptr(h0), _ptr(h), B, L, D, _ptr(ws), ws.numel(),
+                               _ptr(status), ctypes.byref(opts) if opts is not None else None,
+                               _stream_handle(stream))
+    _raise(st, "pararnn_scan_diag")
+    return h
+
+
+def scan_block2(A, b, x0=None, out=None, status=None, opts: Options | None = None, stream=None):
+    """x_t = A_t x_{t-1} + b_t with A [B, L, D, 2, 2] (row-major) and x, b [B, L, D, 2]."""
+    lib = load()
+    B, L, D = A.shape[:3]
+    _check_dev("A", A, torch.float32, (B, L, D, 2, 2))
+    _check_dev("b", b, torch.float32, (B, L, D, 2))
+    _check_dev("x0", x0, torch.float32, (B, D, 2))
+    x = torch.empty_like(b) if out is None else out
+    _check_dev("out", x, torch.float32, (B, L, D, 2))
+    n = workspace_size(OP_SCAN_BLOCK2, B, L, D, 0, opts)
+    ws = _workspace(n, A.device)
+    st = lib.pararnn_scan_block2(_ptr(A), _ptr(b), _ptr(x0), _ptr(x), B, L, D, _ptr(ws),
+                                 ws.numel(), _ptr(status),
+                                 ctypes.byref(opts) if opts is not None else None,
+                                 _stream_handle(stream))
+    _raise(st, "pararnn_scan_block2")
+    return x
+
+
+def _p_dtype(P):
+    if P.dtype == torch.float32:
+        return F32
+    if P.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"P must be float32 or bfloat16, got {P.dtype}")
+
+
+def solve_gru(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
+              opts: Options | None = None, stream=None):
+    """ParaGRU Newton solve.  P [B, L, 3, D] (z, r, c), a [3, D] -> (h [B, L, D], SolveInfo)."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 3:
+        raise ValueError("P must be [B, L, 3, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 3, D))
+    _check_dev("a", a, torch.float32, (3, D))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    h = torch.empty((B, L, D), dtype=torch.float32, device=P.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, L, D))
+    if info is None:
+        info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    n = workspace_size(OP_GRU, B, L, D, max_iters, opts)
+    ws = _workspace(n, P.device)
+    st = lib.pararnn_solve_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D, float(tol),
+                               int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
+                               ctypes.byref(opts) if opts is not None else None,
+                               _stream_handle(stream))
+    _raise(st, "pararnn_solve_gru")
+    return h, SolveInfo(info)
+
+
+def solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
+               opts: Options | None = None, stream=None):
+    """ParaLSTM Newton solve.  P [B, L, 4, D] (i, f, g, o), a [4, D] -> (c, h, SolveInfo)."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 4:
+        raise ValueError("P must be [B, L, 4, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 4, D))
+    _check_dev("a", a, torch.float32, (4, D))
+    _check_dev("c0", c0, torch.float32, (B, D))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    if out is None:
+        c = torch.empty((B, L, D), dtype=torch.float32, device=P.device)
+        h = torch.empty((B, L, D), dtype=torch.float32, device=P.device)
+    else:
+        c, h = out
+    _check_dev("c", c, torch.float32, (B, L, D))
+    _check_dev("h", h, torch.float32, (B, L, D))
+    if info is None:
+        info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    n = workspace_size(OP_LSTM, B, L, D, max_iters, opts)
+    ws = _workspace(n, P.device)
+    st = lib.pararnn_solve_lstm(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h), B, L,
+                                D, float(tol), int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
+                                ctypes.byref(opts) if opts is not None else None,
+                                _stream_handle(stream))
+    _raise(st, "pararnn_solve_lstm")
+    return c, h, SolveInfo(info)

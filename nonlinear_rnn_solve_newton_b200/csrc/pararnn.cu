@@ -1,0 +1,395 @@
+// pararnn.cu -- C ABI of libpararnn.so (declared in include/pararnn.h).
+//
+// Host side: argument validation, the work decomposition (tile width along D,
+// steps per thread, chunks), the workspace layout, and the launches of the
+// kernel in pararnn_kernel.cuh.  Nothing here allocates, frees or synchronises:
+// the caller owns every buffer and the stream.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "pararnn.h"
+#include "pararnn_kernel.cuh"
+
+namespace pararnn {
+namespace {
+
+// Steps per thread for each operation (registers per thread grow with S and
+// with the number of inputs per step).
+constexpr int kStepsScanDiag = 16;
+constexpr int kStepsScanBlock2 = 8;
+constexpr int kStepsGru = 8;
+constexpr int kStepsLstm = 4;
+// Resident CTAs per SM the register allocation is held to (launch bounds).
+constexpr int kMinBlocksScan = 2;
+constexpr int kMinBlocksSolve = 2;
+
+int steps_for(int op) {
+  switch (op) {
+    case kScanDiag: return kStepsScanDiag;
+    case kScanBlock2: return kStepsScanBlock2;
+    case kGru: return kStepsGru;
+    default: return kStepsLstm;
+  }
+}
+int ns_for(int op) { return (op == kScanBlock2 || op == kLstm) ? 2 : 1; }
+int mapw_for(int op) { return (op == kScanBlock2 || op == kLstm) ? 8 : 2; }
+bool is_newton(int op) { return op == kGru || op == kLstm; }
+
+// Channels per tile: 32 (one warp row of 128 B for fp32) once D allows,
+// otherwise the largest power of two not above D.
+int tile_width(long long D) {
+  int cw = 1;
+  while (cw < 32 && (long long)cw * 2 <= D) cw *= 2;
+  return cw;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Plan {
+  int op = 0, CW = 1, S = 1, T = 1, ntd = 0, ntiles = 0, nchunks = 0, nunits = 0;
+  int m_first = 1, m_next = 1, mmax = 1, npasses = 1, max_iters = 0;
+  size_t off_rho = 0, off_ticket = 0, off_flags = 0, zero_bytes = 0;
+  size_t off_agg = 0, off_inc = 0, off_bnd = 0, total = 0;
+  bool ok = false;
+};
+
+int count_sweeps(int m_first, int m_next, int max_iters) {
+  int q = 0, k0 = 0;
+  for (;;) {
+    int m = sweep_len(q, k0, m_first, m_next, max_iters);
+    ++q;
+    if (k0 + m > max_iters) break;
+    k0 += m;
+  }
+  return q;
+}
+
+Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
+               const pararnn_options_t* opts) {
+  Plan pl;
+  pl.op = op;
+  if (B <= 0 || L <= 0 || D <= 0) return pl;
+  if (is_newton(op) && (max_iters < 0 || max_iters > PARARNN_MAX_ITERS)) return pl;
+  pl.CW = tile_width(D);
+  pl.S = steps_for(op);
+  pl.T = (kThreads / pl.CW) * pl.S;
+  long long ntd = (D + pl.CW - 1) / pl.CW;
+  long long ntiles = B * ntd;
+  long long nchunks = (L + pl.T - 1) / pl.T;
+  if (ntiles > INT_MAX / 2 || nchunks > INT_MAX / 2 || ntiles * nchunks > INT_MAX / 2) return pl;
+  pl.ntd = (int)ntd;
+  pl.ntiles = (int)ntiles;
+  pl.nchunks = (int)nchunks;
+  pl.nunits = (int)(ntiles * nchunks);
+  if (is_newton(op)) {
+    pl.max_iters = max_iters;
+    int mf = (opts && opts->iters_first > 0) ? opts->iters_first : 4;
+    int mn = (opts && opts->iters_next > 0) ? opts->iters_next : 2;
+    if (mf > PARARNN_MAX_ITERS + 1) mf = PARARNN_MAX_ITERS + 1;
+    if (mn > PARARNN_MAX_ITERS + 1) mn = PARARNN_MAX_ITERS + 1;
+    pl.m_first = mf;
+    pl.m_next = mn;
+    pl.mmax = mf > mn ? mf : mn;
+    if (pl.mmax > max_iters + 1) pl.mmax = max_iters + 1;
+    pl.npasses = count_sweeps(mf, mn, max_iters);
+  } else {
+    pl.max_iters = 0;
+    pl.m_first = pl.m_next = pl.mmax = 1;
+    pl.npasses = 1;
+  }
+  const int NS = ns_for(op), MAPW = mapw_for(op);
+  size_t off = sizeof(Ctrl);
+  pl.off_rho = off;
+  off += sizeof(unsigned) * (size_t)(pl.max_iters + 1);
+  pl.off_ticket = off;
+  off += sizeof(unsigned) * (size_t)pl.npasses;
+  off = align_up(off, 256);
+  pl.off_flags = off;
+  off += sizeof(unsigned) * (size_t)pl.mmax * pl.nunits;
+  off = align_up(off, 256);
+  pl.zero_bytes = off;
+  pl.off_agg = off;
+  off += sizeof(float) * (size_t)pl.mmax * pl.nunits * pl.CW * MAPW;
+  off = align_up(off, 256);
+  pl.off_inc = off;
+  off += sizeof(float) * (size_t)pl.mmax * pl.nunits * pl.CW * NS;
+  off = align_up(off, 256);
+  pl.off_bnd = off;
+  if (is_newton(op)) off += sizeof(float) * 2 * (size_t)pl.nunits * pl.CW * NS;
+  pl.total = align_up(off, 256);
+  pl.ok = true;
+  return pl;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel selection by tile width.
+// ---------------------------------------------------------------------------
+template <int OP, typename PT, int S, int MINB>
+const void* kernel_for_cw(int cw) {
+  switch (cw) {
+    case 1: return (const void*)pararnn_kernel<OP, PT, 1, S, MINB>;
+    case 2: return (const void*)pararnn_kernel<OP, PT, 2, S, MINB>;
+    case 4: return (const void*)pararnn_kernel<OP, PT, 4, S, MINB>;
+    case 8: return (const void*)pararnn_kernel<OP, PT, 8, S, MINB>;
+    case 16: return (const void*)pararnn_kernel<OP, PT, 16, S, MINB>;
+    default: return (const void*)pararnn_kernel<OP, PT, 32, S, MINB>;
+  }
+}
+
+const void* select_kernel(int op, bool bf16, int cw) {
+  switch (op) {
+    case kScanDiag: return kernel_for_cw<kScanDiag, float, kStepsScanDiag, kMinBlocksScan>(cw);
+    case kScanBlock2:
+      return kernel_for_cw<kScanBlock2, float, kStepsScanBlock2, kMinBlocksScan>(cw);
+    case kGru:
+      return bf16 ? kernel_for_cw<kGru, __nv_bfloat16, kStepsGru, kMinBlocksSolve>(cw)
+                  : kernel_for_cw<kGru, float, kStepsGru, kMinBlocksSolve>(cw);
+    default:
+      return bf16 ? kernel_for_cw<kLstm, __nv_bfloat16, kStepsLstm, kMinBlocksSolve>(cw)
+                  : kernel_for_cw<kLstm, float, kStepsLstm, kMinBlocksSolve>(cw);
+  }
+}
+
+// Resident CTAs per SM for a kernel, cached per (device, kernel).
+struct OccEntry {
+  int dev;
+  const void* fn;
+  int per_sm;
+  int nsm;
+};
+std::mutex g_occ_mu;
+OccEntry g_occ[256];
+int g_occ_n = 0;
+
+cudaError_t resident_ctas(const void* fn, int* total) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    for (int i = 0; i < g_occ_n; ++i)
+      if (g_occ[i].dev == dev && g_occ[i].fn == fn) {
+        *total = g_occ[i].per_sm * g_occ[i].nsm;
+        return cudaSuccess;
+      }
+  }
+  int nsm = 0, per_sm = 0;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    if (g_occ_n < 256) g_occ[g_occ_n++] = OccEntry{dev, fn, per_sm, nsm};
+  }
+  *total = per_sm * nsm;
+  return cudaSuccess;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// Empty problem: no equations, so the solve has converged at k = 0.
+__global__ void empty_info_kernel(pararnn_solve_info_t* info) {
+  info->iterations = 0;
+  info->converged = 1;
+  info->status = 0;
+  info->updates = 0;
+  info->passes = 0;
+  info->reserved = 0;
+  info->max_residual = 0.0f;
+  for (int k = 0; k <= PARARNN_MAX_ITERS; ++k) info->rho[k] = 0.0f;
+}
+
+pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t ws_bytes,
+                        const pararnn_options_t* opts, cudaStream_t stream) {
+  if (!ws || ws_bytes < pl.total || !aligned(ws, 256)) return PARARNN_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  kp.ctrl = reinterpret_cast<Ctrl*>(base);
+  kp.rho_bits = reinterpret_cast<unsigned*>(base + pl.off_rho);
+  kp.ticket = reinterpret_cast<unsigned*>(base + pl.off_ticket);
+  kp.flags = reinterpret_cast<unsigned*>(base + pl.off_flags);
+  kp.agg = reinterpret_cast<float*>(base + pl.off_agg);
+  kp.inc = reinterpret_cast<float*>(base + pl.off_inc);
+  kp.bnd = reinterpret_cast<float*>(base + pl.off_bnd);
+  kp.ntd = pl.ntd;
+  kp.ntiles = pl.ntiles;
+  kp.nchunks = pl.nchunks;
+  kp.nunits = pl.nunits;
+  kp.max_iters = pl.max_iters;
+  kp.m_first = pl.m_first;
+  kp.m_next = pl.m_next;
+  kp.mmax = pl.mmax;
+  kp.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? opts->wait_timeout_ns : 1000000000LL;
+  kp.stall_unit = opts ? opts->debug_stall_unit : -1;
+
+  const void* fn = select_kernel(pl.op, bf16, pl.CW);
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_UNSUPPORTED;
+  }
+  int resident = 0;
+  if (resident_ctas(fn, &resident) != cudaSuccess || resident <= 0) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  int grid = pl.nunits < resident ? pl.nunits : resident;
+
+  if (cudaMemsetAsync(ws, 0, pl.zero_bytes, stream) != cudaSuccess) return PARARNN_ERR_CUDA;
+  if (kp.status_dev && cudaMemsetAsync(kp.status_dev, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return PARARNN_ERR_CUDA;
+
+  void* args[] = {&kp};
+  cudaError_t e;
+  if (is_newton(pl.op)) {
+    // The sweeps are separated by a grid barrier: all CTAs must be resident.
+    e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kThreads), args, 0, stream);
+  } else {
+    // Scans wait only on smaller tickets, which are always held by running CTAs.
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, 0, stream);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  return PARARNN_OK;
+}
+
+}  // namespace
+}  // namespace pararnn
+
+using namespace pararnn;
+
+extern "C" {
+
+int32_t pararnn_version(void) { return PARARNN_VERSION; }
+
+const char* pararnn_status_string(pararnn_status_t s) {
+  switch (s) {
+    case PARARNN_OK: return "ok";
+    case PARARNN_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case PARARNN_ERR_UNSUPPORTED: return "unsupported device (libpararnn needs sm_100a)";
+    case PARARNN_ERR_CUDA: return "CUDA runtime error";
+    case PARARNN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case PARARNN_ERR_NONFINITE: return "non-finite residual";
+    case PARARNN_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+  }
+  return "unknown status";
+}
+
+size_t pararnn_workspace_size(pararnn_op_t op, int64_t B, int64_t L, int64_t D, int32_t max_iters,
+                              const pararnn_options_t* opts) {
+  if ((int)op < 0 || (int)op > 3) return 0;
+  if (B == 0 || L == 0 || D == 0) return 256;
+  Plan pl = make_plan((int)op, B, L, D, max_iters, opts);
+  return pl.ok ? pl.total : 0;
+}
+
+static pararnn_status_t scan_common(int op, const float* A, const float* b, const float* x0,
+                                    float* x, int64_t B, int64_t L, int64_t D, void* ws,
+                                    size_t ws_bytes, int32_t* status_dev,
+                                    const pararnn_options_t* opts, void* stream) {
+  if (B < 0 || L < 0 || D < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (B == 0 || L == 0 || D == 0) {
+    if (status_dev && cudaMemsetAsync(status_dev, 0, sizeof(int32_t), st) != cudaSuccess)
+      return PARARNN_ERR_CUDA;
+    return PARARNN_OK;
+  }
+  if (!A || !b || !x) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (op == kScanBlock2) {
+    if (!aligned(A, 16) || !aligned(b, 8) || !aligned(x, 8) || (x0 && !aligned(x0, 8)))
+      return PARARNN_ERR_INVALID_ARGUMENT;
+  } else {
+    if (!aligned(A, 4) || !aligned(b, 4) || !aligned(x, 4) || (x0 && !aligned(x0, 4)))
+      return PARARNN_ERR_INVALID_ARGUMENT;
+  }
+  Plan pl = make_plan(op, B, L, D, 0, opts);
+  if (!pl.ok) return PARARNN_ERR_INVALID_ARGUMENT;
+  KParams kp = {};
+  kp.in0 = A;
+  kp.in1 = b;
+  kp.x0a = x0;
+  kp.out0 = x;
+  kp.B = B;
+  kp.L = L;
+  kp.D = D;
+  kp.status_dev = status_dev;
+  return launch(pl, kp, false, ws, ws_bytes, opts, st);
+}
+
+pararnn_status_t pararnn_scan_diag(const float* A, const float* b, const float* h0, float* h,
+                                   int64_t B, int64_t L, int64_t D, void* ws, size_t ws_bytes,
+                                   int32_t* status_dev, const pararnn_options_t* opts,
+                                   void* stream) {
+  return scan_common(kScanDiag, A, b, h0, h, B, L, D, ws, ws_bytes, status_dev, opts, stream);
+}
+
+pararnn_status_t pararnn_scan_block2(const float* A, const float* b, const float* x0, float* x,
+                                     int64_t B, int64_t L, int64_t D, void* ws, size_t ws_bytes,
+                                     int32_t* status_dev, const pararnn_options_t* opts,
+                                     void* stream) {
+  return scan_common(kScanBlock2, A, b, x0, x, B, L, D, ws, ws_bytes, status_dev, opts, stream);
+}
+
+static pararnn_status_t solve_common(int op, const void* P, pararnn_dtype_t p_dtype,
+                                     const float* a, const float* x0a, const float* x0b,
+                                     float* out0, float* out1, int64_t B, int64_t L, int64_t D,
+                                     float tol, int32_t max_iters, void* ws, size_t ws_bytes,
+                                     pararnn_solve_info_t* info, const pararnn_options_t* opts,
+                                     void* stream) {
+  if (B < 0 || L < 0 || D < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!info || !aligned(info, 4)) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!(tol >= 0.0f)) return PARARNN_ERR_INVALID_ARGUMENT;  // rejects NaN too
+  if (p_dtype != PARARNN_F32 && p_dtype != PARARNN_BF16) return PARARNN_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (B == 0 || L == 0 || D == 0) {
+    empty_info_kernel<<<1, 1, 0, st>>>(info);
+    return cudaGetLastError() == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA;
+  }
+  if (!P || !a || !out0 || (op == kLstm && !out1)) return PARARNN_ERR_INVALID_ARGUMENT;
+  const size_t esz = p_dtype == PARARNN_BF16 ? 2 : 4;
+  if (!aligned(P, esz) || !aligned(a, 4) || !aligned(out0, 4) || (out1 && !aligned(out1, 4)) ||
+      (x0a && !aligned(x0a, 4)) || (x0b && !aligned(x0b, 4)))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+  Plan pl = make_plan(op, B, L, D, max_iters, opts);
+  if (!pl.ok) return PARARNN_ERR_INVALID_ARGUMENT;
+  KParams kp = {};
+  kp.in0 = P;
+  kp.w = a;
+  kp.x0a = x0a;
+  kp.x0b = x0b;
+  kp.out0 = out0;
+  kp.out1 = out1;
+  kp.B = B;
+  kp.L = L;
+  kp.D = D;
+  kp.tol = tol;
+  kp.info = info;
+  return launch(pl, kp, p_dtype == PARARNN_BF16, ws, ws_bytes, opts, st);
+}
+
+pararnn_status_t pararnn_solve_gru(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                   const float* h0, float* h, int64_t B, int64_t L, int64_t D,
+                                   float tol, int32_t max_iters, void* ws, size_t ws_bytes,
+                                   pararnn_solve_info_t* info, const pararnn_options_t* opts,
+                                   void* stream) {
+  return solve_common(kGru, P, p_dtype, a, h0, nullptr, h, nullptr, B, L, D, tol, max_iters, ws,
+                      ws_bytes, info, opts, stream);
+}
+
+pararnn_status_t pararnn_solve_lstm(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                    const float* c0, const float* h0, float* c, float* h,
+                                    int64_t B, int64_t L, int64_t D, float tol, int32_t max_iters,
+                                    void* ws, size_t ws_bytes, pararnn_solve_info_t* info,
+                                    const pararnn_options_t* opts, void* stream) {
+  return solve_common(kLstm, P, p_dtype, a, c0, h0, c, h, B, L, D, tol, max_iters, ws, ws_bytes,
+                      info, opts, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,906 @@
+// pararnn_kernel.cuh -- the sm_100a kernel behind libpararnn.so.
+//
+// One persistent kernel template serves the four operations of the ParaRNN /
+// DEER hot path ("ParaRNN: Unlocking Parallel Training of Nonlinear RNNs for
+// Large Language Models", TL;DR, Abstract and Figure 2; DEER summary):
+//
+//   * the diagonal and 2x2 affine scans  x_t = A_t x_{t-1} + b_t  (the linear
+//     solve of a Newton step: a block bi-diagonal system), and
+//   * the ParaGRU / ParaLSTM Newton solves of h_t = f(h_{t-1}, P_t), where each
+//     iteration evaluates the cell, its (block-)diagonal Jacobian and the
+//     residual at every step and then solves the bi-diagonal system.
+//
+// Work decomposition.  The trajectory [B, L, D] is cut into units of
+// (CW consecutive channels along D) x (T consecutive steps).  Inside a
+// 256-thread CTA, thread (seg, c) owns channel c of the tile and the S steps
+// [t0 + seg*S, t0 + (seg+1)*S) of the chunk, with NSEG = 256 / CW segments and
+// T = NSEG * S.  Units are handed out by an atomic ticket in chunk-major
+// order, so every predecessor of a unit (the same tile, earlier chunks) was
+// handed out first and is already running: the look-back below always makes
+// progress.
+//
+// One Newton iteration inside a unit (all in registers / shared memory):
+//   1. per step, at the current iterate: f, A = df/dh, the residual
+//      r = f - h^k_t (its max goes to an atomic per iteration), and the affine
+//      map  h^{k+1}_t = A h^{k+1}_{t-1} + (f - A h^k_{t-1});
+//   2. each thread composes its S maps serially;
+//   3. warp shuffles compose the segments inside a warp, shared memory the 8
+//      warps, giving the unit's aggregate map per channel;
+//   4. decoupled look-back along the chunk chain of the tile: publish the
+//      aggregate, walk back over predecessors' aggregates until an inclusive
+//      value, publish the inclusive value (the new state at the chunk end);
+//   5. apply the carried-in state through the maps: h^{k+1} for the S steps.
+// The inputs P stay in registers across the m iterations of a sweep, so a
+// sweep reads P once and h once and writes h once whatever m is.  Sweeps are
+// separated by a grid barrier (the kernel is launched cooperatively, all CTAs
+// resident), after which every CTA reads the per-iteration residual maxima and
+// takes the same stop decision: Newton's stopping rule on the global max, as
+// in the Figure 4 caption.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pararnn {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+enum OpKind : int { kScanDiag = 0, kScanBlock2 = 1, kGru = 2, kLstm = 3 };
+
+// NS: state components per channel (1 diagonal, 2 block).  NI: input values per
+// step held in registers.  MAPW: floats of one published aggregate (padded).
+template <int OP> struct OpT;
+template <> struct OpT<kScanDiag> {
+  static constexpr int NS = 1, NI = 2, MAPW = 2;
+  static constexpr bool newton = false;
+};
+template <> struct OpT<kScanBlock2> {
+  static constexpr int NS = 2, NI = 6, MAPW = 8;
+  static constexpr bool newton = false;
+};
+template <> struct OpT<kGru> {
+  static constexpr int NS = 1, NI = 3, MAPW = 2;
+  static constexpr bool newton = true;
+};
+template <> struct OpT<kLstm> {
+  static constexpr int NS = 2, NI = 4, MAPW = 8;
+  static constexpr bool newton = true;
+};
+
+// ---------------------------------------------------------------------------
+// Workspace control block (zeroed by the host before each launch).
+// ---------------------------------------------------------------------------
+struct Ctrl {
+  unsigned bar_count;
+  unsigned bar_gen;
+  unsigned abort;
+  unsigned status;
+  unsigned pad[12];
+  // followed by: unsigned rho_bits[max_iters + 1]; unsigned ticket[npasses]
+};
+
+struct KParams {
+  const void* in0;       // P (solves) or A (scans)
+  const float* in1;      // b (scans)
+  const float* w;        // recurrence weights [G, D] (solves)
+  const float* x0a;      // h0 (GRU, diag scan), c0 (LSTM), x0 (block scan)
+  const float* x0b;      // h0 (LSTM)
+  float* out0;           // h (GRU, diag scan), c (LSTM), x (block scan)
+  float* out1;           // h (LSTM)
+  long long B, L, D;
+  int ntd;               // tiles along D
+  int ntiles;            // B * ntd
+  int nchunks;
+  int nunits;
+  float tol;
+  int max_iters;
+  int m_first, m_next, mmax;
+  Ctrl* ctrl;
+  unsigned* rho_bits;    // [max_iters + 1]
+  unsigned* ticket;      // [npasses]
+  unsigned* flags;       // [mmax][nunits]
+  float* agg;            // [mmax][nunits][CW][MAPW]
+  float* inc;            // [mmax][nunits][CW][NS]
+  float* bnd;            // [2][nunits][CW][NS]
+  void* info;            // pararnn_solve_info_t* (solves)
+  int* status_dev;       // scans, optional
+  long long timeout_ns;
+  long long stall_unit;
+};
+
+// ---------------------------------------------------------------------------
+// Memory-model helpers (PTX acquire/release at GPU scope, L2-coherent loads).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_volatile(const unsigned* p) {
+  return *reinterpret_cast<const volatile unsigned*>(p);
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ float ldcg(const float* p) { return __ldcg(p); }
+
+// ---------------------------------------------------------------------------
+// Affine maps x -> M x + v and their composition.
+// ---------------------------------------------------------------------------
+template <int NS> struct Map {
+  float m[NS][NS];
+  float v[NS];
+};
+
+template <int NS> __device__ __forceinline__ Map<NS> map_identity() {
+  Map<NS> r;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+#pragma unroll
+    for (int j = 0; j < NS; ++j) r.m[i][j] = (i == j) ? 1.0f : 0.0f;
+    r.v[i] = 0.0f;
+  }
+  return r;
+}
+
+// later o earlier: x -> later(earlier(x))
+template <int NS>
+__device__ __forceinline__ Map<NS> compose(const Map<NS>& later, const Map<NS>& earlier) {
+  Map<NS> r;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+#pragma unroll
+    for (int j = 0; j < NS; ++j) {
+      float s = later.m[i][0] * earlier.m[0][j];
+#pragma unroll
+      for (int k = 1; k < NS; ++k) s = fmaf(later.m[i][k], earlier.m[k][j], s);
+      r.m[i][j] = s;
+    }
+    float s = later.v[i];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) s = fmaf(later.m[i][k], earlier.v[k], s);
+    r.v[i] = s;
+  }
+  return r;
+}
+
+template <int NS> struct Vec {
+  float x[NS];
+};
+
+template <int NS>
+__device__ __forceinline__ Vec<NS> apply(const Map<NS>& M, const Vec<NS>& x) {
+  Vec<NS> y;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    float s = M.v[i];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) s = fmaf(M.m[i][k], x.x[k], s);
+    y.x[i] = s;
+  }
+  return y;
+}
+
+template <int NS>
+__device__ __forceinline__ Map<NS> shfl_up_map(const Map<NS>& a, int delta) {
+  Map<NS> r;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+#pragma unroll
+    for (int j = 0; j < NS; ++j) r.m[i][j] = __shfl_up_sync(0xffffffffu, a.m[i][j], delta);
+    r.v[i] = __shfl_up_sync(0xffffffffu, a.v[i], delta);
+  }
+  return r;
+}
+
+// Published aggregate <-> global memory (MAPW floats, vectorised).
+template <int NS> __device__ __forceinline__ void store_map(float* p, const Map<NS>& a);
+template <> __device__ __forceinline__ void store_map<1>(float* p, const Map<1>& a) {
+  __stcg(reinterpret_cast<float2*>(p), make_float2(a.m[0][0], a.v[0]));
+}
+template <> __device__ __forceinline__ void store_map<2>(float* p, const Map<2>& a) {
+  __stcg(reinterpret_cast<float4*>(p), make_float4(a.m[0][0], a.m[0][1], a.m[1][0], a.m[1][1]));
+  __stcg(reinterpret_cast<float2*>(p + 4), make_float2(a.v[0], a.v[1]));
+}
+template <int NS> __device__ __forceinline__ Map<NS> load_map(const float* p);
+template <> __device__ __forceinline__ Map<1> load_map<1>(const float* p) {
+  float2 q = __ldcg(reinterpret_cast<const float2*>(p));
+  Map<1> a;
+  a.m[0][0] = q.x;
+  a.v[0] = q.y;
+  return a;
+}
+template <> __device__ __forceinline__ Map<2> load_map<2>(const float* p) {
+  float4 q = __ldcg(reinterpret_cast<const float4*>(p));
+  float2 r = __ldcg(reinterpret_cast<const float2*>(p + 4));
+  Map<2> a;
+  a.m[0][0] = q.x;
+  a.m[0][1] = q.y;
+  a.m[1][0] = q.z;
+  a.m[1][1] = q.w;
+  a.v[0] = r.x;
+  a.v[1] = r.y;
+  return a;
+}
+
+// ---------------------------------------------------------------------------
+// Cells.  sigma(x) = 1 / (1 + e^-x) and tanh(x) = 1 - 2 / (1 + e^{2x}), both
+// from the fast exponential and division intrinsics (absolute error well below
+// the 1e-4 parity bound; tanh.approx is not used: its ~2^-11 relative error
+// would bias every step).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float sigm(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+__device__ __forceinline__ float tanh_f(float x) {
+  return 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * x));
+}
+
+// ParaGRU: h' = (1-z) h + z c; returns f and dh'/dh.
+__device__ __forceinline__ void gru_cell(const float* p, const float* w, float h, float& f,
+                                         float& J) {
+  float z = sigm(fmaf(w[0], h, p[0]));
+  float r = sigm(fmaf(w[1], h, p[1]));
+  float rh = r * h;
+  float c = tanh_f(fmaf(w[2], rh, p[2]));
+  float cmh = c - h;
+  f = fmaf(z, cmh, h);
+  float dz = z * (1.0f - z) * w[0];
+  float dr = r * (1.0f - r) * w[1];
+  float du = w[2] * fmaf(h, dr, r);
+  float dc = fmaf(-c, c, 1.0f) * du;
+  J = fmaf(cmh, dz, 1.0f - z) + z * dc;
+}
+
+// ParaLSTM: state (c, h); f = (c', h'), J = d(c',h')/d(c,h) row-major.
+__device__ __forceinline__ void lstm_cell(const float* p, const float* w, float c, float h,
+                                          float& fc, float& fh, float J[2][2]) {
+  float ig = sigm(fmaf(w[0], h, p[0]));
+  float fg = sigm(fmaf(w[1], h, p[1]));
+  float gg = tanh_f(fmaf(w[2], h, p[2]));
+  float og = sigm(fmaf(w[3], h, p[3]));
+  float cn = fmaf(fg, c, ig * gg);
+  float tc = tanh_f(cn);
+  fc = cn;
+  fh = og * tc;
+  float di = ig * (1.0f - ig) * w[0];
+  float df = fg * (1.0f - fg) * w[1];
+  float dg = fmaf(-gg, gg, 1.0f) * w[2];
+  float dov = og * (1.0f - og) * w[3];
+  float dcn_dh = fmaf(df, c, fmaf(di, gg, ig * dg));
+  float odtc = og * fmaf(-tc, tc, 1.0f);
+  J[0][0] = fg;
+  J[0][1] = dcn_dh;
+  J[1][0] = odtc * fg;
+  J[1][1] = fmaf(dov, tc, odtc * dcn_dh);
+}
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// |r| as ordered bits: for non-negative floats the unsigned order is the float
+// order, and NaN (0x7fc00000 after fabs) sorts above +Inf, so a max over bits
+// keeps a NaN visible.
+__device__ __forceinline__ unsigned abs_bits(float r) { return __float_as_uint(fabsf(r)); }
+
+// ---------------------------------------------------------------------------
+// Bounded waits.
+// ---------------------------------------------------------------------------
+// What a bounded wait needs: where to raise an error, and the bound.
+struct WaitCtx {
+  Ctrl* ctrl;
+  int* status_dev;
+  long long timeout_ns;
+};
+
+__device__ __forceinline__ void raise_error(const WaitCtx& w, unsigned code) {
+  atomicCAS(&w.ctrl->status, 0u, code);
+  if (w.status_dev) atomicCAS(w.status_dev, 0, (int)code);
+  __threadfence();
+  atomicExch(&w.ctrl->abort, 1u);
+}
+
+// Warp-wide wait until the flag carries `epoch` with a non-empty state.  All 32
+// lanes load the flag with acquire semantics in the same instruction and must
+// agree, so every lane has synchronised with the release that published the
+// state it acts on.  Returns 1 (aggregate), 2 (inclusive) or 0 on timeout/abort.
+__device__ __noinline__ unsigned wait_flag(const unsigned* addr, unsigned epoch, WaitCtx p) {
+  unsigned long long t_start = 0;
+  unsigned ns = 32;
+  for (int it = 0;; ++it) {
+    unsigned v = ld_acquire(addr);
+    bool ok = (v >> 2) == epoch && (v & 3u) != 0u;
+    unsigned v0 = __shfl_sync(0xffffffffu, v, 0);
+    if (__all_sync(0xffffffffu, ok && v == v0)) return v & 3u;
+    if (it == 0) t_start = globaltimer();
+    const bool aborting = __any_sync(0xffffffffu, ld_volatile(&p.ctrl->abort) != 0u);
+    const bool expired =
+        __any_sync(0xffffffffu, (globaltimer() - t_start) > (unsigned long long)p.timeout_ns);
+    if (aborting || expired) {
+      if ((threadIdx.x & 31) == 0 && !aborting) raise_error(p, 4u /*TIMEOUT*/);
+      return 0u;
+    }
+    __nanosleep(ns);
+    if (ns < 1024) ns <<= 1;
+  }
+}
+
+// Grid-wide barrier (all CTAs are co-resident: cooperative launch).  Bounded;
+// returns false if the kernel is aborting.
+__device__ __noinline__ bool grid_barrier(WaitCtx p) {
+  __shared__ int s_ok;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    unsigned gen = ld_acquire(&p.ctrl->bar_gen);
+    __threadfence();
+    unsigned arrived = atomicAdd(&p.ctrl->bar_count, 1u);
+    if (arrived == gridDim.x - 1) {
+      atomicExch(&p.ctrl->bar_count, 0u);
+      __threadfence();
+      st_release(&p.ctrl->bar_gen, gen + 1u);
+    } else {
+      unsigned long long t0 = globaltimer();
+      unsigned ns = 32;
+      while (ld_acquire(&p.ctrl->bar_gen) == gen) {
+        if (ld_volatile(&p.ctrl->abort) != 0u) {
+          ok = 0;
+          break;
+        }
+        if (globaltimer() - t0 > (unsigned long long)p.timeout_ns) {
+          raise_error(p, 4u);
+          ok = 0;
+          break;
+        }
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+      }
+    }
+    if (ld_volatile(&p.ctrl->abort) != 0u) ok = 0;
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// Iterations evaluated in sweep q that starts at iteration k0.
+__device__ __host__ __forceinline__ int sweep_len(int q, int k0, int m_first, int m_next,
+                                                  int max_iters) {
+  int m = (q == 0) ? m_first : m_next;
+  int left = max_iters + 1 - k0;
+  return m < left ? m : left;
+}
+
+// ---------------------------------------------------------------------------
+// Per-op input and state access.
+// ---------------------------------------------------------------------------
+template <int OP, typename PT> struct IO;
+
+template <typename PT> struct IO<kGru, PT> {
+  __device__ static void load_in(const KParams& p, long long idx_btd, long long b, long long t,
+                                 long long d, float* v) {
+    const PT* P = reinterpret_cast<const PT*>(p.in0);
+    long long base = ((b * p.L + t) * 3) * p.D + d;
+#pragma unroll
+    for (int g = 0; g < 3; ++g) v[g] = to_f(__ldg(P + base + g * p.D));
+  }
+  __device__ static void load_state(const KParams& p, long long i, float* x) {
+    x[0] = ldcg(p.out0 + i);
+  }
+  __device__ static void store_state(const KParams& p, long long i, const float* x) {
+    p.out0[i] = x[0];
+  }
+  __device__ static void init_state(const KParams& p, long long bd, float* x) {
+    x[0] = p.x0a ? p.x0a[bd] : 0.0f;
+  }
+};
+
+template <typename PT> struct IO<kLstm, PT> {
+  __device__ static void load_in(const KParams& p, long long idx_btd, long long b, long long t,
+                                 long long d, float* v) {
+    const PT* P = reinterpret_cast<const PT*>(p.in0);
+    long long base = ((b * p.L + t) * 4) * p.D + d;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) v[g] = to_f(__ldg(P + base + g * p.D));
+  }
+  __device__ static void load_state(const KParams& p, long long i, float* x) {
+    x[0] = ldcg(p.out0 + i);
+    x[1] = ldcg(p.out1 + i);
+  }
+  __device__ static void store_state(const KParams& p, long long i, const float* x) {
+    p.out0[i] = x[0];
+    p.out1[i] = x[1];
+  }
+  __device__ static void init_state(const KParams& p, long long bd, float* x) {
+    x[0] = p.x0a ? p.x0a[bd] : 0.0f;
+    x[1] = p.x0b ? p.x0b[bd] : 0.0f;
+  }
+};
+
+template <typename PT> struct IO<kScanDiag, PT> {
+  __device__ static void load_in(const KParams& p, long long i, long long, long long, long long,
+                                 float* v) {
+    v[0] = __ldg(reinterpret_cast<const float*>(p.in0) + i);
+    v[1] = __ldg(p.in1 + i);
+  }
+  __device__ static void load_state(const KParams& p, long long i, float* x) {
+    x[0] = ldcg(p.out0 + i);
+  }
+  __device__ static void store_state(const KParams& p, long long i, const float* x) {
+    p.out0[i] = x[0];
+  }
+  __device__ static void init_state(const KParams& p, long long bd, float* x) {
+    x[0] = p.x0a ? p.x0a[bd] : 0.0f;
+  }
+};
+
+template <typename PT> struct IO<kScanBlock2, PT> {
+  __device__ static void load_in(const KParams& p, long long i, long long, long long, long long,
+                                 float* v) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p.in0) + i);
+    float2 b = __ldg(reinterpret_cast<const float2*>(p.in1) + i);
+    v[0] = a.x;
+    v[1] = a.y;
+    v[2] = a.z;
+    v[3] = a.w;
+    v[4] = b.x;
+    v[5] = b.y;
+  }
+  __device__ static void load_state(const KParams& p, long long i, float* x) {
+    float2 q = __ldcg(reinterpret_cast<const float2*>(p.out0) + i);
+    x[0] = q.x;
+    x[1] = q.y;
+  }
+  __device__ static void store_state(const KParams& p, long long i, const float* x) {
+    reinterpret_cast<float2*>(p.out0)[i] = make_float2(x[0], x[1]);
+  }
+  __device__ static void init_state(const KParams& p, long long bd, float* x) {
+    if (p.x0a) {
+      float2 q = reinterpret_cast<const float2*>(p.x0a)[bd];
+      x[0] = q.x;
+      x[1] = q.y;
+    } else {
+      x[0] = 0.0f;
+      x[1] = 0.0f;
+    }
+  }
+};
+
+// Map of one step, from the inputs (scans) or from the cell at the iterate.
+template <int OP> struct StepMap;
+template <> struct StepMap<kScanDiag> {
+  __device__ static Map<1> from_inputs(const float* v) {
+    Map<1> m;
+    m.m[0][0] = v[0];
+    m.v[0] = v[1];
+    return m;
+  }
+};
+template <> struct StepMap<kScanBlock2> {
+  __device__ static Map<2> from_inputs(const float* v) {
+    Map<2> m;
+    m.m[0][0] = v[0];
+    m.m[0][1] = v[1];
+    m.m[1][0] = v[2];
+    m.m[1][1] = v[3];
+    m.v[0] = v[4];
+    m.v[1] = v[5];
+    return m;
+  }
+};
+
+// Newton linearisation of one step at the iterate:
+//   map: x_t = J x_{t-1} + (f - J xprev),  residual bits max of |f - xcur|.
+template <int OP>
+__device__ __forceinline__ Map<OpT<OP>::NS> newton_step(const float* pin, const float* w,
+                                                        const Vec<OpT<OP>::NS>& xprev,
+                                                        const Vec<OpT<OP>::NS>& xcur,
+                                                        unsigned& rbits);
+template <>
+__device__ __forceinline__ Map<1> newton_step<kGru>(const float* pin, const float* w,
+                                                    const Vec<1>& xprev, const Vec<1>& xcur,
+                                                    unsigned& rbits) {
+  float f, J;
+  gru_cell(pin, w, xprev.x[0], f, J);
+  rbits = max(rbits, abs_bits(f - xcur.x[0]));
+  Map<1> m;
+  m.m[0][0] = J;
+  m.v[0] = fmaf(-J, xprev.x[0], f);
+  return m;
+}
+template <>
+__device__ __forceinline__ Map<2> newton_step<kLstm>(const float* pin, const float* w,
+                                                     const Vec<2>& xprev, const Vec<2>& xcur,
+                                                     unsigned& rbits) {
+  float fc, fh, J[2][2];
+  lstm_cell(pin, w, xprev.x[0], xprev.x[1], fc, fh, J);
+  rbits = max(rbits, max(abs_bits(fc - xcur.x[0]), abs_bits(fh - xcur.x[1])));
+  Map<2> m;
+  m.m[0][0] = J[0][0];
+  m.m[0][1] = J[0][1];
+  m.m[1][0] = J[1][0];
+  m.m[1][1] = J[1][1];
+  m.v[0] = fc - fmaf(J[0][0], xprev.x[0], J[0][1] * xprev.x[1]);
+  m.v[1] = fh - fmaf(J[1][0], xprev.x[0], J[1][1] * xprev.x[1]);
+  return m;
+}
+
+// ---------------------------------------------------------------------------
+// The kernel.
+// ---------------------------------------------------------------------------
+template <int OP, typename PT, int CW, int S, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p) {
+  using T_ = OpT<OP>;
+  constexpr int NS = T_::NS;
+  constexpr int NI = T_::NI;
+  constexpr int MAPW = T_::MAPW;
+  constexpr bool NEWTON = T_::newton;
+  constexpr int NSEG = kThreads / CW;
+  constexpr int TCH = NSEG * S;  // steps per chunk
+
+  __shared__ Map<NS> s_wagg[kWarps][CW];
+  __shared__ Vec<NS> s_carry[CW];
+  __shared__ unsigned s_rmax[kWarps];
+  __shared__ int s_unit;
+  __shared__ int s_abort;
+  __shared__ int s_done;
+
+  const WaitCtx wctx{p.ctrl, p.status_dev, p.timeout_ns};
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int c = tid % CW;
+  const int seg = tid / CW;
+
+  int k0 = 0;
+  int q = 0;
+  if (tid == 0) {
+    s_abort = 0;
+    s_done = 0;
+  }
+  __syncthreads();
+
+  for (;; ++q) {
+    const int m = NEWTON ? sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) : 1;
+    const unsigned epoch = (unsigned)(q + 1);
+
+    for (;;) {  // units of this sweep
+      if (tid == 0) {
+        int u = (int)atomicAdd(&p.ticket[q], 1u);
+        if (ld_volatile(&p.ctrl->abort) != 0u) u = p.nunits;
+        s_unit = u;
+      }
+      __syncthreads();
+      const int u = s_unit;
+      if (u >= p.nunits) break;
+
+      const int j = u / p.ntiles;
+      const int tile = u - j * p.ntiles;
+      const long long b = tile / p.ntd;
+      const int td = tile - (int)b * p.ntd;
+      const long long d = (long long)td * CW + c;
+      const bool cvalid = d < p.D;
+      const long long t0 = (long long)j * TCH + (long long)seg * S;
+      const long long bd = b * p.D + d;
+      const bool publish = (long long)u != p.stall_unit;
+
+      // ---- stage this unit's inputs in registers -------------------------
+      float vin[S][NI];
+#pragma unroll
+      for (int s = 0; s < S; ++s) {
+        const long long t = t0 + s;
+        if (cvalid && t < p.L) {
+          IO<OP, PT>::load_in(p, (b * p.L + t) * p.D + d, b, t, d, vin[s]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < NI; ++i) vin[s][i] = 0.0f;
+        }
+      }
+      float wv[NEWTON ? NI : 1];
+      if constexpr (NEWTON) {
+#pragma unroll
+        for (int g = 0; g < NI; ++g) wv[g] = cvalid ? __ldg(p.w + (long long)g * p.D + d) : 0.0f;
+      }
+
+      // ---- current iterate of the chunk and the state before each segment --
+      Vec<NS> x[S];
+      Vec<NS> xb;  // state at t0 - 1 for the current iterate
+#pragma unroll
+      for (int i = 0; i < NS; ++i) xb.x[i] = 0.0f;
+      if constexpr (NEWTON) {
+        if (k0 == 0) {
+#pragma unroll
+          for (int s = 0; s < S; ++s)
+#pragma unroll
+            for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
+          if (t0 == 0 && cvalid) IO<OP, PT>::init_state(p, bd, xb.x);
+        } else {
+#pragma unroll
+          for (int s = 0; s < S; ++s) {
+            const long long t = t0 + s;
+            if (cvalid && t < p.L) {
+              IO<OP, PT>::load_state(p, (b * p.L + t) * p.D + d, x[s].x);
+            } else {
+#pragma unroll
+              for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
+            }
+          }
+          if (cvalid) {
+            if (t0 == 0) {
+              IO<OP, PT>::init_state(p, bd, xb.x);
+            } else if (seg == 0) {
+              const float* src = p.bnd + ((size_t)((q - 1) & 1) * p.nunits + (u - p.ntiles)) *
+                                             (size_t)CW * NS + (size_t)c * NS;
+#pragma unroll
+              for (int i = 0; i < NS; ++i) xb.x[i] = ldcg(src + i);
+            } else if (t0 - 1 < p.L) {
+              IO<OP, PT>::load_state(p, (b * p.L + t0 - 1) * p.D + d, xb.x);
+            }
+          }
+        }
+      }
+
+      bool any_update = false;
+      for (int kk = 0; kk < m; ++kk) {
+        const int k = k0 + kk;
+        const bool upd = !NEWTON || k < p.max_iters;
+
+        // ---- 1-2: step maps, residual, thread aggregate --------------------
+        Map<NS> mp[S];
+        Map<NS> agg = map_identity<NS>();
+        unsigned rbits = 0u;
+        Vec<NS> xp = xb;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+          const bool v = cvalid && (t0 + s) < p.L;
+          if (v) {
+            if constexpr (NEWTON) {
+              mp[s] = newton_step<OP>(vin[s], wv, xp, x[s], rbits);
+              xp = x[s];
+            } else {
+              mp[s] = StepMap<OP>::from_inputs(vin[s]);
+            }
+          } else {
+            mp[s] = map_identity<NS>();
+          }
+          agg = compose(mp[s], agg);
+        }
+
+        // warp max of the residual bits
+        if constexpr (NEWTON) {
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1)
+            rbits = max(rbits, __shfl_xor_sync(0xffffffffu, rbits, off));
+        }
+
+        if (!upd) {
+          // residual-only iteration (k == max_iters): no solve, no update
+          if constexpr (NEWTON) {
+            if (lane == 0) s_rmax[warp] = rbits;
+            __syncthreads();
+            if (tid == 0) {
+              unsigned r = s_rmax[0];
+#pragma unroll
+              for (int w2 = 1; w2 < kWarps; ++w2) r = max(r, s_rmax[w2]);
+              atomicMax(&p.rho_bits[k], r);
+            }
+            __syncthreads();
+          }
+          continue;
+        }
+        any_update = true;
+
+        // ---- 3: segmented scan inside the warp (segments stride CW) --------
+        Map<NS> incl = agg;
+        Map<NS> wexcl = map_identity<NS>();
+        if constexpr (CW < 32) {
+#pragma unroll
+          for (int off = CW; off < 32; off <<= 1) {
+            Map<NS> o = shfl_up_map(incl, off);
+            if (lane >= off) incl = compose(incl, o);
+          }
+          Map<NS> e = shfl_up_map(incl, CW);
+          if (lane >= CW) wexcl = e;
+        }
+        if (lane >= 32 - CW) s_wagg[warp][c] = incl;
+        if constexpr (NEWTON) {
+          if (lane == 0) s_rmax[warp] = rbits;
+        }
+        __syncthreads();
+
+        // ---- 4: chunk aggregate, look-back, inclusive value ---------------
+        if (warp == 0) {
+          Map<NS> cta = map_identity<NS>();
+          if (lane < CW) {
+#pragma unroll
+            for (int w2 = 0; w2 < kWarps; ++w2) cta = compose(s_wagg[w2][c], cta);
+          }
+          if constexpr (NEWTON) {
+            if (lane == 0) {
+              unsigned r = s_rmax[0];
+#pragma unroll
+              for (int w2 = 1; w2 < kWarps; ++w2) r = max(r, s_rmax[w2]);
+              atomicMax(&p.rho_bits[k], r);
+            }
+          }
+          const size_t slot = (size_t)kk * p.nunits + u;
+          unsigned* my_flag = p.flags + slot;
+          Vec<NS> carry;
+          bool failed = false;
+          if (j == 0) {
+            if (lane < CW && cvalid) {
+              IO<OP, PT>::init_state(p, bd, carry.x);
+            } else {
+#pragma unroll
+              for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
+            }
+          } else {
+            if (publish) {
+              if (lane < CW) store_map<NS>(p.agg + (slot * CW + c) * MAPW, cta);
+              __threadfence();
+              __syncwarp();
+              if (lane == 0) st_release(my_flag, (epoch << 2) | 1u);
+            }
+            Map<NS> acc = map_identity<NS>();
+            int pu = u - p.ntiles;
+            for (;;) {
+              if (pu < 0) {  // chunk 0 always publishes an inclusive value
+                if (lane == 0) raise_error(wctx, 4u);
+                failed = true;
+#pragma unroll
+                for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
+                break;
+              }
+              const size_t ps = (size_t)kk * p.nunits + pu;
+              unsigned st = wait_flag(p.flags + ps, epoch, wctx);
+              if (st == 0u) {
+                failed = true;
+#pragma unroll
+                for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
+                break;
+              }
+              if (st == 2u) {
+                Vec<NS> v;
+#pragma unroll
+                for (int i = 0; i < NS; ++i) v.x[i] = ldcg(p.inc + (ps * CW + c) * NS + i);
+                carry = apply(acc, v);
+                break;
+              }
+              acc = compose(acc, load_map<NS>(p.agg + (ps * CW + c) * MAPW));
+              pu -= p.ntiles;
+            }
+          }
+          if (publish && !failed) {
+            Vec<NS> xe = apply(cta, carry);
+            if (lane < CW) {
+#pragma unroll
+              for (int i = 0; i < NS; ++i) __stcg(p.inc + (slot * CW + c) * NS + i, xe.x[i]);
+            }
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(my_flag, (epoch << 2) | 2u);
+          }
+          if (lane < CW) s_carry[c] = carry;
+          if (lane == 0 && failed) s_abort = 1;
+        }
+        // prefix of the earlier warps of this chunk, for this thread's channel
+        Map<NS> wpre = map_identity<NS>();
+        for (int w2 = 0; w2 < warp; ++w2) wpre = compose(s_wagg[w2][c], wpre);
+        __syncthreads();
+
+        // ---- 5: carry in, apply the maps -----------------------------------
+        Vec<NS> xin = apply(wexcl, apply(wpre, s_carry[c]));
+        Vec<NS> xr = xin;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+          xr = apply(mp[s], xr);
+          x[s] = xr;
+        }
+        xb = xin;
+        if (s_abort) break;
+      }
+
+      // ---- write the trajectory and the sweep boundary ---------------------
+      if (any_update || k0 == 0 || !NEWTON) {
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+          const long long t = t0 + s;
+          if (cvalid && t < p.L) IO<OP, PT>::store_state(p, (b * p.L + t) * p.D + d, x[s].x);
+        }
+      }
+      if constexpr (NEWTON) {
+        if (seg == NSEG - 1) {
+          float* dst = p.bnd + ((size_t)(q & 1) * p.nunits + u) * (size_t)CW * NS + (size_t)c * NS;
+#pragma unroll
+          for (int i = 0; i < NS; ++i) __stcg(dst + i, x[S - 1].x[i]);
+        }
+      }
+      if (s_abort) break;
+      __syncthreads();  // s_unit is rewritten by the next ticket
+    }
+    if (s_abort) break;
+
+    if constexpr (!NEWTON) {
+      break;
+    } else {
+      if (!grid_barrier(wctx)) {
+        if (tid == 0) s_abort = 1;
+        __syncthreads();
+        break;
+      }
+      // every CTA takes the same decision from the same global residuals
+      if (tid == 0) {
+        int done = 0;
+        for (int kk = 0; kk < m; ++kk) {
+          float r = __uint_as_float(ld_volatile(&p.rho_bits[k0 + kk]));
+          if (!(r <= 3.0e38f)) {  // NaN or Inf
+            done = 1;
+            break;
+          }
+          if (r <= p.tol) done = 1;
+        }
+        if (k0 + m > p.max_iters) done = 1;
+        s_done = done;
+      }
+      __syncthreads();
+      if (s_done) break;
+      k0 += m;
+    }
+  }
+
+  // ---- report ---------------------------------------------------------------
+  if constexpr (NEWTON) {
+    if (blockIdx.x == 0 && tid == 0) {
+      struct Info {
+        int iterations, converged, status, updates, passes, reserved;
+        float max_residual;
+        float rho[128];
+      };
+      Info* info = reinterpret_cast<Info*>(p.info);
+      __threadfence();
+      unsigned status = ld_volatile(&p.ctrl->status);
+      const int last = k0 + sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) - 1;
+      int iters = p.max_iters, conv = 0, nonfinite = 0;
+      float maxres = 0.0f;
+      for (int k = 0; k <= last && k <= p.max_iters; ++k) {
+        float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
+        info->rho[k] = r;
+        if (!(r <= 3.0e38f)) nonfinite = 1;
+      }
+      for (int k = 0; k <= last && k <= p.max_iters; ++k) {
+        float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
+        if (!(r <= 3.0e38f)) {
+          iters = k;
+          maxres = r;
+          break;
+        }
+        if (r <= p.tol) {
+          iters = k;
+          conv = 1;
+          maxres = r;
+          break;
+        }
+        iters = k;
+        maxres = r;
+      }
+      for (int k = last + 1; k <= p.max_iters; ++k) info->rho[k] = 0.0f;
+      if (status == 0u && nonfinite) status = 5u;
+      info->iterations = iters;
+      info->converged = (status == 0u) ? conv : 0;
+      info->status = (int)status;
+      info->updates = last < p.max_iters ? last + 1 : p.max_iters;
+      info->passes = q + 1;
+      info->reserved = 0;
+      info->max_residual = maxres;
+    }
+  }
+  // scans: a device-side error was written to status_dev by raise_error()
+}
+
+}  // namespace pararnn

@@ -1,0 +1,118 @@
+"""CPU-side checks of the C ABI: the library builds, loads, exports every symbol
+that include/pararnn.h declares, sizes workspaces and rejects bad arguments on
+the host (no CUDA work is issued by any call here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pararnn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import nonlinear_rnn_solve_newton_b200 as pr
+
+    return pr.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pararnn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_entry_points():
+    names = declared_functions()
+    for n in ("pararnn_scan_diag", "pararnn_scan_block2", "pararnn_solve_gru",
+              "pararnn_solve_lstm", "pararnn_workspace_size", "pararnn_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.pararnn_version() == 1
+    for code in range(7):
+        s = lib.pararnn_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.pararnn_status_string(99) == b"unknown status"
+
+
+def test_info_struct_layout():
+    import nonlinear_rnn_solve_newton_b200 as pr
+
+    # 6 int32 + 1 float + 128 floats
+    assert pr.INFO_BYTES == 4 * (6 + 1 + 128)
+
+
+def test_workspace_size_host_only():
+    import nonlinear_rnn_solve_newton_b200 as pr
+
+    n1 = pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32)
+    n2 = pr.workspace_size(pr.OP_GRU, 8, 8192, 1024, 32)
+    assert n1 > 0 and n2 > n1 and n1 % 256 == 0
+    assert pr.workspace_size(pr.OP_SCAN_DIAG, 1, 1, 1) > 0
+    assert pr.workspace_size(pr.OP_LSTM, 2, 7, 3, 0) > 0
+    # more iterations per sweep -> more look-back slots
+    o = pr.Options(iters_first=8)
+    assert pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32, o) > n1
+    with pytest.raises(pr.PararnnError):
+        pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 500)   # above the iteration cap
+    with pytest.raises(pr.PararnnError):
+        pr.workspace_size(9, 1, 1, 1)
+
+
+def test_host_validation_rejects_before_any_cuda_call(lib):
+    vp = ctypes.c_void_p
+    fake = vp(4096)  # never dereferenced: validation fails first
+    info = vp(8192)
+    # NULL inputs
+    assert lib.pararnn_solve_gru(None, 0, fake, None, fake, 2, 8, 4, ctypes.c_float(1e-4), 4,
+                                 fake, 1 << 20, info, None, None) == 1
+    # bad dtype
+    assert lib.pararnn_solve_gru(fake, 7, fake, None, fake, 2, 8, 4, ctypes.c_float(1e-4), 4,
+                                 fake, 1 << 20, info, None, None) == 1
+    # max_iters out of range, NaN tolerance, missing info
+    assert lib.pararnn_solve_gru(fake, 0, fake, None, fake, 2, 8, 4, ctypes.c_float(1e-4), 128,
+                                 fake, 1 << 20, info, None, None) == 1
+    assert lib.pararnn_solve_gru(fake, 0, fake, None, fake, 2, 8, 4, ctypes.c_float(float("nan")),
+                                 4, fake, 1 << 20, info, None, None) == 1
+    assert lib.pararnn_solve_gru(fake, 0, fake, None, fake, 2, 8, 4, ctypes.c_float(1e-4), 4,
+                                 fake, 1 << 20, None, None, None) == 1
+    # negative sizes
+    assert lib.pararnn_scan_diag(fake, fake, None, fake, -1, 8, 4, fake, 1 << 20, None, None,
+                                 None) == 1
+    # misaligned fp32 pointer
+    assert lib.pararnn_scan_diag(vp(4098), fake, None, fake, 1, 8, 4, fake, 1 << 20, None, None,
+                                 None) == 1
+    # 2x2 scan needs 16-byte aligned A
+    assert lib.pararnn_scan_block2(vp(4104), fake, None, fake, 1, 8, 4, fake, 1 << 20, None, None,
+                                   None) == 1
+    # workspace too small / misaligned / missing
+    assert lib.pararnn_scan_diag(fake, fake, None, fake, 1, 8, 4, fake, 16, None, None, None) == 6
+    assert lib.pararnn_scan_diag(fake, fake, None, fake, 1, 8, 4, vp(4100), 1 << 20, None, None,
+                                 None) == 6
+    assert lib.pararnn_scan_diag(fake, fake, None, fake, 1, 8, 4, None, 1 << 20, None, None,
+                                 None) == 6
+    # LSTM needs both outputs
+    assert lib.pararnn_solve_lstm(fake, 0, fake, None, None, fake, None, 2, 8, 4,
+                                  ctypes.c_float(1e-4), 4, fake, 1 << 20, info, None, None) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    import nonlinear_rnn_solve_newton_b200 as pr
+
+    A = torch.zeros(1, 4, 2, dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        pr.scan_diag(A, A)
+    P = torch.zeros(1, 4, 3, 2, dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        pr.solve_gru(P, torch.zeros(3, 2, dtype=torch.float32))

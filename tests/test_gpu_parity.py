@@ -1,0 +1,244 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tolerances (written here, derived from the arithmetic):
+* scans: |x - ref| <= 1e-5 * max(1, |ref|) elementwise (fp32 affine scan with
+  contractive maps; rounding of a few ulp per combine does not accumulate).
+* Newton solves: max-abs <= 1e-4 on the whole trajectory against the fp64
+  sequential rollout of the same (bf16-rounded where applicable) inputs --
+  the DEER summary's float32 tolerance.
+* iteration counts: equal to the oracle's serial Newton up to +-1 (a residual
+  that lands within fp32 rounding of tol may fall on either side).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import inputs
+
+pytestmark = pytest.mark.gpu
+
+SCAN_RTOL = 1e-5
+SOLVE_ATOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def pr():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import nonlinear_rnn_solve_newton_b200 as m
+
+    m.load()
+    return m
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def scan_err(got, ref):
+    return np.max(np.abs(got - ref) / np.maximum(1.0, np.abs(ref)))
+
+
+SCAN_SHAPES = [(1, 1, 1), (2, 3, 5), (3, 31, 3), (2, 33, 16), (1, 2049, 1), (2, 1000, 7),
+               (2, 4096 + 17, 64), (1, 300, 33), (4, 129, 1024)]
+
+
+@pytest.mark.parametrize("shape", SCAN_SHAPES)
+def test_scan_diag_parity(pr, shape):
+    B, L, D = shape
+    x = inputs.scan_diag_inputs(B, L, D, seed=[100, B, L, D])
+    h = pr.scan_diag(dev(x["A"]), dev(x["b"]), dev(x["h0"]))
+    torch.cuda.synchronize()
+    ref = oracle.scan_diag(x["A"], x["b"], x["h0"])
+    assert scan_err(h.cpu().numpy(), ref) <= SCAN_RTOL
+
+
+def test_scan_diag_no_h0_and_long_sequence(pr):
+    x = inputs.scan_diag_inputs(2, 40000, 3, seed=101)
+    h = pr.scan_diag(dev(x["A"]), dev(x["b"]))
+    torch.cuda.synchronize()
+    ref = oracle.scan_diag(x["A"], x["b"])
+    assert scan_err(h.cpu().numpy(), ref) <= SCAN_RTOL
+
+
+@pytest.mark.parametrize("shape", SCAN_SHAPES)
+def test_scan_block2_parity(pr, shape):
+    B, L, D = shape
+    x = inputs.scan_block2_inputs(B, L, D, seed=[102, B, L, D])
+    out = pr.scan_block2(dev(x["A"]), dev(x["b"]), dev(x["x0"]))
+    torch.cuda.synchronize()
+    ref = oracle.scan_block2(x["A"], x["b"], x["x0"])
+    assert scan_err(out.cpu().numpy(), ref) <= SCAN_RTOL
+
+
+def test_scan_output_canaries(pr):
+    """Nothing is written outside the output."""
+    B, L, D = 2, 777, 48
+    x = inputs.scan_diag_inputs(B, L, D, seed=103)
+    n = B * L * D
+    buf = torch.full((n + 2048,), 12345.0, device="cuda")
+    out = buf[1024:1024 + n].view(B, L, D)
+    pr.scan_diag(dev(x["A"]), dev(x["b"]), dev(x["h0"]), out=out)
+    torch.cuda.synchronize()
+    b = buf.cpu().numpy()
+    assert np.all(b[:1024] == 12345.0) and np.all(b[1024 + n:] == 12345.0)
+
+
+# --------------------------------------------------------------------------
+# Newton solves
+# --------------------------------------------------------------------------
+GRU_SHAPES = [(2, 512, 16), (1, 1, 1), (2, 3, 5), (3, 31, 3), (1, 2049, 1), (2, 1000, 7),
+              (2, 1100, 64), (1, 300, 33), (4, 257, 128)]
+
+
+@pytest.mark.parametrize("shape", GRU_SHAPES)
+def test_gru_solve_parity(pr, shape):
+    B, L, D = shape
+    x = inputs.gru_inputs(B, L, D, seed=[200, B, L, D])
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), dev(x["h0"]), tol=1e-4, max_iters=32)
+    torch.cuda.synchronize()
+    ref = oracle.rollout_gru(x["P"], x["a"], x["h0"])
+    assert info.status == 0 and info.converged
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
+    orc = oracle.newton_gru(x["P"], x["a"], x["h0"], tol=1e-4, max_iters=32)
+    assert abs(info.iterations - orc.iterations) <= 1, (info.iterations, orc.iterations)
+    assert info.max_residual <= 1e-4
+
+
+def test_gru_solve_nonzero_h0_and_bf16(pr):
+    B, L, D = 3, 700, 40
+    x = inputs.gru_inputs(B, L, D, seed=201, bf16=True, h0_normal=True)
+    P16 = dev(x["P_bits"].view(np.int16)).view(torch.bfloat16)
+    h, info = pr.solve_gru(P16, dev(x["a"]), dev(x["h0"]))
+    torch.cuda.synchronize()
+    ref = oracle.rollout_gru(x["P"], x["a"], x["h0"])   # same bf16-rounded values, in fp64
+    assert info.converged
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
+
+
+def test_gru_unconverged_matches_oracle_iterate(pr):
+    """tol = 0, max_iters = 2: both sides return h^2 and report no convergence."""
+    B, L, D = 2, 300, 8
+    x = inputs.gru_inputs(B, L, D, seed=202)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), tol=0.0, max_iters=2)
+    torch.cuda.synchronize()
+    orc = oracle.newton_gru(x["P"], x["a"], tol=0.0, max_iters=2)
+    assert not info.converged and info.iterations == 2 and info.updates == 2
+    assert np.max(np.abs(h.cpu().numpy() - orc.h)) <= 1e-5
+    np.testing.assert_allclose(info.rho[:3], orc.rho, rtol=1e-4, atol=1e-6)
+
+
+def test_gru_max_iters_zero_returns_initial_guess(pr):
+    x = inputs.gru_inputs(2, 50, 4, seed=203)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), tol=1e-4, max_iters=0)
+    torch.cuda.synchronize()
+    assert info.iterations == 0 and not info.converged and info.updates == 0
+    assert np.all(h.cpu().numpy() == 0.0)
+    orc = oracle.newton_gru(x["P"], x["a"], tol=1e-4, max_iters=0)
+    assert abs(info.rho[0] - orc.rho[0]) <= 1e-5
+
+
+def test_gru_mingru_one_iteration(pr):
+    """a = 0: the cell is affine in h, Newton needs one update and equals a single scan."""
+    B, L, D = 2, 900, 32
+    x = inputs.gru_inputs(B, L, D, seed=204, h0_normal=True)
+    a0 = np.zeros_like(x["a"])
+    h, info = pr.solve_gru(dev(x["P"]), dev(a0), dev(x["h0"]), tol=1e-5)
+    torch.cuda.synchronize()
+    assert info.converged and info.iterations == 1
+    ref = oracle.rollout_gru(x["P"], a0, x["h0"])
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-5
+
+
+def test_gru_iterations_per_sweep_do_not_change_result(pr):
+    B, L, D = 2, 2000, 32
+    x = inputs.gru_inputs(B, L, D, seed=205)
+    ref = oracle.rollout_gru(x["P"], x["a"])
+    counts = set()
+    for first, nxt in ((1, 1), (2, 1), (4, 2), (8, 8)):
+        o = pr.Options(iters_first=first, iters_next=nxt)
+        h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), opts=o)
+        torch.cuda.synchronize()
+        assert info.converged
+        assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
+        counts.add(info.iterations)
+    assert len(counts) == 1   # the stop decision is the same global rule
+
+
+def test_gru_nonfinite_reported(pr):
+    x = inputs.gru_inputs(1, 200, 8, seed=206)
+    P = x["P"].copy()
+    P[0, 77, 1, 3] = np.nan
+    h, info = pr.solve_gru(dev(P), dev(x["a"]))
+    torch.cuda.synchronize()
+    assert info.status == 5 and not info.converged
+
+
+def test_gru_empty_inputs(pr):
+    P = torch.zeros((2, 0, 3, 4), device="cuda")
+    h, info = pr.solve_gru(P, torch.zeros((3, 4), device="cuda"))
+    torch.cuda.synchronize()
+    assert h.shape == (2, 0, 4) and info.converged and info.iterations == 0
+
+
+LSTM_SHAPES = [(2, 512, 16), (1, 1, 1), (2, 5, 3), (1, 1025, 1), (2, 600, 33), (2, 700, 128)]
+
+
+@pytest.mark.parametrize("shape", LSTM_SHAPES)
+def test_lstm_solve_parity(pr, shape):
+    B, L, D = shape
+    x = inputs.lstm_inputs(B, L, D, seed=[300, B, L, D])
+    c, h, info = pr.solve_lstm(dev(x["P"]), dev(x["a"]), dev(x["c0"]), dev(x["h0"]))
+    torch.cuda.synchronize()
+    rc, rh = oracle.rollout_lstm(x["P"], x["a"], x["c0"], x["h0"])
+    assert info.status == 0 and info.converged
+    assert np.max(np.abs(c.cpu().numpy() - rc)) <= SOLVE_ATOL
+    assert np.max(np.abs(h.cpu().numpy() - rh)) <= SOLVE_ATOL
+    orc = oracle.newton_lstm(x["P"], x["a"], x["c0"], x["h0"], tol=1e-4, max_iters=32)
+    assert abs(info.iterations - orc.iterations) <= 1
+
+
+def test_lstm_no_recurrence_two_iterations(pr):
+    x = inputs.lstm_inputs(2, 500, 24, seed=301, h0_normal=True)
+    a0 = np.zeros_like(x["a"])
+    c, h, info = pr.solve_lstm(dev(x["P"]), dev(a0), dev(x["c0"]), dev(x["h0"]), tol=1e-5)
+    torch.cuda.synchronize()
+    assert info.converged and info.iterations == 2
+
+
+def test_lstm_bf16(pr):
+    B, L, D = 2, 400, 64
+    x = inputs.lstm_inputs(B, L, D, seed=302, bf16=True)
+    P16 = dev(x["P_bits"].view(np.int16)).view(torch.bfloat16)
+    c, h, info = pr.solve_lstm(P16, dev(x["a"]))
+    torch.cuda.synchronize()
+    rc, rh = oracle.rollout_lstm(x["P"], x["a"])
+    assert info.converged
+    assert np.max(np.abs(h.cpu().numpy() - rh)) <= SOLVE_ATOL
+    assert np.max(np.abs(c.cpu().numpy() - rc)) <= SOLVE_ATOL
+
+
+# --------------------------------------------------------------------------
+# Failure detection: a bounded wait that runs out
+# --------------------------------------------------------------------------
+def test_stalled_unit_times_out_and_context_survives(pr):
+    """A unit that never publishes (test hook) makes its successors' bounded waits
+    expire: the kernel returns DEVICE_TIMEOUT and the context stays usable."""
+    B, L, D = 1, 4096, 32
+    x = inputs.gru_inputs(B, L, D, seed=400)
+    o = pr.Options(wait_timeout_ns=20_000_000, debug_stall_unit=1)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), opts=o)
+    torch.cuda.synchronize()
+    assert info.status == 4 and not info.converged
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    xs = inputs.scan_diag_inputs(1, 4096, 32, seed=401)
+    pr.scan_diag(dev(xs["A"]), dev(xs["b"]), status=st, opts=o)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
+    # the next normal call is unaffected
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]))
+    torch.cuda.synchronize()
+    assert info.status == 0 and info.converged
+    ref = oracle.rollout_gru(x["P"], x["a"])
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
