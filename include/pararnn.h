@@ -102,12 +102,21 @@ typedef struct {
  *  debug_stall_unit: test hook, -1 = off.  The work unit with this index
  *                 never publishes its look-back status, so the units after it
  *                 run their bounded waits out; the call must then report
- *                 PARARNN_ERR_DEVICE_TIMEOUT. */
+ *                 PARARNN_ERR_DEVICE_TIMEOUT (look-back regime only).
+ *  regime      : how the time chunks of a channel tile are chained.
+ *                0 = automatic; 1 = look-back (chunks of a tile on different
+ *                CTAs, chained through global memory); 2 = walk (one CTA walks
+ *                a tile's chunks in order, no traffic between CTAs).  Both give
+ *                the same result up to fp32 rounding; in walk mode at most 8
+ *                iterations are evaluated per sweep.
+ *  reserved    : must be 0. */
 typedef struct {
   int32_t iters_first;
   int32_t iters_next;
   int64_t wait_timeout_ns;
   int64_t debug_stall_unit;
+  int32_t regime;
+  int32_t reserved;
 } pararnn_options_t;
 
 /* Bytes of workspace the call with the same arguments needs. 0 on bad sizes. */

@@ -11,21 +11,65 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "pararnn.h"
 #include "pararnn_kernel.cuh"
+#include "pararnn_walk.cuh"
 
 namespace pararnn {
 namespace {
 
 // Steps per thread for each operation (registers per thread grow with S and
 // with the number of inputs per step).
-constexpr int kStepsScanDiag = 16;
-constexpr int kStepsScanBlock2 = 8;
-constexpr int kStepsGru = 8;
-constexpr int kStepsLstm = 4;
+// (Overridable at build time for tuning sweeps.)
+#ifndef PARARNN_STEPS_SCAN_DIAG
+#define PARARNN_STEPS_SCAN_DIAG 16
+#endif
+#ifndef PARARNN_STEPS_SCAN_BLOCK2
+#define PARARNN_STEPS_SCAN_BLOCK2 8
+#endif
+#ifndef PARARNN_STEPS_GRU
+#define PARARNN_STEPS_GRU 8
+#endif
+#ifndef PARARNN_STEPS_LSTM
+#define PARARNN_STEPS_LSTM 4
+#endif
+#ifndef PARARNN_MINB_SCAN
+#define PARARNN_MINB_SCAN 2
+#endif
+#ifndef PARARNN_MINB_SOLVE
+#define PARARNN_MINB_SOLVE 2
+#endif
+#ifndef PARARNN_WALK_STEPS_GRU
+#define PARARNN_WALK_STEPS_GRU 8
+#endif
+#ifndef PARARNN_WALK_STEPS_LSTM
+#define PARARNN_WALK_STEPS_LSTM 4
+#endif
+#ifndef PARARNN_WALK_STEPS_SCAN_DIAG
+#define PARARNN_WALK_STEPS_SCAN_DIAG 16
+#endif
+#ifndef PARARNN_WALK_STEPS_SCAN_BLOCK2
+#define PARARNN_WALK_STEPS_SCAN_BLOCK2 8
+#endif
+#ifndef PARARNN_WALK_MINB
+#define PARARNN_WALK_MINB 3
+#endif
+constexpr int kWalkStepsGru = PARARNN_WALK_STEPS_GRU;
+constexpr int kWalkStepsLstm = PARARNN_WALK_STEPS_LSTM;
+constexpr int kWalkStepsScanDiag = PARARNN_WALK_STEPS_SCAN_DIAG;
+constexpr int kWalkStepsScanBlock2 = PARARNN_WALK_STEPS_SCAN_BLOCK2;
+constexpr int kWalkMinBlocks = PARARNN_WALK_MINB;
+constexpr int kStepsScanDiag = PARARNN_STEPS_SCAN_DIAG;
+constexpr int kStepsScanBlock2 = PARARNN_STEPS_SCAN_BLOCK2;
+constexpr int kStepsGru = PARARNN_STEPS_GRU;
+constexpr int kStepsLstm = PARARNN_STEPS_LSTM;
 // Resident CTAs per SM the register allocation is held to (launch bounds).
-constexpr int kMinBlocksScan = 2;
-constexpr int kMinBlocksSolve = 2;
+constexpr int kMinBlocksScan = PARARNN_MINB_SCAN;
+constexpr int kMinBlocksSolve = PARARNN_MINB_SOLVE;
+// Tiles from which one CTA per tile walking its chunks fills the GPU.
+constexpr int kWalkMinTiles = 200;
 
 int steps_for(int op) {
   switch (op) {
@@ -33,6 +77,14 @@ int steps_for(int op) {
     case kScanBlock2: return kStepsScanBlock2;
     case kGru: return kStepsGru;
     default: return kStepsLstm;
+  }
+}
+int walk_steps_for(int op) {
+  switch (op) {
+    case kScanDiag: return kWalkStepsScanDiag;
+    case kScanBlock2: return kWalkStepsScanBlock2;
+    case kGru: return kWalkStepsGru;
+    default: return kWalkStepsLstm;
   }
 }
 int ns_for(int op) { return (op == kScanBlock2 || op == kLstm) ? 2 : 1; }
@@ -50,6 +102,8 @@ int tile_width(long long D) {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
+  bool walk = false;
+  int S_walk = 0;  // steps per thread of the TMA walk kernel (32-wide tiles)
   int op = 0, CW = 1, S = 1, T = 1, ntd = 0, ntiles = 0, nchunks = 0, nunits = 0;
   int m_first = 1, m_next = 1, mmax = 1, npasses = 1, max_iters = 0;
   size_t off_rho = 0, off_ticket = 0, off_flags = 0, zero_bytes = 0;
@@ -85,12 +139,32 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
   pl.ntiles = (int)ntiles;
   pl.nchunks = (int)nchunks;
   pl.nunits = (int)(ntiles * nchunks);
+  // Chain the chunks of a tile inside one CTA when the tiles alone fill the GPU
+  // (about one tile per resident CTA or more); otherwise spread the chunks over
+  // CTAs and chain them by look-back.
+  const int regime = opts ? opts->regime : 0;
+  if (regime == 1) {
+    pl.walk = false;
+  } else if (regime == 2) {
+    pl.walk = true;
+  } else {
+    pl.walk = pl.nchunks > 1 && ntiles >= kWalkMinTiles;
+    if (pl.nchunks == 1) pl.walk = true;
+  }
+  if (pl.walk && pl.CW == 32) {
+    // the TMA walker cuts time into chunks of its own length
+    pl.S_walk = walk_steps_for(op);
+    long long tw = (long long)kWarps * pl.S_walk;
+    long long nchunks_w = (L + tw - 1) / tw;
+    if (nchunks_w > INT_MAX / 2) return pl;
+  }
   if (is_newton(op)) {
     pl.max_iters = max_iters;
     int mf = (opts && opts->iters_first > 0) ? opts->iters_first : 4;
     int mn = (opts && opts->iters_next > 0) ? opts->iters_next : 2;
-    if (mf > PARARNN_MAX_ITERS + 1) mf = PARARNN_MAX_ITERS + 1;
-    if (mn > PARARNN_MAX_ITERS + 1) mn = PARARNN_MAX_ITERS + 1;
+    const int mcap = pl.walk ? kMaxWalkIters : PARARNN_MAX_ITERS + 1;
+    if (mf > mcap) mf = mcap;
+    if (mn > mcap) mn = mcap;
     pl.m_first = mf;
     pl.m_next = mn;
     pl.mmax = mf > mn ? mf : mn;
@@ -109,9 +183,15 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
   off += sizeof(unsigned) * (size_t)pl.npasses;
   off = align_up(off, 256);
   pl.off_flags = off;
-  off += sizeof(unsigned) * (size_t)pl.mmax * pl.nunits;
+  if (!pl.walk) off += sizeof(unsigned) * (size_t)pl.mmax * pl.nunits;
   off = align_up(off, 256);
   pl.zero_bytes = off;
+  if (pl.walk) {  // no look-back slots
+    pl.off_agg = pl.off_inc = pl.off_bnd = off;
+    pl.total = align_up(off, 256);
+    pl.ok = true;
+    return pl;
+  }
   pl.off_agg = off;
   off += sizeof(float) * (size_t)pl.mmax * pl.nunits * pl.CW * MAPW;
   off = align_up(off, 256);
@@ -128,29 +208,34 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
 // ---------------------------------------------------------------------------
 // Kernel selection by tile width.
 // ---------------------------------------------------------------------------
-template <int OP, typename PT, int S, int MINB>
+template <int OP, typename PT, int S, int MINB, bool WALK>
 const void* kernel_for_cw(int cw) {
   switch (cw) {
-    case 1: return (const void*)pararnn_kernel<OP, PT, 1, S, MINB>;
-    case 2: return (const void*)pararnn_kernel<OP, PT, 2, S, MINB>;
-    case 4: return (const void*)pararnn_kernel<OP, PT, 4, S, MINB>;
-    case 8: return (const void*)pararnn_kernel<OP, PT, 8, S, MINB>;
-    case 16: return (const void*)pararnn_kernel<OP, PT, 16, S, MINB>;
-    default: return (const void*)pararnn_kernel<OP, PT, 32, S, MINB>;
+    case 1: return (const void*)pararnn_kernel<OP, PT, 1, S, MINB, WALK>;
+    case 2: return (const void*)pararnn_kernel<OP, PT, 2, S, MINB, WALK>;
+    case 4: return (const void*)pararnn_kernel<OP, PT, 4, S, MINB, WALK>;
+    case 8: return (const void*)pararnn_kernel<OP, PT, 8, S, MINB, WALK>;
+    case 16: return (const void*)pararnn_kernel<OP, PT, 16, S, MINB, WALK>;
+    default: return (const void*)pararnn_kernel<OP, PT, 32, S, MINB, WALK>;
   }
 }
 
-const void* select_kernel(int op, bool bf16, int cw) {
+template <int OP, typename PT, int S, int MINB>
+const void* kernel_for(bool walk, int cw) {
+  return walk ? kernel_for_cw<OP, PT, S, MINB, true>(cw) : kernel_for_cw<OP, PT, S, MINB, false>(cw);
+}
+
+const void* select_kernel(int op, bool bf16, bool walk, int cw) {
   switch (op) {
-    case kScanDiag: return kernel_for_cw<kScanDiag, float, kStepsScanDiag, kMinBlocksScan>(cw);
+    case kScanDiag: return kernel_for<kScanDiag, float, kStepsScanDiag, kMinBlocksScan>(walk, cw);
     case kScanBlock2:
-      return kernel_for_cw<kScanBlock2, float, kStepsScanBlock2, kMinBlocksScan>(cw);
+      return kernel_for<kScanBlock2, float, kStepsScanBlock2, kMinBlocksScan>(walk, cw);
     case kGru:
-      return bf16 ? kernel_for_cw<kGru, __nv_bfloat16, kStepsGru, kMinBlocksSolve>(cw)
-                  : kernel_for_cw<kGru, float, kStepsGru, kMinBlocksSolve>(cw);
+      return bf16 ? kernel_for<kGru, __nv_bfloat16, kStepsGru, kMinBlocksSolve>(walk, cw)
+                  : kernel_for<kGru, float, kStepsGru, kMinBlocksSolve>(walk, cw);
     default:
-      return bf16 ? kernel_for_cw<kLstm, __nv_bfloat16, kStepsLstm, kMinBlocksSolve>(cw)
-                  : kernel_for_cw<kLstm, float, kStepsLstm, kMinBlocksSolve>(cw);
+      return bf16 ? kernel_for<kLstm, __nv_bfloat16, kStepsLstm, kMinBlocksSolve>(walk, cw)
+                  : kernel_for<kLstm, float, kStepsLstm, kMinBlocksSolve>(walk, cw);
   }
 }
 
@@ -165,7 +250,7 @@ std::mutex g_occ_mu;
 OccEntry g_occ[256];
 int g_occ_n = 0;
 
-cudaError_t resident_ctas(const void* fn, int* total) {
+cudaError_t resident_ctas(const void* fn, size_t dyn_smem, int* total) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -180,7 +265,7 @@ cudaError_t resident_ctas(const void* fn, int* total) {
   int nsm = 0, per_sm = 0;
   e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, dyn_smem);
   if (e != cudaSuccess) return e;
   {
     std::lock_guard<std::mutex> lk(g_occ_mu);
@@ -191,6 +276,115 @@ cudaError_t resident_ctas(const void* fn, int* total) {
 }
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// ---------------------------------------------------------------------------
+// Tile-walking kernel with TMA staging (32-channel tiles).
+// ---------------------------------------------------------------------------
+
+template <int OP, typename PT, int S>
+size_t walk_smem_bytes() {
+  constexpr unsigned b = Stage<OP, PT, kWarps * S>::kBytes;
+  return 2 * (size_t)((b + 1023u) / 1024u * 1024u) + 1024;  // + alignment slack
+}
+
+const void* select_walk_kernel(int op, bool bf16, size_t* smem) {
+  switch (op) {
+    case kScanDiag:
+      *smem = walk_smem_bytes<kScanDiag, float, kWalkStepsScanDiag>();
+      return (const void*)pararnn_walk_kernel<kScanDiag, float, kWalkStepsScanDiag, kWalkMinBlocks>;
+    case kScanBlock2:
+      *smem = walk_smem_bytes<kScanBlock2, float, kWalkStepsScanBlock2>();
+      return (const void*)
+          pararnn_walk_kernel<kScanBlock2, float, kWalkStepsScanBlock2, kWalkMinBlocks>;
+    case kGru:
+      if (bf16) {
+        *smem = walk_smem_bytes<kGru, __nv_bfloat16, kWalkStepsGru>();
+        return (const void*)pararnn_walk_kernel<kGru, __nv_bfloat16, kWalkStepsGru, kWalkMinBlocks>;
+      }
+      *smem = walk_smem_bytes<kGru, float, kWalkStepsGru>();
+      return (const void*)pararnn_walk_kernel<kGru, float, kWalkStepsGru, kWalkMinBlocks>;
+    default:
+      if (bf16) {
+        *smem = walk_smem_bytes<kLstm, __nv_bfloat16, kWalkStepsLstm>();
+        return (const void*)
+            pararnn_walk_kernel<kLstm, __nv_bfloat16, kWalkStepsLstm, kWalkMinBlocks>;
+      }
+      *smem = walk_smem_bytes<kLstm, float, kWalkStepsLstm>();
+      return (const void*)pararnn_walk_kernel<kLstm, float, kWalkStepsLstm, kWalkMinBlocks>;
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    else
+      cudaGetLastError();
+  });
+  return g_encode;
+}
+
+// Row-major tensor [outer][mid][inner] (mid = 1 for 2-D), TMA box = inner x mid x rows.
+bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, size_t esize,
+                unsigned long long inner, unsigned long long mid, unsigned long long outer,
+                unsigned box_inner, unsigned box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  CUresult r;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  if (mid > 1) {
+    const cuuint64_t dims[3] = {inner, mid, outer};
+    const cuuint64_t strides[2] = {inner * esize, inner * mid * esize};
+    const cuuint32_t box[3] = {box_inner, (cuuint32_t)mid, box_rows};
+    r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * esize};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS;
+}
+
+// Tensor maps for the walk kernel, or false if the shapes or pointers do not
+// meet TMA's rules (16-byte aligned base, row pitch a multiple of 16 bytes).
+bool make_walk_maps(int op, bool bf16, const KParams& kp, int T, TmaMaps* tm) {
+  const long long B = kp.B, L = kp.L, D = kp.D;
+  if (D < 32 || B * L >= (1LL << 31)) return false;
+  const size_t es = bf16 ? 2 : 4;
+  const CUtensorMapDataType dt =
+      bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const unsigned long long rows = (unsigned long long)(B * L);
+  switch (op) {
+    case kGru:
+    case kLstm: {
+      const int G = op == kGru ? 3 : 4;
+      if (!aligned(kp.in0, 16) || (D * (long long)es) % 16 != 0) return false;
+      return encode_map(&tm->in0, kp.in0, dt, es, D, G, rows, 32, T);
+    }
+    case kScanDiag:
+      if (!aligned(kp.in0, 16) || !aligned(kp.in1, 16) || (D * 4) % 16 != 0) return false;
+      return encode_map(&tm->in0, kp.in0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, 1, rows, 32, T) &&
+             encode_map(&tm->in1, kp.in1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, 1, rows, 32, T);
+    default:
+      if (!aligned(kp.in0, 16) || !aligned(kp.in1, 16)) return false;
+      return encode_map(&tm->in0, kp.in0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 4 * D, 1, rows,
+                        128, T) &&
+             encode_map(&tm->in1, kp.in1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 2 * D, 1, rows, 64,
+                        T);
+  }
+}
 
 // Empty problem: no equations, so the solve has converged at k = 0.
 __global__ void empty_info_kernel(pararnn_solve_info_t* info) {
@@ -226,31 +420,52 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
   kp.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? opts->wait_timeout_ns : 1000000000LL;
   kp.stall_unit = opts ? opts->debug_stall_unit : -1;
 
-  const void* fn = select_kernel(pl.op, bf16, pl.CW);
+  // The TMA tile walker when the tiles are 32 wide and TMA's rules hold;
+  // otherwise the general kernel (look-back or register-staged walk).
+  TmaMaps tm;
+  const bool tma_walk = pl.walk && pl.CW == 32 && pl.S_walk > 0 &&
+                        make_walk_maps(pl.op, bf16, kp, kWarps * pl.S_walk, &tm);
+  const void* fn;
+  size_t dyn_smem = 0;
+  if (tma_walk) {
+    fn = select_walk_kernel(pl.op, bf16, &dyn_smem);
+    kp.nchunks = (int)((kp.L + kWarps * pl.S_walk - 1) / (kWarps * pl.S_walk));
+  } else {
+    fn = select_kernel(pl.op, bf16, pl.walk, pl.CW);
+  }
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
     return PARARNN_ERR_UNSUPPORTED;
   }
-  int resident = 0;
-  if (resident_ctas(fn, &resident) != cudaSuccess || resident <= 0) {
+  if (dyn_smem > 0 &&
+      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem) !=
+          cudaSuccess) {
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }
-  int grid = pl.nunits < resident ? pl.nunits : resident;
+  int resident = 0;
+  if (resident_ctas(fn, dyn_smem, &resident) != cudaSuccess || resident <= 0) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  const int nwork = pl.walk ? pl.ntiles : pl.nunits;
+  int grid = nwork < resident ? nwork : resident;
 
   if (cudaMemsetAsync(ws, 0, pl.zero_bytes, stream) != cudaSuccess) return PARARNN_ERR_CUDA;
   if (kp.status_dev && cudaMemsetAsync(kp.status_dev, 0, sizeof(int32_t), stream) != cudaSuccess)
     return PARARNN_ERR_CUDA;
 
-  void* args[] = {&kp};
+  void* args_plain[] = {&kp};
+  void* args_tma[] = {&kp, &tm};
+  void** args = tma_walk ? args_tma : args_plain;
   cudaError_t e;
   if (is_newton(pl.op)) {
     // The sweeps are separated by a grid barrier: all CTAs must be resident.
-    e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kThreads), args, 0, stream);
+    e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kThreads), args, dyn_smem, stream);
   } else {
     // Scans wait only on smaller tickets, which are always held by running CTAs.
-    e = cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, 0, stream);
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, dyn_smem, stream);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();

@@ -533,8 +533,20 @@ __device__ __forceinline__ Map<2> newton_step<kLstm>(const float* pin, const flo
 
 // ---------------------------------------------------------------------------
 // The kernel.
+//
+// Two ways to chain the time chunks of a tile (both exact, same arithmetic):
+//  WALK = true   one CTA takes a whole tile and walks its chunks in time order;
+//                the state entering chunk j at every iteration of the sweep is
+//                the one chunk j-1 produced, kept in shared memory.  No traffic
+//                between CTAs.  Used when there are enough tiles to fill the GPU.
+//  WALK = false  a unit is one (tile, chunk); chunks of a tile run on different
+//                CTAs at once and are chained by decoupled look-back through
+//                global memory.  Used when the channels are few and the time
+//                axis must provide the parallelism (e.g. one channel, 2^20 steps).
 // ---------------------------------------------------------------------------
-template <int OP, typename PT, int CW, int S, int MINB>
+constexpr int kMaxWalkIters = 8;  // iterations per sweep kept in shared memory (WALK)
+
+template <int OP, typename PT, int CW, int S, int MINB, bool WALK>
 __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p) {
   using T_ = OpT<OP>;
   constexpr int NS = T_::NS;
@@ -543,10 +555,14 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
   constexpr bool NEWTON = T_::newton;
   constexpr int NSEG = kThreads / CW;
   constexpr int TCH = NSEG * S;  // steps per chunk
+  constexpr int WM = WALK ? kMaxWalkIters : 1;
 
   __shared__ Map<NS> s_wagg[kWarps][CW];
   __shared__ Vec<NS> s_carry[CW];
   __shared__ unsigned s_rmax[kWarps];
+  __shared__ Vec<NS> s_inc[WALK ? 2 : 1][WM][CW];   // WALK: chunk-end state per iteration
+  __shared__ Vec<NS> s_pend[WALK ? 2 : 1][CW];      // WALK: chunk-end state of the loaded iterate
+  __shared__ unsigned s_racc[WM];                   // WALK: residual max per iteration
   __shared__ int s_unit;
   __shared__ int s_abort;
   __shared__ int s_done;
@@ -557,6 +573,7 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
   const int warp = tid >> 5;
   const int c = tid % CW;
   const int seg = tid / CW;
+  const int nwork = WALK ? p.ntiles : p.nunits;
 
   int k0 = 0;
   int q = 0;
@@ -570,259 +587,290 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
     const int m = NEWTON ? sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) : 1;
     const unsigned epoch = (unsigned)(q + 1);
 
-    for (;;) {  // units of this sweep
+    for (;;) {  // work items of this sweep: tiles (WALK) or (tile, chunk) units
       if (tid == 0) {
         int u = (int)atomicAdd(&p.ticket[q], 1u);
-        if (ld_volatile(&p.ctrl->abort) != 0u) u = p.nunits;
+        if (ld_volatile(&p.ctrl->abort) != 0u) u = nwork;
         s_unit = u;
       }
+      if (WALK && tid < WM) s_racc[tid] = 0u;
       __syncthreads();
-      const int u = s_unit;
-      if (u >= p.nunits) break;
+      const int item = s_unit;
+      if (item >= nwork) break;
 
-      const int j = u / p.ntiles;
-      const int tile = u - j * p.ntiles;
+      const int jbeg = WALK ? 0 : item / p.ntiles;
+      const int jend = WALK ? p.nchunks : jbeg + 1;
+      const int tile = WALK ? item : item - jbeg * p.ntiles;
       const long long b = tile / p.ntd;
       const int td = tile - (int)b * p.ntd;
       const long long d = (long long)td * CW + c;
       const bool cvalid = d < p.D;
-      const long long t0 = (long long)j * TCH + (long long)seg * S;
       const long long bd = b * p.D + d;
-      const bool publish = (long long)u != p.stall_unit;
 
-      // ---- stage this unit's inputs in registers -------------------------
-      float vin[S][NI];
-#pragma unroll
-      for (int s = 0; s < S; ++s) {
-        const long long t = t0 + s;
-        if (cvalid && t < p.L) {
-          IO<OP, PT>::load_in(p, (b * p.L + t) * p.D + d, b, t, d, vin[s]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < NI; ++i) vin[s][i] = 0.0f;
-        }
-      }
       float wv[NEWTON ? NI : 1];
       if constexpr (NEWTON) {
 #pragma unroll
         for (int g = 0; g < NI; ++g) wv[g] = cvalid ? __ldg(p.w + (long long)g * p.D + d) : 0.0f;
       }
 
-      // ---- current iterate of the chunk and the state before each segment --
-      Vec<NS> x[S];
-      Vec<NS> xb;  // state at t0 - 1 for the current iterate
-#pragma unroll
-      for (int i = 0; i < NS; ++i) xb.x[i] = 0.0f;
-      if constexpr (NEWTON) {
-        if (k0 == 0) {
-#pragma unroll
-          for (int s = 0; s < S; ++s)
-#pragma unroll
-            for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
-          if (t0 == 0 && cvalid) IO<OP, PT>::init_state(p, bd, xb.x);
-        } else {
-#pragma unroll
-          for (int s = 0; s < S; ++s) {
-            const long long t = t0 + s;
-            if (cvalid && t < p.L) {
-              IO<OP, PT>::load_state(p, (b * p.L + t) * p.D + d, x[s].x);
-            } else {
-#pragma unroll
-              for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
-            }
-          }
-          if (cvalid) {
-            if (t0 == 0) {
-              IO<OP, PT>::init_state(p, bd, xb.x);
-            } else if (seg == 0) {
-              const float* src = p.bnd + ((size_t)((q - 1) & 1) * p.nunits + (u - p.ntiles)) *
-                                             (size_t)CW * NS + (size_t)c * NS;
-#pragma unroll
-              for (int i = 0; i < NS; ++i) xb.x[i] = ldcg(src + i);
-            } else if (t0 - 1 < p.L) {
-              IO<OP, PT>::load_state(p, (b * p.L + t0 - 1) * p.D + d, xb.x);
-            }
-          }
-        }
-      }
+      for (int j = jbeg; j < jend; ++j) {
+        const int u = j * p.ntiles + tile;  // unit index (look-back slots)
+        const long long t0 = (long long)j * TCH + (long long)seg * S;
+        const bool publish = (long long)u != p.stall_unit;
 
-      bool any_update = false;
-      for (int kk = 0; kk < m; ++kk) {
-        const int k = k0 + kk;
-        const bool upd = !NEWTON || k < p.max_iters;
-
-        // ---- 1-2: step maps, residual, thread aggregate --------------------
-        Map<NS> mp[S];
-        Map<NS> agg = map_identity<NS>();
-        unsigned rbits = 0u;
-        Vec<NS> xp = xb;
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-          const bool v = cvalid && (t0 + s) < p.L;
-          if (v) {
-            if constexpr (NEWTON) {
-              mp[s] = newton_step<OP>(vin[s], wv, xp, x[s], rbits);
-              xp = x[s];
-            } else {
-              mp[s] = StepMap<OP>::from_inputs(vin[s]);
-            }
-          } else {
-            mp[s] = map_identity<NS>();
-          }
-          agg = compose(mp[s], agg);
-        }
-
-        // warp max of the residual bits
-        if constexpr (NEWTON) {
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1)
-            rbits = max(rbits, __shfl_xor_sync(0xffffffffu, rbits, off));
-        }
-
-        if (!upd) {
-          // residual-only iteration (k == max_iters): no solve, no update
-          if constexpr (NEWTON) {
-            if (lane == 0) s_rmax[warp] = rbits;
-            __syncthreads();
-            if (tid == 0) {
-              unsigned r = s_rmax[0];
-#pragma unroll
-              for (int w2 = 1; w2 < kWarps; ++w2) r = max(r, s_rmax[w2]);
-              atomicMax(&p.rho_bits[k], r);
-            }
-            __syncthreads();
-          }
-          continue;
-        }
-        any_update = true;
-
-        // ---- 3: segmented scan inside the warp (segments stride CW) --------
-        Map<NS> incl = agg;
-        Map<NS> wexcl = map_identity<NS>();
-        if constexpr (CW < 32) {
-#pragma unroll
-          for (int off = CW; off < 32; off <<= 1) {
-            Map<NS> o = shfl_up_map(incl, off);
-            if (lane >= off) incl = compose(incl, o);
-          }
-          Map<NS> e = shfl_up_map(incl, CW);
-          if (lane >= CW) wexcl = e;
-        }
-        if (lane >= 32 - CW) s_wagg[warp][c] = incl;
-        if constexpr (NEWTON) {
-          if (lane == 0) s_rmax[warp] = rbits;
-        }
-        __syncthreads();
-
-        // ---- 4: chunk aggregate, look-back, inclusive value ---------------
-        if (warp == 0) {
-          Map<NS> cta = map_identity<NS>();
-          if (lane < CW) {
-#pragma unroll
-            for (int w2 = 0; w2 < kWarps; ++w2) cta = compose(s_wagg[w2][c], cta);
-          }
-          if constexpr (NEWTON) {
-            if (lane == 0) {
-              unsigned r = s_rmax[0];
-#pragma unroll
-              for (int w2 = 1; w2 < kWarps; ++w2) r = max(r, s_rmax[w2]);
-              atomicMax(&p.rho_bits[k], r);
-            }
-          }
-          const size_t slot = (size_t)kk * p.nunits + u;
-          unsigned* my_flag = p.flags + slot;
-          Vec<NS> carry;
-          bool failed = false;
-          if (j == 0) {
-            if (lane < CW && cvalid) {
-              IO<OP, PT>::init_state(p, bd, carry.x);
-            } else {
-#pragma unroll
-              for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
-            }
-          } else {
-            if (publish) {
-              if (lane < CW) store_map<NS>(p.agg + (slot * CW + c) * MAPW, cta);
-              __threadfence();
-              __syncwarp();
-              if (lane == 0) st_release(my_flag, (epoch << 2) | 1u);
-            }
-            Map<NS> acc = map_identity<NS>();
-            int pu = u - p.ntiles;
-            for (;;) {
-              if (pu < 0) {  // chunk 0 always publishes an inclusive value
-                if (lane == 0) raise_error(wctx, 4u);
-                failed = true;
-#pragma unroll
-                for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
-                break;
-              }
-              const size_t ps = (size_t)kk * p.nunits + pu;
-              unsigned st = wait_flag(p.flags + ps, epoch, wctx);
-              if (st == 0u) {
-                failed = true;
-#pragma unroll
-                for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
-                break;
-              }
-              if (st == 2u) {
-                Vec<NS> v;
-#pragma unroll
-                for (int i = 0; i < NS; ++i) v.x[i] = ldcg(p.inc + (ps * CW + c) * NS + i);
-                carry = apply(acc, v);
-                break;
-              }
-              acc = compose(acc, load_map<NS>(p.agg + (ps * CW + c) * MAPW));
-              pu -= p.ntiles;
-            }
-          }
-          if (publish && !failed) {
-            Vec<NS> xe = apply(cta, carry);
-            if (lane < CW) {
-#pragma unroll
-              for (int i = 0; i < NS; ++i) __stcg(p.inc + (slot * CW + c) * NS + i, xe.x[i]);
-            }
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(my_flag, (epoch << 2) | 2u);
-          }
-          if (lane < CW) s_carry[c] = carry;
-          if (lane == 0 && failed) s_abort = 1;
-        }
-        // prefix of the earlier warps of this chunk, for this thread's channel
-        Map<NS> wpre = map_identity<NS>();
-        for (int w2 = 0; w2 < warp; ++w2) wpre = compose(s_wagg[w2][c], wpre);
-        __syncthreads();
-
-        // ---- 5: carry in, apply the maps -----------------------------------
-        Vec<NS> xin = apply(wexcl, apply(wpre, s_carry[c]));
-        Vec<NS> xr = xin;
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-          xr = apply(mp[s], xr);
-          x[s] = xr;
-        }
-        xb = xin;
-        if (s_abort) break;
-      }
-
-      // ---- write the trajectory and the sweep boundary ---------------------
-      if (any_update || k0 == 0 || !NEWTON) {
+        // ---- stage this chunk's inputs in registers ------------------------
+        float vin[S][NI];
 #pragma unroll
         for (int s = 0; s < S; ++s) {
           const long long t = t0 + s;
-          if (cvalid && t < p.L) IO<OP, PT>::store_state(p, (b * p.L + t) * p.D + d, x[s].x);
-        }
-      }
-      if constexpr (NEWTON) {
-        if (seg == NSEG - 1) {
-          float* dst = p.bnd + ((size_t)(q & 1) * p.nunits + u) * (size_t)CW * NS + (size_t)c * NS;
+          if (cvalid && t < p.L) {
+            IO<OP, PT>::load_in(p, (b * p.L + t) * p.D + d, b, t, d, vin[s]);
+          } else {
 #pragma unroll
-          for (int i = 0; i < NS; ++i) __stcg(dst + i, x[S - 1].x[i]);
+            for (int i = 0; i < NI; ++i) vin[s][i] = 0.0f;
+          }
         }
+
+        // ---- current iterate of the chunk and the state before each segment
+        Vec<NS> x[S];
+        Vec<NS> xb;  // state at t0 - 1 for the current iterate
+#pragma unroll
+        for (int i = 0; i < NS; ++i) xb.x[i] = 0.0f;
+        if constexpr (NEWTON) {
+          if (k0 == 0) {
+#pragma unroll
+            for (int s = 0; s < S; ++s)
+#pragma unroll
+              for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
+            if (t0 == 0 && cvalid) IO<OP, PT>::init_state(p, bd, xb.x);
+          } else {
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+              const long long t = t0 + s;
+              if (cvalid && t < p.L) {
+                IO<OP, PT>::load_state(p, (b * p.L + t) * p.D + d, x[s].x);
+              } else {
+#pragma unroll
+                for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
+              }
+            }
+            if (cvalid) {
+              if (t0 == 0) {
+                IO<OP, PT>::init_state(p, bd, xb.x);
+              } else if (seg == 0) {
+                if constexpr (WALK) {
+                  xb = s_pend[(j - 1) & 1][c];
+                } else {
+                  const float* src = p.bnd + ((size_t)((q - 1) & 1) * p.nunits + (u - p.ntiles)) *
+                                                 (size_t)CW * NS + (size_t)c * NS;
+#pragma unroll
+                  for (int i = 0; i < NS; ++i) xb.x[i] = ldcg(src + i);
+                }
+              } else if (t0 - 1 < p.L) {
+                IO<OP, PT>::load_state(p, (b * p.L + t0 - 1) * p.D + d, xb.x);
+              }
+            }
+          }
+          if constexpr (WALK) {
+            // the loaded iterate's chunk end, for the next chunk's first segment
+            if (seg == NSEG - 1) s_pend[j & 1][c] = x[S - 1];
+          }
+        }
+
+        bool any_update = false;
+        for (int kk = 0; kk < m; ++kk) {
+          const int k = k0 + kk;
+          const bool upd = !NEWTON || k < p.max_iters;
+
+          // ---- step maps, residual, thread aggregate -----------------------
+          Map<NS> mp[S];
+          Map<NS> agg = map_identity<NS>();
+          unsigned rbits = 0u;
+          Vec<NS> xp = xb;
+#pragma unroll
+          for (int s = 0; s < S; ++s) {
+            const bool v = cvalid && (t0 + s) < p.L;
+            if (v) {
+              if constexpr (NEWTON) {
+                mp[s] = newton_step<OP>(vin[s], wv, xp, x[s], rbits);
+                xp = x[s];
+              } else {
+                mp[s] = StepMap<OP>::from_inputs(vin[s]);
+              }
+            } else {
+              mp[s] = map_identity<NS>();
+            }
+            agg = compose(mp[s], agg);
+          }
+          if constexpr (NEWTON) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+              rbits = max(rbits, __shfl_xor_sync(0xffffffffu, rbits, off));
+          }
+
+          if (!upd) {
+            // residual-only iteration (k == max_iters): no solve, no update
+            if constexpr (NEWTON) {
+              if (lane == 0) s_rmax[warp] = rbits;
+              __syncthreads();
+              if (tid == 0) {
+                unsigned r = s_rmax[0];
+#pragma unroll
+                for (int w2 = 1; w2 < kWarps; ++w2) r = max(r, s_rmax[w2]);
+                if constexpr (WALK) {
+                  s_racc[kk] = max(s_racc[kk], r);
+                } else {
+                  atomicMax(&p.rho_bits[k], r);
+                }
+              }
+              __syncthreads();
+            }
+            continue;
+          }
+          any_update = true;
+
+          // ---- segmented scan inside the warp (segments stride CW) ---------
+          Map<NS> incl = agg;
+          Map<NS> wexcl = map_identity<NS>();
+          if constexpr (CW < 32) {
+#pragma unroll
+            for (int off = CW; off < 32; off <<= 1) {
+              Map<NS> o = shfl_up_map(incl, off);
+              if (lane >= off) incl = compose(incl, o);
+            }
+            Map<NS> e = shfl_up_map(incl, CW);
+            if (lane >= CW) wexcl = e;
+          }
+          if (lane >= 32 - CW) s_wagg[warp][c] = incl;
+          if constexpr (NEWTON) {
+            if (lane == 0) s_rmax[warp] = rbits;
+          }
+          __syncthreads();
+
+          // ---- chunk aggregate and the state carried into the chunk --------
+          if (warp == 0) {
+            Map<NS> cta = map_identity<NS>();
+            if (lane < CW) {
+#pragma unroll
+              for (int w2 = 0; w2 < kWarps; ++w2) cta = compose(s_wagg[w2][c], cta);
+            }
+            if constexpr (NEWTON) {
+              if (lane == 0) {
+                unsigned r = s_rmax[0];
+#pragma unroll
+                for (int w2 = 1; w2 < kWarps; ++w2) r = max(r, s_rmax[w2]);
+                if constexpr (WALK) {
+                  s_racc[kk] = max(s_racc[kk], r);
+                } else {
+                  atomicMax(&p.rho_bits[k], r);
+                }
+              }
+            }
+            Vec<NS> carry;
+            bool failed = false;
+            if (j == 0) {
+              if (lane < CW && cvalid) {
+                IO<OP, PT>::init_state(p, bd, carry.x);
+              } else {
+#pragma unroll
+                for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
+              }
+            } else if constexpr (WALK) {
+              carry = s_inc[(j - 1) & 1][kk][c];
+            } else {
+              const size_t slot = (size_t)kk * p.nunits + u;
+              if (publish) {
+                if (lane < CW) store_map<NS>(p.agg + (slot * CW + c) * MAPW, cta);
+                __syncwarp();
+                if (lane == 0) st_release(p.flags + slot, (epoch << 2) | 1u);
+              }
+              Map<NS> acc = map_identity<NS>();
+              int pu = u - p.ntiles;
+              for (;;) {
+                if (pu < 0) {  // chunk 0 always publishes an inclusive value
+                  if (lane == 0) raise_error(wctx, 4u);
+                  failed = true;
+#pragma unroll
+                  for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
+                  break;
+                }
+                const size_t ps = (size_t)kk * p.nunits + pu;
+                unsigned st = wait_flag(p.flags + ps, epoch, wctx);
+                if (st == 0u) {
+                  failed = true;
+#pragma unroll
+                  for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
+                  break;
+                }
+                if (st == 2u) {
+                  Vec<NS> v;
+#pragma unroll
+                  for (int i = 0; i < NS; ++i) v.x[i] = ldcg(p.inc + (ps * CW + c) * NS + i);
+                  carry = apply(acc, v);
+                  break;
+                }
+                acc = compose(acc, load_map<NS>(p.agg + (ps * CW + c) * MAPW));
+                pu -= p.ntiles;
+              }
+            }
+            const Vec<NS> xe = apply(cta, carry);
+            if constexpr (WALK) {
+              if (lane < CW) s_inc[j & 1][kk][c] = xe;
+            } else {
+              if (publish && !failed) {
+                const size_t slot = (size_t)kk * p.nunits + u;
+                if (lane < CW) {
+#pragma unroll
+                  for (int i = 0; i < NS; ++i) __stcg(p.inc + (slot * CW + c) * NS + i, xe.x[i]);
+                }
+                __syncwarp();
+                if (lane == 0) st_release(p.flags + slot, (epoch << 2) | 2u);
+              }
+            }
+            if (lane < CW) s_carry[c] = carry;
+            if (lane == 0 && failed) s_abort = 1;
+          }
+          // prefix of the earlier warps of this chunk, for this thread's channel
+          Map<NS> wpre = map_identity<NS>();
+          for (int w2 = 0; w2 < warp; ++w2) wpre = compose(s_wagg[w2][c], wpre);
+          __syncthreads();
+
+          // ---- carry in, apply the maps ------------------------------------
+          const Vec<NS> xin = apply(wexcl, apply(wpre, s_carry[c]));
+          Vec<NS> xr = xin;
+#pragma unroll
+          for (int s = 0; s < S; ++s) {
+            xr = apply(mp[s], xr);
+            x[s] = xr;
+          }
+          xb = xin;
+          if (s_abort) break;
+        }
+
+        // ---- write the trajectory and the sweep boundary --------------------
+        if (any_update || k0 == 0 || !NEWTON) {
+#pragma unroll
+          for (int s = 0; s < S; ++s) {
+            const long long t = t0 + s;
+            if (cvalid && t < p.L) IO<OP, PT>::store_state(p, (b * p.L + t) * p.D + d, x[s].x);
+          }
+        }
+        if constexpr (NEWTON && !WALK) {
+          if (seg == NSEG - 1) {
+            float* dst =
+                p.bnd + ((size_t)(q & 1) * p.nunits + u) * (size_t)CW * NS + (size_t)c * NS;
+#pragma unroll
+            for (int i = 0; i < NS; ++i) __stcg(dst + i, x[S - 1].x[i]);
+          }
+        }
+        if (s_abort) break;
+      }
+      if constexpr (NEWTON && WALK) {
+        __syncthreads();
+        if (tid < m) atomicMax(&p.rho_bits[k0 + tid], s_racc[tid]);
       }
       if (s_abort) break;
-      __syncthreads();  // s_unit is rewritten by the next ticket
+      __syncthreads();  // s_unit and s_racc are rewritten for the next item
     }
     if (s_abort) break;
 
@@ -875,19 +923,13 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
       }
       for (int k = 0; k <= last && k <= p.max_iters; ++k) {
         float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
-        if (!(r <= 3.0e38f)) {
-          iters = k;
-          maxres = r;
-          break;
-        }
-        if (r <= p.tol) {
-          iters = k;
-          conv = 1;
-          maxres = r;
-          break;
-        }
         iters = k;
         maxres = r;
+        if (!(r <= 3.0e38f)) break;
+        if (r <= p.tol) {
+          conv = 1;
+          break;
+        }
       }
       for (int k = last + 1; k <= p.max_iters; ++k) info->rho[k] = 0.0f;
       if (status == 0u && nonfinite) status = 5u;

@@ -1,0 +1,470 @@
+// pararnn_walk.cuh -- the tile-walking kernel: one CTA per tile of 32 channels,
+// time chunks staged in shared memory by TMA, all iterations of a sweep on chip.
+//
+// Same method and arithmetic as pararnn_kernel (ParaRNN TL;DR / Abstract: Newton
+// on the stacked system, each step a bi-diagonal solve by a parallel
+// reduction), organised for the case where the channel tiles alone fill the
+// GPU (LM-width layers):
+//   * the CTA walks the chunks of its tile in time order; the state entering
+//     chunk j at iteration k (h^{k+1} at the chunk start, and h^k for the
+//     Jacobian) is what chunk j-1 produced at the same iteration, kept in
+//     shared memory -- no traffic between CTAs at all;
+//   * the projected inputs of chunk j+1 are fetched by one TMA tensor copy
+//     (cp.async.bulk.tensor, box = 32 channels x gates x T steps) into the other
+//     half of a double buffer while chunk j is being iterated, so registers hold
+//     only the iterate and the step maps;
+//   * one __syncthreads per Newton iteration: every warp composes the
+//     aggregates of the warps before it (double-buffered shared array) and
+//     applies them to the carry it already has.
+#pragma once
+
+#include <cuda.h>
+
+#include "pararnn_kernel.cuh"
+
+namespace pararnn {
+
+struct TmaMaps {
+  CUtensorMap in0;  // P (solves) or A (scans)
+  CUtensorMap in1;  // b (scans)
+};
+
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<unsigned long long>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<unsigned long long>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory image of one time chunk, per op (32 channels wide).
+template <int OP, typename PT, int TCH> struct Stage;
+template <typename PT, int TCH> struct Stage<kGru, PT, TCH> {
+  static constexpr unsigned kBytes = TCH * 3 * 32 * sizeof(PT);
+  __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
+                               unsigned long long* bar) {
+    mbar_expect_tx(bar, kBytes);
+    tma_load_3d(s, &tm.in0, d0, 0, row, bar);
+  }
+  __device__ static void read(const unsigned char* s, int tl, int c, float* v) {
+    const PT* q = reinterpret_cast<const PT*>(s) + tl * 96 + c;
+    v[0] = to_f(q[0]);
+    v[1] = to_f(q[32]);
+    v[2] = to_f(q[64]);
+  }
+};
+template <typename PT, int TCH> struct Stage<kLstm, PT, TCH> {
+  static constexpr unsigned kBytes = TCH * 4 * 32 * sizeof(PT);
+  __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
+                               unsigned long long* bar) {
+    mbar_expect_tx(bar, kBytes);
+    tma_load_3d(s, &tm.in0, d0, 0, row, bar);
+  }
+  __device__ static void read(const unsigned char* s, int tl, int c, float* v) {
+    const PT* q = reinterpret_cast<const PT*>(s) + tl * 128 + c;
+    v[0] = to_f(q[0]);
+    v[1] = to_f(q[32]);
+    v[2] = to_f(q[64]);
+    v[3] = to_f(q[96]);
+  }
+};
+template <typename PT, int TCH> struct Stage<kScanDiag, PT, TCH> {
+  static constexpr unsigned kHalf = TCH * 32 * 4;
+  static constexpr unsigned kBytes = 2 * kHalf;
+  __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
+                               unsigned long long* bar) {
+    mbar_expect_tx(bar, kBytes);
+    tma_load_2d(s, &tm.in0, d0, row, bar);
+    tma_load_2d(s + kHalf, &tm.in1, d0, row, bar);
+  }
+  __device__ static void read(const unsigned char* s, int tl, int c, float* v) {
+    v[0] = reinterpret_cast<const float*>(s)[tl * 32 + c];
+    v[1] = reinterpret_cast<const float*>(s + kHalf)[tl * 32 + c];
+  }
+};
+template <typename PT, int TCH> struct Stage<kScanBlock2, PT, TCH> {
+  static constexpr unsigned kA = TCH * 32 * 16;
+  static constexpr unsigned kBytes = kA + TCH * 32 * 8;
+  __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
+                               unsigned long long* bar) {
+    mbar_expect_tx(bar, kBytes);
+    tma_load_2d(s, &tm.in0, 4 * d0, row, bar);
+    tma_load_2d(s + kA, &tm.in1, 2 * d0, row, bar);
+  }
+  __device__ static void read(const unsigned char* s, int tl, int c, float* v) {
+    const float4 a = reinterpret_cast<const float4*>(s)[tl * 32 + c];
+    const float2 b = reinterpret_cast<const float2*>(s + kA)[tl * 32 + c];
+    v[0] = a.x;
+    v[1] = a.y;
+    v[2] = a.z;
+    v[3] = a.w;
+    v[4] = b.x;
+    v[5] = b.y;
+  }
+};
+
+// Bounded wait for a stage's bytes to land.
+__device__ __forceinline__ bool stage_wait(unsigned long long* bar, unsigned parity,
+                                           const WaitCtx& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > (unsigned long long)w.timeout_ns) return false;
+  }
+}
+
+template <int OP, typename PT, int S, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
+    pararnn_walk_kernel(const __grid_constant__ KParams p, const __grid_constant__ TmaMaps tm) {
+  using T_ = OpT<OP>;
+  constexpr int NS = T_::NS;
+  constexpr int NI = T_::NI;
+  constexpr bool NEWTON = T_::newton;
+  constexpr int CW = 32;
+  constexpr int TCH = kWarps * S;  // steps per chunk (one segment of S steps per warp)
+  using St = Stage<OP, PT, TCH>;
+  constexpr unsigned kStageBytes = (St::kBytes + 1023u) / 1024u * 1024u;
+  constexpr int WM = kMaxWalkIters;
+
+  extern __shared__ __align__(1024) unsigned char dsmem[];
+  __shared__ unsigned long long s_bar[2];
+  __shared__ Map<NS> s_wagg[2][kWarps][CW];  // per-warp aggregates, double-buffered by iteration
+  __shared__ unsigned s_rmax[2][kWarps];
+  __shared__ Vec<NS> s_inc[2][WM][CW];       // chunk-end state per iteration, by chunk parity
+  __shared__ Vec<NS> s_pend[2][CW];          // chunk-end state of the loaded iterate
+  __shared__ unsigned s_racc[WM];
+  __shared__ int s_item;
+  __shared__ int s_flag;
+
+  const WaitCtx wctx{p.ctrl, p.status_dev, p.timeout_ns};
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int c = lane;
+  const int seg = warp;
+
+  if (tid == 0) {
+    mbar_init(&s_bar[0], 1);
+    mbar_init(&s_bar[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+
+  unsigned phase = 0u;    // parity of the next wait, per stage (bit s)
+  unsigned pending = 0u;  // stages with a copy in flight (thread 0's view)
+  int k0 = 0;
+  int q = 0;
+  bool aborted = false;
+
+  for (;; ++q) {
+    const int m = NEWTON ? sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) : 1;
+
+    for (;;) {  // tiles
+      if (tid == 0) {
+        int u = (int)atomicAdd(&p.ticket[q], 1u);
+        if (ld_volatile(&p.ctrl->abort) != 0u) u = p.ntiles;
+        s_item = u;
+      }
+      if (tid < WM) s_racc[tid] = 0u;
+      __syncthreads();
+      const int tile = s_item;
+      if (tile >= p.ntiles) break;
+
+      const long long b = tile / p.ntd;
+      const int td = tile - (int)b * p.ntd;
+      const int d0 = td * CW;
+      const long long d = d0 + c;
+      const bool cvalid = d < p.D;
+      const long long bd = b * p.D + d;
+      const int row0 = (int)(b * p.L);
+
+      float wv[NEWTON ? NI : 1];
+      Vec<NS> x0v;
+#pragma unroll
+      for (int i = 0; i < NS; ++i) x0v.x[i] = 0.0f;
+      if (cvalid) IO<OP, PT>::init_state(p, bd, x0v.x);
+      if constexpr (NEWTON) {
+#pragma unroll
+        for (int g = 0; g < NI; ++g) wv[g] = cvalid ? __ldg(p.w + (long long)g * p.D + d) : 0.0f;
+      }
+
+      // first two chunks of the tile in flight
+      if (tid == 0) {
+        for (int jj = 0; jj < 2 && jj < p.nchunks; ++jj) {
+          St::issue(dsmem + jj * kStageBytes, tm, d0, row0 + jj * TCH, &s_bar[jj]);
+          pending |= 1u << jj;
+        }
+      }
+
+      for (int j = 0; j < p.nchunks; ++j) {
+        const int st = j & 1;
+        const unsigned char* stage = dsmem + st * kStageBytes;
+        const long long t0 = (long long)j * TCH + (long long)seg * S;
+        const bool full = cvalid && (t0 + S) <= p.L;
+
+        // ---- current iterate and the state before this segment -----------
+        Vec<NS> x[S];
+        Vec<NS> xb;
+#pragma unroll
+        for (int i = 0; i < NS; ++i) xb.x[i] = 0.0f;
+        if constexpr (NEWTON) {
+          if (k0 == 0) {
+#pragma unroll
+            for (int s = 0; s < S; ++s)
+#pragma unroll
+              for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
+            if (t0 == 0) xb = x0v;
+          } else {
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+              const long long t = t0 + s;
+              if (cvalid && t < p.L) {
+                IO<OP, PT>::load_state(p, (b * p.L + t) * p.D + d, x[s].x);
+              } else {
+#pragma unroll
+                for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
+              }
+            }
+            if (t0 == 0) {
+              xb = x0v;
+            } else if (seg == 0) {
+              xb = s_pend[(j - 1) & 1][c];
+            } else if (cvalid && t0 - 1 < p.L) {
+              IO<OP, PT>::load_state(p, (b * p.L + t0 - 1) * p.D + d, xb.x);
+            }
+            if (seg == kWarps - 1) s_pend[j & 1][c] = x[S - 1];
+          }
+        }
+
+        // ---- this chunk's inputs have landed ------------------------------
+        const bool ok = stage_wait(&s_bar[st], (phase >> st) & 1u, wctx);
+        phase ^= 1u << st;
+        if (tid == 0) pending &= ~(1u << st);
+        if (!__syncthreads_and(ok ? 1 : 0)) {
+          if (tid == 0) raise_error(wctx, 4u);
+          aborted = true;
+          break;
+        }
+
+        bool any_update = false;
+        for (int kk = 0; kk < m; ++kk) {
+          const int k = k0 + kk;
+          const bool upd = !NEWTON || k < p.max_iters;
+          const int buf = kk & 1;
+
+          Map<NS> mp[S];
+          Map<NS> agg = map_identity<NS>();
+          unsigned rbits = 0u;
+          Vec<NS> xp = xb;
+          if (full) {
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+              float vin[NI];
+              St::read(stage, seg * S + s, c, vin);
+              if constexpr (NEWTON) {
+                mp[s] = newton_step<OP>(vin, wv, xp, x[s], rbits);
+                xp = x[s];
+              } else {
+                mp[s] = StepMap<OP>::from_inputs(vin);
+              }
+              agg = compose(mp[s], agg);
+            }
+          } else {
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+              if (cvalid && (t0 + s) < p.L) {
+                float vin[NI];
+                St::read(stage, seg * S + s, c, vin);
+                if constexpr (NEWTON) {
+                  mp[s] = newton_step<OP>(vin, wv, xp, x[s], rbits);
+                  xp = x[s];
+                } else {
+                  mp[s] = StepMap<OP>::from_inputs(vin);
+                }
+              } else {
+                mp[s] = map_identity<NS>();
+              }
+              agg = compose(mp[s], agg);
+            }
+          }
+          if constexpr (NEWTON) {
+            rbits = __reduce_max_sync(0xffffffffu, rbits);
+            if (lane == 0) s_rmax[buf][warp] = rbits;
+          }
+
+          if (!upd) {  // residual-only iteration (k == max_iters)
+            __syncthreads();
+            if (tid == 0) {
+              unsigned r = s_racc[kk];
+#pragma unroll
+              for (int w2 = 0; w2 < kWarps; ++w2) r = max(r, s_rmax[buf][w2]);
+              s_racc[kk] = r;
+            }
+            continue;
+          }
+          any_update = true;
+
+          s_wagg[buf][warp][c] = agg;
+          __syncthreads();
+
+          // prefix of the earlier warps, carry into the chunk, chunk-end state
+          Map<NS> pre = map_identity<NS>();
+#pragma unroll
+          for (int w2 = 0; w2 < kWarps - 1; ++w2)
+            if (w2 < warp) pre = compose(s_wagg[buf][w2][c], pre);
+          Vec<NS> carry = (j == 0) ? x0v : s_inc[(j - 1) & 1][kk][c];
+          const Vec<NS> xin = apply(pre, carry);
+          if (warp == kWarps - 1) s_inc[j & 1][kk][c] = apply(agg, xin);
+          if constexpr (NEWTON) {
+            if (tid == 0) {
+              unsigned r = s_racc[kk];
+#pragma unroll
+              for (int w2 = 0; w2 < kWarps; ++w2) r = max(r, s_rmax[buf][w2]);
+              s_racc[kk] = r;
+            }
+          }
+          Vec<NS> xr = xin;
+#pragma unroll
+          for (int s = 0; s < S; ++s) {
+            xr = apply(mp[s], xr);
+            x[s] = xr;
+          }
+          xb = xin;
+        }
+
+        // ---- write the chunk; refill its stage with chunk j + 2 -----------
+        if (any_update || k0 == 0 || !NEWTON) {
+          if (full) {
+#pragma unroll
+            for (int s = 0; s < S; ++s)
+              IO<OP, PT>::store_state(p, (b * p.L + t0 + s) * p.D + d, x[s].x);
+          } else {
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+              const long long t = t0 + s;
+              if (cvalid && t < p.L) IO<OP, PT>::store_state(p, (b * p.L + t) * p.D + d, x[s].x);
+            }
+          }
+        }
+        __syncthreads();  // every warp is done reading this stage
+        if (tid == 0 && j + 2 < p.nchunks) {
+          St::issue(dsmem + st * kStageBytes, tm, d0, row0 + (j + 2) * TCH, &s_bar[st]);
+          pending |= 1u << st;
+        }
+      }
+      if (aborted) break;
+      if constexpr (NEWTON) {
+        if (tid < m) atomicMax(&p.rho_bits[k0 + tid], s_racc[tid]);
+      }
+      __syncthreads();
+    }
+    if (aborted) break;
+
+    if constexpr (!NEWTON) {
+      break;
+    } else {
+      if (!grid_barrier(wctx)) {
+        aborted = true;
+        break;
+      }
+      if (tid == 0) {
+        int done = 0;
+        for (int kk = 0; kk < m; ++kk) {
+          const float r = __uint_as_float(ld_volatile(&p.rho_bits[k0 + kk]));
+          if (!(r <= 3.0e38f)) {
+            done = 1;
+            break;
+          }
+          if (r <= p.tol) done = 1;
+        }
+        if (k0 + m > p.max_iters) done = 1;
+        s_flag = done;
+      }
+      __syncthreads();
+      if (s_flag) break;
+      k0 += m;
+    }
+  }
+
+  // No copy may still be writing this CTA's shared memory when it exits.
+  if (tid == 0 && pending) {
+    for (int st = 0; st < 2; ++st)
+      if (pending & (1u << st)) stage_wait(&s_bar[st], (phase >> st) & 1u, wctx);
+  }
+
+  if constexpr (NEWTON) {
+    if (blockIdx.x == 0 && tid == 0) {
+      struct Info {
+        int iterations, converged, status, updates, passes, reserved;
+        float max_residual;
+        float rho[128];
+      };
+      Info* info = reinterpret_cast<Info*>(p.info);
+      __threadfence();
+      unsigned status = ld_volatile(&p.ctrl->status);
+      const int last = k0 + sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) - 1;
+      int iters = p.max_iters, conv = 0, nonfinite = 0;
+      float maxres = 0.0f;
+      for (int k = 0; k <= last && k <= p.max_iters; ++k) {
+        const float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
+        info->rho[k] = r;
+        if (!(r <= 3.0e38f)) nonfinite = 1;
+      }
+      for (int k = 0; k <= last && k <= p.max_iters; ++k) {
+        const float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
+        iters = k;
+        maxres = r;
+        if (!(r <= 3.0e38f)) break;
+        if (r <= p.tol) {
+          conv = 1;
+          break;
+        }
+      }
+      for (int k = last + 1; k <= p.max_iters; ++k) info->rho[k] = 0.0f;
+      if (status == 0u && nonfinite) status = 5u;
+      info->iterations = iters;
+      info->converged = (status == 0u) ? conv : 0;
+      info->status = (int)status;
+      info->updates = last < p.max_iters ? last + 1 : p.max_iters;
+      info->passes = q + 1;
+      info->reserved = 0;
+      info->max_residual = maxres;
+    }
+  }
+}
+
+}  // namespace pararnn

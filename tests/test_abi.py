@@ -54,14 +54,18 @@ def test_info_struct_layout():
 def test_workspace_size_host_only():
     import nonlinear_rnn_solve_newton_b200 as pr
 
-    n1 = pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32)
-    n2 = pr.workspace_size(pr.OP_GRU, 8, 8192, 1024, 32)
+    lb = pr.Options(regime=pr.Options.LOOKBACK)
+    n1 = pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32, lb)
+    n2 = pr.workspace_size(pr.OP_GRU, 8, 8192, 1024, 32, lb)
     assert n1 > 0 and n2 > n1 and n1 % 256 == 0
     assert pr.workspace_size(pr.OP_SCAN_DIAG, 1, 1, 1) > 0
     assert pr.workspace_size(pr.OP_LSTM, 2, 7, 3, 0) > 0
     # more iterations per sweep -> more look-back slots
-    o = pr.Options(iters_first=8)
+    o = pr.Options(iters_first=8, regime=pr.Options.LOOKBACK)
     assert pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32, o) > n1
+    # a CTA walking its tile needs no look-back slots: only the control block
+    walk = pr.Options(regime=pr.Options.WALK)
+    assert pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32, walk) <= 4096
     with pytest.raises(pr.PararnnError):
         pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 500)   # above the iteration cap
     with pytest.raises(pr.PararnnError):

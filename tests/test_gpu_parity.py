@@ -242,3 +242,65 @@ def test_stalled_unit_times_out_and_context_survives(pr):
     assert info.status == 0 and info.converged
     ref = oracle.rollout_gru(x["P"], x["a"])
     assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
+
+
+# --------------------------------------------------------------------------
+# Both ways of chaining time chunks (look-back across CTAs, or one CTA walking
+# a tile) must give the oracle's result.
+# --------------------------------------------------------------------------
+REGIME_SHAPES = [(2, 700, 64), (1, 2049, 1), (3, 300, 33), (2, 1500, 96)]
+
+
+@pytest.mark.parametrize("regime", [1, 2])
+@pytest.mark.parametrize("shape", REGIME_SHAPES)
+def test_regimes_gru(pr, regime, shape):
+    B, L, D = shape
+    x = inputs.gru_inputs(B, L, D, seed=[500, B, L, D], h0_normal=True)
+    o = pr.Options(regime=regime)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), dev(x["h0"]), opts=o)
+    torch.cuda.synchronize()
+    ref = oracle.rollout_gru(x["P"], x["a"], x["h0"])
+    assert info.converged
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
+    orc = oracle.newton_gru(x["P"], x["a"], x["h0"], tol=1e-4, max_iters=32)
+    assert abs(info.iterations - orc.iterations) <= 1
+
+
+@pytest.mark.parametrize("regime", [1, 2])
+@pytest.mark.parametrize("shape", REGIME_SHAPES)
+def test_regimes_lstm(pr, regime, shape):
+    B, L, D = shape
+    x = inputs.lstm_inputs(B, L, D, seed=[501, B, L, D])
+    o = pr.Options(regime=regime)
+    c, h, info = pr.solve_lstm(dev(x["P"]), dev(x["a"]), opts=o)
+    torch.cuda.synchronize()
+    rc, rh = oracle.rollout_lstm(x["P"], x["a"])
+    assert info.converged
+    assert np.max(np.abs(h.cpu().numpy() - rh)) <= SOLVE_ATOL
+    assert np.max(np.abs(c.cpu().numpy() - rc)) <= SOLVE_ATOL
+
+
+@pytest.mark.parametrize("regime", [1, 2])
+@pytest.mark.parametrize("shape", REGIME_SHAPES)
+def test_regimes_scans(pr, regime, shape):
+    B, L, D = shape
+    o = pr.Options(regime=regime)
+    x = inputs.scan_diag_inputs(B, L, D, seed=[502, B, L, D])
+    h = pr.scan_diag(dev(x["A"]), dev(x["b"]), dev(x["h0"]), opts=o)
+    y = inputs.scan_block2_inputs(B, L, D, seed=[503, B, L, D])
+    xo = pr.scan_block2(dev(y["A"]), dev(y["b"]), dev(y["x0"]), opts=o)
+    torch.cuda.synchronize()
+    assert scan_err(h.cpu().numpy(), oracle.scan_diag(x["A"], x["b"], x["h0"])) <= SCAN_RTOL
+    assert scan_err(xo.cpu().numpy(), oracle.scan_block2(y["A"], y["b"], y["x0"])) <= SCAN_RTOL
+
+
+def test_walk_regime_unconverged_iterate(pr):
+    """Walk regime, tol = 0, max_iters = 3: h^3 of the oracle's serial Newton."""
+    B, L, D = 2, 900, 64
+    x = inputs.gru_inputs(B, L, D, seed=504)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), tol=0.0, max_iters=3,
+                           opts=pr.Options(regime=2, iters_first=2, iters_next=1))
+    torch.cuda.synchronize()
+    orc = oracle.newton_gru(x["P"], x["a"], tol=0.0, max_iters=3)
+    assert not info.converged and info.iterations == 3 and info.updates == 3
+    assert np.max(np.abs(h.cpu().numpy() - orc.h)) <= 1e-5
