@@ -171,6 +171,38 @@ pararnn_status_t pararnn_solve_lstm(const void* P, pararnn_dtype_t p_dtype, cons
                                     void* ws, size_t ws_bytes, pararnn_solve_info_t* info,
                                     const pararnn_options_t* opts, void* stream);
 
+/* Allocation-free variant of pararnn_solve_gru (the pages have no counterpart:
+ * this is an interface convenience of this library).
+ * For callers that cannot allocate device memory where they solve -- their
+ * device memory is fully reserved by another allocator, they sit behind a
+ * plug-in interface that passes inputs and outputs but no workspace, or they
+ * run in a latency-critical loop where an allocation (which may synchronise
+ * the device) is not allowed.  Same arguments and results as
+ * pararnn_solve_gru without ws / ws_bytes: the scratch is a device array of
+ * PARARNN_NOALLOC_SCRATCH_BYTES inside the library, present on every GPU that
+ * loads it until the process exits.
+ *  - Problems whose pararnn_workspace_size(PARARNN_OP_GRU, ...) exceeds
+ *    PARARNN_NOALLOC_SCRATCH_BYTES are rejected with PARARNN_ERR_WORKSPACE
+ *    before any work is enqueued.  (In the walk regime -- the automatic
+ *    choice once there are at least 200 tiles of 32 channels -- the scratch
+ *    needed stays under 4 KB whatever L is.)
+ *  - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
+ *    library routine.  The part of the scratch that must start at zero is
+ *    cleared on the stream at every call.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current (a one-time set-up per device); make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array, which keeps what the last
+ *    call left: calls whose kernels may overlap on the GPU (different streams
+ *    without ordering, several host threads) race on it and must be
+ *    serialised by the caller. */
+#define PARARNN_NOALLOC_SCRATCH_BYTES (4u << 20)
+pararnn_status_t pararnn_solve_gru_noalloc(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                           const float* h0, float* h, int64_t B, int64_t L,
+                                           int64_t D, float tol, int32_t max_iters,
+                                           pararnn_solve_info_t* info,
+                                           const pararnn_options_t* opts, void* stream);
+
 /* Static description of a status code (never NULL). */
 const char* pararnn_status_string(pararnn_status_t status);
 

@@ -23,7 +23,8 @@ import torch
 
 from . import build as _build
 
-__all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "workspace_size",
+__all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc",
+           "workspace_size",
            "SolveInfo", "Options", "PararnnError", "library_path", "load", "MAX_ITERS"]
 
 MAX_ITERS = 127
@@ -98,6 +99,10 @@ def load(build_if_missing: bool = True):
                                                _i64, _i64, ctypes.c_float, ctypes.c_int32, _vp,
                                                ctypes.c_size_t, _vp, _vp, _vp]
             lib.pararnn_solve_lstm.restype = ctypes.c_int
+            lib.pararnn_solve_gru_noalloc.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64,
+                                                      _i64, _i64, ctypes.c_float, ctypes.c_int32,
+                                                      _vp, _vp, _vp]
+            lib.pararnn_solve_gru_noalloc.restype = ctypes.c_int
             lib.pararnn_status_string.argtypes = [ctypes.c_int]
             lib.pararnn_status_string.restype = ctypes.c_char_p
             lib.pararnn_version.restype = ctypes.c_int32
@@ -302,3 +307,34 @@ def solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32, out=None, info=No
                                 _stream_handle(stream))
     _raise(st, "pararnn_solve_lstm")
     return c, h, SolveInfo(info)
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def solve_gru_noalloc(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
+                      opts: Options | None = None, stream=None):
+    """ParaGRU Newton solve through ``pararnn_solve_gru_noalloc``: the library
+    allocates nothing and uses its own fixed device scratch array instead of a
+    workspace (for callers that cannot allocate device memory where they
+    solve).  Calls on one device share that array, so they must not overlap on
+    the GPU.  ``out`` and ``info`` may be passed to keep this call itself free
+    of allocations."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 3:
+        raise ValueError("P must be [B, L, 3, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 3, D))
+    _check_dev("a", a, torch.float32, (3, D))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    h = torch.empty((B, L, D), dtype=torch.float32, device=P.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, L, D))
+    if info is None:
+        info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    st = lib.pararnn_solve_gru_noalloc(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D,
+                                       float(tol), int(max_iters), _ptr(info),
+                                       ctypes.byref(opts) if opts is not None else None,
+                                       _stream_handle(stream))
+    _raise(st, "pararnn_solve_gru_noalloc")
+    return h, SolveInfo(info)

@@ -608,3 +608,65 @@ pararnn_status_t pararnn_solve_lstm(const void* P, pararnn_dtype_t p_dtype, cons
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free ParaGRU solve.
+//
+// Some callers cannot allocate device memory at the point where they solve:
+// code whose device memory is entirely reserved by another allocator, a
+// framework plug-in interface that hands over inputs and outputs but no
+// workspace, or a latency-critical loop where an allocation (which may
+// synchronise the device) is not allowed.  For them the scratch the kernel
+// needs lives in the library itself: one file-scope device array of
+// PARARNN_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
+// until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PARARNN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  Resolved once per
+// device, on the first call made with that device current; the name of the
+// array is only a host-side stand-in and must never be handed to a kernel.
+pararnn_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return PARARNN_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return PARARNN_OK;
+}
+
+}  // namespace
+
+extern "C" pararnn_status_t pararnn_solve_gru_noalloc(const void* P, pararnn_dtype_t p_dtype,
+                                                      const float* a, const float* h0, float* h,
+                                                      int64_t B, int64_t L, int64_t D, float tol,
+                                                      int32_t max_iters,
+                                                      pararnn_solve_info_t* info,
+                                                      const pararnn_options_t* opts,
+                                                      void* stream) {
+  if (B < 0 || L < 0 || D < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  const size_t need = pararnn_workspace_size(PARARNN_OP_GRU, B, L, D, max_iters, opts);
+  if (need == 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (need > (size_t)PARARNN_NOALLOC_SCRATCH_BYTES) return PARARNN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  pararnn_status_t st = noalloc_scratch(&scratch);
+  if (st != PARARNN_OK) return st;
+  return pararnn_solve_gru(P, p_dtype, a, h0, h, B, L, D, tol, max_iters, scratch,
+                           (size_t)PARARNN_NOALLOC_SCRATCH_BYTES, info, opts, stream);
+}
