@@ -169,6 +169,13 @@ def barrier(world):
         dist.barrier()
 
 
+def aggregate(ms_local, world, units_per_rank, device):
+    """Whole-job throughput under weak scaling: every rank processed
+    `units_per_rank` channel-steps per step; the step time is the slowest rank's."""
+    ms = max_over_ranks(ms_local, world, device)
+    return ms, world * units_per_rank / (ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------
 # sweep accounting (mirrors the kernel's schedule: m_first then m_next per sweep)
 # ---------------------------------------------------------------------------
@@ -256,8 +263,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
     ms_local = evs[0].elapsed_time(evs[K]) / K
-    ms = max_over_ranks(ms_local, world, device)
-    value = world * N / (ms * 1e-3)
+    ms, value = aggregate(ms_local, world, N, device)
     clocks = clk.summary()
 
     # dominant kernel: the fused Newton kernel, one launch per solve.  Its

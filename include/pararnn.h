@@ -109,14 +109,16 @@ typedef struct {
  *                a tile's chunks in order, no traffic between CTAs).  Both give
  *                the same result up to fp32 rounding; in walk mode at most 8
  *                iterations are evaluated per sweep.
- *  reserved    : must be 0. */
+ *  walk_warps  : warps per CTA in the walk regime with 32-channel tiles:
+ *                0 = automatic (16 for the GRU solve and the diagonal scan
+ *                below 512 tiles, else 8), 8 or 16. */
 typedef struct {
   int32_t iters_first;
   int32_t iters_next;
   int64_t wait_timeout_ns;
   int64_t debug_stall_unit;
   int32_t regime;
-  int32_t reserved;
+  int32_t walk_warps;
 } pararnn_options_t;
 
 /* Bytes of workspace the call with the same arguments needs. 0 on bad sizes. */

@@ -51,7 +51,7 @@ namespace {
 #define PARARNN_WALK_STEPS_SCAN_DIAG 16
 #endif
 #ifndef PARARNN_WALK_STEPS_SCAN_BLOCK2
-#define PARARNN_WALK_STEPS_SCAN_BLOCK2 8
+#define PARARNN_WALK_STEPS_SCAN_BLOCK2 4
 #endif
 #ifndef PARARNN_WALK_MINB
 #define PARARNN_WALK_MINB 3
@@ -70,6 +70,8 @@ constexpr int kMinBlocksScan = PARARNN_MINB_SCAN;
 constexpr int kMinBlocksSolve = PARARNN_MINB_SOLVE;
 // Tiles from which one CTA per tile walking its chunks fills the GPU.
 constexpr int kWalkMinTiles = 200;
+// Below this many tiles the walker uses 16-warp CTAs.
+constexpr int kWalkWideTiles = 512;
 
 int steps_for(int op) {
   switch (op) {
@@ -103,7 +105,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
   bool walk = false;
-  int S_walk = 0;  // steps per thread of the TMA walk kernel (32-wide tiles)
+  int S_walk = 0;   // steps per thread of the TMA walk kernel (32-wide tiles)
+  int NW_walk = 8;  // warps per CTA of the TMA walk kernel
   int op = 0, CW = 1, S = 1, T = 1, ntd = 0, ntiles = 0, nchunks = 0, nunits = 0;
   int m_first = 1, m_next = 1, mmax = 1, npasses = 1, max_iters = 0;
   size_t off_rho = 0, off_ticket = 0, off_flags = 0, zero_bytes = 0;
@@ -154,7 +157,12 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
   if (pl.walk && pl.CW == 32) {
     // the TMA walker cuts time into chunks of its own length
     pl.S_walk = walk_steps_for(op);
-    long long tw = (long long)kWarps * pl.S_walk;
+    const int want = opts ? opts->walk_warps : 0;
+    // 16-warp CTAs only help the GRU and the diagonal scan when tiles are few
+    // (measured on B200); the 2x2 ops keep 8 warps, whose CTAs fit more per SM.
+    const bool wide = (op == kGru || op == kScanDiag) && ntiles < kWalkWideTiles;
+    pl.NW_walk = (want == 8 || want == 16) ? want : (wide ? 16 : 8);
+    long long tw = (long long)pl.NW_walk * pl.S_walk;
     long long nchunks_w = (L + tw - 1) / tw;
     if (nchunks_w > INT_MAX / 2) return pl;
   }
@@ -250,7 +258,7 @@ std::mutex g_occ_mu;
 OccEntry g_occ[256];
 int g_occ_n = 0;
 
-cudaError_t resident_ctas(const void* fn, size_t dyn_smem, int* total) {
+cudaError_t resident_ctas(const void* fn, int threads, size_t dyn_smem, int* total) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -265,7 +273,7 @@ cudaError_t resident_ctas(const void* fn, size_t dyn_smem, int* total) {
   int nsm = 0, per_sm = 0;
   e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, dyn_smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, dyn_smem);
   if (e != cudaSuccess) return e;
   {
     std::lock_guard<std::mutex> lk(g_occ_mu);
@@ -281,36 +289,34 @@ bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 // Tile-walking kernel with TMA staging (32-channel tiles).
 // ---------------------------------------------------------------------------
 
-template <int OP, typename PT, int S>
+template <int OP, typename PT, int S, int NW>
 size_t walk_smem_bytes() {
-  constexpr unsigned b = Stage<OP, PT, kWarps * S>::kBytes;
+  constexpr unsigned b = Stage<OP, PT, NW * S>::kBytes;
   return 2 * (size_t)((b + 1023u) / 1024u * 1024u) + 1024;  // + alignment slack
 }
 
-const void* select_walk_kernel(int op, bool bf16, size_t* smem) {
+// Warps per CTA of the walker: 8, or 16 when the tiles are too few to fill the
+// SMs with 8-warp CTAs (more warps per tile then hide more latency).
+template <int OP, typename PT, int S>
+const void* walk_kernel_nw(int nw, size_t* smem) {
+  if (nw == 16) {
+    *smem = walk_smem_bytes<OP, PT, S, 16>();
+    return (const void*)pararnn_walk_kernel<OP, PT, S, 16, (kWalkMinBlocks + 1) / 2>;
+  }
+  *smem = walk_smem_bytes<OP, PT, S, 8>();
+  return (const void*)pararnn_walk_kernel<OP, PT, S, 8, kWalkMinBlocks>;
+}
+
+const void* select_walk_kernel(int op, bool bf16, int nw, size_t* smem) {
   switch (op) {
-    case kScanDiag:
-      *smem = walk_smem_bytes<kScanDiag, float, kWalkStepsScanDiag>();
-      return (const void*)pararnn_walk_kernel<kScanDiag, float, kWalkStepsScanDiag, kWalkMinBlocks>;
-    case kScanBlock2:
-      *smem = walk_smem_bytes<kScanBlock2, float, kWalkStepsScanBlock2>();
-      return (const void*)
-          pararnn_walk_kernel<kScanBlock2, float, kWalkStepsScanBlock2, kWalkMinBlocks>;
+    case kScanDiag: return walk_kernel_nw<kScanDiag, float, kWalkStepsScanDiag>(nw, smem);
+    case kScanBlock2: return walk_kernel_nw<kScanBlock2, float, kWalkStepsScanBlock2>(nw, smem);
     case kGru:
-      if (bf16) {
-        *smem = walk_smem_bytes<kGru, __nv_bfloat16, kWalkStepsGru>();
-        return (const void*)pararnn_walk_kernel<kGru, __nv_bfloat16, kWalkStepsGru, kWalkMinBlocks>;
-      }
-      *smem = walk_smem_bytes<kGru, float, kWalkStepsGru>();
-      return (const void*)pararnn_walk_kernel<kGru, float, kWalkStepsGru, kWalkMinBlocks>;
+      return bf16 ? walk_kernel_nw<kGru, __nv_bfloat16, kWalkStepsGru>(nw, smem)
+                  : walk_kernel_nw<kGru, float, kWalkStepsGru>(nw, smem);
     default:
-      if (bf16) {
-        *smem = walk_smem_bytes<kLstm, __nv_bfloat16, kWalkStepsLstm>();
-        return (const void*)
-            pararnn_walk_kernel<kLstm, __nv_bfloat16, kWalkStepsLstm, kWalkMinBlocks>;
-      }
-      *smem = walk_smem_bytes<kLstm, float, kWalkStepsLstm>();
-      return (const void*)pararnn_walk_kernel<kLstm, float, kWalkStepsLstm, kWalkMinBlocks>;
+      return bf16 ? walk_kernel_nw<kLstm, __nv_bfloat16, kWalkStepsLstm>(nw, smem)
+                  : walk_kernel_nw<kLstm, float, kWalkStepsLstm>(nw, smem);
   }
 }
 
@@ -424,12 +430,14 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
   // otherwise the general kernel (look-back or register-staged walk).
   TmaMaps tm;
   const bool tma_walk = pl.walk && pl.CW == 32 && pl.S_walk > 0 &&
-                        make_walk_maps(pl.op, bf16, kp, kWarps * pl.S_walk, &tm);
+                        make_walk_maps(pl.op, bf16, kp, pl.NW_walk * pl.S_walk, &tm);
   const void* fn;
   size_t dyn_smem = 0;
+  int threads = kThreads;
   if (tma_walk) {
-    fn = select_walk_kernel(pl.op, bf16, &dyn_smem);
-    kp.nchunks = (int)((kp.L + kWarps * pl.S_walk - 1) / (kWarps * pl.S_walk));
+    fn = select_walk_kernel(pl.op, bf16, pl.NW_walk, &dyn_smem);
+    kp.nchunks = (int)((kp.L + pl.NW_walk * pl.S_walk - 1) / (pl.NW_walk * pl.S_walk));
+    threads = 32 * pl.NW_walk;
   } else {
     fn = select_kernel(pl.op, bf16, pl.walk, pl.CW);
   }
@@ -445,7 +453,7 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
     return PARARNN_ERR_CUDA;
   }
   int resident = 0;
-  if (resident_ctas(fn, dyn_smem, &resident) != cudaSuccess || resident <= 0) {
+  if (resident_ctas(fn, threads, dyn_smem, &resident) != cudaSuccess || resident <= 0) {
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }
@@ -462,10 +470,10 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
   cudaError_t e;
   if (is_newton(pl.op)) {
     // The sweeps are separated by a grid barrier: all CTAs must be resident.
-    e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kThreads), args, dyn_smem, stream);
+    e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(threads), args, dyn_smem, stream);
   } else {
     // Scans wait only on smaller tickets, which are always held by running CTAs.
-    e = cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, dyn_smem, stream);
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, dyn_smem, stream);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();

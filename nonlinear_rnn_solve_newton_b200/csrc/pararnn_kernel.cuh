@@ -200,6 +200,19 @@ __device__ __forceinline__ Map<NS> shfl_up_map(const Map<NS>& a, int delta) {
   return r;
 }
 
+// Shuffle up within independent groups of `width` lanes.
+template <int NS>
+__device__ __forceinline__ Map<NS> shfl_up_map_w(const Map<NS>& a, int delta, int width) {
+  Map<NS> r;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+#pragma unroll
+    for (int j = 0; j < NS; ++j) r.m[i][j] = __shfl_up_sync(0xffffffffu, a.m[i][j], delta, width);
+    r.v[i] = __shfl_up_sync(0xffffffffu, a.v[i], delta, width);
+  }
+  return r;
+}
+
 // Published aggregate <-> global memory (MAPW floats, vectorised).
 template <int NS> __device__ __forceinline__ void store_map(float* p, const Map<NS>& a);
 template <> __device__ __forceinline__ void store_map<1>(float* p, const Map<1>& a) {
@@ -231,14 +244,37 @@ template <> __device__ __forceinline__ Map<2> load_map<2>(const float* p) {
 }
 
 // ---------------------------------------------------------------------------
-// Cells.  sigma(x) = 1 / (1 + e^-x) and tanh(x) = 1 - 2 / (1 + e^{2x}), both
-// from the fast exponential and division intrinsics (absolute error well below
-// the 1e-4 parity bound; tanh.approx is not used: its ~2^-11 relative error
-// would bias every step).
+// Cells.  From the identities e^x = 2^(x log2 e),
+//   sigma(x) = 1 / (1 + 2^(-x log2 e)),   tanh(x) = 1 - 2 / (1 + 2^(2 x log2 e)),
+// each evaluated with one hardware base-2 exponential and one hardware
+// reciprocal (PTX ex2.approx / rcp.approx: relative errors near 2^-22, so the
+// per-step absolute error stays ~1e-7, far inside the 1e-4 parity bound).
+// The limits are exact: 2^(+inf) = inf gives 1/inf = 0, 2^(-inf) = 0 gives 1.
+// tanh.approx is not used: its ~2^-11 relative error would bias every step.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float sigm(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float sigm(float x) {
+  return rcp_approx(1.0f + ex2_approx(-kLog2e * x));
+}
 __device__ __forceinline__ float tanh_f(float x) {
-  return 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * x));
+  return fmaf(-2.0f, rcp_approx(1.0f + ex2_approx((2.0f * kLog2e) * x)), 1.0f);
+}
+// max(m, |r|) that keeps a NaN (PTX max.NaN): a NaN residual must stop the solve.
+__device__ __forceinline__ float max_abs_nan(float m, float r) {
+  float y;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(m), "f"(fabsf(r)));
+  return y;
 }
 
 // ParaGRU: h' = (1-z) h + z c; returns f and dh'/dh.
@@ -283,10 +319,9 @@ __device__ __forceinline__ void lstm_cell(const float* p, const float* w, float 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// |r| as ordered bits: for non-negative floats the unsigned order is the float
-// order, and NaN (0x7fc00000 after fabs) sorts above +Inf, so a max over bits
-// keeps a NaN visible.
-__device__ __forceinline__ unsigned abs_bits(float r) { return __float_as_uint(fabsf(r)); }
+// Residual maxima travel as the bits of a non-negative float: for those the
+// unsigned order is the float order, and a NaN (0x7fc00000 or above) sorts
+// above +Inf, so integer max reductions and atomics keep it visible.
 
 // ---------------------------------------------------------------------------
 // Bounded waits.
@@ -496,19 +531,19 @@ template <> struct StepMap<kScanBlock2> {
 };
 
 // Newton linearisation of one step at the iterate:
-//   map: x_t = J x_{t-1} + (f - J xprev),  residual bits max of |f - xcur|.
+//   map: x_t = J x_{t-1} + (f - J xprev),  rmax = max(rmax, |f - xcur|).
 template <int OP>
 __device__ __forceinline__ Map<OpT<OP>::NS> newton_step(const float* pin, const float* w,
                                                         const Vec<OpT<OP>::NS>& xprev,
                                                         const Vec<OpT<OP>::NS>& xcur,
-                                                        unsigned& rbits);
+                                                        float& rmax);
 template <>
 __device__ __forceinline__ Map<1> newton_step<kGru>(const float* pin, const float* w,
                                                     const Vec<1>& xprev, const Vec<1>& xcur,
-                                                    unsigned& rbits) {
+                                                    float& rmax) {
   float f, J;
   gru_cell(pin, w, xprev.x[0], f, J);
-  rbits = max(rbits, abs_bits(f - xcur.x[0]));
+  rmax = max_abs_nan(rmax, f - xcur.x[0]);
   Map<1> m;
   m.m[0][0] = J;
   m.v[0] = fmaf(-J, xprev.x[0], f);
@@ -517,10 +552,10 @@ __device__ __forceinline__ Map<1> newton_step<kGru>(const float* pin, const floa
 template <>
 __device__ __forceinline__ Map<2> newton_step<kLstm>(const float* pin, const float* w,
                                                      const Vec<2>& xprev, const Vec<2>& xcur,
-                                                     unsigned& rbits) {
+                                                     float& rmax) {
   float fc, fh, J[2][2];
   lstm_cell(pin, w, xprev.x[0], xprev.x[1], fc, fh, J);
-  rbits = max(rbits, max(abs_bits(fc - xcur.x[0]), abs_bits(fh - xcur.x[1])));
+  rmax = max_abs_nan(max_abs_nan(rmax, fc - xcur.x[0]), fh - xcur.x[1]);
   Map<2> m;
   m.m[0][0] = J[0][0];
   m.m[0][1] = J[0][1];
@@ -685,14 +720,14 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
           // ---- step maps, residual, thread aggregate -----------------------
           Map<NS> mp[S];
           Map<NS> agg = map_identity<NS>();
-          unsigned rbits = 0u;
+          float rmax = 0.0f;
           Vec<NS> xp = xb;
 #pragma unroll
           for (int s = 0; s < S; ++s) {
             const bool v = cvalid && (t0 + s) < p.L;
             if (v) {
               if constexpr (NEWTON) {
-                mp[s] = newton_step<OP>(vin[s], wv, xp, x[s], rbits);
+                mp[s] = newton_step<OP>(vin[s], wv, xp, x[s], rmax);
                 xp = x[s];
               } else {
                 mp[s] = StepMap<OP>::from_inputs(vin[s]);
@@ -702,11 +737,8 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
             }
             agg = compose(mp[s], agg);
           }
-          if constexpr (NEWTON) {
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-              rbits = max(rbits, __shfl_xor_sync(0xffffffffu, rbits, off));
-          }
+          unsigned rbits = 0u;
+          if constexpr (NEWTON) rbits = __reduce_max_sync(0xffffffffu, __float_as_uint(rmax));
 
           if (!upd) {
             // residual-only iteration (k == max_iters): no solve, no update

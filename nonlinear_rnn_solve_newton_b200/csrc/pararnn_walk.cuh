@@ -146,25 +146,29 @@ __device__ __forceinline__ bool stage_wait(unsigned long long* bar, unsigned par
   }
 }
 
-template <int OP, typename PT, int S, int MINB>
-__global__ void __launch_bounds__(kThreads, MINB)
+template <int OP, typename PT, int S, int NW, int MINB>
+__global__ void __launch_bounds__(NW * 32, MINB)
     pararnn_walk_kernel(const __grid_constant__ KParams p, const __grid_constant__ TmaMaps tm) {
   using T_ = OpT<OP>;
   constexpr int NS = T_::NS;
   constexpr int NI = T_::NI;
   constexpr bool NEWTON = T_::newton;
   constexpr int CW = 32;
-  constexpr int TCH = kWarps * S;  // steps per chunk (one segment of S steps per warp)
+  constexpr int TCH = NW * S;  // steps per chunk (one segment of S steps per warp)
   using St = Stage<OP, PT, TCH>;
   constexpr unsigned kStageBytes = (St::kBytes + 1023u) / 1024u * 1024u;
   constexpr int WM = kMaxWalkIters;
 
+  constexpr int CPW = CW / NW;  // channels each warp scans across the NW segments
+  static_assert(CW % NW == 0, "warps per CTA must divide 32");
+
   extern __shared__ __align__(1024) unsigned char dsmem[];
   __shared__ unsigned long long s_bar[2];
-  __shared__ Map<NS> s_wagg[2][kWarps][CW];  // per-warp aggregates, double-buffered by iteration
-  __shared__ unsigned s_rmax[2][kWarps];
-  __shared__ Vec<NS> s_inc[2][WM][CW];       // chunk-end state per iteration, by chunk parity
-  __shared__ Vec<NS> s_pend[2][CW];          // chunk-end state of the loaded iterate
+  __shared__ Map<NS> s_wagg[NW][CW];      // per-segment aggregates of the iteration
+  __shared__ Map<NS> s_pre[NW][CW];       // exclusive prefix over the segments before
+  __shared__ Vec<NS> s_inc[2][WM][CW];    // chunk-end state per iteration, by chunk parity
+  __shared__ Vec<NS> s_pend[2][CW];       // chunk-end state of the loaded iterate
+  __shared__ Vec<NS> s_x0[CW];            // initial state of each channel of the tile
   __shared__ unsigned s_racc[WM];
   __shared__ int s_item;
   __shared__ int s_flag;
@@ -217,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
 #pragma unroll
       for (int i = 0; i < NS; ++i) x0v.x[i] = 0.0f;
       if (cvalid) IO<OP, PT>::init_state(p, bd, x0v.x);
+      if (warp == 0) s_x0[c] = x0v;
       if constexpr (NEWTON) {
 #pragma unroll
         for (int g = 0; g < NI; ++g) wv[g] = cvalid ? __ldg(p.w + (long long)g * p.D + d) : 0.0f;
@@ -266,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
             } else if (cvalid && t0 - 1 < p.L) {
               IO<OP, PT>::load_state(p, (b * p.L + t0 - 1) * p.D + d, xb.x);
             }
-            if (seg == kWarps - 1) s_pend[j & 1][c] = x[S - 1];
+            if (seg == NW - 1) s_pend[j & 1][c] = x[S - 1];
           }
         }
 
@@ -284,11 +289,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
         for (int kk = 0; kk < m; ++kk) {
           const int k = k0 + kk;
           const bool upd = !NEWTON || k < p.max_iters;
-          const int buf = kk & 1;
 
           Map<NS> mp[S];
           Map<NS> agg = map_identity<NS>();
-          unsigned rbits = 0u;
+          float rmax = 0.0f;
           Vec<NS> xp = xb;
           if (full) {
 #pragma unroll
@@ -296,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
               float vin[NI];
               St::read(stage, seg * S + s, c, vin);
               if constexpr (NEWTON) {
-                mp[s] = newton_step<OP>(vin, wv, xp, x[s], rbits);
+                mp[s] = newton_step<OP>(vin, wv, xp, x[s], rmax);
                 xp = x[s];
               } else {
                 mp[s] = StepMap<OP>::from_inputs(vin);
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
                 float vin[NI];
                 St::read(stage, seg * S + s, c, vin);
                 if constexpr (NEWTON) {
-                  mp[s] = newton_step<OP>(vin, wv, xp, x[s], rbits);
+                  mp[s] = newton_step<OP>(vin, wv, xp, x[s], rmax);
                   xp = x[s];
                 } else {
                   mp[s] = StepMap<OP>::from_inputs(vin);
@@ -322,41 +326,37 @@ __global__ void __launch_bounds__(kThreads, MINB)
             }
           }
           if constexpr (NEWTON) {
-            rbits = __reduce_max_sync(0xffffffffu, rbits);
-            if (lane == 0) s_rmax[buf][warp] = rbits;
+            const unsigned rbits = __reduce_max_sync(0xffffffffu, __float_as_uint(rmax));
+            if (lane == 0) atomicMax(&s_racc[kk], rbits);
           }
-
-          if (!upd) {  // residual-only iteration (k == max_iters)
-            __syncthreads();
-            if (tid == 0) {
-              unsigned r = s_racc[kk];
-#pragma unroll
-              for (int w2 = 0; w2 < kWarps; ++w2) r = max(r, s_rmax[buf][w2]);
-              s_racc[kk] = r;
-            }
-            continue;
-          }
+          if (!upd) continue;  // residual-only iteration (k == max_iters)
           any_update = true;
 
-          s_wagg[buf][warp][c] = agg;
+          // ---- combine the NW segments of each channel ----------------------
+          // Warp w scans channels [w*CPW, (w+1)*CPW): lane -> (channel, segment),
+          // a Kogge-Stone scan over the segment index within groups of NW lanes.
+          s_wagg[warp][c] = agg;
           __syncthreads();
-
-          // prefix of the earlier warps, carry into the chunk, chunk-end state
-          Map<NS> pre = map_identity<NS>();
+          {
+            const int ch = warp * CPW + lane / NW;
+            const int sg = lane % NW;
+            Map<NS> v = s_wagg[sg][ch];
 #pragma unroll
-          for (int w2 = 0; w2 < kWarps - 1; ++w2)
-            if (w2 < warp) pre = compose(s_wagg[buf][w2][c], pre);
-          Vec<NS> carry = (j == 0) ? x0v : s_inc[(j - 1) & 1][kk][c];
-          const Vec<NS> xin = apply(pre, carry);
-          if (warp == kWarps - 1) s_inc[j & 1][kk][c] = apply(agg, xin);
-          if constexpr (NEWTON) {
-            if (tid == 0) {
-              unsigned r = s_racc[kk];
-#pragma unroll
-              for (int w2 = 0; w2 < kWarps; ++w2) r = max(r, s_rmax[buf][w2]);
-              s_racc[kk] = r;
+            for (int off = 1; off < NW; off <<= 1) {
+              const Map<NS> o = shfl_up_map_w(v, off, NW);
+              if (sg >= off) v = compose(v, o);
+            }
+            Map<NS> ex = shfl_up_map_w(v, 1, NW);
+            if (sg == 0) ex = map_identity<NS>();
+            s_pre[sg][ch] = ex;
+            if (sg == NW - 1) {
+              const Vec<NS> cin = (j == 0) ? s_x0[ch] : s_inc[(j - 1) & 1][kk][ch];
+              s_inc[j & 1][kk][ch] = apply(v, cin);
             }
           }
+          __syncthreads();
+          const Vec<NS> carry = (j == 0) ? x0v : s_inc[(j - 1) & 1][kk][c];
+          const Vec<NS> xin = apply(s_pre[warp][c], carry);
           Vec<NS> xr = xin;
 #pragma unroll
           for (int s = 0; s < S; ++s) {
