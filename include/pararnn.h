@@ -110,8 +110,8 @@ typedef struct {
  *                the same result up to fp32 rounding; in walk mode at most 8
  *                iterations are evaluated per sweep.
  *  walk_warps  : warps per CTA in the walk regime with 32-channel tiles:
- *                0 = automatic (16 for the GRU solve and the diagonal scan
- *                below 512 tiles, else 8), 8 or 16. */
+ *                0 = automatic (16 for the diagonal scan below 512 tiles,
+ *                else 8), 8 or 16. */
 typedef struct {
   int32_t iters_first;
   int32_t iters_next;

@@ -42,10 +42,10 @@ namespace {
 #define PARARNN_MINB_SOLVE 2
 #endif
 #ifndef PARARNN_WALK_STEPS_GRU
-#define PARARNN_WALK_STEPS_GRU 8
+#define PARARNN_WALK_STEPS_GRU 16
 #endif
 #ifndef PARARNN_WALK_STEPS_LSTM
-#define PARARNN_WALK_STEPS_LSTM 4
+#define PARARNN_WALK_STEPS_LSTM 8
 #endif
 #ifndef PARARNN_WALK_STEPS_SCAN_DIAG
 #define PARARNN_WALK_STEPS_SCAN_DIAG 16
@@ -53,14 +53,21 @@ namespace {
 #ifndef PARARNN_WALK_STEPS_SCAN_BLOCK2
 #define PARARNN_WALK_STEPS_SCAN_BLOCK2 4
 #endif
+// Resident 8-warp CTAs per SM the walker's registers are held to: 3 where the
+// staged chunk is small (scans, bf16 GRU), 2 for fp32 GRU and LSTM, whose
+// larger per-thread state would otherwise spill (chosen by measurement).
 #ifndef PARARNN_WALK_MINB
 #define PARARNN_WALK_MINB 3
+#endif
+#ifndef PARARNN_WALK_MINB_WIDE
+#define PARARNN_WALK_MINB_WIDE 2
 #endif
 constexpr int kWalkStepsGru = PARARNN_WALK_STEPS_GRU;
 constexpr int kWalkStepsLstm = PARARNN_WALK_STEPS_LSTM;
 constexpr int kWalkStepsScanDiag = PARARNN_WALK_STEPS_SCAN_DIAG;
 constexpr int kWalkStepsScanBlock2 = PARARNN_WALK_STEPS_SCAN_BLOCK2;
 constexpr int kWalkMinBlocks = PARARNN_WALK_MINB;
+constexpr int kWalkMinBlocksWide = PARARNN_WALK_MINB_WIDE;
 constexpr int kStepsScanDiag = PARARNN_STEPS_SCAN_DIAG;
 constexpr int kStepsScanBlock2 = PARARNN_STEPS_SCAN_BLOCK2;
 constexpr int kStepsGru = PARARNN_STEPS_GRU;
@@ -158,9 +165,9 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
     // the TMA walker cuts time into chunks of its own length
     pl.S_walk = walk_steps_for(op);
     const int want = opts ? opts->walk_warps : 0;
-    // 16-warp CTAs only help the GRU and the diagonal scan when tiles are few
-    // (measured on B200); the 2x2 ops keep 8 warps, whose CTAs fit more per SM.
-    const bool wide = (op == kGru || op == kScanDiag) && ntiles < kWalkWideTiles;
+    // 16-warp CTAs only help the diagonal scan when tiles are few (measured on
+    // B200); the solves and the 2x2 scan keep 8 warps.
+    const bool wide = op == kScanDiag && ntiles < kWalkWideTiles;
     pl.NW_walk = (want == 8 || want == 16) ? want : (wide ? 16 : 8);
     long long tw = (long long)pl.NW_walk * pl.S_walk;
     long long nchunks_w = (L + tw - 1) / tw;
@@ -297,26 +304,29 @@ size_t walk_smem_bytes() {
 
 // Warps per CTA of the walker: 8, or 16 when the tiles are too few to fill the
 // SMs with 8-warp CTAs (more warps per tile then hide more latency).
-template <int OP, typename PT, int S>
+template <int OP, typename PT, int S, int MINB>
 const void* walk_kernel_nw(int nw, size_t* smem) {
   if (nw == 16) {
     *smem = walk_smem_bytes<OP, PT, S, 16>();
-    return (const void*)pararnn_walk_kernel<OP, PT, S, 16, (kWalkMinBlocks + 1) / 2>;
+    return (const void*)pararnn_walk_kernel<OP, PT, S, 16, (MINB + 1) / 2>;
   }
   *smem = walk_smem_bytes<OP, PT, S, 8>();
-  return (const void*)pararnn_walk_kernel<OP, PT, S, 8, kWalkMinBlocks>;
+  return (const void*)pararnn_walk_kernel<OP, PT, S, 8, MINB>;
 }
 
 const void* select_walk_kernel(int op, bool bf16, int nw, size_t* smem) {
   switch (op) {
-    case kScanDiag: return walk_kernel_nw<kScanDiag, float, kWalkStepsScanDiag>(nw, smem);
-    case kScanBlock2: return walk_kernel_nw<kScanBlock2, float, kWalkStepsScanBlock2>(nw, smem);
+    case kScanDiag:
+      return walk_kernel_nw<kScanDiag, float, kWalkStepsScanDiag, kWalkMinBlocks>(nw, smem);
+    case kScanBlock2:
+      return walk_kernel_nw<kScanBlock2, float, kWalkStepsScanBlock2, kWalkMinBlocks>(nw, smem);
     case kGru:
-      return bf16 ? walk_kernel_nw<kGru, __nv_bfloat16, kWalkStepsGru>(nw, smem)
-                  : walk_kernel_nw<kGru, float, kWalkStepsGru>(nw, smem);
+      return bf16 ? walk_kernel_nw<kGru, __nv_bfloat16, kWalkStepsGru, kWalkMinBlocks>(nw, smem)
+                  : walk_kernel_nw<kGru, float, kWalkStepsGru, kWalkMinBlocksWide>(nw, smem);
     default:
-      return bf16 ? walk_kernel_nw<kLstm, __nv_bfloat16, kWalkStepsLstm>(nw, smem)
-                  : walk_kernel_nw<kLstm, float, kWalkStepsLstm>(nw, smem);
+      return bf16
+                 ? walk_kernel_nw<kLstm, __nv_bfloat16, kWalkStepsLstm, kWalkMinBlocksWide>(nw, smem)
+                 : walk_kernel_nw<kLstm, float, kWalkStepsLstm, kWalkMinBlocksWide>(nw, smem);
   }
 }
 

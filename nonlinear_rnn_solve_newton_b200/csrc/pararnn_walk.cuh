@@ -159,16 +159,11 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   constexpr unsigned kStageBytes = (St::kBytes + 1023u) / 1024u * 1024u;
   constexpr int WM = kMaxWalkIters;
 
-  constexpr int CPW = CW / NW;  // channels each warp scans across the NW segments
-  static_assert(CW % NW == 0, "warps per CTA must divide 32");
-
   extern __shared__ __align__(1024) unsigned char dsmem[];
   __shared__ unsigned long long s_bar[2];
-  __shared__ Map<NS> s_wagg[NW][CW];      // per-segment aggregates of the iteration
-  __shared__ Map<NS> s_pre[NW][CW];       // exclusive prefix over the segments before
+  __shared__ Map<NS> s_wagg[2][NW][CW];   // per-segment aggregates, double-buffered by iteration
   __shared__ Vec<NS> s_inc[2][WM][CW];    // chunk-end state per iteration, by chunk parity
   __shared__ Vec<NS> s_pend[2][CW];       // chunk-end state of the loaded iterate
-  __shared__ Vec<NS> s_x0[CW];            // initial state of each channel of the tile
   __shared__ unsigned s_racc[WM];
   __shared__ int s_item;
   __shared__ int s_flag;
@@ -221,7 +216,6 @@ __global__ void __launch_bounds__(NW * 32, MINB)
 #pragma unroll
       for (int i = 0; i < NS; ++i) x0v.x[i] = 0.0f;
       if (cvalid) IO<OP, PT>::init_state(p, bd, x0v.x);
-      if (warp == 0) s_x0[c] = x0v;
       if constexpr (NEWTON) {
 #pragma unroll
         for (int g = 0; g < NI; ++g) wv[g] = cvalid ? __ldg(p.w + (long long)g * p.D + d) : 0.0f;
@@ -332,31 +326,20 @@ __global__ void __launch_bounds__(NW * 32, MINB)
           if (!upd) continue;  // residual-only iteration (k == max_iters)
           any_update = true;
 
-          // ---- combine the NW segments of each channel ----------------------
-          // Warp w scans channels [w*CPW, (w+1)*CPW): lane -> (channel, segment),
-          // a Kogge-Stone scan over the segment index within groups of NW lanes.
-          s_wagg[warp][c] = agg;
+          // ---- combine the segments: one barrier per iteration ---------------
+          // Each warp composes the aggregates of the warps before it (the shared
+          // array alternates between iterations, so the next iteration's writes
+          // cannot overtake a slow warp's reads) and applies the prefix to the
+          // state carried in from the previous chunk at this iteration.
+          const int buf = kk & 1;
+          s_wagg[buf][warp][c] = agg;
           __syncthreads();
-          {
-            const int ch = warp * CPW + lane / NW;
-            const int sg = lane % NW;
-            Map<NS> v = s_wagg[sg][ch];
-#pragma unroll
-            for (int off = 1; off < NW; off <<= 1) {
-              const Map<NS> o = shfl_up_map_w(v, off, NW);
-              if (sg >= off) v = compose(v, o);
-            }
-            Map<NS> ex = shfl_up_map_w(v, 1, NW);
-            if (sg == 0) ex = map_identity<NS>();
-            s_pre[sg][ch] = ex;
-            if (sg == NW - 1) {
-              const Vec<NS> cin = (j == 0) ? s_x0[ch] : s_inc[(j - 1) & 1][kk][ch];
-              s_inc[j & 1][kk][ch] = apply(v, cin);
-            }
-          }
-          __syncthreads();
+          Map<NS> pre = map_identity<NS>();
+#pragma unroll 4
+          for (int w2 = 0; w2 < warp; ++w2) pre = compose(s_wagg[buf][w2][c], pre);
           const Vec<NS> carry = (j == 0) ? x0v : s_inc[(j - 1) & 1][kk][c];
-          const Vec<NS> xin = apply(s_pre[warp][c], carry);
+          const Vec<NS> xin = apply(pre, carry);
+          if (warp == NW - 1) s_inc[j & 1][kk][c] = apply(agg, xin);
           Vec<NS> xr = xin;
 #pragma unroll
           for (int s = 0; s < S; ++s) {
