@@ -97,7 +97,8 @@ int walk_steps_for(int op) {
   }
 }
 int ns_for(int op) { return (op == kScanBlock2 || op == kLstm) ? 2 : 1; }
-int mapw_for(int op) { return (op == kScanBlock2 || op == kLstm) ? 8 : 2; }
+// 64-bit words of one look-back record (aggregate, then chunk-end state).
+int rec_words_for(int op) { return ns_for(op) == 2 ? Rec<2>::kWords : Rec<1>::kWords; }
 bool is_newton(int op) { return op == kGru || op == kLstm; }
 
 // Channels per tile: 32 (one warp row of 128 B for fp32) once D allows,
@@ -116,8 +117,8 @@ struct Plan {
   int NW_walk = 8;  // warps per CTA of the TMA walk kernel
   int op = 0, CW = 1, S = 1, T = 1, ntd = 0, ntiles = 0, nchunks = 0, nunits = 0;
   int m_first = 1, m_next = 1, mmax = 1, npasses = 1, max_iters = 0;
-  size_t off_rho = 0, off_ticket = 0, off_flags = 0, zero_bytes = 0;
-  size_t off_agg = 0, off_inc = 0, off_bnd = 0, total = 0;
+  size_t off_rho = 0, off_ticket = 0, off_rec = 0, zero_bytes = 0;
+  size_t off_bnd = 0, total = 0;
   bool ok = false;
 };
 
@@ -190,31 +191,20 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
     pl.m_first = pl.m_next = pl.mmax = 1;
     pl.npasses = 1;
   }
-  const int NS = ns_for(op), MAPW = mapw_for(op);
+  const int NS = ns_for(op);
   size_t off = sizeof(Ctrl);
   pl.off_rho = off;
   off += sizeof(unsigned) * (size_t)(pl.max_iters + 1);
   pl.off_ticket = off;
   off += sizeof(unsigned) * (size_t)pl.npasses;
   off = align_up(off, 256);
-  pl.off_flags = off;
-  if (!pl.walk) off += sizeof(unsigned) * (size_t)pl.mmax * pl.nunits;
+  pl.off_rec = off;  // look-back records: zeroed with the control block
+  if (!pl.walk) off += sizeof(unsigned long long) * (size_t)pl.mmax * pl.nunits * pl.CW *
+                       (size_t)rec_words_for(op);
   off = align_up(off, 256);
   pl.zero_bytes = off;
-  if (pl.walk) {  // no look-back slots
-    pl.off_agg = pl.off_inc = pl.off_bnd = off;
-    pl.total = align_up(off, 256);
-    pl.ok = true;
-    return pl;
-  }
-  pl.off_agg = off;
-  off += sizeof(float) * (size_t)pl.mmax * pl.nunits * pl.CW * MAPW;
-  off = align_up(off, 256);
-  pl.off_inc = off;
-  off += sizeof(float) * (size_t)pl.mmax * pl.nunits * pl.CW * NS;
-  off = align_up(off, 256);
   pl.off_bnd = off;
-  if (is_newton(op)) off += sizeof(float) * 2 * (size_t)pl.nunits * pl.CW * NS;
+  if (!pl.walk && is_newton(op)) off += sizeof(float) * 2 * (size_t)pl.nunits * pl.CW * NS;
   pl.total = align_up(off, 256);
   pl.ok = true;
   return pl;
@@ -421,9 +411,13 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
   kp.ctrl = reinterpret_cast<Ctrl*>(base);
   kp.rho_bits = reinterpret_cast<unsigned*>(base + pl.off_rho);
   kp.ticket = reinterpret_cast<unsigned*>(base + pl.off_ticket);
-  kp.flags = reinterpret_cast<unsigned*>(base + pl.off_flags);
-  kp.agg = reinterpret_cast<float*>(base + pl.off_agg);
-  kp.inc = reinterpret_cast<float*>(base + pl.off_inc);
+  kp.rec = reinterpret_cast<unsigned long long*>(base + pl.off_rec);
+  // D == 1: a thread's S steps form one contiguous block; 16-byte vectors need
+  // every array aligned and each block start on a 16-byte boundary (L % 8 == 0
+  // covers the narrowest element, bf16 gate triples).
+  kp.vec1 = kp.D == 1 && kp.L % 8 == 0 && aligned(kp.in0, 16) &&
+            (!kp.in1 || aligned(kp.in1, 16)) && aligned(kp.out0, 16) &&
+            (!kp.out1 || aligned(kp.out1, 16));
   kp.bnd = reinterpret_cast<float*>(base + pl.off_bnd);
   kp.ntd = pl.ntd;
   kp.ntiles = pl.ntiles;

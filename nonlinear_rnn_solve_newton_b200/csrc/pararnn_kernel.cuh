@@ -41,6 +41,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace pararnn {
 
@@ -50,22 +51,22 @@ constexpr int kWarps = kThreads / 32;
 enum OpKind : int { kScanDiag = 0, kScanBlock2 = 1, kGru = 2, kLstm = 3 };
 
 // NS: state components per channel (1 diagonal, 2 block).  NI: input values per
-// step held in registers.  MAPW: floats of one published aggregate (padded).
+// step held in registers.
 template <int OP> struct OpT;
 template <> struct OpT<kScanDiag> {
-  static constexpr int NS = 1, NI = 2, MAPW = 2;
+  static constexpr int NS = 1, NI = 2;
   static constexpr bool newton = false;
 };
 template <> struct OpT<kScanBlock2> {
-  static constexpr int NS = 2, NI = 6, MAPW = 8;
+  static constexpr int NS = 2, NI = 6;
   static constexpr bool newton = false;
 };
 template <> struct OpT<kGru> {
-  static constexpr int NS = 1, NI = 3, MAPW = 2;
+  static constexpr int NS = 1, NI = 3;
   static constexpr bool newton = true;
 };
 template <> struct OpT<kLstm> {
-  static constexpr int NS = 2, NI = 4, MAPW = 8;
+  static constexpr int NS = 2, NI = 4;
   static constexpr bool newton = true;
 };
 
@@ -100,10 +101,10 @@ struct KParams {
   Ctrl* ctrl;
   unsigned* rho_bits;    // [max_iters + 1]
   unsigned* ticket;      // [npasses]
-  unsigned* flags;       // [mmax][nunits]
-  float* agg;            // [mmax][nunits][CW][MAPW]
-  float* inc;            // [mmax][nunits][CW][NS]
+  unsigned long long* rec;  // look-back records [mmax][nunits][CW][Rec<NS>::kWords]
   float* bnd;            // [2][nunits][CW][NS]
+  int vec1;              // D == 1 and every array 16-byte aligned with L % 8 == 0:
+                         // a thread's S steps are one contiguous, aligned block
   void* info;            // pararnn_solve_info_t* (solves)
   int* status_dev;       // scans, optional
   long long timeout_ns;
@@ -213,34 +214,47 @@ __device__ __forceinline__ Map<NS> shfl_up_map_w(const Map<NS>& a, int delta, in
   return r;
 }
 
-// Published aggregate <-> global memory (MAPW floats, vectorised).
-template <int NS> __device__ __forceinline__ void store_map(float* p, const Map<NS>& a);
-template <> __device__ __forceinline__ void store_map<1>(float* p, const Map<1>& a) {
-  __stcg(reinterpret_cast<float2*>(p), make_float2(a.m[0][0], a.v[0]));
+// ---------------------------------------------------------------------------
+// Look-back records.  Every published number travels in its own aligned 64-bit
+// word together with the sweep's tag (high 32 bits = tag, low 32 = the float).
+// An aligned 64-bit access is single-copy atomic, so a reader validates each
+// word by its tag alone: the writer needs no fence and the reader no separate
+// flag round trip.  Per (iteration slot, unit, channel) the record holds the
+// chunk aggregate (NS*NS matrix entries, then NS offsets) and the chunk-end
+// state (NS words).  The records are zeroed before every call; tag 0 = empty.
+// ---------------------------------------------------------------------------
+template <int NS> struct Rec {
+  static constexpr int kAgg = NS * NS + NS;
+  static constexpr int kWords = kAgg + NS;
+};
+
+__device__ __forceinline__ unsigned long long tagged(unsigned tag, float v) {
+  return ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(v);
 }
-template <> __device__ __forceinline__ void store_map<2>(float* p, const Map<2>& a) {
-  __stcg(reinterpret_cast<float4*>(p), make_float4(a.m[0][0], a.m[0][1], a.m[1][0], a.m[1][1]));
-  __stcg(reinterpret_cast<float2*>(p + 4), make_float2(a.v[0], a.v[1]));
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
-template <int NS> __device__ __forceinline__ Map<NS> load_map(const float* p);
-template <> __device__ __forceinline__ Map<1> load_map<1>(const float* p) {
-  float2 q = __ldcg(reinterpret_cast<const float2*>(p));
-  Map<1> a;
-  a.m[0][0] = q.x;
-  a.v[0] = q.y;
-  return a;
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-template <> __device__ __forceinline__ Map<2> load_map<2>(const float* p) {
-  float4 q = __ldcg(reinterpret_cast<const float4*>(p));
-  float2 r = __ldcg(reinterpret_cast<const float2*>(p + 4));
-  Map<2> a;
-  a.m[0][0] = q.x;
-  a.m[0][1] = q.y;
-  a.m[1][0] = q.z;
-  a.m[1][1] = q.w;
-  a.v[0] = r.x;
-  a.v[1] = r.y;
-  return a;
+
+template <int NS>
+__device__ __forceinline__ void publish_agg(unsigned long long* rec, unsigned tag,
+                                            const Map<NS>& a) {
+#pragma unroll
+  for (int i = 0; i < NS; ++i)
+#pragma unroll
+    for (int j = 0; j < NS; ++j) st_relaxed_u64(rec + i * NS + j, tagged(tag, a.m[i][j]));
+#pragma unroll
+  for (int i = 0; i < NS; ++i) st_relaxed_u64(rec + NS * NS + i, tagged(tag, a.v[i]));
+}
+template <int NS>
+__device__ __forceinline__ void publish_inc(unsigned long long* rec, unsigned tag,
+                                            const Vec<NS>& x) {
+#pragma unroll
+  for (int i = 0; i < NS; ++i) st_relaxed_u64(rec + Rec<NS>::kAgg + i, tagged(tag, x.x[i]));
 }
 
 // ---------------------------------------------------------------------------
@@ -340,28 +354,47 @@ __device__ __forceinline__ void raise_error(const WaitCtx& w, unsigned code) {
   atomicExch(&w.ctrl->abort, 1u);
 }
 
-// Warp-wide wait until the flag carries `epoch` with a non-empty state.  All 32
-// lanes load the flag with acquire semantics in the same instruction and must
-// agree, so every lane has synchronised with the release that published the
-// state it acts on.  Returns 1 (aggregate), 2 (inclusive) or 0 on timeout/abort.
-__device__ __noinline__ unsigned wait_flag(const unsigned* addr, unsigned epoch, WaitCtx p) {
+// Warp-wide read of a predecessor's look-back record (all 32 lanes, each for
+// its own channel).  Returns 2 with the chunk-end state in `inc` if every lane
+// sees it, else 1 with the aggregate in `agg` if every lane sees that, waiting
+// (bounded) until one holds; 0 on timeout or abort.
+template <int NS>
+__device__ __forceinline__ unsigned read_record(const unsigned long long* rec, unsigned tag,
+                                                Map<NS>& agg, Vec<NS>& inc, const WaitCtx& w) {
   unsigned long long t_start = 0;
   unsigned ns = 32;
   for (int it = 0;; ++it) {
-    unsigned v = ld_acquire(addr);
-    bool ok = (v >> 2) == epoch && (v & 3u) != 0u;
-    unsigned v0 = __shfl_sync(0xffffffffu, v, 0);
-    if (__all_sync(0xffffffffu, ok && v == v0)) return v & 3u;
+    unsigned long long q[Rec<NS>::kWords];
+#pragma unroll
+    for (int i = 0; i < Rec<NS>::kWords; ++i) q[i] = ld_relaxed_u64(rec + i);
+    bool iok = true, aok = true;
+#pragma unroll
+    for (int i = 0; i < Rec<NS>::kAgg; ++i) aok = aok && (unsigned)(q[i] >> 32) == tag;
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+      iok = iok && (unsigned)(q[Rec<NS>::kAgg + i] >> 32) == tag;
+      inc.x[i] = __uint_as_float((unsigned)q[Rec<NS>::kAgg + i]);
+    }
+    if (__all_sync(0xffffffffu, iok)) return 2u;
+    if (__all_sync(0xffffffffu, aok)) {
+#pragma unroll
+      for (int i = 0; i < NS; ++i)
+#pragma unroll
+        for (int j = 0; j < NS; ++j) agg.m[i][j] = __uint_as_float((unsigned)q[i * NS + j]);
+#pragma unroll
+      for (int i = 0; i < NS; ++i) agg.v[i] = __uint_as_float((unsigned)q[NS * NS + i]);
+      return 1u;
+    }
     if (it == 0) t_start = globaltimer();
-    const bool aborting = __any_sync(0xffffffffu, ld_volatile(&p.ctrl->abort) != 0u);
+    const bool aborting = __any_sync(0xffffffffu, ld_volatile(&w.ctrl->abort) != 0u);
     const bool expired =
-        __any_sync(0xffffffffu, (globaltimer() - t_start) > (unsigned long long)p.timeout_ns);
+        __any_sync(0xffffffffu, (globaltimer() - t_start) > (unsigned long long)w.timeout_ns);
     if (aborting || expired) {
-      if ((threadIdx.x & 31) == 0 && !aborting) raise_error(p, 4u /*TIMEOUT*/);
+      if ((threadIdx.x & 31) == 0 && !aborting) raise_error(w, 4u /*TIMEOUT*/);
       return 0u;
     }
     __nanosleep(ns);
-    if (ns < 1024) ns <<= 1;
+    if (ns < 512) ns <<= 1;
   }
 }
 
@@ -507,6 +540,147 @@ template <typename PT> struct IO<kScanBlock2, PT> {
   }
 };
 
+// ---------------------------------------------------------------------------
+// D == 1: a thread's S consecutive steps of one channel are one contiguous
+// block of memory; move it with 16-byte vector accesses (the host checks the
+// alignment and sets p.vec1).
+// ---------------------------------------------------------------------------
+template <typename T, int N>
+__device__ __forceinline__ void ld_block(const T* src, float* dst) {
+  constexpr int V = 16 / (int)sizeof(T);
+  static_assert((N * (int)sizeof(T)) % 16 == 0, "block must be whole 16-byte vectors");
+#pragma unroll
+  for (int i = 0; i < N / V; ++i) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(src) + i);
+    T tmp[V];
+    memcpy(tmp, &q, 16);
+#pragma unroll
+    for (int k = 0; k < V; ++k) dst[i * V + k] = to_f(tmp[k]);
+  }
+}
+template <int N>
+__device__ __forceinline__ void ld_block_cg(const float* src, float* dst) {
+  static_assert(N % 4 == 0, "block must be whole float4s");
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i) {
+    const float4 q = __ldcg(reinterpret_cast<const float4*>(src) + i);
+    dst[4 * i] = q.x;
+    dst[4 * i + 1] = q.y;
+    dst[4 * i + 2] = q.z;
+    dst[4 * i + 3] = q.w;
+  }
+}
+template <int N>
+__device__ __forceinline__ void st_block(float* dst, const float* src) {
+  static_assert(N % 4 == 0, "block must be whole float4s");
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i)
+    reinterpret_cast<float4*>(dst)[i] =
+        make_float4(src[4 * i], src[4 * i + 1], src[4 * i + 2], src[4 * i + 3]);
+}
+
+// Per op: inputs of S steps [t0, t0+S) of channel b (D == 1) into vin[s][i], and
+// the state block into / out of x[s].
+template <int OP, typename PT, int S> struct Block1;
+template <typename PT, int S> struct Block1<kGru, PT, S> {
+  __device__ static void load_in(const KParams& p, long long b, long long t0, float (*vin)[3]) {
+    ld_block<PT, 3 * S>(reinterpret_cast<const PT*>(p.in0) + (b * p.L + t0) * 3, &vin[0][0]);
+  }
+  __device__ static void load_state(const KParams& p, long long i0, Vec<1>* x) {
+    float t[S];
+    ld_block_cg<S>(p.out0 + i0, t);
+#pragma unroll
+    for (int s = 0; s < S; ++s) x[s].x[0] = t[s];
+  }
+  __device__ static void store_state(const KParams& p, long long i0, const Vec<1>* x) {
+    float t[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) t[s] = x[s].x[0];
+    st_block<S>(p.out0 + i0, t);
+  }
+};
+template <typename PT, int S> struct Block1<kLstm, PT, S> {
+  __device__ static void load_in(const KParams& p, long long b, long long t0, float (*vin)[4]) {
+    ld_block<PT, 4 * S>(reinterpret_cast<const PT*>(p.in0) + (b * p.L + t0) * 4, &vin[0][0]);
+  }
+  __device__ static void load_state(const KParams& p, long long i0, Vec<2>* x) {
+    float tc[S], th[S];
+    ld_block_cg<S>(p.out0 + i0, tc);
+    ld_block_cg<S>(p.out1 + i0, th);
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      x[s].x[0] = tc[s];
+      x[s].x[1] = th[s];
+    }
+  }
+  __device__ static void store_state(const KParams& p, long long i0, const Vec<2>* x) {
+    float tc[S], th[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      tc[s] = x[s].x[0];
+      th[s] = x[s].x[1];
+    }
+    st_block<S>(p.out0 + i0, tc);
+    st_block<S>(p.out1 + i0, th);
+  }
+};
+template <typename PT, int S> struct Block1<kScanDiag, PT, S> {
+  __device__ static void load_in(const KParams& p, long long b, long long t0, float (*vin)[2]) {
+    float ta[S], tb[S];
+    ld_block<float, S>(reinterpret_cast<const float*>(p.in0) + b * p.L + t0, ta);
+    ld_block<float, S>(p.in1 + b * p.L + t0, tb);
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      vin[s][0] = ta[s];
+      vin[s][1] = tb[s];
+    }
+  }
+  __device__ static void load_state(const KParams& p, long long i0, Vec<1>* x) {
+    float t[S];
+    ld_block_cg<S>(p.out0 + i0, t);
+#pragma unroll
+    for (int s = 0; s < S; ++s) x[s].x[0] = t[s];
+  }
+  __device__ static void store_state(const KParams& p, long long i0, const Vec<1>* x) {
+    float t[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) t[s] = x[s].x[0];
+    st_block<S>(p.out0 + i0, t);
+  }
+};
+template <typename PT, int S> struct Block1<kScanBlock2, PT, S> {
+  __device__ static void load_in(const KParams& p, long long b, long long t0, float (*vin)[6]) {
+    float ta[4 * S], tb[2 * S];
+    ld_block<float, 4 * S>(reinterpret_cast<const float*>(p.in0) + (b * p.L + t0) * 4, ta);
+    ld_block<float, 2 * S>(p.in1 + (b * p.L + t0) * 2, tb);
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) vin[s][i] = ta[4 * s + i];
+      vin[s][4] = tb[2 * s];
+      vin[s][5] = tb[2 * s + 1];
+    }
+  }
+  __device__ static void load_state(const KParams& p, long long i0, Vec<2>* x) {
+    float t[2 * S];
+    ld_block_cg<2 * S>(p.out0 + 2 * i0, t);
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      x[s].x[0] = t[2 * s];
+      x[s].x[1] = t[2 * s + 1];
+    }
+  }
+  __device__ static void store_state(const KParams& p, long long i0, const Vec<2>* x) {
+    float t[2 * S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      t[2 * s] = x[s].x[0];
+      t[2 * s + 1] = x[s].x[1];
+    }
+    st_block<2 * S>(p.out0 + 2 * i0, t);
+  }
+};
+
 // Map of one step, from the inputs (scans) or from the cell at the iterate.
 template <int OP> struct StepMap;
 template <> struct StepMap<kScanDiag> {
@@ -586,7 +760,6 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
   using T_ = OpT<OP>;
   constexpr int NS = T_::NS;
   constexpr int NI = T_::NI;
-  constexpr int MAPW = T_::MAPW;
   constexpr bool NEWTON = T_::newton;
   constexpr int NSEG = kThreads / CW;
   constexpr int TCH = NSEG * S;  // steps per chunk
@@ -654,15 +827,22 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
         const bool publish = (long long)u != p.stall_unit;
 
         // ---- stage this chunk's inputs in registers ------------------------
+        // (D == 1 and aligned: the S steps are one contiguous block)
+        bool blk = false;
+        if constexpr (CW == 1) blk = p.vec1 && cvalid && t0 + S <= p.L;
         float vin[S][NI];
+        if (blk) {
+          if constexpr (CW == 1) Block1<OP, PT, S>::load_in(p, b, t0, vin);
+        } else {
 #pragma unroll
-        for (int s = 0; s < S; ++s) {
-          const long long t = t0 + s;
-          if (cvalid && t < p.L) {
-            IO<OP, PT>::load_in(p, (b * p.L + t) * p.D + d, b, t, d, vin[s]);
-          } else {
+          for (int s = 0; s < S; ++s) {
+            const long long t = t0 + s;
+            if (cvalid && t < p.L) {
+              IO<OP, PT>::load_in(p, (b * p.L + t) * p.D + d, b, t, d, vin[s]);
+            } else {
 #pragma unroll
-            for (int i = 0; i < NI; ++i) vin[s][i] = 0.0f;
+              for (int i = 0; i < NI; ++i) vin[s][i] = 0.0f;
+            }
           }
         }
 
@@ -679,14 +859,18 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
               for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
             if (t0 == 0 && cvalid) IO<OP, PT>::init_state(p, bd, xb.x);
           } else {
+            if (blk) {
+              if constexpr (CW == 1) Block1<OP, PT, S>::load_state(p, b * p.L + t0, x);
+            } else {
 #pragma unroll
-            for (int s = 0; s < S; ++s) {
-              const long long t = t0 + s;
-              if (cvalid && t < p.L) {
-                IO<OP, PT>::load_state(p, (b * p.L + t) * p.D + d, x[s].x);
-              } else {
+              for (int s = 0; s < S; ++s) {
+                const long long t = t0 + s;
+                if (cvalid && t < p.L) {
+                  IO<OP, PT>::load_state(p, (b * p.L + t) * p.D + d, x[s].x);
+                } else {
 #pragma unroll
-                for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
+                  for (int i = 0; i < NS; ++i) x[s].x[i] = 0.0f;
+                }
               }
             }
             if (cvalid) {
@@ -810,12 +994,10 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
             } else if constexpr (WALK) {
               carry = s_inc[(j - 1) & 1][kk][c];
             } else {
-              const size_t slot = (size_t)kk * p.nunits + u;
-              if (publish) {
-                if (lane < CW) store_map<NS>(p.agg + (slot * CW + c) * MAPW, cta);
-                __syncwarp();
-                if (lane == 0) st_release(p.flags + slot, (epoch << 2) | 1u);
-              }
+              constexpr int RW = Rec<NS>::kWords;
+              unsigned long long* my_rec =
+                  p.rec + (((size_t)kk * p.nunits + u) * CW + c) * RW;
+              if (publish && lane < CW) publish_agg<NS>(my_rec, epoch, cta);
               Map<NS> acc = map_identity<NS>();
               int pu = u - p.ntiles;
               for (;;) {
@@ -826,8 +1008,11 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
                   for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
                   break;
                 }
-                const size_t ps = (size_t)kk * p.nunits + pu;
-                unsigned st = wait_flag(p.flags + ps, epoch, wctx);
+                const unsigned long long* prec =
+                    p.rec + (((size_t)kk * p.nunits + pu) * CW + c) * RW;
+                Map<NS> pagg;
+                Vec<NS> pinc;
+                const unsigned st = read_record<NS>(prec, epoch, pagg, pinc, wctx);
                 if (st == 0u) {
                   failed = true;
 #pragma unroll
@@ -835,13 +1020,10 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
                   break;
                 }
                 if (st == 2u) {
-                  Vec<NS> v;
-#pragma unroll
-                  for (int i = 0; i < NS; ++i) v.x[i] = ldcg(p.inc + (ps * CW + c) * NS + i);
-                  carry = apply(acc, v);
+                  carry = apply(acc, pinc);
                   break;
                 }
-                acc = compose(acc, load_map<NS>(p.agg + (ps * CW + c) * MAPW));
+                acc = compose(acc, pagg);
                 pu -= p.ntiles;
               }
             }
@@ -849,14 +1031,9 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
             if constexpr (WALK) {
               if (lane < CW) s_inc[j & 1][kk][c] = xe;
             } else {
-              if (publish && !failed) {
-                const size_t slot = (size_t)kk * p.nunits + u;
-                if (lane < CW) {
-#pragma unroll
-                  for (int i = 0; i < NS; ++i) __stcg(p.inc + (slot * CW + c) * NS + i, xe.x[i]);
-                }
-                __syncwarp();
-                if (lane == 0) st_release(p.flags + slot, (epoch << 2) | 2u);
+              if (publish && !failed && lane < CW) {
+                constexpr int RW = Rec<NS>::kWords;
+                publish_inc<NS>(p.rec + (((size_t)kk * p.nunits + u) * CW + c) * RW, epoch, xe);
               }
             }
             if (lane < CW) s_carry[c] = carry;
@@ -881,10 +1058,14 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
 
         // ---- write the trajectory and the sweep boundary --------------------
         if (any_update || k0 == 0 || !NEWTON) {
+          if (blk) {
+            if constexpr (CW == 1) Block1<OP, PT, S>::store_state(p, b * p.L + t0, x);
+          } else {
 #pragma unroll
-          for (int s = 0; s < S; ++s) {
-            const long long t = t0 + s;
-            if (cvalid && t < p.L) IO<OP, PT>::store_state(p, (b * p.L + t) * p.D + d, x[s].x);
+            for (int s = 0; s < S; ++s) {
+              const long long t = t0 + s;
+              if (cvalid && t < p.L) IO<OP, PT>::store_state(p, (b * p.L + t) * p.D + d, x[s].x);
+            }
           }
         }
         if constexpr (NEWTON && !WALK) {
