@@ -189,15 +189,115 @@ def evaluated_iterations(passes, max_iters, m_first=4, m_next=2):
     return total
 
 
-def algorithmic_bytes(op, bf16, B, L, D, passes):
-    """Bytes a launch must move: each sweep reads P once, reads the iterate
-    (not in the first sweep: h^0 = 0) and writes the new iterate."""
+def algorithmic_bytes(op, bf16, B, L, D, passes=1):
+    """Bytes one launch must move.  Solves: each sweep reads P once, reads the
+    iterate (not in the first sweep: h^0 = 0) and writes the new iterate.
+    Scans: read A and b, write the state once."""
+    N = B * L * D
+    if op == "scan_diag":
+        return 12 * N
+    if op == "scan_block2":
+        return 32 * N
     G = 3 if op == "gru" else 4
     ns = 1 if op == "gru" else 2
     pbytes = G * (2 if bf16 else 4)
     first = pbytes + 4 * ns
     later = pbytes + 8 * ns
-    return B * L * D * (first + later * (passes - 1))
+    return N * (first + later * (passes - 1))
+
+
+def kernel_source_digest():
+    """sha256 of the CUDA sources: ties a recorded ncu traffic figure to the
+    kernel it was measured on."""
+    import hashlib
+
+    hsh = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nonlinear_rnn_solve_newton_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            hsh.update(name.encode() + b"\0" + f.read())
+    return hsh.hexdigest()
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch measured by ncu (profiles/traffic.json), or None
+    if no capture exists or the kernels changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+    except Exception:
+        return None, "no capture recorded"
+    if rec.get("source_sha256") != kernel_source_digest():
+        return None, "kernels changed since the capture"
+    k = rec.get("kernels", {}).get(workload)
+    if not k:
+        return None, "no capture for this workload"
+    return int(k["dram_bytes_per_launch"]), "ncu " + k.get("capture", "")
+
+
+# ---------------------------------------------------------------------------
+# workloads: device inputs, one step, host copies for the end-to-end leg
+# ---------------------------------------------------------------------------
+class Case:
+    def __init__(self, name, rank, device):
+        import torch
+
+        import nonlinear_rnn_solve_newton_b200 as pr
+
+        self.pr = pr
+        self.name = name
+        w = dict(inputs.WORKLOADS[name])
+        self.w = w
+        self.op, self.B, self.L, self.D, self.bf16 = w["op"], w["B"], w["L"], w["D"], w["bf16"]
+        self.N = self.B * self.L * self.D
+        self.device = device
+        self.tol, self.max_iters = 1e-4, 32
+        seed = w["seed"] if rank == 0 else [w["seed"], 1000 + rank]
+        B, L, D = self.B, self.L, self.D
+        if self.op in ("gru", "lstm"):
+            x = (inputs.gru_inputs if self.op == "gru" else inputs.lstm_inputs)(B, L, D, seed,
+                                                                                  self.bf16)
+            if self.bf16:
+                P = torch.from_numpy(x["P_bits"].view(np.int16)).view(torch.bfloat16)
+            else:
+                P = torch.from_numpy(x["P"])
+            self.host = {"P": P, "a": torch.from_numpy(x["a"]), "h0": torch.from_numpy(x["h0"])}
+            if self.op == "lstm":
+                self.host["c0"] = torch.from_numpy(x["c0"])
+            self.out_shapes = [(B, L, D)] * (2 if self.op == "lstm" else 1)
+        elif self.op == "scan_diag":
+            x = inputs.scan_diag_inputs(B, L, D, seed)
+            self.host = {k: torch.from_numpy(v) for k, v in x.items()}
+            self.out_shapes = [(B, L, D)]
+        else:
+            x = inputs.scan_block2_inputs(B, L, D, seed)
+            self.host = {k: torch.from_numpy(v) for k, v in x.items()}
+            self.out_shapes = [(B, L, D, 2)]
+        self.x = x
+        self.dev = {k: v.to(device) for k, v in self.host.items()}
+        self.outs = [torch.empty(sh, dtype=torch.float32, device=device) for sh in self.out_shapes]
+        self.info_t = torch.empty(pr.INFO_BYTES // 4, dtype=torch.int32, device=device)
+
+    def run(self, d, outs):
+        pr, op = self.pr, self.op
+        if op == "gru":
+            pr.solve_gru(d["P"], d["a"], d["h0"], self.tol, self.max_iters, out=outs[0],
+                         info=self.info_t)
+        elif op == "lstm":
+            pr.solve_lstm(d["P"], d["a"], d["c0"], d["h0"], self.tol, self.max_iters,
+                          out=(outs[0], outs[1]), info=self.info_t)
+        elif op == "scan_diag":
+            pr.scan_diag(d["A"], d["b"], d["h0"], out=outs[0])
+        else:
+            pr.scan_block2(d["A"], d["b"], d["x0"], out=outs[0])
+
+    def step(self):
+        self.run(self.dev, self.outs)
+
+    def solve_info(self):
+        if self.op in ("gru", "lstm"):
+            return self.pr.SolveInfo(self.info_t)
+        return None
 
 
 # ---------------------------------------------------------------------------
@@ -212,44 +312,28 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     maybe_init_pg(world, "nccl")
     pr.load()
-    w = dict(inputs.WORKLOADS[args.workload])
-    op, B, L, D, bf16 = w["op"], w["B"], w["L"], w["D"], w["bf16"]
-    seed = w["seed"] if rank == 0 else [w["seed"], 1000 + rank]
-    if op == "gru":
-        x = inputs.gru_inputs(B, L, D, seed, bf16)
-    else:
-        x = inputs.lstm_inputs(B, L, D, seed, bf16)
-    if bf16:
-        P_host = torch.from_numpy(x["P_bits"].view(np.int16)).view(torch.bfloat16)
-    else:
-        P_host = torch.from_numpy(x["P"])
-    P = P_host.to(device)
-    a = torch.from_numpy(x["a"]).to(device)
-    h0 = torch.from_numpy(x["h0"]).to(device)
-    c0 = torch.from_numpy(x["c0"]).to(device) if op == "lstm" else None
-    tol, max_iters = 1e-4, 32
-    N = B * L * D
+    cs = Case(args.workload, rank, device)
+    op, B, L, D, bf16, N = cs.op, cs.B, cs.L, cs.D, cs.bf16, cs.N
     stream = torch.cuda.current_stream()
 
-    h = torch.empty((B, L, D), dtype=torch.float32, device=device)
-    c = torch.empty_like(h) if op == "lstm" else None
-    info_t = torch.empty(pr.INFO_BYTES // 4, dtype=torch.int32, device=device)
-
-    def step():
-        if op == "gru":
-            pr.solve_gru(P, a, h0, tol, max_iters, out=h, info=info_t)
-        else:
-            pr.solve_lstm(P, a, c0, h0, tol, max_iters, out=(c, h), info=info_t)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
+    # Warm-up: at least W steps (and at least 3), continued until the GPU has
+    # run the workload for --warmup-seconds so clocks and memory have settled;
+    # the count actually run is reported as "warmup".
+    W = 0
+    t_w = time.perf_counter()
+    while W < max(args.warmup, 3) or time.perf_counter() - t_w < args.warmup_seconds:
+        cs.step()
+        W += 1
+        if W % 8 == 0 or W >= max(args.warmup, 3):
+            torch.cuda.synchronize()
     torch.cuda.synchronize()
-    info = pr.SolveInfo(info_t)
-    if info.status != 0 or not info.converged:
+    info = cs.solve_info()
+    if info is not None and (info.status != 0 or not info.converged):
         raise SystemExit(f"solve did not converge: {info.as_dict()}")
-    iters, passes = info.iterations, info.passes
+    iters = info.iterations if info else None
+    passes = info.passes if info else 1
 
-    # ---- timed region: exactly K solves --------------------------------------
+    # ---- timed region: exactly K steps ---------------------------------------
     K = args.steps
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
     barrier(world)
@@ -257,7 +341,7 @@ def run_ours(args, world, rank, local):
     with ClockSampler(local) as clk:
         evs[0].record(stream)
         for i in range(K):
-            step()
+            cs.step()
             evs[i + 1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -266,120 +350,126 @@ def run_ours(args, world, rank, local):
     ms, value = aggregate(ms_local, world, N, device)
     clocks = clk.summary()
 
-    # dominant kernel: the fused Newton kernel, one launch per solve.  Its
-    # per-launch time is bracketed by events on the launching stream; the
-    # bracket also holds the 1-2 us zeroing of the look-back flags.
+    # ---- roofline of the step's one kernel launch ----------------------------
+    # Per-launch times are CUDA events around each call on the launching stream
+    # (they also hold the ~2 us zeroing of the workspace control block).
     launch_ms = statistics.mean(per_step)
     hbm_peak, peak_kind, pk = peaks()
     bytes_launch = algorithmic_bytes(op, bf16, B, L, D, passes)
     achieved_gbs = bytes_launch / (launch_ms * 1e-3) / 1e9
-    ev_iters = evaluated_iterations(passes, max_iters)
-    mufu_ops = N * ev_iters * MUFU_PER_STEP[op]
-    sm_mhz = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
-    mufu_peak = SMS * MUFU_PER_SM_PER_CLK * sm_mhz * 1e6
-    mufu_frac = mufu_ops / (launch_ms * 1e-3) / mufu_peak
     hbm_frac = achieved_gbs / hbm_peak
-    if mufu_frac > hbm_frac:
-        roofline = {"bound": "alu", "achieved": mufu_ops / (launch_ms * 1e-3) / 1e12,
-                    "peak": mufu_peak / 1e12, "unit": "Tops/s (MUFU ex2+rcp)",
-                    "frac": mufu_frac, "traffic": None,
-                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                            "frac": hbm_frac, "peak_kind": peak_kind}}
+    traffic, traffic_src = recorded_traffic(args.workload)
+    hbm = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+           "frac": hbm_frac, "traffic": traffic, "peak_kind": peak_kind,
+           "algorithmic_bytes_per_launch": bytes_launch}
+    if op in ("gru", "lstm"):
+        ev_iters = evaluated_iterations(passes, cs.max_iters, m_first=5 if op == "lstm" else 4)
+        mufu_ops = N * ev_iters * MUFU_PER_STEP[op]
+        sm_mhz = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
+        mufu_peak = SMS * MUFU_PER_SM_PER_CLK * sm_mhz * 1e6
+        alu = {"bound": "alu", "achieved": mufu_ops / (launch_ms * 1e-3) / 1e12,
+               "peak": mufu_peak / 1e12, "unit": "Tops/s (MUFU ex2+rcp)",
+               "frac": mufu_ops / (launch_ms * 1e-3) / mufu_peak, "traffic": traffic,
+               "peak_kind": "derived: 148 SMs x 16 MUFU/clk x sampled SM clock",
+               "mufu_ops_per_launch": mufu_ops}
+        if alu["frac"] >= hbm_frac:
+            roofline = dict(alu)
+            roofline["hbm"] = {k: hbm[k] for k in ("achieved", "peak", "unit", "frac",
+                                                    "algorithmic_bytes_per_launch")}
+        else:
+            roofline = dict(hbm)
+            roofline["alu"] = {k: alu[k] for k in ("achieved", "peak", "unit", "frac")}
     else:
-        roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": hbm_frac, "traffic": None, "peak_kind": peak_kind,
-                    "alu": {"achieved": mufu_ops / (launch_ms * 1e-3) / 1e12,
-                            "peak": mufu_peak / 1e12, "unit": "Tops/s (MUFU ex2+rcp)",
-                            "frac": mufu_frac}}
-    roofline["kernel"] = "pararnn_kernel<GRU>" if op == "gru" else "pararnn_kernel<LSTM>"
-    roofline["algorithmic_bytes_per_launch"] = bytes_launch
+        ev_iters = None
+        roofline = dict(hbm)
+    roofline["kernel"] = {"gru": "pararnn Newton kernel (GRU)", "lstm":
+                          "pararnn Newton kernel (LSTM)", "scan_diag": "pararnn scan (diagonal)",
+                          "scan_block2": "pararnn scan (2x2)"}[op]
     roofline["launch_ms"] = launch_ms
+    roofline["traffic_source"] = traffic_src
 
     # ---- the diagonal scan at the same shape (the scan half of the metric) ---
     scan = None
     if args.workload == "gru_l" and not args.no_scan:
-        xs = inputs.scan_diag_inputs(B, L, D, inputs.WORKLOADS["scan"]["seed"])
-        A_s = torch.from_numpy(xs["A"]).to(device)
-        b_s = torch.from_numpy(xs["b"]).to(device)
-        h0_s = torch.from_numpy(xs["h0"]).to(device)
-        hs = torch.empty_like(A_s)
-        for _ in range(max(args.warmup, 3)):
-            pr.scan_diag(A_s, b_s, h0_s, out=hs)
-        torch.cuda.synchronize()
+        sc = Case("scan", rank, device)
+        t_w = time.perf_counter()
+        n_w = 0
+        while n_w < W or time.perf_counter() - t_w < args.warmup_seconds:
+            sc.step()
+            n_w += 1
+            torch.cuda.synchronize()
         sev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         barrier(world)
         sev[0].record(stream)
         for _ in range(K):
-            pr.scan_diag(A_s, b_s, h0_s, out=hs)
+            sc.step()
         sev[1].record(stream)
         torch.cuda.synchronize()
         sms = max_over_ranks(sev[0].elapsed_time(sev[1]) / K, world, device)
-        sbytes = 12 * B * L * D
+        sbytes = algorithmic_bytes("scan_diag", False, sc.B, sc.L, sc.D)
         sgbs = sbytes / (sms * 1e-3) / 1e9
-        scan = {"workload": f"diagonal scan fp32 B={B} L={L} D={D}", "ms": sms,
-                "channel_steps_per_s": world * B * L * D / (sms * 1e-3),
-                "achieved_gbs": sgbs, "algorithmic_bytes": sbytes,
-                "frac_of_measured_hbm": sgbs / hbm_peak, "frac_of_8tbs": sgbs / 8000.0}
-        del A_s, b_s, h0_s, hs
+        st, ssrc = recorded_traffic("scan")
+        scan = {"workload": f"diagonal scan fp32 B={sc.B} L={sc.L} D={sc.D}", "ms": sms,
+                "channel_steps_per_s": world * sc.N / (sms * 1e-3), "achieved_gbs": sgbs,
+                "algorithmic_bytes": sbytes, "frac_of_measured_hbm": sgbs / hbm_peak,
+                "frac_of_8tbs": sgbs / 8000.0, "traffic": st, "traffic_source": ssrc}
+        del sc
 
     # ---- end to end through the public API with pinned host buffers ---------
-    P_pin = P_host.pin_memory()
-    a_pin = torch.from_numpy(x["a"]).pin_memory()
-    h0_pin = torch.from_numpy(x["h0"]).pin_memory()
-    out_pin = torch.empty((B, L, D), dtype=torch.float32).pin_memory()
-    out2_pin = torch.empty((B, L, D), dtype=torch.float32).pin_memory() if op == "lstm" else None
+    e2e = None
+    if not args.no_e2e:
+        pin = {k: v.pin_memory() for k, v in cs.host.items()}
+        outs_pin = [torch.empty(sh, dtype=torch.float32).pin_memory() for sh in cs.out_shapes]
 
-    def e2e_step():
-        Pd = P_pin.to(device, non_blocking=True)
-        ad = a_pin.to(device, non_blocking=True)
-        h0d = h0_pin.to(device, non_blocking=True)
-        if op == "gru":
-            hd, _ = pr.solve_gru(Pd, ad, h0d, tol, max_iters, out=h, info=info_t)
-            out_pin.copy_(hd, non_blocking=True)
-        else:
-            cd, hd, _ = pr.solve_lstm(Pd, ad, None, h0d, tol, max_iters, out=(c, h), info=info_t)
-            out_pin.copy_(hd, non_blocking=True)
-            out2_pin.copy_(cd, non_blocking=True)
+        def e2e_step():
+            d = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
+            cs.run(d, cs.outs)
+            for o_pin, o_dev in zip(outs_pin, cs.outs):
+                o_pin.copy_(o_dev, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    ee = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    Ke = min(K, 5)
-    barrier(world)
-    ee[0].record(stream)
-    for _ in range(Ke):
         e2e_step()
-    ee[1].record(stream)
-    torch.cuda.synchronize()
-    ems = max_over_ranks(ee[0].elapsed_time(ee[1]) / Ke, world, device)
-    h2d = P_host.numel() * P_host.element_size() + 4 * a_pin.numel() + 4 * h0_pin.numel()
-    d2h = 4 * N * (2 if op == "lstm" else 1)
-    e2e = {"value": world * N / (ems * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+        torch.cuda.synchronize()
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        Ke = min(K, 5)
+        barrier(world)
+        ee[0].record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        ee[1].record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(ee[0].elapsed_time(ee[1]) / Ke, world, device)
+        h2d = sum(v.numel() * v.element_size() for v in pin.values())
+        d2h = sum(o.numel() * o.element_size() for o in outs_pin)
+        e2e = {"value": world * N / (ems * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems}
 
     # ---- the oracle on the host cores (rank 0, N = 1 only) -------------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(x, op, B, L, D, budget_s=args.cpu_seconds)
+        cpu = cpu_baseline(cs.x, op, B, L, D, budget_s=args.cpu_seconds)
 
     if rank == 0:
         wl = {"gru_l": "ParaGRU Newton solve fp32",
               "lm": "ParaGRU Newton solve, bf16 P, fp32 state",
               "deer": "ParaGRU Newton solve fp32 (DEER shape)",
               "gru_s": "ParaGRU Newton solve fp32 (small)",
-              "lstm": "ParaLSTM Newton solve fp32"}[args.workload]
+              "lstm": "ParaLSTM Newton solve fp32",
+              "scan": "diagonal affine scan fp32",
+              "block2": "2x2 block affine scan fp32"}[args.workload]
+        cfg = {"workload": f"{wl} B={B} L={L} D={D}", "B": B, "L": L, "D": D,
+               "parallelism": f"replicas x{world} (independent batches)",
+               "l2": "inputs larger than L2 (%.0f MB per step), no flush needed" % (
+                   sum(v.numel() * v.element_size() for v in cs.host.values()) / 1e6)}
+        if op in ("gru", "lstm"):
+            cfg.update({"tol": cs.tol, "max_iters": cs.max_iters, "newton_iterations": iters,
+                        "sweeps": passes, "evaluated_iterations": ev_iters})
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32" if not bf16 else "bf16-in/f32",
-            "data": "synthetic (seeded numpy: P~N(0,1), a~U(-0.5,0.5), h0=0)",
-            "config": {"workload": f"{wl} B={B} L={L} D={D}", "B": B, "L": L, "D": D,
-                       "tol": tol, "max_iters": max_iters, "newton_iterations": iters,
-                       "sweeps": passes, "evaluated_iterations": ev_iters,
-                       "parallelism": f"replicas x{world} (independent batches)",
-                       "l2": "inputs larger than L2 (P alone is %.0f MB)" % (
-                           P_host.numel() * P_host.element_size() / 1e6)},
-            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "warmup": W, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if not bf16 else "bf16-in/f32",
+            "data": "synthetic (seeded numpy; see tests/inputs.py)",
+            "config": cfg, "roofline": roofline, "clocks": clocks, "e2e": e2e,
             "gpu_launches": K, "scan": scan, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -392,11 +482,20 @@ def run_ours(args, world, rank, local):
 def cpu_baseline(x, op, B, L, D, budget_s=15.0):
     """The oracle's serial Newton (and its sequential rollout) on the host cores,
     on a bounded sample of the workload: the first batch rows, as many channels
-    as fit the time budget (estimated from a short calibration run)."""
+    as fit the time budget (estimated from a short calibration run).  For the
+    scans, the oracle's sequential scan over the whole workload."""
     import oracle
 
     oracle.build()
     cores = oracle.get_threads()
+    if op in ("scan_diag", "scan_block2"):
+        fn = oracle.scan_diag if op == "scan_diag" else oracle.scan_block2
+        args = (x["A"], x["b"], x["h0"] if op == "scan_diag" else x["x0"])
+        t0 = time.perf_counter()
+        fn(*args)
+        dt = time.perf_counter() - t0
+        return {"value": B * L * D / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"sequential fp64 scan over the whole workload ({dt:.1f} s)"}
     # calibrate on 64 channels
     nd = min(D, 64)
     Pc = x["P"][:1, :, :, :nd]
@@ -443,16 +542,29 @@ def run_reference(args, world, rank, local):
     oracle.build()
     w = dict(inputs.WORKLOADS[args.workload])
     op, B, L, D, bf16 = w["op"], w["B"], w["L"], w["D"], w["bf16"]
-    x = (inputs.gru_inputs if op == "gru" else inputs.lstm_inputs)(B, L, D, w["seed"], bf16)
     cores = oracle.get_threads()
-    # each step: the serial Newton on one batch row's first channels (bounded)
+    # each step: the oracle on one batch row's first channels (a bounded sample)
     nd = min(D, 256)
-    Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
-    as_ = np.ascontiguousarray(x["a"][:, :nd])
-    fn = oracle.newton_gru if op == "gru" else oracle.newton_lstm
+    x = inputs.workload_inputs(args.workload)  # the same draws as the GPU arm, then sliced
+    if op in ("gru", "lstm"):
+        Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
+        as_ = np.ascontiguousarray(x["a"][:, :nd])
+        fn = oracle.newton_gru if op == "gru" else oracle.newton_lstm
 
-    def step():
-        return fn(Ps, as_, tol=1e-4, max_iters=32)
+        def step():
+            return fn(Ps, as_, tol=1e-4, max_iters=32)
+        what = "serial fp64 Newton"
+    else:
+        if op == "scan_diag":
+            sargs = (x["A"][:1, :, :nd], x["b"][:1, :, :nd], x["h0"][:1, :nd])
+            fn = oracle.scan_diag
+        else:
+            sargs = (x["A"][:1, :, :nd], x["b"][:1, :, :nd], x["x0"][:1, :nd])
+            fn = oracle.scan_block2
+
+        def step():
+            return fn(*sargs)
+        what = "sequential fp64 scan"
 
     for _ in range(max(args.warmup, 1)):
         step()
@@ -466,7 +578,7 @@ def run_reference(args, world, rank, local):
             "steps": args.steps, "warmup": max(args.warmup, 1), "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded numpy)",
-            "config": {"workload": f"oracle serial Newton, sample of B=1 x D={nd} x L={L} "
+            "config": {"workload": f"oracle {what}, sample of B=1 x D={nd} x L={L} "
                                    f"from the {args.workload} workload (B={B}, D={D})"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"B=1, D={nd}, L={L} per step"},
@@ -481,10 +593,14 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="gru_l", choices=["gru_l", "lm", "deer", "gru_s", "lstm"])
+    ap.add_argument("--workload", default="gru_l",
+                    choices=["gru_l", "lm", "deer", "gru_s", "lstm", "scan", "block2"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--no-scan", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-scan", action="store_true", help="skip the scan leg (gru_l)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
+    ap.add_argument("--warmup-seconds", type=float, default=0.5,
+                    help="keep warming up until this much time has passed (after W steps)")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     if args.impl == "reference":

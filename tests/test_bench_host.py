@@ -1,0 +1,35 @@
+"""Host-side arithmetic of bench.py (CPU only): the algorithmic bytes and MUFU
+operation counts that the roofline figures divide by, and the sweep schedule
+the kernels follow."""
+import bench
+
+
+def test_algorithmic_bytes_per_channel_step():
+    N = 8 * 4096 * 1024
+    # scans: read A and b, write the state
+    assert bench.algorithmic_bytes("scan_diag", False, 8, 4096, 1024) == 12 * N
+    assert bench.algorithmic_bytes("scan_block2", False, 8, 4096, 1024) == 32 * N
+    # GRU, one sweep: P (3 gates) read once, h written once; h^0 = 0 is not read
+    assert bench.algorithmic_bytes("gru", False, 8, 4096, 1024, passes=1) == 16 * N
+    assert bench.algorithmic_bytes("gru", True, 8, 4096, 1024, passes=1) == 10 * N
+    # a second sweep re-reads P and reads + writes the iterate
+    assert bench.algorithmic_bytes("gru", False, 8, 4096, 1024, passes=2) == (16 + 20) * N
+    # LSTM: 4 gates, (c, h) state
+    assert bench.algorithmic_bytes("lstm", False, 8, 4096, 1024, passes=1) == 24 * N
+    assert bench.algorithmic_bytes("lstm", False, 8, 4096, 1024, passes=2) == (24 + 32) * N
+
+
+def test_sweep_schedule_matches_kernel_defaults():
+    # 4 iterations in the first sweep, 2 per later sweep, capped at max_iters + 1
+    assert bench.evaluated_iterations(1, 32) == 4
+    assert bench.evaluated_iterations(2, 32) == 6
+    assert bench.evaluated_iterations(3, 32) == 8
+    assert bench.evaluated_iterations(1, 2) == 3
+    assert bench.evaluated_iterations(2, 4) == 5
+
+
+def test_traffic_record_is_tied_to_kernel_sources():
+    d1 = bench.kernel_source_digest()
+    assert d1 == bench.kernel_source_digest() and len(d1) == 64
+    traffic, why = bench.recorded_traffic("no-such-workload")
+    assert traffic is None
