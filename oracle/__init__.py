@@ -58,32 +58,45 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def _bind(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    lib.oracle_scan_diag.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+    lib.oracle_scan_block2.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+    lib.oracle_gru_cell.argtypes = [_f64p, _f64p, ctypes.c_double, _f64p, _f64p]
+    lib.oracle_lstm_cell.argtypes = [_f64p, _f64p, ctypes.c_double, ctypes.c_double,
+                                     _f64p, _f64p, _f64p]
+    lib.oracle_rollout_gru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+    lib.oracle_rollout_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
+                                        _i64, _i64, _i64]
+    lib.oracle_newton_gru.argtypes = [_f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_int,
+                                      _i64, _i64, _i64, _f64p, _f64p, _i32p, _intp, _intp]
+    lib.oracle_newton_gru.restype = ctypes.c_int
+    lib.oracle_newton_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, ctypes.c_double,
+                                       ctypes.c_int, _i64, _i64, _i64, _f64p, _f64p,
+                                       _f64p, _i32p, _intp, _intp]
+    lib.oracle_newton_lstm.restype = ctypes.c_int
+    lib.oracle_residual_gru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+    lib.oracle_residual_gru.restype = ctypes.c_double
+    lib.oracle_set_threads.argtypes = [ctypes.c_int]
+    lib.oracle_get_threads.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            lib.oracle_scan_diag.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
-            lib.oracle_scan_block2.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
-            lib.oracle_gru_cell.argtypes = [_f64p, _f64p, ctypes.c_double, _f64p, _f64p]
-            lib.oracle_lstm_cell.argtypes = [_f64p, _f64p, ctypes.c_double, ctypes.c_double,
-                                             _f64p, _f64p, _f64p]
-            lib.oracle_rollout_gru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
-            lib.oracle_rollout_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
-                                                _i64, _i64, _i64]
-            lib.oracle_newton_gru.argtypes = [_f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_int,
-                                              _i64, _i64, _i64, _f64p, _f64p, _i32p, _intp, _intp]
-            lib.oracle_newton_gru.restype = ctypes.c_int
-            lib.oracle_newton_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, ctypes.c_double,
-                                               ctypes.c_int, _i64, _i64, _i64, _f64p, _f64p,
-                                               _f64p, _i32p, _intp, _intp]
-            lib.oracle_newton_lstm.restype = ctypes.c_int
-            lib.oracle_residual_gru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
-            lib.oracle_residual_gru.restype = ctypes.c_double
-            lib.oracle_set_threads.argtypes = [ctypes.c_int]
-            lib.oracle_get_threads.restype = ctypes.c_int
-            _lib = lib
+            _lib = _bind(ctypes.CDLL(build()))
     return _lib
+
+
+def compile_variant(src_path: str, out_path: str):
+    """Build and bind another copy of oracle.c (used by the tests that plant a
+    mistake in the oracle to check that the pins catch it)."""
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fno-fast-math",
+                           "-ffp-contract=off", "-std=c11", src_path, "-o", out_path, "-lm",
+                           "-lpthread"])
+    return _bind(ctypes.CDLL(out_path))
 
 
 def set_threads(n: int) -> None:

@@ -1,0 +1,88 @@
+"""The pins catch plausible mistakes in the oracle (CPU only).
+
+Each case plants one mistake in a copy of oracle.c -- a dropped Jacobian term,
+a flipped sign, an index off by one step, a transposed 2x2 operand, swapped
+LSTM gates, a forgotten initial state -- builds it, points the oracle package
+at it and runs the pins of tests/test_oracle_pins.py.  At least one pin must
+fail for every mistake; the unmodified oracle passes them all.
+"""
+import inspect
+import os
+import shutil
+
+import pytest
+import torch
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(os.path.abspath(oracle.__file__)), "oracle.c")
+
+MUTANTS = {
+    "gru_jacobian_drops_c_dz": ("*J = (1.0 - z) - h * dz + c * dz + z * dc;",
+                                "*J = (1.0 - z) - h * dz + z * dc;"),
+    "gru_jacobian_dr_sign": ("double du = w[2] * (r + h * dr);", "double du = w[2] * (r - h * dr);"),
+    "newton_residual_sign": ("x->rt[i] = f - x->h[i];", "x->rt[i] = x->h[i] - f;"),
+    "newton_previous_step_index": (
+        "x->h[IDX3(bb, t - 1, d, L, D)];\n"
+        "    double pg[3];\n"
+        "    for (int g = 0; g < 3; ++g) pg[g] = x->P[IDXP(bb, t, g, d, L, 3, D)];\n"
+        "    double f, J;",
+        "x->h[IDX3(bb, t, d, L, D)];\n"
+        "    double pg[3];\n"
+        "    for (int g = 0; g < 3; ++g) pg[g] = x->P[IDXP(bb, t, g, d, L, 3, D)];\n"
+        "    double f, J;"),
+    "scan_diag_misplaced_offset": ("x = c->A[i] * x + c->b[i];", "x = c->A[i] * (x + c->b[i]);"),
+    "scan_block2_transposed": (
+        "double n0 = M[0] * u0 + M[1] * u1 + c->b[2 * i + 0];\n"
+        "    double n1 = M[2] * u0 + M[3] * u1 + c->b[2 * i + 1];",
+        "double n0 = M[0] * u0 + M[2] * u1 + c->b[2 * i + 0];\n"
+        "    double n1 = M[1] * u0 + M[3] * u1 + c->b[2 * i + 1];"),
+    "lstm_gates_swapped": ("double cn = f * c + i * g;", "double cn = i * c + f * g;"),
+    "lstm_jacobian_drops_o": ("J[2] = o * dtc * dcn_dc;", "J[2] = dtc * dcn_dc;"),
+    "gru_rollout_ignores_h0": ("double s = x->h0 ? x->h0[bb * D + d] : 0.0;", "double s = 0.0;"),
+    "newton_solve_drops_carry": ("delta = x->Jt[i] * delta + x->rt[i];", "delta = x->rt[i];"),
+}
+
+
+def _pin_functions():
+    out = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if name.startswith("test_") and "oracle" in inspect.signature(fn).parameters:
+            out.append(fn)
+    return out
+
+
+def _failures_with(lib):
+    saved = oracle._lib
+    old_dtype = torch.get_default_dtype()
+    failed = []
+    try:
+        oracle._lib = lib
+        torch.set_default_dtype(torch.float64)
+        for fn in _pin_functions():
+            try:
+                fn(oracle)
+            except AssertionError:
+                failed.append(fn.__name__)
+    finally:
+        oracle._lib = saved
+        torch.set_default_dtype(old_dtype)
+    return failed
+
+
+def test_unmodified_oracle_passes_every_pin(tmp_path):
+    shutil.copy(SRC, tmp_path / "o.c")
+    lib = oracle.compile_variant(str(tmp_path / "o.c"), str(tmp_path / "o.so"))
+    assert _failures_with(lib) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(tmp_path, name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    (tmp_path / "o.c").write_text(src.replace(old, new))
+    lib = oracle.compile_variant(str(tmp_path / "o.c"), str(tmp_path / "o.so"))
+    failed = _failures_with(lib)
+    assert failed, f"no pin caught the planted mistake {name}"
