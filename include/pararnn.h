@@ -96,7 +96,8 @@ typedef struct {
 } pararnn_solve_info_t;
 
 /* Optional tuning and test hooks (host struct; pass NULL for defaults).
- *  iters_first : Newton iterations evaluated in the first sweep (0 = 4).
+ *  iters_first : Newton iterations evaluated in the first sweep
+ *                (0 = 4 for GRU, 5 for LSTM).
  *  iters_next  : Newton iterations per later sweep (0 = 2).
  *  wait_timeout_ns : bound on every device-side wait (0 = 1e9, i.e. 1 s).
  *  debug_stall_unit: test hook, -1 = off.  The work unit with this index

@@ -176,7 +176,10 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
   }
   if (is_newton(op)) {
     pl.max_iters = max_iters;
-    int mf = (opts && opts->iters_first > 0) ? opts->iters_first : 4;
+    // Iterations in the first sweep: Newton on these cells needs rho_0..rho_3
+    // (GRU) or rho_0..rho_4 (LSTM, whose 2x2 coupling converges a step later)
+    // for tol = 1e-4 at every workload measured, so one sweep usually suffices.
+    int mf = (opts && opts->iters_first > 0) ? opts->iters_first : (op == kLstm ? 5 : 4);
     int mn = (opts && opts->iters_next > 0) ? opts->iters_next : 2;
     const int mcap = pl.walk ? kMaxWalkIters : PARARNN_MAX_ITERS + 1;
     if (mf > mcap) mf = mcap;

@@ -354,47 +354,137 @@ __device__ __forceinline__ void raise_error(const WaitCtx& w, unsigned code) {
   atomicExch(&w.ctrl->abort, 1u);
 }
 
-// Warp-wide read of a predecessor's look-back record (all 32 lanes, each for
-// its own channel).  Returns 2 with the chunk-end state in `inc` if every lane
-// sees it, else 1 with the aggregate in `agg` if every lane sees that, waiting
-// (bounded) until one holds; 0 on timeout or abort.
+// One non-blocking read of a look-back record by this lane: 2 = chunk-end state
+// valid (in `inc`), 1 = aggregate valid (in `agg`), 0 = not yet published.
 template <int NS>
-__device__ __forceinline__ unsigned read_record(const unsigned long long* rec, unsigned tag,
-                                                Map<NS>& agg, Vec<NS>& inc, const WaitCtx& w) {
+__device__ __forceinline__ unsigned poll_record(const unsigned long long* rec, unsigned tag,
+                                                Map<NS>& agg, Vec<NS>& inc) {
+  unsigned long long q[Rec<NS>::kWords];
+#pragma unroll
+  for (int i = 0; i < Rec<NS>::kWords; ++i) q[i] = ld_relaxed_u64(rec + i);
+  bool iok = true, aok = true;
+#pragma unroll
+  for (int i = 0; i < Rec<NS>::kAgg; ++i) aok = aok && (unsigned)(q[i] >> 32) == tag;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    iok = iok && (unsigned)(q[Rec<NS>::kAgg + i] >> 32) == tag;
+    inc.x[i] = __uint_as_float((unsigned)q[Rec<NS>::kAgg + i]);
+  }
+#pragma unroll
+  for (int i = 0; i < NS; ++i)
+#pragma unroll
+    for (int j = 0; j < NS; ++j) agg.m[i][j] = __uint_as_float((unsigned)q[i * NS + j]);
+#pragma unroll
+  for (int i = 0; i < NS; ++i) agg.v[i] = __uint_as_float((unsigned)q[NS * NS + i]);
+  return iok ? 2u : (aok ? 1u : 0u);
+}
+
+template <int NS>
+__device__ __forceinline__ Map<NS> shfl_down_map(const Map<NS>& a, int delta) {
+  Map<NS> r;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+#pragma unroll
+    for (int j = 0; j < NS; ++j) r.m[i][j] = __shfl_down_sync(0xffffffffu, a.m[i][j], delta);
+    r.v[i] = __shfl_down_sync(0xffffffffu, a.v[i], delta);
+  }
+  return r;
+}
+template <int NS>
+__device__ __forceinline__ Vec<NS> shfl_vec(const Vec<NS>& a, int src) {
+  Vec<NS> r;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) r.x[i] = __shfl_sync(0xffffffffu, a.x[i], src);
+  return r;
+}
+
+// Windowed look-back (all 32 lanes of one warp).  Lane (w, c) = (lane / CW,
+// lane % CW) reads the record of predecessor w (counting back from the nearest,
+// `first_pred`) for channel c, so one round trip covers WIN = min(32 / CW, 4)
+// predecessors (a wider window measured slower: the nearest record is usually
+// ready, and polling more of them costs more than the round trips it saves).  Per channel: the nearest predecessor holding a chunk-end state
+// is found; the aggregates in front of it are composed by a shuffle tree
+// (nearest = latest map first) and applied to that state.  A window of
+// aggregates only is folded into `acc` and the window moves back; a window with
+// an unpublished slot in front of the nearest state is re-read.  Returns false
+// on timeout or abort; on success lanes < CW hold their channel's carry.
+#ifndef PARARNN_LOOKBACK_WINDOW
+#define PARARNN_LOOKBACK_WINDOW 4
+#endif
+template <int NS, int CW>
+__device__ __forceinline__ bool window_lookback(const unsigned long long* rec_base,
+                                                size_t unit_words, int first_pred, int unit_step,
+                                                unsigned tag, Vec<NS>& carry, const WaitCtx& wc) {
+  constexpr int WIN_MAX = 32 / CW;
+  constexpr int WIN = WIN_MAX < PARARNN_LOOKBACK_WINDOW ? WIN_MAX : PARARNN_LOOKBACK_WINDOW;
+  constexpr int RW = Rec<NS>::kWords;
+  const int lane = threadIdx.x & 31;
+  const int c = lane % CW;
+  const int wi = lane / CW;
+  Map<NS> acc = map_identity<NS>();  // windows already folded in, nearest first
+  bool done = false;
+  int base = first_pred;
   unsigned long long t_start = 0;
+  bool timing = false;
   unsigned ns = 32;
-  for (int it = 0;; ++it) {
-    unsigned long long q[Rec<NS>::kWords];
+  for (;;) {
+    const int pu = base - wi * unit_step;
+    Map<NS> agg = map_identity<NS>();
+    Vec<NS> inc;
 #pragma unroll
-    for (int i = 0; i < Rec<NS>::kWords; ++i) q[i] = ld_relaxed_u64(rec + i);
-    bool iok = true, aok = true;
-#pragma unroll
-    for (int i = 0; i < Rec<NS>::kAgg; ++i) aok = aok && (unsigned)(q[i] >> 32) == tag;
-#pragma unroll
-    for (int i = 0; i < NS; ++i) {
-      iok = iok && (unsigned)(q[Rec<NS>::kAgg + i] >> 32) == tag;
-      inc.x[i] = __uint_as_float((unsigned)q[Rec<NS>::kAgg + i]);
+    for (int i = 0; i < NS; ++i) inc.x[i] = 0.0f;
+    unsigned st = 0u;
+    if (wi < WIN && pu >= 0 && !done)
+      st = poll_record<NS>(rec_base + (size_t)pu * unit_words + (size_t)c * RW, tag, agg, inc);
+    const unsigned inc_mask = __ballot_sync(0xffffffffu, st == 2u);
+    const unsigned rdy_mask = __ballot_sync(0xffffffffu, st != 0u);
+    int fw = WIN;
+    bool gap = false;
+#pragma unroll 1
+    for (int w = 0; w < WIN; ++w) {
+      const unsigned bit = 1u << (w * CW + c);
+      if (inc_mask & bit) {
+        fw = w;
+        break;
+      }
+      if (!(rdy_mask & bit)) {
+        gap = true;
+        break;
+      }
     }
-    if (__all_sync(0xffffffffu, iok)) return 2u;
-    if (__all_sync(0xffffffffu, aok)) {
+    if (done) gap = false;
+    if (!__any_sync(0xffffffffu, gap)) {
+      Map<NS> m = (wi < fw) ? agg : map_identity<NS>();
 #pragma unroll
-      for (int i = 0; i < NS; ++i)
-#pragma unroll
-        for (int j = 0; j < NS; ++j) agg.m[i][j] = __uint_as_float((unsigned)q[i * NS + j]);
-#pragma unroll
-      for (int i = 0; i < NS; ++i) agg.v[i] = __uint_as_float((unsigned)q[NS * NS + i]);
-      return 1u;
+      for (int off = CW; off < CW * WIN; off <<= 1) {
+        const Map<NS> o = shfl_down_map(m, off);
+        if (wi + off / CW < WIN) m = compose(m, o);
+      }
+      const Vec<NS> v = shfl_vec(inc, (fw < WIN ? fw : 0) * CW + c);
+      if (!done) {
+        acc = compose(acc, m);
+        if (fw < WIN) {
+          carry = apply(acc, v);
+          done = true;
+        }
+      }
+      if (__all_sync(0xffffffffu, done || wi != 0)) return true;
+      base -= WIN * unit_step;
+      continue;
     }
-    if (it == 0) t_start = globaltimer();
-    const bool aborting = __any_sync(0xffffffffu, ld_volatile(&w.ctrl->abort) != 0u);
+    if (!timing) {
+      t_start = globaltimer();
+      timing = true;
+    }
+    const bool aborting = __any_sync(0xffffffffu, ld_volatile(&wc.ctrl->abort) != 0u);
     const bool expired =
-        __any_sync(0xffffffffu, (globaltimer() - t_start) > (unsigned long long)w.timeout_ns);
+        __any_sync(0xffffffffu, (globaltimer() - t_start) > (unsigned long long)wc.timeout_ns);
     if (aborting || expired) {
-      if ((threadIdx.x & 31) == 0 && !aborting) raise_error(w, 4u /*TIMEOUT*/);
-      return 0u;
+      if (lane == 0 && !aborting) raise_error(wc, 4u /*TIMEOUT*/);
+      return false;
     }
     __nanosleep(ns);
-    if (ns < 512) ns <<= 1;
+    if (ns < 256) ns <<= 1;
   }
 }
 
@@ -998,34 +1088,11 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
               unsigned long long* my_rec =
                   p.rec + (((size_t)kk * p.nunits + u) * CW + c) * RW;
               if (publish && lane < CW) publish_agg<NS>(my_rec, epoch, cta);
-              Map<NS> acc = map_identity<NS>();
-              int pu = u - p.ntiles;
-              for (;;) {
-                if (pu < 0) {  // chunk 0 always publishes an inclusive value
-                  if (lane == 0) raise_error(wctx, 4u);
-                  failed = true;
 #pragma unroll
-                  for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
-                  break;
-                }
-                const unsigned long long* prec =
-                    p.rec + (((size_t)kk * p.nunits + pu) * CW + c) * RW;
-                Map<NS> pagg;
-                Vec<NS> pinc;
-                const unsigned st = read_record<NS>(prec, epoch, pagg, pinc, wctx);
-                if (st == 0u) {
-                  failed = true;
-#pragma unroll
-                  for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
-                  break;
-                }
-                if (st == 2u) {
-                  carry = apply(acc, pinc);
-                  break;
-                }
-                acc = compose(acc, pagg);
-                pu -= p.ntiles;
-              }
+              for (int i = 0; i < NS; ++i) carry.x[i] = 0.0f;
+              failed = !window_lookback<NS, CW>(p.rec + (size_t)kk * p.nunits * CW * RW,
+                                                (size_t)CW * RW, u - p.ntiles, p.ntiles, epoch,
+                                                carry, wctx);
             }
             const Vec<NS> xe = apply(cta, carry);
             if constexpr (WALK) {
