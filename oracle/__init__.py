@@ -19,6 +19,8 @@ What each function computes, and the passage it follows:
   serial, with the max-abs residual over the whole batch as the stopping
   test (ParaRNN abstract and Figure 4 caption; DEER summary: tolerance 1e-4).
 * ``gru_cell`` / ``lstm_cell``: one cell step and its Jacobian.
+* ``backward_gru`` / ``backward_lstm``: gradients of a loss through the solved
+  trajectory by the adjoint (reverse-time, transposed bi-diagonal) recursion.
 
 Parity status: every function above is pinned in ``tests/test_oracle_pins.py``
 against closed forms, brute force, PyTorch's fp64 ``GRUCell``/``LSTMCell`` and
@@ -77,6 +79,10 @@ def _bind(lib):
     lib.oracle_newton_lstm.restype = ctypes.c_int
     lib.oracle_residual_gru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
     lib.oracle_residual_gru.restype = ctypes.c_double
+    lib.oracle_backward_gru.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
+                                        _i64, _i64, _i64]
+    lib.oracle_backward_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
+                                         _f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_get_threads.restype = ctypes.c_int
     return lib
@@ -234,3 +240,37 @@ def residual_gru(P, a, h, h0=None):
     B, L, G, D = P.shape
     h0 = None if h0 is None else _d(h0).reshape(B, D)
     return _load().oracle_residual_gru(_p(P), _p(a), _p(h0), _p(h), B, L, D)
+
+
+def backward_gru(P, a, h, gh, h0=None):
+    """Gradients of a loss through the ParaGRU trajectory h (the forward solution).
+
+    gh = dl/dh [B,L,D].  Returns (dP [B,L,3,D], da [3,D], dh0 [B,D]) by the adjoint
+    recursion lambda_t = g_t + J_{t+1}^T lambda_{t+1}, evaluated backwards in time."""
+    P, a, h, gh = _d(P), _d(a), _d(h), _d(gh)
+    B, L, G, D = P.shape
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    dP = np.empty_like(P)
+    da = np.empty((3, D))
+    dh0 = np.empty((B, D))
+    _load().oracle_backward_gru(_p(P), _p(a), _p(h0), _p(h), _p(gh), _p(dP), _p(da), _p(dh0),
+                                B, L, D)
+    return dP, da, dh0
+
+
+def backward_lstm(P, a, c, h, gc, gh, c0=None, h0=None):
+    """Gradients through the ParaLSTM trajectory (c, h): gc = dl/dc, gh = dl/dh (either
+    may be None = 0).  Returns (dP [B,L,4,D], da [4,D], dc0 [B,D], dh0 [B,D])."""
+    P, a, c, h = _d(P), _d(a), _d(c), _d(h)
+    B, L, G, D = P.shape
+    gc = None if gc is None else _d(gc)
+    gh = None if gh is None else _d(gh)
+    c0 = None if c0 is None else _d(c0).reshape(B, D)
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    dP = np.empty_like(P)
+    da = np.empty((4, D))
+    dc0 = np.empty((B, D))
+    dh0 = np.empty((B, D))
+    _load().oracle_backward_lstm(_p(P), _p(a), _p(c0), _p(h0), _p(c), _p(h), _p(gc), _p(gh),
+                                 _p(dP), _p(da), _p(dc0), _p(dh0), B, L, D)
+    return dP, da, dc0, dh0

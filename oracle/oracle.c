@@ -480,3 +480,139 @@ double oracle_residual_gru(const double* P, const double* a, const double* h0, c
   free(x.cmax);
   return m;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Gradients of the solved trajectory (the backward pass).                    */
+/* ------------------------------------------------------------------------- */
+/*
+ * For a loss whose gradient with respect to the trajectory is g_t = dl/dh_t
+ * (t = 1..L), the total gradient lambda_t = dl/dh_t through the recurrence
+ * obeys the adjoint recursion
+ *     lambda_L = g_L,   lambda_t = g_t + J_{t+1}^T lambda_{t+1},
+ * with J_t = df/dh at (h_{t-1}, P_t).  Then
+ *     dl/dP_t  = lambda_t^T df/dP_t (h_{t-1}, P_t),
+ *     dl/da    = sum_t lambda_t^T df/da (h_{t-1}, P_t),
+ *     dl/dh0   = J_1^T lambda_1.
+ * The trajectory h is the solution of the forward system (given, not
+ * recomputed).  Evaluated sequentially from t = L down to 1, in fp64.
+ */
+typedef struct {
+  const double *P, *a, *c0, *h0, *c, *h, *gc, *gh;
+  double *dP, *da_part, *dc0, *dh0;
+  int64_t L, D;
+} bwd_ctx;
+
+/* GRU: df/dPz = (c-h) z(1-z), df/dPc = z(1-c^2), df/dPr = z(1-c^2) ac h r(1-r);
+ * df/da_g = df/dP_g * (h for z and r, r*h for c). */
+static void backward_gru_chan(void* p, int64_t ch) {
+  bwd_ctx* x = (bwd_ctx*)p;
+  int64_t L = x->L, D = x->D, bb = ch / D, d = ch % D;
+  double w[3] = {x->a[0 * D + d], x->a[1 * D + d], x->a[2 * D + d]};
+  double da[3] = {0.0, 0.0, 0.0};
+  double lam_next = 0.0; /* J_{t+1}^T lambda_{t+1}, zero after the last step */
+  double mu = 0.0;
+  for (int64_t t = L - 1; t >= 0; --t) {
+    double hp = (t == 0) ? (x->h0 ? x->h0[bb * D + d] : 0.0) : x->h[IDX3(bb, t - 1, d, L, D)];
+    double pg[3];
+    for (int g = 0; g < 3; ++g) pg[g] = x->P[IDXP(bb, t, g, d, L, 3, D)];
+    double lam = x->gh[IDX3(bb, t, d, L, D)] + lam_next;
+    double z = sig(pg[0] + w[0] * hp);
+    double r = sig(pg[1] + w[1] * hp);
+    double c = tanh(pg[2] + w[2] * (r * hp));
+    double dfdz = (c - hp) * z * (1.0 - z);      /* d h'/d Pz */
+    double dfdu = z * (1.0 - c * c);             /* d h'/d Pc */
+    double dfdr = dfdu * w[2] * hp * r * (1.0 - r); /* d h'/d Pr */
+    x->dP[IDXP(bb, t, 0, d, L, 3, D)] = lam * dfdz;
+    x->dP[IDXP(bb, t, 1, d, L, 3, D)] = lam * dfdr;
+    x->dP[IDXP(bb, t, 2, d, L, 3, D)] = lam * dfdu;
+    da[0] += lam * dfdz * hp;
+    da[1] += lam * dfdr * hp;
+    da[2] += lam * dfdu * r * hp;
+    double f, J;
+    oracle_gru_cell(pg, w, hp, &f, &J);
+    mu = J * lam;
+    lam_next = mu;
+  }
+  if (x->dh0) x->dh0[bb * D + d] = mu;
+  for (int g = 0; g < 3; ++g) x->da_part[ch * 3 + g] = da[g];
+}
+
+void oracle_backward_gru(const double* P, const double* a, const double* h0, const double* h,
+                         const double* gh, double* dP, double* da, double* dh0, int64_t B,
+                         int64_t L, int64_t D) {
+  bwd_ctx x = {P, a, NULL, h0, NULL, h, NULL, gh, dP, NULL, NULL, dh0, L, D};
+  x.da_part = (double*)malloc((size_t)(B * D) * 3 * sizeof(double));
+  for_channels(B * D, backward_gru_chan, &x);
+  for (int64_t g = 0; g < 3; ++g)
+    for (int64_t d = 0; d < D; ++d) {
+      double s = 0.0;
+      for (int64_t bb = 0; bb < B; ++bb) s += x.da_part[(bb * D + d) * 3 + g];
+      da[g * D + d] = s;
+    }
+  free(x.da_part);
+}
+
+/* LSTM, state (c, h), lambda = (lambda_c, lambda_h).  With u_x = P_x + a_x h:
+ *   dc'/du_i = g i(1-i), dc'/du_f = c f(1-f), dc'/du_g = i(1-g^2), dc'/du_o = 0,
+ *   dh'/du_x = o (1 - tanh(c')^2) dc'/du_x  (x = i, f, g),  dh'/du_o = tanh(c') o(1-o);
+ *   dl/dP_x = lambda_c dc'/du_x + lambda_h dh'/du_x,   dl/da_x += dl/dP_x * h. */
+static void backward_lstm_chan(void* p, int64_t ch) {
+  bwd_ctx* x = (bwd_ctx*)p;
+  int64_t L = x->L, D = x->D, bb = ch / D, d = ch % D;
+  double w[4] = {x->a[0 * D + d], x->a[1 * D + d], x->a[2 * D + d], x->a[3 * D + d]};
+  double da[4] = {0.0, 0.0, 0.0, 0.0};
+  double mc = 0.0, mh = 0.0; /* J_{t+1}^T lambda_{t+1} */
+  for (int64_t t = L - 1; t >= 0; --t) {
+    double cp, hp;
+    if (t == 0) {
+      cp = x->c0 ? x->c0[bb * D + d] : 0.0;
+      hp = x->h0 ? x->h0[bb * D + d] : 0.0;
+    } else {
+      cp = x->c[IDX3(bb, t - 1, d, L, D)];
+      hp = x->h[IDX3(bb, t - 1, d, L, D)];
+    }
+    double pg[4];
+    for (int g = 0; g < 4; ++g) pg[g] = x->P[IDXP(bb, t, g, d, L, 4, D)];
+    double lc = (x->gc ? x->gc[IDX3(bb, t, d, L, D)] : 0.0) + mc;
+    double lh = (x->gh ? x->gh[IDX3(bb, t, d, L, D)] : 0.0) + mh;
+    double ig = sig(pg[0] + w[0] * hp);
+    double fg = sig(pg[1] + w[1] * hp);
+    double gg = tanh(pg[2] + w[2] * hp);
+    double og = sig(pg[3] + w[3] * hp);
+    double cn = fg * cp + ig * gg;
+    double tc = tanh(cn);
+    double dc[4] = {gg * ig * (1.0 - ig), cp * fg * (1.0 - fg), ig * (1.0 - gg * gg), 0.0};
+    double dh[4];
+    for (int g = 0; g < 3; ++g) dh[g] = og * (1.0 - tc * tc) * dc[g];
+    dh[3] = tc * og * (1.0 - og);
+    for (int g = 0; g < 4; ++g) {
+      double v = lc * dc[g] + lh * dh[g];
+      x->dP[IDXP(bb, t, g, d, L, 4, D)] = v;
+      da[g] += v * hp;
+    }
+    double fc, fh, J[4];
+    oracle_lstm_cell(pg, w, cp, hp, &fc, &fh, J);
+    /* J^T lambda: J = [[dc'/dc, dc'/dh], [dh'/dc, dh'/dh]] */
+    mc = J[0] * lc + J[2] * lh;
+    mh = J[1] * lc + J[3] * lh;
+  }
+  if (x->dc0) x->dc0[bb * D + d] = mc;
+  if (x->dh0) x->dh0[bb * D + d] = mh;
+  for (int g = 0; g < 4; ++g) x->da_part[ch * 4 + g] = da[g];
+}
+
+void oracle_backward_lstm(const double* P, const double* a, const double* c0, const double* h0,
+                          const double* c, const double* h, const double* gc, const double* gh,
+                          double* dP, double* da, double* dc0, double* dh0, int64_t B, int64_t L,
+                          int64_t D) {
+  bwd_ctx x = {P, a, c0, h0, c, h, gc, gh, dP, NULL, dc0, dh0, L, D};
+  x.da_part = (double*)malloc((size_t)(B * D) * 4 * sizeof(double));
+  for_channels(B * D, backward_lstm_chan, &x);
+  for (int64_t g = 0; g < 4; ++g)
+    for (int64_t d = 0; d < D; ++d) {
+      double s = 0.0;
+      for (int64_t bb = 0; bb < B; ++bb) s += x.da_part[(bb * D + d) * 4 + g];
+      da[g * D + d] = s;
+    }
+  free(x.da_part);
+}

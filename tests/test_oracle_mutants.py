@@ -42,6 +42,12 @@ MUTANTS = {
     "lstm_jacobian_drops_o": ("J[2] = o * dtc * dcn_dc;", "J[2] = dtc * dcn_dc;"),
     "gru_rollout_ignores_h0": ("double s = x->h0 ? x->h0[bb * D + d] : 0.0;", "double s = 0.0;"),
     "newton_solve_drops_carry": ("delta = x->Jt[i] * delta + x->rt[i];", "delta = x->rt[i];"),
+    "backward_gru_drops_r_derivative": ("double dfdr = dfdu * w[2] * hp * r * (1.0 - r);",
+                                        "double dfdr = dfdu * w[2] * hp * r;"),
+    "backward_lstm_untransposed_jacobian": ("mc = J[0] * lc + J[2] * lh;\n    mh = J[1] * lc + J[3] * lh;",
+                                            "mc = J[0] * lc + J[1] * lh;\n    mh = J[2] * lc + J[3] * lh;"),
+    "backward_gru_forward_time": ("double lam = x->gh[IDX3(bb, t, d, L, D)] + lam_next;",
+                                  "double lam = x->gh[IDX3(bb, t, d, L, D)];"),
 }
 
 

@@ -432,3 +432,89 @@ def test_inputs_are_deterministic():
     np.testing.assert_array_equal(a["P"], b["P"])
     assert a["P"].dtype == np.float32 and a["P"].shape == (2, 10, 3, 3)
     assert np.all(np.abs(a["a"]) <= 0.5)
+
+
+# --------------------------------------------------------------------------
+# Backward pass: the adjoint recursion against autograd through the library cells
+# --------------------------------------------------------------------------
+def _autograd_gru(P, a, h0, gh):
+    """dl/dP, dl/da, dl/dh0 for l = sum_t <gh_t, h_t>, with torch's GRU cell
+    (weights built from a, so autograd reaches a through the diagonal)."""
+    P = torch.tensor(np.asarray(P, np.float64), requires_grad=True)
+    a = torch.tensor(np.asarray(a, np.float64), requires_grad=True)
+    h = torch.tensor(np.asarray(h0, np.float64), requires_grad=True)
+    B, L, _, D = P.shape
+    w_ih = torch.eye(3 * D)
+    w_hh = torch.cat([torch.diag(a[1]), torch.diag(-a[0]), torch.diag(a[2])])
+    hs = []
+    ht = h
+    for t in range(L):
+        x = torch.cat([P[:, t, 1], -P[:, t, 0], P[:, t, 2]], dim=-1)
+        ht = torch._VF.gru_cell(x, ht, w_ih, w_hh, None, None)
+        hs.append(ht)
+    loss = (torch.stack(hs, 1) * torch.tensor(np.asarray(gh, np.float64))).sum()
+    loss.backward()
+    return P.grad.numpy(), a.grad.numpy(), h.grad.numpy()
+
+
+def _autograd_lstm(P, a, c0, h0, gc, gh):
+    P = torch.tensor(np.asarray(P, np.float64), requires_grad=True)
+    a = torch.tensor(np.asarray(a, np.float64), requires_grad=True)
+    c = torch.tensor(np.asarray(c0, np.float64), requires_grad=True)
+    h = torch.tensor(np.asarray(h0, np.float64), requires_grad=True)
+    B, L, _, D = P.shape
+    w_ih = torch.eye(4 * D)
+    w_hh = torch.cat([torch.diag(a[g]) for g in range(4)])
+    cs, hs = [], []
+    ct, ht = c, h
+    for t in range(L):
+        ht, ct = torch._VF.lstm_cell(P[:, t].reshape(B, 4 * D), (ht, ct), w_ih, w_hh, None, None)
+        cs.append(ct)
+        hs.append(ht)
+    loss = (torch.stack(cs, 1) * torch.tensor(np.asarray(gc, np.float64))).sum() + \
+        (torch.stack(hs, 1) * torch.tensor(np.asarray(gh, np.float64))).sum()
+    loss.backward()
+    return P.grad.numpy(), a.grad.numpy(), c.grad.numpy(), h.grad.numpy()
+
+
+def test_backward_gru_matches_autograd(oracle):
+    x = inputs.gru_inputs(2, 40, 5, seed=40, h0_normal=True)
+    gh = np.random.default_rng(41).standard_normal((2, 40, 5))
+    h = oracle.rollout_gru(x["P"], x["a"], x["h0"])
+    dP, da, dh0 = oracle.backward_gru(x["P"], x["a"], h, gh, x["h0"])
+    rP, ra, rh0 = _autograd_gru(x["P"], x["a"], x["h0"], gh)
+    np.testing.assert_allclose(dP, rP, atol=1e-12, rtol=1e-10)
+    np.testing.assert_allclose(da, ra, atol=1e-11, rtol=1e-10)
+    np.testing.assert_allclose(dh0, rh0, atol=1e-12, rtol=1e-10)
+
+
+def test_backward_lstm_matches_autograd(oracle):
+    x = inputs.lstm_inputs(2, 40, 5, seed=42, h0_normal=True)
+    rng = np.random.default_rng(43)
+    gc = rng.standard_normal((2, 40, 5))
+    gh = rng.standard_normal((2, 40, 5))
+    c, h = oracle.rollout_lstm(x["P"], x["a"], x["c0"], x["h0"])
+    dP, da, dc0, dh0 = oracle.backward_lstm(x["P"], x["a"], c, h, gc, gh, x["c0"], x["h0"])
+    rP, ra, rc0, rh0 = _autograd_lstm(x["P"], x["a"], x["c0"], x["h0"], gc, gh)
+    np.testing.assert_allclose(dP, rP, atol=1e-12, rtol=1e-10)
+    np.testing.assert_allclose(da, ra, atol=1e-11, rtol=1e-10)
+    np.testing.assert_allclose(dc0, rc0, atol=1e-12, rtol=1e-10)
+    np.testing.assert_allclose(dh0, rh0, atol=1e-12, rtol=1e-10)
+
+
+def test_backward_linear_recurrence_is_a_reverse_scan(oracle):
+    """a = 0 (minGRU): J_t = 1 - z_t does not depend on h, so lambda is the reverse
+    scan lambda_t = g_t + (1 - z_{t+1}) lambda_{t+1}, and dh0 = (1 - z_1) lambda_1."""
+    x = inputs.gru_inputs(1, 25, 3, seed=44, h0_normal=True)
+    a0 = np.zeros_like(x["a"])
+    gh = np.random.default_rng(45).standard_normal((1, 25, 3))
+    h = oracle.rollout_gru(x["P"], a0, x["h0"])
+    dP, da, dh0 = oracle.backward_gru(x["P"], a0, h, gh, x["h0"])
+    z = sigmoid(x["P"].astype(np.float64)[:, :, 0])                     # [1, L, D]
+    # reverse scan as a forward scan over reversed time
+    lam = oracle.scan_diag(np.concatenate([np.zeros((1, 1, 3)), (1 - z)[:, :0:-1]], 1),
+                           gh[:, ::-1])[:, ::-1]
+    np.testing.assert_allclose(dh0, (1 - z[:, 0]) * lam[:, 0], atol=1e-12)
+    c = np.tanh(x["P"].astype(np.float64)[:, :, 2])
+    hp = np.concatenate([x["h0"][:, None].astype(np.float64), h[:, :-1]], 1)
+    np.testing.assert_allclose(dP[:, :, 0], lam * (c - hp) * z * (1 - z), atol=1e-12)
