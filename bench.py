@@ -198,6 +198,10 @@ def algorithmic_bytes(op, bf16, B, L, D, passes=1):
         return 12 * N
     if op == "scan_block2":
         return 32 * N
+    if op == "gru_bwd":   # read P, h_{t-1}, dl/dh; write dP
+        return N * (3 * (2 if bf16 else 4) + 4 + 4 + 12)
+    if op == "lstm_bwd":  # read P, (c, h)_{t-1}, dl/dc, dl/dh; write dP
+        return N * (4 * (2 if bf16 else 4) + 8 + 8 + 16)
     G = 3 if op == "gru" else 4
     ns = 1 if op == "gru" else 2
     pbytes = G * (2 if bf16 else 4)
@@ -254,7 +258,29 @@ class Case:
         self.tol, self.max_iters = 1e-4, 32
         seed = w["seed"] if rank == 0 else [w["seed"], 1000 + rank]
         B, L, D = self.B, self.L, self.D
-        if self.op in ("gru", "lstm"):
+        if self.op in ("gru_bwd", "lstm_bwd"):
+            # the backward pass differentiates the forward solution: solve once here
+            cell = self.op[:-4]
+            x = (inputs.gru_inputs if cell == "gru" else inputs.lstm_inputs)(B, L, D, seed,
+                                                                               self.bf16)
+            P = torch.from_numpy(x["P"])
+            self.host = {"P": P, "a": torch.from_numpy(x["a"]), "h0": torch.from_numpy(x["h0"])}
+            grads = inputs.upstream_gradients(B, L, D, w["seed"], 2 if cell == "lstm" else 1)
+            self.host["gh"] = torch.from_numpy(grads[0])
+            if cell == "lstm":
+                self.host["c0"] = torch.from_numpy(x["c0"])
+                self.host["gc"] = torch.from_numpy(grads[1])
+            dv = {k: v.to(device) for k, v in self.host.items()}
+            if cell == "gru":
+                hs, info = pr.solve_gru(dv["P"], dv["a"], dv["h0"])
+                self.host["h"] = hs.cpu()
+            else:
+                cs_, hs, info = pr.solve_lstm(dv["P"], dv["a"], dv["c0"], dv["h0"])
+                self.host["c"] = cs_.cpu()
+                self.host["h"] = hs.cpu()
+            G = 3 if cell == "gru" else 4
+            self.out_shapes = [(B, L, G, D), (G, D), (B, D)] + ([(B, D)] if cell == "lstm" else [])
+        elif self.op in ("gru", "lstm"):
             x = (inputs.gru_inputs if self.op == "gru" else inputs.lstm_inputs)(B, L, D, seed,
                                                                                   self.bf16)
             if self.bf16:
@@ -286,6 +312,12 @@ class Case:
         elif op == "lstm":
             pr.solve_lstm(d["P"], d["a"], d["c0"], d["h0"], self.tol, self.max_iters,
                           out=(outs[0], outs[1]), info=self.info_t)
+        elif op == "gru_bwd":
+            pr.solve_gru_backward(d["P"], d["a"], d["h"], d["gh"], d["h0"],
+                                  out=(outs[0], outs[1], outs[2]))
+        elif op == "lstm_bwd":
+            pr.solve_lstm_backward(d["P"], d["a"], d["c"], d["h"], d["gc"], d["gh"], d["c0"],
+                                   d["h0"], out=(outs[0], outs[1], outs[2], outs[3]))
         elif op == "scan_diag":
             pr.scan_diag(d["A"], d["b"], d["h0"], out=outs[0])
         else:
@@ -362,9 +394,13 @@ def run_ours(args, world, rank, local):
     hbm = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
            "frac": hbm_frac, "traffic": traffic, "peak_kind": peak_kind,
            "algorithmic_bytes_per_launch": bytes_launch}
-    if op in ("gru", "lstm"):
-        ev_iters = evaluated_iterations(passes, cs.max_iters, m_first=5 if op == "lstm" else 4)
-        mufu_ops = N * ev_iters * MUFU_PER_STEP[op]
+    if op in ("gru", "lstm", "gru_bwd", "lstm_bwd"):
+        if op in ("gru", "lstm"):
+            ev_iters = evaluated_iterations(passes, cs.max_iters,
+                                            m_first=5 if op == "lstm" else 4)
+        else:
+            ev_iters = 1  # the backward evaluates each step once
+        mufu_ops = N * ev_iters * MUFU_PER_STEP[op[:4].rstrip("_")]
         sm_mhz = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
         mufu_peak = SMS * MUFU_PER_SM_PER_CLK * sm_mhz * 1e6
         alu = {"bound": "alu", "achieved": mufu_ops / (launch_ms * 1e-3) / 1e12,
@@ -384,7 +420,9 @@ def run_ours(args, world, rank, local):
         roofline = dict(hbm)
     roofline["kernel"] = {"gru": "pararnn Newton kernel (GRU)", "lstm":
                           "pararnn Newton kernel (LSTM)", "scan_diag": "pararnn scan (diagonal)",
-                          "scan_block2": "pararnn scan (2x2)"}[op]
+                          "scan_block2": "pararnn scan (2x2)",
+                          "gru_bwd": "pararnn backward kernel (GRU)",
+                          "lstm_bwd": "pararnn backward kernel (LSTM)"}[op]
     roofline["launch_ms"] = launch_ms
     roofline["traffic_source"] = traffic_src
 
@@ -455,7 +493,9 @@ def run_ours(args, world, rank, local):
               "gru_s": "ParaGRU Newton solve fp32 (small)",
               "lstm": "ParaLSTM Newton solve fp32",
               "scan": "diagonal affine scan fp32",
-              "block2": "2x2 block affine scan fp32"}[args.workload]
+              "block2": "2x2 block affine scan fp32",
+              "gru_bwd": "ParaGRU backward pass fp32",
+              "lstm_bwd": "ParaLSTM backward pass fp32"}[args.workload]
         cfg = {"workload": f"{wl} B={B} L={L} D={D}", "B": B, "L": L, "D": D,
                "parallelism": f"replicas x{world} (independent batches)",
                "l2": "inputs larger than L2 (%.0f MB per step), no flush needed" % (
@@ -488,6 +528,21 @@ def cpu_baseline(x, op, B, L, D, budget_s=15.0):
 
     oracle.build()
     cores = oracle.get_threads()
+    if op in ("gru_bwd", "lstm_bwd"):
+        nb = 1
+        nd = min(D, 256)
+        Ps = x["P"][:nb, :, :, :nd]
+        as_ = x["a"][:, :nd]
+        t0 = time.perf_counter()
+        if op == "gru_bwd":
+            hh = oracle.rollout_gru(Ps, as_)
+            oracle.backward_gru(Ps, as_, hh, hh)
+        else:
+            cc, hh = oracle.rollout_lstm(Ps, as_)
+            oracle.backward_lstm(Ps, as_, cc, hh, cc, hh)
+        dt = time.perf_counter() - t0
+        return {"value": nb * L * nd / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"fp64 rollout + adjoint on B={nb} x D={nd} x L={L} ({dt:.1f} s)"}
     if op in ("scan_diag", "scan_block2"):
         fn = oracle.scan_diag if op == "scan_diag" else oracle.scan_block2
         args = (x["A"], x["b"], x["h0"] if op == "scan_diag" else x["x0"])
@@ -545,8 +600,30 @@ def run_reference(args, world, rank, local):
     cores = oracle.get_threads()
     # each step: the oracle on one batch row's first channels (a bounded sample)
     nd = min(D, 256)
-    x = inputs.workload_inputs(args.workload)  # the same draws as the GPU arm, then sliced
-    if op in ("gru", "lstm"):
+    if op in ("gru_bwd", "lstm_bwd"):
+        cell = op[:-4]
+        x = (inputs.gru_inputs if cell == "gru" else inputs.lstm_inputs)(B, L, D, w["seed"])
+        Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
+        as_ = np.ascontiguousarray(x["a"][:, :nd])
+        g = [v[:1, :, :nd] for v in inputs.upstream_gradients(B, L, D, w["seed"],
+                                                              2 if cell == "lstm" else 1)]
+        if cell == "gru":
+            hh = oracle.rollout_gru(Ps, as_)
+
+            def step():
+                return oracle.backward_gru(Ps, as_, hh, g[0])
+        else:
+            cc, hh = oracle.rollout_lstm(Ps, as_)
+
+            def step():
+                return oracle.backward_lstm(Ps, as_, cc, hh, g[1], g[0])
+        what = "adjoint (backward) recursion"
+        x = None
+    else:
+        x = inputs.workload_inputs(args.workload)  # the same draws as the GPU arm, then sliced
+    if op in ("gru_bwd", "lstm_bwd"):
+        pass
+    elif op in ("gru", "lstm"):
         Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
         as_ = np.ascontiguousarray(x["a"][:, :nd])
         fn = oracle.newton_gru if op == "gru" else oracle.newton_lstm
@@ -594,7 +671,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gru_l",
-                    choices=["gru_l", "lm", "deer", "gru_s", "lstm", "scan", "block2"])
+                    choices=["gru_l", "lm", "deer", "gru_s", "lstm", "scan", "block2",
+                             "gru_bwd", "lstm_bwd"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-scan", action="store_true", help="skip the scan leg (gru_l)")

@@ -65,7 +65,9 @@ typedef enum {
   PARARNN_OP_SCAN_DIAG = 0,
   PARARNN_OP_SCAN_BLOCK2 = 1,
   PARARNN_OP_GRU = 2,
-  PARARNN_OP_LSTM = 3
+  PARARNN_OP_LSTM = 3,
+  PARARNN_OP_GRU_BACKWARD = 4,
+  PARARNN_OP_LSTM_BACKWARD = 5
 } pararnn_op_t;
 
 /* Device-side outcome of a solve (caller-owned DEVICE memory, written by the
@@ -173,6 +175,43 @@ pararnn_status_t pararnn_solve_lstm(const void* P, pararnn_dtype_t p_dtype, cons
                                     int64_t B, int64_t L, int64_t D, float tol, int32_t max_iters,
                                     void* ws, size_t ws_bytes, pararnn_solve_info_t* info,
                                     const pararnn_options_t* opts, void* stream);
+
+/* Backward pass of the ParaGRU solve: gradients of a loss through the solved
+ * trajectory (DEER summary: "forward plus gradients"; ParaRNN trains with
+ * them).  With g_t = dl/dh_t given, the total gradient lambda_t obeys the
+ * adjoint recursion lambda_t = g_t + J_{t+1}^T lambda_{t+1} -- the transposed
+ * bi-diagonal system of a Newton step, run backwards in time -- and
+ *   dP_t = lambda_t df/dP_t,  da = sum over (b, t) of lambda_t df/da,
+ *   dh0 = J_1^T lambda_1,
+ * with every derivative taken at the forward solution.  One pass, no Newton
+ * iterations.
+ *  P, p_dtype, a, h0 : as given to pararnn_solve_gru.
+ *  h  : [B, L, D] fp32, the forward solution (t = 1..L).
+ *  dh : [B, L, D] fp32 upstream gradient dl/dh_t.
+ *  dP : [B, L, 3, D] fp32 output.   da : [3, D] fp32 output (overwritten; the
+ *       sum over b and t is accumulated with atomics, so its last bits depend
+ *       on the order of addition).   dh0 : [B, D] fp32 output or NULL.
+ *  status_dev : optional device int32 for the device-side status.
+ *  ws : pararnn_workspace_size(PARARNN_OP_GRU_BACKWARD, B, L, D, 0, opts). */
+pararnn_status_t pararnn_solve_gru_backward(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                            const float* h0, const float* h, const float* dh,
+                                            float* dP, float* da, float* dh0, int64_t B,
+                                            int64_t L, int64_t D, void* ws, size_t ws_bytes,
+                                            int32_t* status_dev, const pararnn_options_t* opts,
+                                            void* stream);
+
+/* Backward pass of the ParaLSTM solve, state (c, h) and 2x2 transposed
+ * Jacobians.  c, h : the forward solution.  dc, dh : upstream gradients
+ * dl/dc_t and dl/dh_t (either may be NULL = 0, not both).  Outputs dP
+ * [B, L, 4, D], da [4, D] (overwritten, atomically accumulated), dc0 and dh0
+ * [B, D] (each may be NULL).  Workspace for PARARNN_OP_LSTM_BACKWARD. */
+pararnn_status_t pararnn_solve_lstm_backward(const void* P, pararnn_dtype_t p_dtype,
+                                             const float* a, const float* c0, const float* h0,
+                                             const float* c, const float* h, const float* dc,
+                                             const float* dh, float* dP, float* da, float* dc0,
+                                             float* dh0, int64_t B, int64_t L, int64_t D,
+                                             void* ws, size_t ws_bytes, int32_t* status_dev,
+                                             const pararnn_options_t* opts, void* stream);
 
 /* Allocation-free variant of pararnn_solve_gru (the pages have no counterpart:
  * this is an interface convenience of this library).

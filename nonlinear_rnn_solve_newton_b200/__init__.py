@@ -12,6 +12,7 @@ Entry points (same names as the C ABI, without the ``pararnn_`` prefix):
 * ``scan_block2(A, b, x0=None)``    x_t = A_t x_{t-1} + b_t, 2x2 blocks  [B, L, D, 2]
 * ``solve_gru(P, a, h0=None, tol=1e-4, max_iters=32)``   ParaGRU Newton solve
 * ``solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32)``  ParaLSTM Newton solve
+* ``solve_gru_backward`` / ``solve_lstm_backward``  gradients through the solution
 """
 from __future__ import annotations
 
@@ -24,6 +25,7 @@ import torch
 from . import build as _build
 
 __all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc",
+           "solve_gru_backward", "solve_lstm_backward",
            "workspace_size",
            "SolveInfo", "Options", "PararnnError", "library_path", "load", "MAX_ITERS"]
 
@@ -32,6 +34,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libpararnn.so")
 
 OP_SCAN_DIAG, OP_SCAN_BLOCK2, OP_GRU, OP_LSTM = 0, 1, 2, 3
+OP_GRU_BACKWARD, OP_LSTM_BACKWARD = 4, 5
 F32, BF16 = 0, 1
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA runtime error",
@@ -100,6 +103,14 @@ def load(build_if_missing: bool = True):
                                                _i64, _i64, ctypes.c_float, ctypes.c_int32, _vp,
                                                ctypes.c_size_t, _vp, _vp, _vp]
             lib.pararnn_solve_lstm.restype = ctypes.c_int
+            lib.pararnn_solve_gru_backward.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+                                                       _vp, _vp, _i64, _i64, _i64, _vp,
+                                                       ctypes.c_size_t, _vp, _vp, _vp]
+            lib.pararnn_solve_gru_backward.restype = ctypes.c_int
+            lib.pararnn_solve_lstm_backward.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+                                                        _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                                        _i64, _vp, ctypes.c_size_t, _vp, _vp, _vp]
+            lib.pararnn_solve_lstm_backward.restype = ctypes.c_int
             lib.pararnn_solve_gru_noalloc.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64,
                                                       _i64, _i64, ctypes.c_float, ctypes.c_int32,
                                                       _vp, _vp, _vp]
@@ -339,3 +350,72 @@ def solve_gru_noalloc(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None
                                        _stream_handle(stream))
     _raise(st, "pararnn_solve_gru_noalloc")
     return h, SolveInfo(info)
+
+
+def solve_gru_backward(P, a, h, dh, h0=None, out=None, status=None,
+                       opts: Options | None = None, stream=None):
+    """Gradients of a loss through the ParaGRU solution h, given dh = dl/dh.
+
+    Returns (dP [B, L, 3, D] fp32, da [3, D], dh0 [B, D])."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 3:
+        raise ValueError("P must be [B, L, 3, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 3, D))
+    _check_dev("a", a, torch.float32, (3, D))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    _check_dev("h", h, torch.float32, (B, L, D))
+    _check_dev("dh", dh, torch.float32, (B, L, D))
+    if out is None:
+        dP = torch.empty((B, L, 3, D), dtype=torch.float32, device=P.device)
+        da = torch.empty((3, D), dtype=torch.float32, device=P.device)
+        dh0 = torch.empty((B, D), dtype=torch.float32, device=P.device)
+    else:
+        dP, da, dh0 = out
+    _check_dev("dP", dP, torch.float32, (B, L, 3, D))
+    _check_dev("da", da, torch.float32, (3, D))
+    _check_dev("dh0", dh0, torch.float32, (B, D))
+    n = workspace_size(OP_GRU_BACKWARD, B, L, D, 0, opts)
+    ws = _workspace(n, P.device)
+    st = lib.pararnn_solve_gru_backward(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), _ptr(dh),
+                                        _ptr(dP), _ptr(da), _ptr(dh0), B, L, D, _ptr(ws),
+                                        ws.numel(), _ptr(status),
+                                        ctypes.byref(opts) if opts is not None else None,
+                                        _stream_handle(stream))
+    _raise(st, "pararnn_solve_gru_backward")
+    return dP, da, dh0
+
+
+def solve_lstm_backward(P, a, c, h, dc, dh, c0=None, h0=None, out=None, status=None,
+                        opts: Options | None = None, stream=None):
+    """Gradients through the ParaLSTM solution (c, h), given dc = dl/dc and dh = dl/dh
+    (either may be None).  Returns (dP [B, L, 4, D], da [4, D], dc0 [B, D], dh0 [B, D])."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 4:
+        raise ValueError("P must be [B, L, 4, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 4, D))
+    _check_dev("a", a, torch.float32, (4, D))
+    for nm, t in (("c0", c0), ("h0", h0)):
+        _check_dev(nm, t, torch.float32, (B, D))
+    for nm, t in (("c", c), ("h", h), ("dc", dc), ("dh", dh)):
+        _check_dev(nm, t, torch.float32, (B, L, D))
+    if out is None:
+        dP = torch.empty((B, L, 4, D), dtype=torch.float32, device=P.device)
+        da = torch.empty((4, D), dtype=torch.float32, device=P.device)
+        dc0 = torch.empty((B, D), dtype=torch.float32, device=P.device)
+        dh0 = torch.empty((B, D), dtype=torch.float32, device=P.device)
+    else:
+        dP, da, dc0, dh0 = out
+    n = workspace_size(OP_LSTM_BACKWARD, B, L, D, 0, opts)
+    ws = _workspace(n, P.device)
+    st = lib.pararnn_solve_lstm_backward(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c),
+                                         _ptr(h), _ptr(dc), _ptr(dh), _ptr(dP), _ptr(da),
+                                         _ptr(dc0), _ptr(dh0), B, L, D, _ptr(ws), ws.numel(),
+                                         _ptr(status),
+                                         ctypes.byref(opts) if opts is not None else None,
+                                         _stream_handle(stream))
+    _raise(st, "pararnn_solve_lstm_backward")
+    return dP, da, dc0, dh0

@@ -14,6 +14,7 @@
 #include <cudaTypedefs.h>
 
 #include "pararnn.h"
+#include "pararnn_bwd.cuh"
 #include "pararnn_kernel.cuh"
 #include "pararnn_walk.cuh"
 
@@ -80,11 +81,16 @@ constexpr int kWalkMinTiles = 200;
 // Below this many tiles the walker uses 16-warp CTAs.
 constexpr int kWalkWideTiles = 512;
 
+constexpr int kStepsGruBwd = 8;
+constexpr int kStepsLstmBwd = 4;
+
 int steps_for(int op) {
   switch (op) {
     case kScanDiag: return kStepsScanDiag;
     case kScanBlock2: return kStepsScanBlock2;
     case kGru: return kStepsGru;
+    case kGruBwd: return kStepsGruBwd;
+    case kLstmBwd: return kStepsLstmBwd;
     default: return kStepsLstm;
   }
 }
@@ -96,7 +102,8 @@ int walk_steps_for(int op) {
     default: return kWalkStepsLstm;
   }
 }
-int ns_for(int op) { return (op == kScanBlock2 || op == kLstm) ? 2 : 1; }
+int ns_for(int op) { return (op == kScanBlock2 || op == kLstm || op == kLstmBwd) ? 2 : 1; }
+bool is_backward(int op) { return op == kGruBwd || op == kLstmBwd; }
 // 64-bit words of one look-back record (aggregate, then chunk-end state).
 int rec_words_for(int op) { return ns_for(op) == 2 ? Rec<2>::kWords : Rec<1>::kWords; }
 bool is_newton(int op) { return op == kGru || op == kLstm; }
@@ -162,7 +169,7 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
     pl.walk = pl.nchunks > 1 && ntiles >= kWalkMinTiles;
     if (pl.nchunks == 1) pl.walk = true;
   }
-  if (pl.walk && pl.CW == 32) {
+  if (pl.walk && pl.CW == 32 && !is_backward(op)) {
     // the TMA walker cuts time into chunks of its own length
     pl.S_walk = walk_steps_for(op);
     const int want = opts ? opts->walk_warps : 0;
@@ -245,6 +252,26 @@ const void* select_kernel(int op, bool bf16, bool walk, int cw) {
       return bf16 ? kernel_for<kLstm, __nv_bfloat16, kStepsLstm, kMinBlocksSolve>(walk, cw)
                   : kernel_for<kLstm, float, kStepsLstm, kMinBlocksSolve>(walk, cw);
   }
+}
+
+template <int OP, typename PT, int S, bool WALK>
+const void* bwd_kernel_for_cw(int cw) {
+  switch (cw) {
+    case 1: return (const void*)pararnn_bwd_kernel<OP, PT, 1, S, 2, WALK>;
+    case 2: return (const void*)pararnn_bwd_kernel<OP, PT, 2, S, 2, WALK>;
+    case 4: return (const void*)pararnn_bwd_kernel<OP, PT, 4, S, 2, WALK>;
+    case 8: return (const void*)pararnn_bwd_kernel<OP, PT, 8, S, 2, WALK>;
+    case 16: return (const void*)pararnn_bwd_kernel<OP, PT, 16, S, 2, WALK>;
+    default: return (const void*)pararnn_bwd_kernel<OP, PT, 32, S, 2, WALK>;
+  }
+}
+
+template <int OP, int S>
+const void* bwd_kernel_for(bool bf16, bool walk, int cw) {
+  if (bf16)
+    return walk ? bwd_kernel_for_cw<OP, __nv_bfloat16, S, true>(cw)
+                : bwd_kernel_for_cw<OP, __nv_bfloat16, S, false>(cw);
+  return walk ? bwd_kernel_for_cw<OP, float, S, true>(cw) : bwd_kernel_for_cw<OP, float, S, false>(cw);
 }
 
 // Resident CTAs per SM for a kernel, cached per (device, kernel).
@@ -489,6 +516,48 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
   return PARARNN_OK;
 }
 
+pararnn_status_t launch_bwd(const Plan& pl, BwdParams& bp, bool bf16, void* ws, size_t ws_bytes,
+                            const pararnn_options_t* opts, cudaStream_t stream) {
+  if (!ws || ws_bytes < pl.total || !aligned(ws, 256)) return PARARNN_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  bp.ctrl = reinterpret_cast<Ctrl*>(base);
+  bp.ticket = reinterpret_cast<unsigned*>(base + pl.off_ticket);
+  bp.rec = reinterpret_cast<unsigned long long*>(base + pl.off_rec);
+  bp.ntd = pl.ntd;
+  bp.ntiles = pl.ntiles;
+  bp.nchunks = pl.nchunks;
+  bp.nunits = pl.nunits;
+  bp.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? opts->wait_timeout_ns : 1000000000LL;
+  bp.stall_unit = opts ? opts->debug_stall_unit : -1;
+  const void* fn = pl.op == kGruBwd ? bwd_kernel_for<kGruBwd, kStepsGruBwd>(bf16, pl.walk, pl.CW)
+                                    : bwd_kernel_for<kLstmBwd, kStepsLstmBwd>(bf16, pl.walk, pl.CW);
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_UNSUPPORTED;
+  }
+  int resident = 0;
+  if (resident_ctas(fn, kThreads, 0, &resident) != cudaSuccess || resident <= 0) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  const int nwork = pl.walk ? pl.ntiles : pl.nunits;
+  const int grid = nwork < resident ? nwork : resident;
+  const int G = pl.op == kGruBwd ? 3 : 4;
+  if (cudaMemsetAsync(ws, 0, pl.zero_bytes, stream) != cudaSuccess ||
+      cudaMemsetAsync(bp.da, 0, sizeof(float) * G * (size_t)bp.D, stream) != cudaSuccess)
+    return PARARNN_ERR_CUDA;
+  if (bp.status_dev && cudaMemsetAsync(bp.status_dev, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return PARARNN_ERR_CUDA;
+  void* args[] = {&bp};
+  // Waits are only on smaller tickets, which running CTAs hold: no grid barrier.
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, 0, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  return PARARNN_OK;
+}
+
 }  // namespace
 }  // namespace pararnn
 
@@ -513,7 +582,7 @@ const char* pararnn_status_string(pararnn_status_t s) {
 
 size_t pararnn_workspace_size(pararnn_op_t op, int64_t B, int64_t L, int64_t D, int32_t max_iters,
                               const pararnn_options_t* opts) {
-  if ((int)op < 0 || (int)op > 3) return 0;
+  if ((int)op < 0 || (int)op > 5) return 0;
   if (B == 0 || L == 0 || D == 0) return 256;
   Plan pl = make_plan((int)op, B, L, D, max_iters, opts);
   return pl.ok ? pl.total : 0;
@@ -684,4 +753,79 @@ extern "C" pararnn_status_t pararnn_solve_gru_noalloc(const void* P, pararnn_dty
   if (st != PARARNN_OK) return st;
   return pararnn_solve_gru(P, p_dtype, a, h0, h, B, L, D, tol, max_iters, scratch,
                            (size_t)PARARNN_NOALLOC_SCRATCH_BYTES, info, opts, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Backward pass.
+// ---------------------------------------------------------------------------
+static pararnn_status_t backward_common(int op, const void* P, pararnn_dtype_t p_dtype,
+                                        const float* a, const float* x0a, const float* x0b,
+                                        const float* tr0, const float* tr1, const float* g0,
+                                        const float* g1, float* dP, float* da, float* d0a,
+                                        float* d0b, int64_t B, int64_t L, int64_t D, void* ws,
+                                        size_t ws_bytes, int32_t* status_dev,
+                                        const pararnn_options_t* opts, void* stream) {
+  if (B < 0 || L < 0 || D < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (p_dtype != PARARNN_F32 && p_dtype != PARARNN_BF16) return PARARNN_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = op == kGruBwd ? 3 : 4;
+  if (B == 0 || L == 0 || D == 0) {
+    // no steps: every gradient is zero
+    if (da && D > 0 && cudaMemsetAsync(da, 0, sizeof(float) * G * (size_t)D, st) != cudaSuccess)
+      return PARARNN_ERR_CUDA;
+    if (B > 0 && D > 0) {
+      if (d0a && cudaMemsetAsync(d0a, 0, sizeof(float) * (size_t)(B * D), st) != cudaSuccess)
+        return PARARNN_ERR_CUDA;
+      if (d0b && cudaMemsetAsync(d0b, 0, sizeof(float) * (size_t)(B * D), st) != cudaSuccess)
+        return PARARNN_ERR_CUDA;
+    }
+    if (status_dev && cudaMemsetAsync(status_dev, 0, sizeof(int32_t), st) != cudaSuccess)
+      return PARARNN_ERR_CUDA;
+    return PARARNN_OK;
+  }
+  if (!P || !a || !tr0 || !dP || !da) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (op == kGruBwd && !g0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (op == kLstmBwd && (!tr1 || (!g0 && !g1))) return PARARNN_ERR_INVALID_ARGUMENT;
+  const size_t esz = p_dtype == PARARNN_BF16 ? 2 : 4;
+  const void* ptrs4[] = {a, x0a, x0b, tr0, tr1, g0, g1, dP, da, d0a, d0b};
+  for (const void* q : ptrs4)
+    if (q && !aligned(q, 4)) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!aligned(P, esz)) return PARARNN_ERR_INVALID_ARGUMENT;
+  Plan pl = make_plan(op, B, L, D, 0, opts);
+  if (!pl.ok) return PARARNN_ERR_INVALID_ARGUMENT;
+  BwdParams bp = {};
+  bp.P = P;
+  bp.w = a;
+  bp.x0a = x0a;
+  bp.x0b = x0b;
+  bp.tr0 = tr0;
+  bp.tr1 = tr1;
+  bp.g0 = g0;
+  bp.g1 = g1;
+  bp.dP = dP;
+  bp.da = da;
+  bp.d0a = d0a;
+  bp.d0b = d0b;
+  bp.B = B;
+  bp.L = L;
+  bp.D = D;
+  bp.status_dev = status_dev;
+  return launch_bwd(pl, bp, p_dtype == PARARNN_BF16, ws, ws_bytes, opts, st);
+}
+
+extern "C" pararnn_status_t pararnn_solve_gru_backward(
+    const void* P, pararnn_dtype_t p_dtype, const float* a, const float* h0, const float* h,
+    const float* dh, float* dP, float* da, float* dh0, int64_t B, int64_t L, int64_t D, void* ws,
+    size_t ws_bytes, int32_t* status_dev, const pararnn_options_t* opts, void* stream) {
+  return backward_common(kGruBwd, P, p_dtype, a, h0, nullptr, h, nullptr, dh, nullptr, dP, da,
+                         dh0, nullptr, B, L, D, ws, ws_bytes, status_dev, opts, stream);
+}
+
+extern "C" pararnn_status_t pararnn_solve_lstm_backward(
+    const void* P, pararnn_dtype_t p_dtype, const float* a, const float* c0, const float* h0,
+    const float* c, const float* h, const float* dc, const float* dh, float* dP, float* da,
+    float* dc0, float* dh0, int64_t B, int64_t L, int64_t D, void* ws, size_t ws_bytes,
+    int32_t* status_dev, const pararnn_options_t* opts, void* stream) {
+  return backward_common(kLstmBwd, P, p_dtype, a, c0, h0, c, h, dc, dh, dP, da, dc0, dh0, B, L, D,
+                         ws, ws_bytes, status_dev, opts, stream);
 }

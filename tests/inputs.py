@@ -16,6 +16,8 @@ name     operation                              shape (B, L, D)
 gru_s    ParaGRU solve, fp32                    2, 512, 16
 scan     diagonal affine scan, fp32             8, 4096, 1024
 gru_l    ParaGRU solve, fp32, L sweep 2^6..2^14 8, L, 1024
+gru_bwd  ParaGRU backward pass, fp32           8, 4096, 1024
+lstm_bwd ParaLSTM backward pass, fp32          8, 4096, 1024
 lstm     ParaLSTM solve, fp32 (+ block scan)    8, 4096, 1024
 deer     ParaGRU solve, fp32, DEER shape        16, 2^20, 1
 lm       ParaGRU solve, bf16 P, fp32 state      8, 8192, 4096
@@ -25,6 +27,8 @@ Distributions: projected gate inputs P ~ N(0, 1); diagonal recurrence weights
 a ~ U(-0.5, 0.5); h0 = c0 = 0 for the solves.  Diagonal scan: A ~ U(0, 1),
 b ~ N(0, 1), h0 ~ N(0, 1).  Block scan: A entries ~ U(-0.5, 0.5), b ~ N(0, 1),
 x0 ~ N(0, 1).  Draw order: P (or A) first, then a (or b), then h0 (or x0).
+Backward passes: the forward workload's inputs, and upstream gradients
+dl/dh (and dl/dc) ~ N(0, 1) from their own generator.
 """
 from __future__ import annotations
 
@@ -38,6 +42,8 @@ WORKLOADS = {
     "block2": dict(op="scan_block2", B=8, L=4096, D=1024, seed=3, bf16=False),
     "deer": dict(op="gru", B=16, L=1 << 20, D=1, seed=4, bf16=False),
     "lm": dict(op="gru", B=8, L=8192, D=4096, seed=5, bf16=True),
+    "gru_bwd": dict(op="gru_bwd", B=8, L=4096, D=1024, seed=2, bf16=False),
+    "lstm_bwd": dict(op="lstm_bwd", B=8, L=4096, D=1024, seed=3, bf16=False),
 }
 
 L_SWEEP = [1 << e for e in range(6, 15)]
@@ -133,3 +139,9 @@ def workload_inputs(name, L=None):
     if op == "scan_block2":
         return scan_block2_inputs(w["B"], w["L"], w["D"], seed)
     raise KeyError(op)
+
+
+def upstream_gradients(B, L, D, seed, n=1):
+    """n arrays [B, L, D] of fp32 N(0, 1) draws: the upstream gradients dl/dh (, dl/dc)."""
+    rng = _rng([seed, 97])
+    return [_normal(rng, (B, L, D)) for _ in range(n)]

@@ -130,3 +130,26 @@ def test_lstm_fullsize(pr):
         rc, rh = oracle.rollout_lstm(P, x["a"][:, d:d + 1])
         assert np.max(np.abs(c[b, :, d].cpu().numpy() - rc[0, :, 0])) <= 1e-4
         assert np.max(np.abs(h[b, :, d].cpu().numpy() - rh[0, :, 0])) <= 1e-4
+
+
+def test_gru_backward_fullsize(pr):
+    """Backward pass at the B=8, L=4096, D=1024 shape: the GPU differentiates its own
+    forward solution; sampled channels are compared with the oracle's adjoint on the
+    same (fp32) trajectory and gradients."""
+    w = inputs.WORKLOADS["gru_bwd"]
+    B, L, D = w["B"], w["L"], w["D"]
+    x = inputs.gru_inputs(B, L, D, w["seed"])
+    (gh,) = inputs.upstream_gradients(B, L, D, w["seed"], 1)
+    P, a = dev(x["P"]), dev(x["a"])
+    h, info = pr.solve_gru(P, a)
+    dP, da, dh0 = pr.solve_gru_backward(P, a, h, dev(gh))
+    torch.cuda.synchronize()
+    assert info.converged and bool(torch.isfinite(dP).all())
+    hh = h.cpu().numpy()
+    for b, d in sample_channels(B, D, 32, 7):
+        Pc = x["P"][b, :, :, d][None, :, :, None]
+        rP, ra, rh0 = oracle.backward_gru(Pc, x["a"][:, d:d + 1], hh[b, :, d][None, :, None],
+                                          gh[b, :, d][None, :, None])
+        got = dP[b, :, :, d].cpu().numpy()
+        assert np.max(np.abs(got - rP[0, :, :, 0]) / np.maximum(1, np.abs(rP[0, :, :, 0]))) <= 1e-4
+        assert abs(float(dh0[b, d]) - rh0[0, 0]) <= 1e-4 * max(1.0, abs(rh0[0, 0]))
