@@ -453,6 +453,62 @@ def run_ours(args, world, rank, local):
                 "frac_of_8tbs": sgbs / 8000.0, "traffic": st, "traffic_source": ssrc}
         del sc
 
+    # ---- context: sequential application on the same GPU ---------------------
+    # (ParaRNN's abstract measures its speedup against naive sequential
+    # application: one launch per time step.  Also timed: the one-thread-per-
+    # channel rollout, whose time is L x the cell's dependency chain.)
+    sequential = None
+    if op in ("gru", "lstm") and not args.no_sequential:
+        try:
+            seq_fn = pr.rollout_gru if op == "gru" else pr.rollout_lstm
+            d = cs.dev
+            seq_args = (d["P"], d["a"], d["h0"]) if op == "gru" else (d["P"], d["a"], d["c0"],
+                                                                      d["h0"])
+            for _ in range(2):
+                seq_fn(*seq_args)
+            torch.cuda.synchronize()
+            qev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            Kq = max(1, min(K, 5))
+            qev[0].record(stream)
+            for _ in range(Kq):
+                seq_fn(*seq_args)
+            qev[1].record(stream)
+            torch.cuda.synchronize()
+            roll_ms = qev[0].elapsed_time(qev[1]) / Kq
+            # naive loop: one decode-step launch per time step, over a bounded
+            # number of steps, scaled to L
+            nsteps = min(L, 2048)
+            G = 3 if op == "gru" else 4
+            Pt = d["P"][:, :nsteps].transpose(0, 1).contiguous()      # [n, B, G, D]
+            hs = torch.empty((nsteps, B, D), dtype=torch.float32, device=device)
+            cs_ = torch.empty_like(hs) if op == "lstm" else None
+
+            def naive():
+                prev_h = d["h0"]
+                prev_c = d["c0"] if op == "lstm" else None
+                for t in range(nsteps):
+                    if op == "gru":
+                        pr.step_gru(Pt[t], d["a"], prev_h, out=hs[t])
+                    else:
+                        pr.step_lstm(Pt[t], d["a"], prev_c, prev_h, out=(cs_[t], hs[t]))
+                        prev_c = cs_[t]
+                    prev_h = hs[t]
+            naive()
+            torch.cuda.synchronize()
+            qev[0].record(stream)
+            naive()
+            qev[1].record(stream)
+            torch.cuda.synchronize()
+            naive_ms = qev[0].elapsed_time(qev[1]) * L / nsteps
+            sequential = {"rollout_one_thread_per_channel_ms": roll_ms,
+                          "naive_step_loop_ms": naive_ms,
+                          "naive_step_loop_sample": f"{nsteps} of {L} steps, scaled",
+                          "newton_speedup_vs_rollout": roll_ms / ms,
+                          "newton_speedup_vs_naive_loop": naive_ms / ms}
+            del Pt, hs, cs_
+        except Exception as e:  # context only; never fails the benchmark
+            sequential = {"error": str(e)[:200]}
+
     # ---- end to end through the public API with pinned host buffers ---------
     e2e = None
     if not args.no_e2e:
@@ -511,6 +567,7 @@ def run_ours(args, world, rank, local):
             "data": "synthetic (seeded numpy; see tests/inputs.py)",
             "config": cfg, "roofline": roofline, "clocks": clocks, "e2e": e2e,
             "gpu_launches": K, "scan": scan, "cpu_baseline": cpu,
+            "sequential_gpu": sequential,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -677,6 +734,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-scan", action="store_true", help="skip the scan leg (gru_l)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
+    ap.add_argument("--no-sequential", action="store_true",
+                    help="skip the sequential-application context timings")
     ap.add_argument("--warmup-seconds", type=float, default=0.5,
                     help="keep warming up until this much time has passed (after W steps)")
     args = ap.parse_args()

@@ -213,6 +213,32 @@ pararnn_status_t pararnn_solve_lstm_backward(const void* P, pararnn_dtype_t p_dt
                                              void* ws, size_t ws_bytes, int32_t* status_dev,
                                              const pararnn_options_t* opts, void* stream);
 
+/* One cell step for every channel: h_next = f(h_prev, P) -- a decode step when
+ * generating token by token (ParaRNN Figure 3 caption: generation
+ * throughput).  P : [B, 3, D] (z, r, c) for one time step, fp32 or bf16;
+ * a : [3, D]; h_prev : [B, D] or NULL (= 0); h_next : [B, D].  No workspace;
+ * h_next may not alias h_prev's storage of another step being read. */
+pararnn_status_t pararnn_step_gru(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                  const float* h_prev, float* h_next, int64_t B, int64_t D,
+                                  void* stream);
+/* ParaLSTM decode step: P : [B, 4, D]; (c_prev, h_prev) -> (c_next, h_next). */
+pararnn_status_t pararnn_step_lstm(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                   const float* c_prev, const float* h_prev, float* c_next,
+                                   float* h_next, int64_t B, int64_t D, void* stream);
+
+/* Sequential application of the cell over the whole sequence on the GPU, one
+ * thread per channel walking t = 1..L in order (the "sequential application"
+ * that ParaRNN's abstract and the DEER summary compare the parallel solve
+ * against).  Same arguments and layout as pararnn_solve_gru / _lstm without
+ * tol, max_iters, workspace or info.  Its time is L times the cell's
+ * dependency chain, independent of B * D up to the GPU's thread count. */
+pararnn_status_t pararnn_rollout_gru(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                     const float* h0, float* h, int64_t B, int64_t L, int64_t D,
+                                     void* stream);
+pararnn_status_t pararnn_rollout_lstm(const void* P, pararnn_dtype_t p_dtype, const float* a,
+                                      const float* c0, const float* h0, float* c, float* h,
+                                      int64_t B, int64_t L, int64_t D, void* stream);
+
 /* Allocation-free variant of pararnn_solve_gru (the pages have no counterpart:
  * this is an interface convenience of this library).
  * For callers that cannot allocate device memory where they solve -- their

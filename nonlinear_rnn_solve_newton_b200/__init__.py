@@ -25,7 +25,8 @@ import torch
 from . import build as _build
 
 __all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc",
-           "solve_gru_backward", "solve_lstm_backward",
+           "solve_gru_backward", "solve_lstm_backward", "step_gru", "step_lstm",
+           "rollout_gru", "rollout_lstm",
            "workspace_size",
            "SolveInfo", "Options", "PararnnError", "library_path", "load", "MAX_ITERS"]
 
@@ -111,6 +112,17 @@ def load(build_if_missing: bool = True):
                                                         _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
                                                         _i64, _vp, ctypes.c_size_t, _vp, _vp, _vp]
             lib.pararnn_solve_lstm_backward.restype = ctypes.c_int
+            lib.pararnn_step_gru.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _vp]
+            lib.pararnn_step_gru.restype = ctypes.c_int
+            lib.pararnn_step_lstm.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i64,
+                                              _i64, _vp]
+            lib.pararnn_step_lstm.restype = ctypes.c_int
+            lib.pararnn_rollout_gru.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64,
+                                                _vp]
+            lib.pararnn_rollout_gru.restype = ctypes.c_int
+            lib.pararnn_rollout_lstm.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i64,
+                                                 _i64, _i64, _vp]
+            lib.pararnn_rollout_lstm.restype = ctypes.c_int
             lib.pararnn_solve_gru_noalloc.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64,
                                                       _i64, _i64, ctypes.c_float, ctypes.c_int32,
                                                       _vp, _vp, _vp]
@@ -419,3 +431,79 @@ def solve_lstm_backward(P, a, c, h, dc, dh, c0=None, h0=None, out=None, status=N
                                          _stream_handle(stream))
     _raise(st, "pararnn_solve_lstm_backward")
     return dP, da, dc0, dh0
+
+
+def step_gru(P, a, h_prev=None, out=None, stream=None):
+    """One ParaGRU step for every channel (decode): P [B, 3, D] -> h_next [B, D]."""
+    lib = load()
+    B, G, D = P.shape
+    if G != 3:
+        raise ValueError("P must be [B, 3, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, 3, D))
+    _check_dev("a", a, torch.float32, (3, D))
+    _check_dev("h_prev", h_prev, torch.float32, (B, D))
+    h = torch.empty((B, D), dtype=torch.float32, device=P.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, D))
+    _raise(lib.pararnn_step_gru(_ptr(P), dt, _ptr(a), _ptr(h_prev), _ptr(h), B, D,
+                                _stream_handle(stream)), "pararnn_step_gru")
+    return h
+
+
+def step_lstm(P, a, c_prev=None, h_prev=None, out=None, stream=None):
+    """One ParaLSTM step for every channel: P [B, 4, D] -> (c_next, h_next)."""
+    lib = load()
+    B, G, D = P.shape
+    if G != 4:
+        raise ValueError("P must be [B, 4, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, 4, D))
+    _check_dev("a", a, torch.float32, (4, D))
+    _check_dev("c_prev", c_prev, torch.float32, (B, D))
+    _check_dev("h_prev", h_prev, torch.float32, (B, D))
+    if out is None:
+        c = torch.empty((B, D), dtype=torch.float32, device=P.device)
+        h = torch.empty((B, D), dtype=torch.float32, device=P.device)
+    else:
+        c, h = out
+    _raise(lib.pararnn_step_lstm(_ptr(P), dt, _ptr(a), _ptr(c_prev), _ptr(h_prev), _ptr(c),
+                                 _ptr(h), B, D, _stream_handle(stream)), "pararnn_step_lstm")
+    return c, h
+
+
+def rollout_gru(P, a, h0=None, out=None, stream=None):
+    """Sequential ParaGRU application on the GPU (one thread per channel)."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 3:
+        raise ValueError("P must be [B, L, 3, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 3, D))
+    _check_dev("a", a, torch.float32, (3, D))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    h = torch.empty((B, L, D), dtype=torch.float32, device=P.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, L, D))
+    _raise(lib.pararnn_rollout_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D,
+                                   _stream_handle(stream)), "pararnn_rollout_gru")
+    return h
+
+
+def rollout_lstm(P, a, c0=None, h0=None, out=None, stream=None):
+    """Sequential ParaLSTM application on the GPU (one thread per channel)."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 4:
+        raise ValueError("P must be [B, L, 4, D]")
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 4, D))
+    _check_dev("a", a, torch.float32, (4, D))
+    _check_dev("c0", c0, torch.float32, (B, D))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    if out is None:
+        c = torch.empty((B, L, D), dtype=torch.float32, device=P.device)
+        h = torch.empty((B, L, D), dtype=torch.float32, device=P.device)
+    else:
+        c, h = out
+    _raise(lib.pararnn_rollout_lstm(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h),
+                                    B, L, D, _stream_handle(stream)), "pararnn_rollout_lstm")
+    return c, h

@@ -16,6 +16,7 @@
 #include "pararnn.h"
 #include "pararnn_bwd.cuh"
 #include "pararnn_kernel.cuh"
+#include "pararnn_seq.cuh"
 #include "pararnn_walk.cuh"
 
 namespace pararnn {
@@ -828,4 +829,86 @@ extern "C" pararnn_status_t pararnn_solve_lstm_backward(
     int32_t* status_dev, const pararnn_options_t* opts, void* stream) {
   return backward_common(kLstmBwd, P, p_dtype, a, c0, h0, c, h, dc, dh, dP, da, dc0, dh0, B, L, D,
                          ws, ws_bytes, status_dev, opts, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Sequential application on the GPU: one step (decode) and the full rollout.
+// ---------------------------------------------------------------------------
+static pararnn_status_t seq_common(bool rollout, int op, const void* P, pararnn_dtype_t p_dtype,
+                                   const float* a, const float* x0a, const float* x0b,
+                                   float* out0, float* out1, int64_t B, int64_t L, int64_t D,
+                                   void* stream) {
+  if (B < 0 || L < 0 || D < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (p_dtype != PARARNN_F32 && p_dtype != PARARNN_BF16) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (B == 0 || L == 0 || D == 0) return PARARNN_OK;
+  if (!P || !a || !out0 || (op == kLstm && !out1)) return PARARNN_ERR_INVALID_ARGUMENT;
+  const size_t esz = p_dtype == PARARNN_BF16 ? 2 : 4;
+  const void* ptrs[] = {a, x0a, x0b, out0, out1};
+  for (const void* q : ptrs)
+    if (q && !aligned(q, 4)) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!aligned(P, esz)) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (B * D > (1LL << 40)) return PARARNN_ERR_INVALID_ARGUMENT;
+  SeqParams sp = {P, a, x0a, x0b, out0, out1, B, L, D};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = p_dtype == PARARNN_BF16;
+  const long long n = B * D;
+  if (rollout) {
+    const int threads = 128;
+    const unsigned blocks = (unsigned)((n + threads - 1) / threads);
+    if (op == kGru) {
+      if (bf16)
+        pararnn_rollout_kernel<kGru, __nv_bfloat16, 16><<<blocks, threads, 0, st>>>(sp);
+      else
+        pararnn_rollout_kernel<kGru, float, 16><<<blocks, threads, 0, st>>>(sp);
+    } else {
+      if (bf16)
+        pararnn_rollout_kernel<kLstm, __nv_bfloat16, 8><<<blocks, threads, 0, st>>>(sp);
+      else
+        pararnn_rollout_kernel<kLstm, float, 8><<<blocks, threads, 0, st>>>(sp);
+    }
+  } else {
+    const int threads = 256;
+    long long blocks = (n + threads - 1) / threads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (op == kGru) {
+      if (bf16)
+        pararnn_step_kernel<kGru, __nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(sp);
+      else
+        pararnn_step_kernel<kGru, float><<<(unsigned)blocks, threads, 0, st>>>(sp);
+    } else {
+      if (bf16)
+        pararnn_step_kernel<kLstm, __nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(sp);
+      else
+        pararnn_step_kernel<kLstm, float><<<(unsigned)blocks, threads, 0, st>>>(sp);
+    }
+  }
+  if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
+  return PARARNN_OK;
+}
+
+extern "C" pararnn_status_t pararnn_step_gru(const void* P, pararnn_dtype_t p_dtype,
+                                             const float* a, const float* h_prev, float* h_next,
+                                             int64_t B, int64_t D, void* stream) {
+  return seq_common(false, kGru, P, p_dtype, a, h_prev, nullptr, h_next, nullptr, B, 1, D,
+                    stream);
+}
+
+extern "C" pararnn_status_t pararnn_step_lstm(const void* P, pararnn_dtype_t p_dtype,
+                                              const float* a, const float* c_prev,
+                                              const float* h_prev, float* c_next, float* h_next,
+                                              int64_t B, int64_t D, void* stream) {
+  return seq_common(false, kLstm, P, p_dtype, a, c_prev, h_prev, c_next, h_next, B, 1, D, stream);
+}
+
+extern "C" pararnn_status_t pararnn_rollout_gru(const void* P, pararnn_dtype_t p_dtype,
+                                                const float* a, const float* h0, float* h,
+                                                int64_t B, int64_t L, int64_t D, void* stream) {
+  return seq_common(true, kGru, P, p_dtype, a, h0, nullptr, h, nullptr, B, L, D, stream);
+}
+
+extern "C" pararnn_status_t pararnn_rollout_lstm(const void* P, pararnn_dtype_t p_dtype,
+                                                 const float* a, const float* c0, const float* h0,
+                                                 float* c, float* h, int64_t B, int64_t L,
+                                                 int64_t D, void* stream) {
+  return seq_common(true, kLstm, P, p_dtype, a, c0, h0, c, h, B, L, D, stream);
 }
