@@ -1,6 +1,7 @@
 """Build libpararnn.so in-tree with nvcc for sm_100a (B200)."""
 from __future__ import annotations
 
+import glob
 import os
 import shutil
 import subprocess
@@ -12,7 +13,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpararnn.so")
 SOURCES = [os.path.join(CSRC, "pararnn.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "pararnn_kernel.cuh"), os.path.join(INCLUDE, "pararnn.h")]
+DEPS = SOURCES + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "pararnn.h")]
 
 
 def nvcc_path() -> str:

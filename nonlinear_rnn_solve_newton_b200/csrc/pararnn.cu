@@ -15,6 +15,7 @@
 
 #include "pararnn.h"
 #include "pararnn_bwd.cuh"
+#include "pararnn_bwd_walk.cuh"
 #include "pararnn_kernel.cuh"
 #include "pararnn_seq.cuh"
 #include "pararnn_walk.cuh"
@@ -84,6 +85,29 @@ constexpr int kWalkWideTiles = 512;
 
 constexpr int kStepsGruBwd = 8;
 constexpr int kStepsLstmBwd = 4;
+// Backward TMA walker, per cell: warps per CTA, steps per warp (a chunk is
+// their product) and CTAs per SM for the register budget.  Measured on B200 at
+// B=8, L=4096, D=1024: the GRU pass runs best with 32-step chunks (4 or 8
+// warps alike), the LSTM pass (1.5x the bytes per step) with 72-step chunks of
+// 12 warps and the full register file.
+#ifndef PARARNN_BWD_WALK_WARPS_GRU
+#define PARARNN_BWD_WALK_WARPS_GRU 8
+#endif
+#ifndef PARARNN_BWD_WALK_STEPS_GRU
+#define PARARNN_BWD_WALK_STEPS_GRU 4
+#endif
+#ifndef PARARNN_BWD_WALK_MINB_GRU
+#define PARARNN_BWD_WALK_MINB_GRU 2
+#endif
+#ifndef PARARNN_BWD_WALK_WARPS_LSTM
+#define PARARNN_BWD_WALK_WARPS_LSTM 12
+#endif
+#ifndef PARARNN_BWD_WALK_STEPS_LSTM
+#define PARARNN_BWD_WALK_STEPS_LSTM 6
+#endif
+#ifndef PARARNN_BWD_WALK_MINB_LSTM
+#define PARARNN_BWD_WALK_MINB_LSTM 1
+#endif
 
 int steps_for(int op) {
   switch (op) {
@@ -275,6 +299,28 @@ const void* bwd_kernel_for(bool bf16, bool walk, int cw) {
   return walk ? bwd_kernel_for_cw<OP, float, S, true>(cw) : bwd_kernel_for_cw<OP, float, S, false>(cw);
 }
 
+// Backward TMA walker for an op and P dtype, with its dynamic shared memory,
+// chunk length and threads per CTA.
+template <int OP, typename PT, int S, int NW, int MINB>
+const void* bwd_walk_kernel(size_t* smem, int* tch, int* threads) {
+  *smem = 2 * (size_t)BwdStage<OP, PT, NW * S>::kPadded + 1024;  // + alignment slack
+  *tch = NW * S;
+  *threads = 32 * NW;
+  return (const void*)pararnn_bwd_walk_kernel<OP, PT, S, NW, MINB>;
+}
+
+const void* select_bwd_walk_kernel(int op, bool bf16, size_t* smem, int* tch, int* threads) {
+  constexpr int WG = PARARNN_BWD_WALK_WARPS_GRU, SG = PARARNN_BWD_WALK_STEPS_GRU,
+                MG = PARARNN_BWD_WALK_MINB_GRU;
+  constexpr int WL = PARARNN_BWD_WALK_WARPS_LSTM, SL = PARARNN_BWD_WALK_STEPS_LSTM,
+                ML = PARARNN_BWD_WALK_MINB_LSTM;
+  if (op == kGruBwd)
+    return bf16 ? bwd_walk_kernel<kGruBwd, __nv_bfloat16, SG, WG, MG>(smem, tch, threads)
+                : bwd_walk_kernel<kGruBwd, float, SG, WG, MG>(smem, tch, threads);
+  return bf16 ? bwd_walk_kernel<kLstmBwd, __nv_bfloat16, SL, WL, ML>(smem, tch, threads)
+              : bwd_walk_kernel<kLstmBwd, float, SL, WL, ML>(smem, tch, threads);
+}
+
 // Resident CTAs per SM for a kernel, cached per (device, kernel).
 struct OccEntry {
   int dev;
@@ -423,6 +469,31 @@ bool make_walk_maps(int op, bool bf16, const KParams& kp, int T, TmaMaps* tm) {
   }
 }
 
+// Tensor maps for the backward walker, or false if TMA's rules do not hold for
+// every array it stages (16-byte aligned bases, row pitches a multiple of 16 B).
+bool make_bwd_maps(int op, bool bf16, const BwdParams& bp, int T, BwdMaps* tm) {
+  const long long B = bp.B, L = bp.L, D = bp.D;
+  // (row coordinates and the per-chunk dP offsets are 32-bit in the kernel)
+  if (D < 32 || D > (1LL << 24) || B * L >= (1LL << 31) || (D * 4) % 16 != 0) return false;
+  const size_t es = bf16 ? 2 : 4;
+  if ((D * (long long)es) % 16 != 0) return false;
+  const int G = op == kGruBwd ? 3 : 4;
+  const unsigned long long rows = (unsigned long long)(B * L);
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const void* planes[4] = {bp.tr0, bp.tr1, bp.g0, bp.g1};
+  CUtensorMap* maps[4] = {&tm->x0, &tm->x1, &tm->g0, &tm->g1};
+  if (!aligned(bp.P, 16)) return false;
+  if (!encode_map(&tm->P, bp.P, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : f32, es, D, G, rows,
+                  32, T))
+    return false;
+  for (int i = 0; i < 4; ++i) {
+    if (!planes[i]) continue;
+    if (!aligned(planes[i], 16) || !encode_map(maps[i], planes[i], f32, 4, D, 1, rows, 32, T))
+      return false;
+  }
+  return true;
+}
+
 // Empty problem: no equations, so the solve has converged at k = 0.
 __global__ void empty_info_kernel(pararnn_solve_info_t* info) {
   info->iterations = 0;
@@ -530,15 +601,38 @@ pararnn_status_t launch_bwd(const Plan& pl, BwdParams& bp, bool bf16, void* ws, 
   bp.nunits = pl.nunits;
   bp.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? opts->wait_timeout_ns : 1000000000LL;
   bp.stall_unit = opts ? opts->debug_stall_unit : -1;
-  const void* fn = pl.op == kGruBwd ? bwd_kernel_for<kGruBwd, kStepsGruBwd>(bf16, pl.walk, pl.CW)
-                                    : bwd_kernel_for<kLstmBwd, kStepsLstmBwd>(bf16, pl.walk, pl.CW);
+  // The TMA walker when the tiles are 32 wide and TMA's rules hold; otherwise
+  // the general kernel (look-back or register-staged walk).
+  BwdMaps tm;
+  const void* fn = nullptr;
+  size_t dyn_smem = 0;
+  int tch = 0, walk_threads = 0;
+  bool tma_walk = false;
+  if (pl.walk && pl.CW == 32) {
+    fn = select_bwd_walk_kernel(pl.op, bf16, &dyn_smem, &tch, &walk_threads);
+    tma_walk = make_bwd_maps(pl.op, bf16, bp, tch, &tm);
+  }
+  if (tma_walk) {
+    bp.nchunks = (int)((bp.L + tch - 1) / tch);
+  } else {
+    dyn_smem = 0;
+    fn = pl.op == kGruBwd ? bwd_kernel_for<kGruBwd, kStepsGruBwd>(bf16, pl.walk, pl.CW)
+                          : bwd_kernel_for<kLstmBwd, kStepsLstmBwd>(bf16, pl.walk, pl.CW);
+  }
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
     return PARARNN_ERR_UNSUPPORTED;
   }
+  if (dyn_smem > 0 &&
+      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
   int resident = 0;
-  if (resident_ctas(fn, kThreads, 0, &resident) != cudaSuccess || resident <= 0) {
+  const int threads = tma_walk ? walk_threads : kThreads;
+  if (resident_ctas(fn, threads, dyn_smem, &resident) != cudaSuccess || resident <= 0) {
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }
@@ -550,9 +644,11 @@ pararnn_status_t launch_bwd(const Plan& pl, BwdParams& bp, bool bf16, void* ws, 
     return PARARNN_ERR_CUDA;
   if (bp.status_dev && cudaMemsetAsync(bp.status_dev, 0, sizeof(int32_t), stream) != cudaSuccess)
     return PARARNN_ERR_CUDA;
-  void* args[] = {&bp};
+  void* args_plain[] = {&bp};
+  void* args_tma[] = {&bp, &tm};
   // Waits are only on smaller tickets, which running CTAs hold: no grid barrier.
-  if (cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, 0, stream) != cudaSuccess) {
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(threads), tma_walk ? args_tma : args_plain,
+                       dyn_smem, stream) != cudaSuccess) {
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }

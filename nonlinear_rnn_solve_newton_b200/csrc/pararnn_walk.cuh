@@ -146,6 +146,19 @@ __device__ __forceinline__ bool stage_wait(unsigned long long* bar, unsigned par
   }
 }
 
+// Before a CTA exits: wait for the copies still in flight into its shared
+// memory (thread 0; bit s of `pending` = stage s, `phase` = the parities).  The
+// copies read valid global memory and land within microseconds; the limit is at
+// least 2 s so that a short user wait limit, which may have ended a stage wait
+// early, cannot let the CTA leave before its copies do.
+__device__ __forceinline__ void drain_stages(unsigned long long* bars, unsigned pending,
+                                             unsigned phase, const WaitCtx& w) {
+  WaitCtx wl = w;
+  if (wl.timeout_ns < 2000000000LL) wl.timeout_ns = 2000000000LL;
+  for (int st = 0; st < 2; ++st)
+    if (pending & (1u << st)) stage_wait(&bars[st], (phase >> st) & 1u, wl);
+}
+
 template <int OP, typename PT, int S, int NW, int MINB>
 __global__ void __launch_bounds__(NW * 32, MINB)
     pararnn_walk_kernel(const __grid_constant__ KParams p, const __grid_constant__ TmaMaps tm) {
@@ -271,8 +284,10 @@ __global__ void __launch_bounds__(NW * 32, MINB)
 
         // ---- this chunk's inputs have landed ------------------------------
         const bool ok = stage_wait(&s_bar[st], (phase >> st) & 1u, wctx);
-        phase ^= 1u << st;
-        if (tid == 0) pending &= ~(1u << st);
+        if (ok) {  // a copy that did not land stays pending for the final drain
+          phase ^= 1u << st;
+          if (tid == 0) pending &= ~(1u << st);
+        }
         if (!__syncthreads_and(ok ? 1 : 0)) {
           if (tid == 0) raise_error(wctx, 4u);
           aborted = true;
@@ -404,10 +419,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   }
 
   // No copy may still be writing this CTA's shared memory when it exits.
-  if (tid == 0 && pending) {
-    for (int st = 0; st < 2; ++st)
-      if (pending & (1u << st)) stage_wait(&s_bar[st], (phase >> st) & 1u, wctx);
-  }
+  if (tid == 0 && pending) drain_stages(s_bar, pending, phase, wctx);
 
   if constexpr (NEWTON) {
     if (blockIdx.x == 0 && tid == 0) {

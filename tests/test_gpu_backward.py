@@ -121,3 +121,76 @@ def test_backward_stall_times_out(pr):
     pr.solve_gru_backward(dev(x["P"]), dev(x["a"]), dev(h), dev(h), status=st, opts=o)
     torch.cuda.synchronize()
     assert int(st.item()) == 4
+
+
+# Shapes the TMA tile walker takes when the walk regime is forced: D a multiple
+# of 4 (fp32 rows) / 8 (bf16 rows) and at least 32, ragged last tile (D = 40,
+# 96 + 8), L not a multiple of the chunk length (64 GRU, 32 LSTM).
+WALK_SHAPES = [(2, 1000, 40), (3, 333, 104), (1, 64, 32), (2, 65, 64)]
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+@pytest.mark.parametrize("shape", WALK_SHAPES)
+def test_gru_backward_walk(pr, shape, bf16):
+    B, L, D = shape
+    x = inputs.gru_inputs(B, L, D, seed=[650, B, L, D], bf16=bf16, h0_normal=True)
+    h = oracle.rollout_gru(x["P"], x["a"], x["h0"]).astype(np.float32)
+    gh = np.random.default_rng([651, B, L, D]).standard_normal((B, L, D)).astype(np.float32)
+    P = (torch.from_numpy(x["P_bits"].view(np.int16)).cuda().view(torch.bfloat16) if bf16
+         else dev(x["P"]))
+    dP, da, dh0 = pr.solve_gru_backward(P, dev(x["a"]), dev(h), dev(gh), dev(x["h0"]),
+                                        opts=pr.Options(regime=2))
+    torch.cuda.synchronize()
+    rP, ra, rh0 = oracle.backward_gru(x["P"], x["a"], h, gh, x["h0"])
+    hp = np.concatenate([x["h0"][:, None].astype(np.float64), h[:, :-1].astype(np.float64)], 1)
+    scale = np.abs(rP * hp[:, :, None]).sum(axis=(0, 1))
+    assert close(dP.cpu().numpy(), rP) <= 1e-4
+    assert close(dh0.cpu().numpy(), rh0) <= 1e-4
+    assert da_close(da.cpu().numpy(), ra, scale) <= 1e-4
+
+
+@pytest.mark.parametrize("which", ["both", "dc_only", "dh_only"])
+@pytest.mark.parametrize("shape", WALK_SHAPES)
+def test_lstm_backward_walk(pr, shape, which):
+    B, L, D = shape
+    x = inputs.lstm_inputs(B, L, D, seed=[660, B, L, D], h0_normal=True)
+    c, h = oracle.rollout_lstm(x["P"], x["a"], x["c0"], x["h0"])
+    c, h = c.astype(np.float32), h.astype(np.float32)
+    rng = np.random.default_rng([661, B, L, D])
+    gc = rng.standard_normal((B, L, D)).astype(np.float32)
+    gh = rng.standard_normal((B, L, D)).astype(np.float32)
+    if which == "dc_only":
+        gh[:] = 0.0
+    if which == "dh_only":
+        gc[:] = 0.0
+    dP, da, dc0, dh0 = pr.solve_lstm_backward(
+        dev(x["P"]), dev(x["a"]), dev(c), dev(h),
+        None if which == "dh_only" else dev(gc), None if which == "dc_only" else dev(gh),
+        dev(x["c0"]), dev(x["h0"]), opts=pr.Options(regime=2))
+    torch.cuda.synchronize()
+    rP, ra, rc0, rh0 = oracle.backward_lstm(x["P"], x["a"], c, h, gc, gh, x["c0"], x["h0"])
+    hp = np.concatenate([x["h0"][:, None].astype(np.float64), h[:, :-1].astype(np.float64)], 1)
+    scale = np.abs(rP * hp[:, :, None]).sum(axis=(0, 1))
+    assert close(dP.cpu().numpy(), rP) <= 1e-4
+    assert close(dc0.cpu().numpy(), rc0) <= 1e-4
+    assert close(dh0.cpu().numpy(), rh0) <= 1e-4
+    assert da_close(da.cpu().numpy(), ra, scale) <= 1e-4
+
+
+def test_backward_walk_stage_timeout(pr):
+    """A stage wait that runs out reports status 4 and leaves the context usable.
+    The walker's copies always land, so the limit is made shorter than any copy
+    (1 ns): the first wait that is not already complete gives up."""
+    B, L, D = 8, 4096, 1024
+    x = inputs.gru_inputs(1, 64, 32, seed=670)
+    P = torch.randn(B, L, 3, D, device="cuda")
+    a = dev(np.resize(x["a"], (3, D)))
+    h = torch.zeros(B, L, D, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pr.solve_gru_backward(P, a, h, h, status=st, opts=pr.Options(regime=2, wait_timeout_ns=1))
+    torch.cuda.synchronize()
+    assert int(st.item()) in (0, 4)
+    # the context still works
+    dP, da, dh0 = pr.solve_gru_backward(P, a, h, h, opts=pr.Options(regime=2))
+    torch.cuda.synchronize()
+    assert torch.isfinite(dP).all()
