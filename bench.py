@@ -198,6 +198,8 @@ def algorithmic_bytes(op, bf16, B, L, D, passes=1):
         return 12 * N
     if op == "scan_block2":
         return 32 * N
+    if op == "proj":      # handled by projection_bytes (depends on K and G)
+        raise ValueError("use projection_bytes for the input projection")
     if op == "gru_bwd":   # read P, h_{t-1}, dl/dh; write dP
         return N * (3 * (2 if bf16 else 4) + 4 + 4 + 12)
     if op == "lstm_bwd":  # read P, (c, h)_{t-1}, dl/dc, dl/dh; write dP
@@ -208,6 +210,11 @@ def algorithmic_bytes(op, bf16, B, L, D, passes=1):
     first = pbytes + 4 * ns
     later = pbytes + 8 * ns
     return N * (first + later * (passes - 1))
+
+
+def projection_bytes(M, N, K, out_bf16):
+    """Bytes the projection must move: x and W once (bf16), the bias, P once."""
+    return 2 * M * K + 2 * N * K + 4 * N + (2 if out_bf16 else 4) * M * N
 
 
 def kernel_source_digest():
@@ -258,7 +265,21 @@ class Case:
         self.tol, self.max_iters = 1e-4, 32
         seed = w["seed"] if rank == 0 else [w["seed"], 1000 + rank]
         B, L, D = self.B, self.L, self.D
-        if self.op in ("gru_bwd", "lstm_bwd"):
+        self.out_dtype = None
+        if self.op == "proj":
+            # x [B, L, K] -> P [B, L, G, D]: M = B * L rows, N = G * D features
+            self.K, self.G = w["K"], w["G"]
+            M, Nf = B * L, w["G"] * D
+            x = inputs.projection_inputs(M, Nf, self.K, seed)
+            x["G"] = self.G
+            self.host = {
+                "x": torch.from_numpy(x["x_bits"].view(np.int16)).view(torch.bfloat16).view(
+                    B, L, self.K),
+                "W": torch.from_numpy(x["W_bits"].view(np.int16)).view(torch.bfloat16),
+                "bias": torch.from_numpy(x["bias"])}
+            self.out_dtype = torch.bfloat16 if self.bf16 else torch.float32
+            self.out_shapes = [(B, L, Nf)]
+        elif self.op in ("gru_bwd", "lstm_bwd"):
             # the backward pass differentiates the forward solution: solve once here
             cell = self.op[:-4]
             x = (inputs.gru_inputs if cell == "gru" else inputs.lstm_inputs)(B, L, D, seed,
@@ -301,7 +322,8 @@ class Case:
             self.out_shapes = [(B, L, D, 2)]
         self.x = x
         self.dev = {k: v.to(device) for k, v in self.host.items()}
-        self.outs = [torch.empty(sh, dtype=torch.float32, device=device) for sh in self.out_shapes]
+        odt = self.out_dtype or torch.float32
+        self.outs = [torch.empty(sh, dtype=odt, device=device) for sh in self.out_shapes]
         self.info_t = torch.empty(pr.INFO_BYTES // 4, dtype=torch.int32, device=device)
 
     def run(self, d, outs):
@@ -312,6 +334,8 @@ class Case:
         elif op == "lstm":
             pr.solve_lstm(d["P"], d["a"], d["c0"], d["h0"], self.tol, self.max_iters,
                           out=(outs[0], outs[1]), info=self.info_t)
+        elif op == "proj":
+            pr.input_projection(d["x"], d["W"], d["bias"], out=outs[0], out_dtype=self.out_dtype)
         elif op == "gru_bwd":
             pr.solve_gru_backward(d["P"], d["a"], d["h"], d["gh"], d["h0"],
                                   out=(outs[0], outs[1], outs[2]))
@@ -387,7 +411,8 @@ def run_ours(args, world, rank, local):
     # (they also hold the ~2 us zeroing of the workspace control block).
     launch_ms = statistics.mean(per_step)
     hbm_peak, peak_kind, pk = peaks()
-    bytes_launch = algorithmic_bytes(op, bf16, B, L, D, passes)
+    bytes_launch = (projection_bytes(B * L, cs.G * D, cs.K, bf16) if op == "proj"
+                    else algorithmic_bytes(op, bf16, B, L, D, passes))
     achieved_gbs = bytes_launch / (launch_ms * 1e-3) / 1e9
     hbm_frac = achieved_gbs / hbm_peak
     traffic, traffic_src = recorded_traffic(args.workload)
@@ -415,6 +440,19 @@ def run_ours(args, world, rank, local):
         else:
             roofline = dict(hbm)
             roofline["alu"] = {k: alu[k] for k in ("achieved", "peak", "unit", "frac")}
+    elif op == "proj":
+        ev_iters = None
+        flops = 2.0 * (B * L) * (cs.G * D) * cs.K
+        tf_peak = pk.get("bf16_tflops")
+        tf_kind = "measured burst (cuBLAS bf16 GEMM, MEASURED_PEAKS)"
+        if not tf_peak:
+            tf_peak, tf_kind = 1590.0, "fallback"
+        tflops = flops / (launch_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": tflops, "peak": tf_peak, "unit": "TFLOP/s",
+                    "frac": tflops / tf_peak, "traffic": traffic, "peak_kind": tf_kind,
+                    "flops_per_launch": flops,
+                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": hbm_frac, "algorithmic_bytes_per_launch": bytes_launch}}
     else:
         ev_iters = None
         roofline = dict(hbm)
@@ -422,7 +460,8 @@ def run_ours(args, world, rank, local):
                           "pararnn Newton kernel (LSTM)", "scan_diag": "pararnn scan (diagonal)",
                           "scan_block2": "pararnn scan (2x2)",
                           "gru_bwd": "pararnn backward kernel (GRU)",
-                          "lstm_bwd": "pararnn backward kernel (LSTM)"}[op]
+                          "lstm_bwd": "pararnn backward kernel (LSTM)",
+                          "proj": "pararnn input projection (tcgen05)"}[op]
     roofline["launch_ms"] = launch_ms
     roofline["traffic_source"] = traffic_src
 
@@ -513,7 +552,8 @@ def run_ours(args, world, rank, local):
     e2e = None
     if not args.no_e2e:
         pin = {k: v.pin_memory() for k, v in cs.host.items()}
-        outs_pin = [torch.empty(sh, dtype=torch.float32).pin_memory() for sh in cs.out_shapes]
+        outs_pin = [torch.empty(sh, dtype=cs.out_dtype or torch.float32).pin_memory()
+                    for sh in cs.out_shapes]
 
         def e2e_step():
             d = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
@@ -551,8 +591,14 @@ def run_ours(args, world, rank, local):
               "scan": "diagonal affine scan fp32",
               "block2": "2x2 block affine scan fp32",
               "gru_bwd": "ParaGRU backward pass fp32",
-              "lstm_bwd": "ParaLSTM backward pass fp32"}[args.workload]
-        cfg = {"workload": f"{wl} B={B} L={L} D={D}", "B": B, "L": L, "D": D,
+              "lstm_bwd": "ParaLSTM backward pass fp32",
+              "proj": "input projection x W^T + bias, bf16 in, fp32 out (tcgen05)",
+              "proj_lm": "input projection x W^T + bias, bf16 in, bf16 out (tcgen05)",
+              }[args.workload]
+        wlname = f"{wl} B={B} L={L} D={D}"
+        if op == "proj":
+            wlname += f" K={cs.K} G={cs.G} (M={B * L}, N={cs.G * D})"
+        cfg = {"workload": wlname, "B": B, "L": L, "D": D,
                "parallelism": f"replicas x{world} (independent batches)",
                "l2": "inputs larger than L2 (%.0f MB per step), no flush needed" % (
                    sum(v.numel() * v.element_size() for v in cs.host.values()) / 1e6)}
@@ -563,7 +609,8 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32" if not bf16 else "bf16-in/f32",
+            "dtype": ("bf16-in/f32-acc" if op == "proj" else
+                      "f32" if not bf16 else "bf16-in/f32"),
             "data": "synthetic (seeded numpy; see tests/inputs.py)",
             "config": cfg, "roofline": roofline, "clocks": clocks, "e2e": e2e,
             "gpu_launches": K, "scan": scan, "cpu_baseline": cpu,
@@ -585,6 +632,21 @@ def cpu_baseline(x, op, B, L, D, budget_s=15.0):
 
     oracle.build()
     cores = oracle.get_threads()
+    if op == "proj":
+        # rows of the projection (each row is L-independent work: N x K sums)
+        Wd = x["W"]
+        t0 = time.perf_counter()
+        oracle.input_projection(x["x"][:8], Wd, x["bias"])
+        per_row = max((time.perf_counter() - t0) / 8, 1e-6)
+        nrows = int(max(8, min(x["x"].shape[0], budget_s / per_row)))
+        t0 = time.perf_counter()
+        oracle.input_projection(x["x"][:nrows], Wd, x["bias"])
+        dt = time.perf_counter() - t0
+        Nf = Wd.shape[0]
+        return {"value": nrows * (Nf // x["G"]) / dt, "unit": UNIT, "cores": cores,
+                "kind": "oracle",
+                "sample": f"fp64 projection of {nrows} of {x['x'].shape[0]} rows "
+                          f"(N={Nf}, K={Wd.shape[1]}; {dt:.1f} s)"}
     if op in ("gru_bwd", "lstm_bwd"):
         nb = 1
         nd = min(D, 256)
@@ -676,9 +738,18 @@ def run_reference(args, world, rank, local):
                 return oracle.backward_lstm(Ps, as_, cc, hh, g[1], g[0])
         what = "adjoint (backward) recursion"
         x = None
+    elif op == "proj":
+        Nf, K = w["G"] * D, w["K"]
+        x = inputs.projection_inputs(B * L, Nf, K, w["seed"])
+        nrows = max(1, min(B * L, int(2e8 // max(Nf * K, 1))))  # about 0.2 G multiply-adds
+        xs = np.ascontiguousarray(x["x"][:nrows])
+
+        def step():
+            return oracle.input_projection(xs, x["W"], x["bias"])
+        what = f"fp64 input projection ({nrows} rows x N={Nf} x K={K})"
     else:
         x = inputs.workload_inputs(args.workload)  # the same draws as the GPU arm, then sliced
-    if op in ("gru_bwd", "lstm_bwd"):
+    if op in ("gru_bwd", "lstm_bwd", "proj"):
         pass
     elif op in ("gru", "lstm"):
         Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
@@ -706,16 +777,17 @@ def run_reference(args, world, rank, local):
     for _ in range(args.steps):
         step()
     dt = (time.perf_counter() - t0) / args.steps
-    steps = L * nd
+    steps = nrows * D if op == "proj" else L * nd
     value = steps / dt
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": max(args.warmup, 1), "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded numpy)",
-            "config": {"workload": f"oracle {what}, sample of B=1 x D={nd} x L={L} "
-                                   f"from the {args.workload} workload (B={B}, D={D})"},
+            "config": {"workload": (f"oracle {what} from the {args.workload} workload" if op == "proj"
+                                    else f"oracle {what}, sample of B=1 x D={nd} x L={L} "
+                                         f"from the {args.workload} workload (B={B}, D={D})")},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"B=1, D={nd}, L={L} per step"},
+                             "sample": (what if op == "proj" else f"B=1, D={nd}, L={L} per step")},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -729,7 +801,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gru_l",
                     choices=["gru_l", "lm", "deer", "gru_s", "lstm", "scan", "block2",
-                             "gru_bwd", "lstm_bwd"])
+                             "gru_bwd", "lstm_bwd", "proj", "proj_lm"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-scan", action="store_true", help="skip the scan leg (gru_l)")

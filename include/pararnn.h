@@ -239,6 +239,26 @@ pararnn_status_t pararnn_rollout_lstm(const void* P, pararnn_dtype_t p_dtype, co
                                       const float* c0, const float* h0, float* c, float* h,
                                       int64_t B, int64_t L, int64_t D, void* stream);
 
+/* Input projection P = x W^T + bias on the tensor cores (tcgen05, bf16 inputs,
+ * fp32 accumulation): the projected gate pre-activations that the cells take
+ * as inputs (ParaRNN TL;DR: the recurrence keeps only diagonal weights, the
+ * dense weights act on the inputs; Figure 2 caption).  For a layer of G gates
+ * and D channels, N = G * D and P is [M, N] = [B, L, G, D] with M = B * L, the
+ * layout pararnn_solve_gru / _lstm read.
+ *   x    : [M, K] bf16, row-major (K contiguous), 16-byte aligned;
+ *   W    : [N, K] bf16, row-major (the nn.Linear weight layout), 16-byte aligned;
+ *   bias : [N] fp32 or NULL (= 0);
+ *   P    : [M, N], fp32 (p_dtype = PARARNN_F32) or bf16 (round to nearest even),
+ *          16-byte aligned; must not overlap x, W or bias.
+ * N and K must be multiples of 8 (16-byte rows for the tensor copies) and M, N,
+ * K below 2^31; otherwise PARARNN_ERR_INVALID_ARGUMENT.  K = 0 writes the bias
+ * (or zeros).  No workspace.  status_dev (optional, zeroed by the call) reads 4
+ * if a device-side wait ran out.  Needs sm_100a (PARARNN_ERR_UNSUPPORTED). */
+pararnn_status_t pararnn_input_projection(const void* x, const void* W, const float* bias,
+                                          void* P, pararnn_dtype_t p_dtype, int64_t M,
+                                          int64_t N, int64_t K, int32_t* status_dev,
+                                          void* stream);
+
 /* Allocation-free variant of pararnn_solve_gru (the pages have no counterpart:
  * this is an interface convenience of this library).
  * For callers that cannot allocate device memory where they solve -- their

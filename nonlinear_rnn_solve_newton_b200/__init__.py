@@ -127,6 +127,9 @@ def load(build_if_missing: bool = True):
                                                       _i64, _i64, ctypes.c_float, ctypes.c_int32,
                                                       _vp, _vp, _vp]
             lib.pararnn_solve_gru_noalloc.restype = ctypes.c_int
+            lib.pararnn_input_projection.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i64,
+                                                     _i64, _i64, _vp, _vp]
+            lib.pararnn_input_projection.restype = ctypes.c_int
             lib.pararnn_status_string.argtypes = [ctypes.c_int]
             lib.pararnn_status_string.restype = ctypes.c_char_p
             lib.pararnn_version.restype = ctypes.c_int32
@@ -448,6 +451,38 @@ def step_gru(P, a, h_prev=None, out=None, stream=None):
     _raise(lib.pararnn_step_gru(_ptr(P), dt, _ptr(a), _ptr(h_prev), _ptr(h), B, D,
                                 _stream_handle(stream)), "pararnn_step_gru")
     return h
+
+
+def input_projection(x, W, bias=None, out=None, out_dtype=torch.float32, status=None,
+                     stream=None):
+    """P = x W^T + bias on the tensor cores: x [..., K] bf16, W [N, K] bf16,
+    bias [N] fp32 or None -> P [..., N] (fp32 or bf16).  With N = G * D and x
+    [B, L, K], P.view(B, L, G, D) is the solve's input."""
+    lib = load()
+    if x.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise TypeError("x and W must be bf16")
+    if W.dim() != 2 or x.shape[-1] != W.shape[1]:
+        raise ValueError(f"x [..., K] and W [N, K] do not match: {tuple(x.shape)}, {tuple(W.shape)}")
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    N, K = W.shape
+    lead = tuple(x.shape[:-1])
+    M = 1
+    for n in lead:
+        M *= n
+    if not x.is_contiguous() or not W.is_contiguous():
+        raise ValueError("x and W must be contiguous")
+    _check_dev("x", x, torch.bfloat16, lead + (K,))
+    _check_dev("W", W, torch.bfloat16, (N, K))
+    _check_dev("bias", bias, torch.float32, (N,))
+    P = torch.empty(lead + (N,), dtype=out_dtype, device=x.device) if out is None else out
+    _check_dev("out", P, out_dtype, lead + (N,))
+    _check_dev("status", status, torch.int32, (1,))
+    dt = BF16 if out_dtype == torch.bfloat16 else F32
+    _raise(lib.pararnn_input_projection(_ptr(x), _ptr(W), _ptr(bias), _ptr(P), dt, M, N, K,
+                                        _ptr(status), _stream_handle(stream)),
+           "pararnn_input_projection")
+    return P
 
 
 def step_lstm(P, a, c_prev=None, h_prev=None, out=None, stream=None):

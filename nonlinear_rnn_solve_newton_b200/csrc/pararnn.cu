@@ -17,6 +17,7 @@
 #include "pararnn_bwd.cuh"
 #include "pararnn_bwd_walk.cuh"
 #include "pararnn_kernel.cuh"
+#include "pararnn_proj.cuh"
 #include "pararnn_seq.cuh"
 #include "pararnn_walk.cuh"
 
@@ -1007,4 +1008,108 @@ extern "C" pararnn_status_t pararnn_rollout_lstm(const void* P, pararnn_dtype_t 
                                                  float* c, float* h, int64_t B, int64_t L,
                                                  int64_t D, void* stream) {
   return seq_common(true, kLstm, P, p_dtype, a, c0, h0, c, h, B, L, D, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Input projection P = x W^T + bias (tcgen05 tensor cores).
+// ---------------------------------------------------------------------------
+namespace pararnn {
+namespace {
+
+#ifndef PARARNN_PROJ_STAGES
+#define PARARNN_PROJ_STAGES 4
+#endif
+constexpr int kProjStages = PARARNN_PROJ_STAGES;
+
+// K = 0: P is the bias broadcast over rows (or zero).
+__global__ void proj_fill_kernel(const float* bias, void* out, long long M, long long N,
+                                 int out_bf16) {
+  const long long n = M * N;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float v = bias ? bias[i % N] : 0.0f;
+    if (out_bf16)
+      static_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(out)[i] = v;
+  }
+}
+
+// bf16 row-major [outer][inner] operand, box = 64 (one 128-byte swizzle row) x rows.
+bool encode_map_sw128(CUtensorMap* m, const void* base, unsigned long long inner,
+                      unsigned long long outer, unsigned box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace pararnn
+
+extern "C" pararnn_status_t pararnn_input_projection(const void* x, const void* W,
+                                                     const float* bias, void* P,
+                                                     pararnn_dtype_t p_dtype, int64_t M,
+                                                     int64_t N, int64_t K, int32_t* status_dev,
+                                                     void* stream) {
+  if (M < 0 || N < 0 || K < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (p_dtype != PARARNN_F32 && p_dtype != PARARNN_BF16) return PARARNN_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (status_dev && cudaMemsetAsync(status_dev, 0, sizeof(int32_t), st) != cudaSuccess)
+    return PARARNN_ERR_CUDA;
+  if (M == 0 || N == 0) return PARARNN_OK;
+  if (!P || N % 8 != 0 || K % 8 != 0 || M >= (1LL << 31) || N >= (1LL << 31) ||
+      K >= (1LL << 31))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!aligned(P, 16) || (bias && !aligned(bias, 4))) return PARARNN_ERR_INVALID_ARGUMENT;
+  const int out_bf16 = p_dtype == PARARNN_BF16 ? 1 : 0;
+  if (K == 0) {
+    long long blocks = (M * N + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    proj_fill_kernel<<<(unsigned)blocks, 256, 0, st>>>(bias, P, M, N, out_bf16);
+    return cudaGetLastError() == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA;
+  }
+  if (!x || !W || !aligned(x, 16) || !aligned(W, 16)) return PARARNN_ERR_INVALID_ARGUMENT;
+  const long long ntm = (M + kProjBM - 1) / kProjBM, ntn = (N + kProjBN - 1) / kProjBN;
+  if (ntm * ntn >= (1LL << 31)) return PARARNN_ERR_INVALID_ARGUMENT;
+
+  const void* fn = (const void*)pararnn_proj_kernel<kProjStages>;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_UNSUPPORTED;
+  }
+  const size_t smem = proj_smem_bytes<kProjStages>();
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  ProjMaps tm;
+  if (!encode_map_sw128(&tm.x, x, (unsigned long long)K, (unsigned long long)M, kProjBM) ||
+      !encode_map_sw128(&tm.w, W, (unsigned long long)K, (unsigned long long)N, kProjBN))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+  ProjParams pp;
+  pp.bias = bias;
+  pp.out = P;
+  pp.M = (int)M;
+  pp.N = (int)N;
+  pp.K = (int)K;
+  pp.ntn = (int)ntn;
+  pp.out_bf16 = out_bf16;
+  pp.status_dev = status_dev;
+  pp.timeout_ns = 1000000000LL;
+  void* args[] = {&pp, &tm};
+  if (cudaLaunchKernel(fn, dim3((unsigned)(ntm * ntn)), dim3(128), args, smem, st) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  return PARARNN_OK;
 }

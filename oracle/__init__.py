@@ -21,6 +21,9 @@ What each function computes, and the passage it follows:
 * ``gru_cell`` / ``lstm_cell``: one cell step and its Jacobian.
 * ``backward_gru`` / ``backward_lstm``: gradients of a loss through the solved
   trajectory by the adjoint (reverse-time, transposed bi-diagonal) recursion.
+* ``input_projection``: P = x W^T + bias, the projected gate inputs of the
+  cells (ParaRNN TL;DR: dense weights act on the inputs, the recurrence keeps
+  diagonal ones), as plain fp64 sums.
 
 Parity status: every function above is pinned in ``tests/test_oracle_pins.py``
 against closed forms, brute force, PyTorch's fp64 ``GRUCell``/``LSTMCell`` and
@@ -83,6 +86,7 @@ def _bind(lib):
                                         _i64, _i64, _i64]
     lib.oracle_backward_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
                                          _f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+    lib.oracle_input_projection.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_get_threads.restype = ctypes.c_int
     return lib
@@ -274,3 +278,16 @@ def backward_lstm(P, a, c, h, gc, gh, c0=None, h0=None):
     _load().oracle_backward_lstm(_p(P), _p(a), _p(c0), _p(h0), _p(c), _p(h), _p(gc), _p(gh),
                                  _p(dP), _p(da), _p(dc0), _p(dh0), B, L, D)
     return dP, da, dc0, dh0
+
+
+def input_projection(x, W, bias=None):
+    """P = x W^T + bias in fp64: x [..., K], W [N, K], bias [N] or None -> P [..., N]."""
+    x, W = _d(x), _d(W)
+    N, K = W.shape
+    lead = x.shape[:-1]
+    M = int(np.prod(lead, dtype=np.int64))
+    x2 = np.ascontiguousarray(x.reshape(M, K))
+    bias = None if bias is None else _d(bias).reshape(N)
+    P = np.empty((M, N))
+    _load().oracle_input_projection(_p(x2), _p(W), _p(bias), _p(P), M, N, K)
+    return P.reshape(lead + (N,))

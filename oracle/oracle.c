@@ -616,3 +616,30 @@ void oracle_backward_lstm(const double* P, const double* a, const double* c0, co
     }
   free(x.da_part);
 }
+
+/* ------------------------------------------------------------------------
+ * Input projection P = x W^T + bias: the projected gate pre-activations the
+ * cells take as inputs (ParaRNN TL;DR: the recurrence keeps diagonal weights
+ * only, the dense weights act on the inputs).  x [M,K], W [N,K] (one row of W
+ * per output feature), bias [N] or NULL, P [M,N]; plain sums in k order.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  const double *x, *W, *bias;
+  double* P;
+  int64_t N, K;
+} proj_ctx;
+
+static void projection_row(void* p, int64_t m) {
+  const proj_ctx* c = (const proj_ctx*)p;
+  for (int64_t n = 0; n < c->N; ++n) {
+    double s = c->bias ? c->bias[n] : 0.0;
+    for (int64_t k = 0; k < c->K; ++k) s += c->x[m * c->K + k] * c->W[n * c->K + k];
+    c->P[m * c->N + n] = s;
+  }
+}
+
+void oracle_input_projection(const double* x, const double* W, const double* bias, double* P,
+                             int64_t M, int64_t N, int64_t K) {
+  proj_ctx c = {x, W, bias, P, N, K};
+  for_channels(M, projection_row, &c);
+}

@@ -21,6 +21,8 @@ lstm_bwd ParaLSTM backward pass, fp32          8, 4096, 1024
 lstm     ParaLSTM solve, fp32 (+ block scan)    8, 4096, 1024
 deer     ParaGRU solve, fp32, DEER shape        16, 2^20, 1
 lm       ParaGRU solve, bf16 P, fp32 state      8, 8192, 4096
+proj     input projection x W^T (+bias), G=3    8, 4096, 1024, K = 1024
+proj_lm  input projection, LM width, G=3        8, 8192, 4096, K = 4096
 =======  =====================================  ==========================
 
 Distributions: projected gate inputs P ~ N(0, 1); diagonal recurrence weights
@@ -29,6 +31,9 @@ b ~ N(0, 1), h0 ~ N(0, 1).  Block scan: A entries ~ U(-0.5, 0.5), b ~ N(0, 1),
 x0 ~ N(0, 1).  Draw order: P (or A) first, then a (or b), then h0 (or x0).
 Backward passes: the forward workload's inputs, and upstream gradients
 dl/dh (and dl/dc) ~ N(0, 1) from their own generator.
+Input projection: x ~ N(0, 1) and W ~ N(0, 1/K), both rounded to bf16 once,
+bias ~ N(0, 0.1^2) fp32 (draw order x, W, bias), so that P = x W^T + bias has
+about the N(0, 1) spread of the solves' P.
 """
 from __future__ import annotations
 
@@ -44,6 +49,8 @@ WORKLOADS = {
     "lm": dict(op="gru", B=8, L=8192, D=4096, seed=5, bf16=True),
     "gru_bwd": dict(op="gru_bwd", B=8, L=4096, D=1024, seed=2, bf16=False),
     "lstm_bwd": dict(op="lstm_bwd", B=8, L=4096, D=1024, seed=3, bf16=False),
+    "proj": dict(op="proj", B=8, L=4096, D=1024, K=1024, G=3, seed=6, bf16=False),
+    "proj_lm": dict(op="proj", B=8, L=8192, D=4096, K=4096, G=3, seed=7, bf16=True),
 }
 
 L_SWEEP = [1 << e for e in range(6, 15)]
@@ -145,3 +152,13 @@ def upstream_gradients(B, L, D, seed, n=1):
     """n arrays [B, L, D] of fp32 N(0, 1) draws: the upstream gradients dl/dh (, dl/dc)."""
     rng = _rng([seed, 97])
     return [_normal(rng, (B, L, D)) for _ in range(n)]
+
+
+def projection_inputs(M, N, K, seed):
+    """x [M, K] and W [N, K] as bf16 (bits uint16, values fp32), bias [N] fp32."""
+    rng = _rng(seed)
+    x_bits, x = round_to_bf16(_normal(rng, (M, K)))
+    w32 = (_normal(rng, (N, K)) * np.float32(1.0 / np.sqrt(max(K, 1)))).astype(np.float32)
+    w_bits, W = round_to_bf16(w32)
+    bias = (_normal(rng, (N,)) * np.float32(0.1)).astype(np.float32)
+    return dict(x=x, x_bits=x_bits, W=W, W_bits=w_bits, bias=bias)

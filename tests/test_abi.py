@@ -109,6 +109,24 @@ def test_host_validation_rejects_before_any_cuda_call(lib):
                                   ctypes.c_float(1e-4), 4, fake, 1 << 20, info, None, None) == 1
 
 
+def test_input_projection_host_validation(lib):
+    vp = ctypes.c_void_p
+    fake = vp(4096)  # never dereferenced: validation fails first
+    # N and K must be multiples of 8
+    assert lib.pararnn_input_projection(fake, fake, None, fake, 0, 16, 12, 64, None, None) == 1
+    assert lib.pararnn_input_projection(fake, fake, None, fake, 0, 16, 16, 60, None, None) == 1
+    # negative sizes, unknown dtype, misaligned P / x
+    assert lib.pararnn_input_projection(fake, fake, None, fake, 0, -1, 16, 64, None, None) == 1
+    assert lib.pararnn_input_projection(fake, fake, None, fake, 3, 16, 16, 64, None, None) == 1
+    assert lib.pararnn_input_projection(fake, fake, None, vp(4104), 0, 16, 16, 64, None,
+                                        None) == 1
+    assert lib.pararnn_input_projection(vp(4100), fake, None, fake, 0, 16, 16, 64, None,
+                                        None) == 1
+    # M = 0 or N = 0: nothing to do, nothing launched
+    assert lib.pararnn_input_projection(fake, fake, None, fake, 0, 0, 16, 64, None, None) == 0
+    assert lib.pararnn_input_projection(fake, fake, None, fake, 1, 16, 0, 64, None, None) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
 

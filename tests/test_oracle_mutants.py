@@ -46,6 +46,11 @@ MUTANTS = {
                                         "double dfdr = dfdu * w[2] * hp * r;"),
     "backward_lstm_untransposed_jacobian": ("mc = J[0] * lc + J[2] * lh;\n    mh = J[1] * lc + J[3] * lh;",
                                             "mc = J[0] * lc + J[1] * lh;\n    mh = J[2] * lc + J[3] * lh;"),
+    "projection_transposed_w": ("s += c->x[m * c->K + k] * c->W[n * c->K + k];",
+                                "s += c->x[m * c->K + k] * c->W[k * c->N + n];"),
+    "projection_drops_bias": ("double s = c->bias ? c->bias[n] : 0.0;", "double s = 0.0;"),
+    "projection_skips_first_k": ("for (int64_t k = 0; k < c->K; ++k) s +=",
+                                 "for (int64_t k = 1; k < c->K; ++k) s +="),
     "backward_gru_forward_time": ("double lam = x->gh[IDX3(bb, t, d, L, D)] + lam_next;",
                                   "double lam = x->gh[IDX3(bb, t, d, L, D)];"),
 }

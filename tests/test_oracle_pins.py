@@ -518,3 +518,71 @@ def test_backward_linear_recurrence_is_a_reverse_scan(oracle):
     c = np.tanh(x["P"].astype(np.float64)[:, :, 2])
     hp = np.concatenate([x["h0"][:, None].astype(np.float64), h[:, :-1]], 1)
     np.testing.assert_allclose(dP[:, :, 0], lam * (c - hp) * z * (1 - z), atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Input projection P = x W^T + bias
+# --------------------------------------------------------------------------
+def test_projection_selects_permuted_columns(oracle):
+    """W with a single 1 per row, W[n, pi(n)] = 1, picks column pi(n) of x.  pi is
+    a 7-cycle (not its own inverse), so a transposed W would pick pi^-1(n)."""
+    rng = np.random.default_rng(700)
+    K = 7
+    pi = np.array([1, 2, 3, 4, 5, 6, 0])
+    W = np.zeros((K, K))
+    W[np.arange(K), pi] = 1.0
+    x = rng.standard_normal((5, K))
+    b = rng.standard_normal(K)
+    assert np.array_equal(oracle.input_projection(x, W, b), x[:, pi] + b)
+
+
+def test_projection_rectangular_selection(oracle):
+    """N != K: each output feature is a scaled copy of one input feature."""
+    rng = np.random.default_rng(701)
+    M, N, K = 4, 3, 10
+    W = np.zeros((N, K))
+    W[[0, 1, 2], [7, 2, 9]] = [2.0, -1.0, 0.5]
+    x = rng.standard_normal((M, K))
+    expect = np.stack([2.0 * x[:, 7], -x[:, 2], 0.5 * x[:, 9]], axis=1)
+    assert np.array_equal(oracle.input_projection(x, W), expect)
+
+
+def test_projection_bias_only(oracle):
+    rng = np.random.default_rng(702)
+    b = rng.standard_normal(6)
+    P = oracle.input_projection(rng.standard_normal((3, 5)), np.zeros((6, 5)), b)
+    assert np.array_equal(P, np.broadcast_to(b, (3, 6)))
+    P0 = oracle.input_projection(np.zeros((3, 0)), np.zeros((6, 0)), b)
+    assert np.array_equal(P0, np.broadcast_to(b, (3, 6)))
+
+
+def test_projection_small_integers_brute_force(oracle):
+    """Integer operands: the sums are exact, so brute force in Python integers
+    must agree bit for bit."""
+    rng = np.random.default_rng(703)
+    M, N, K = 3, 4, 5
+    x = rng.integers(-3, 4, (M, K))
+    W = rng.integers(-3, 4, (N, K))
+    b = rng.integers(-5, 6, N)
+    P = oracle.input_projection(x, W, b)
+    for m in range(M):
+        for n in range(N):
+            s = int(b[n])
+            for k in range(K):
+                s += int(x[m, k]) * int(W[n, k])
+            assert P[m, n] == s
+
+
+def test_projection_rank_one(oracle):
+    """x = u v^T  =>  P = u (W v)^T."""
+    rng = np.random.default_rng(704)
+    u, v = rng.standard_normal(6), rng.standard_normal(9)
+    W = rng.standard_normal((5, 9))
+    P = oracle.input_projection(np.outer(u, v), W)
+    assert np.allclose(P, np.outer(u, W @ v), rtol=0, atol=1e-12)
+
+
+def test_projection_matches_library_matmul(oracle):
+    rng = np.random.default_rng(705)
+    x, W, b = rng.standard_normal((33, 70)), rng.standard_normal((24, 70)), rng.standard_normal(24)
+    assert np.allclose(oracle.input_projection(x, W, b), x @ W.T + b, rtol=0, atol=1e-12)
