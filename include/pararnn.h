@@ -247,7 +247,7 @@ pararnn_status_t pararnn_rollout_lstm(const void* P, pararnn_dtype_t p_dtype, co
  * layout pararnn_solve_gru / _lstm read.
  *   x    : [M, K] bf16, row-major (K contiguous), 16-byte aligned;
  *   W    : [N, K] bf16, row-major (the nn.Linear weight layout), 16-byte aligned;
- *   bias : [N] fp32 or NULL (= 0);
+ *   bias : [N] fp32 or NULL (= 0), 16-byte aligned;
  *   P    : [M, N], fp32 (p_dtype = PARARNN_F32) or bf16 (round to nearest even),
  *          16-byte aligned; must not overlap x, W or bias.
  * N and K must be multiples of 8 (16-byte rows for the tensor copies) and M, N,

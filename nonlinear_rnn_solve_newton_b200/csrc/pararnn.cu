@@ -1050,6 +1050,23 @@ bool encode_map_sw128(CUtensorMap* m, const void* base, unsigned long long inner
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// P [M, N] (fp32 or bf16) for the epilogue's tensor stores: box = 128 bytes of
+// columns x 32 rows, 128-byte swizzle.
+bool encode_map_out(CUtensorMap* m, void* base, unsigned long long N, unsigned long long M,
+                    bool bf16) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const size_t es = bf16 ? 2 : 4;
+  const cuuint64_t dims[2] = {N, M};
+  const cuuint64_t strides[1] = {N * es};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / es), 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+             base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 }  // namespace pararnn
 
@@ -1067,7 +1084,7 @@ extern "C" pararnn_status_t pararnn_input_projection(const void* x, const void* 
   if (!P || N % 8 != 0 || K % 8 != 0 || M >= (1LL << 31) || N >= (1LL << 31) ||
       K >= (1LL << 31))
     return PARARNN_ERR_INVALID_ARGUMENT;
-  if (!aligned(P, 16) || (bias && !aligned(bias, 4))) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!aligned(P, 16) || (bias && !aligned(bias, 16))) return PARARNN_ERR_INVALID_ARGUMENT;
   const int out_bf16 = p_dtype == PARARNN_BF16 ? 1 : 0;
   if (K == 0) {
     long long blocks = (M * N + 255) / 256;
@@ -1079,7 +1096,8 @@ extern "C" pararnn_status_t pararnn_input_projection(const void* x, const void* 
   const long long ntm = (M + kProjBM - 1) / kProjBM, ntn = (N + kProjBN - 1) / kProjBN;
   if (ntm * ntn >= (1LL << 31)) return PARARNN_ERR_INVALID_ARGUMENT;
 
-  const void* fn = (const void*)pararnn_proj_kernel<kProjStages>;
+  const void* fn = out_bf16 ? (const void*)pararnn_proj_kernel<kProjStages, true>
+                            : (const void*)pararnn_proj_kernel<kProjStages, false>;
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
@@ -1093,7 +1111,8 @@ extern "C" pararnn_status_t pararnn_input_projection(const void* x, const void* 
   }
   ProjMaps tm;
   if (!encode_map_sw128(&tm.x, x, (unsigned long long)K, (unsigned long long)M, kProjBM) ||
-      !encode_map_sw128(&tm.w, W, (unsigned long long)K, (unsigned long long)N, kProjBN))
+      !encode_map_sw128(&tm.w, W, (unsigned long long)K, (unsigned long long)N, kProjBN) ||
+      !encode_map_out(&tm.p, P, (unsigned long long)N, (unsigned long long)M, out_bf16 != 0))
     return PARARNN_ERR_INVALID_ARGUMENT;
   ProjParams pp;
   pp.bias = bias;
@@ -1105,9 +1124,16 @@ extern "C" pararnn_status_t pararnn_input_projection(const void* x, const void* 
   pp.out_bf16 = out_bf16;
   pp.status_dev = status_dev;
   pp.timeout_ns = 1000000000LL;
+  // persistent: one CTA per SM (the ring and both accumulators fill an SM)
+  int resident = 0;
+  if (resident_ctas(fn, kProjThreads, smem, &resident) != cudaSuccess || resident <= 0) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  const long long ntiles = ntm * ntn;
+  const unsigned grid = (unsigned)(ntiles < resident ? ntiles : resident);
   void* args[] = {&pp, &tm};
-  if (cudaLaunchKernel(fn, dim3((unsigned)(ntm * ntn)), dim3(128), args, smem, st) !=
-      cudaSuccess) {
+  if (cudaLaunchKernel(fn, dim3(grid), dim3(kProjThreads), args, smem, st) != cudaSuccess) {
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }

@@ -7,14 +7,19 @@
 // W is [N, K] bf16 (N = G*D output features, the nn.Linear layout), P is [M, N]
 // fp32 or bf16 -- i.e. [B, L, G, D], the layout the Newton solve reads.
 //
-// One CTA computes one 128 x 256 tile of P with tcgen05:
+// A persistent CTA per SM computes 128 x 256 tiles of P with tcgen05:
 //   * warp 0, one thread: TMA copies of the x and W k-blocks (64 deep, 128-byte
-//     swizzle) into a ring of shared-memory stages (mbarrier completion);
+//     swizzle) into a ring of shared-memory stages (mbarrier completion); the
+//     ring runs on from one tile to the next;
 //   * warp 1, one thread: per stage, four tcgen05.mma (M=128, N=256, K=16, bf16
-//     in, fp32 accumulate) into a 256-column TMEM accumulator, then
-//     tcgen05.commit to release the stage;
-//   * all four warps: the epilogue reads the accumulator with tcgen05.ld (warp w
-//     owns TMEM lanes = rows 32w..32w+31), adds the bias and stores P.
+//     in, fp32 accumulate) into one of two 256-column TMEM accumulators, then
+//     tcgen05.commit to release the stage (and, after the last k-block, to
+//     hand the accumulator to the epilogue);
+//   * warps 2-9: the epilogue reads an accumulator with tcgen05.ld (warp w owns
+//     TMEM lanes = rows 32 (w mod 4) .. + 31 and one half of the columns),
+//     adds the bias, writes P by tensor stores of 32-row boxes staged in
+//     shared memory and frees the accumulator -- while the MMAs of the next
+//     tile run.
 // Every wait is bounded; a wait that runs out sets status 4 and the CTA still
 // frees its TMEM before it returns.
 #pragma once
@@ -33,8 +38,16 @@ constexpr unsigned kProjABytes = kProjBM * kProjBK * 2;
 constexpr unsigned kProjBBytes = kProjBN * kProjBK * 2;
 constexpr unsigned kProjStageBytes = kProjABytes + kProjBBytes;
 
+// Epilogue: 8 warps, two per TMEM lane quarter (each takes 128 of the 256
+// columns), each staging one 32-row x 128-byte box at a time.
+constexpr int kProjEpiWarps = 8;
+constexpr int kProjThreads = 32 * (2 + kProjEpiWarps);
+constexpr unsigned kProjEpiBox = 32 * 128;
+constexpr unsigned kProjEpiBytes = kProjEpiWarps * kProjEpiBox;
+
 template <int ST> constexpr size_t proj_smem_bytes() {
-  return (size_t)ST * kProjStageBytes + 1024;  // + alignment slack for the 1024-byte swizzle atoms
+  // + alignment slack for the 1024-byte swizzle atoms
+  return (size_t)ST * kProjStageBytes + kProjEpiBytes + 1024;
 }
 
 struct ProjParams {
@@ -50,6 +63,7 @@ struct ProjParams {
 struct ProjMaps {
   CUtensorMap x;  // 2-D {K, M}, box {64, 128}, 128-byte swizzle
   CUtensorMap w;  // 2-D {K, N}, box {64, 256}, 128-byte swizzle
+  CUtensorMap p;  // 2-D {N, M}, box {128 bytes of columns, 32 rows}, 128-byte swizzle
 };
 
 // Shared-memory matrix descriptor of a K-major operand tile written by TMA with
@@ -119,19 +133,135 @@ __device__ __forceinline__ void tmem_ld16(unsigned taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <int ST>
-__global__ void __launch_bounds__(128, 1)
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Tensor store of a 32-row x 128-byte box from shared memory (bulk group).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, unsigned src, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<unsigned long long>(map)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// The TMEM columns of one box row: 32 (fp32 out) or 64 (bf16 out), loads
+// issued without waiting (tcgen05.wait::ld completes them).
+template <bool OB>
+__device__ __forceinline__ void tmem_ld_box_async(unsigned taddr, unsigned* r) {
+#define PARARNN_LD16(OFF, R)                                                                    \
+  asm volatile(                                                                                 \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "   \
+      "%11, %12, %13, %14, %15}, [%16];"                                                        \
+      : "=r"(R[0]), "=r"(R[1]), "=r"(R[2]), "=r"(R[3]), "=r"(R[4]), "=r"(R[5]), "=r"(R[6]),     \
+        "=r"(R[7]), "=r"(R[8]), "=r"(R[9]), "=r"(R[10]), "=r"(R[11]), "=r"(R[12]), "=r"(R[13]), \
+        "=r"(R[14]), "=r"(R[15])                                                                \
+      : "r"(taddr + (OFF)))
+  PARARNN_LD16(0u, (r + 0));
+  PARARNN_LD16(16u, (r + 16));
+  if constexpr (OB) {
+    PARARNN_LD16(32u, (r + 32));
+    PARARNN_LD16(48u, (r + 48));
+  }
+#undef PARARNN_LD16
+}
+
+// Epilogue of one tile for one warp: TMEM columns [c_lo, c_lo + 128) of its
+// 32 lanes (rows y0 .. y0 + 31) -> + bias -> 128-byte-swizzled box in shared
+// memory (16-byte chunk j of row r at chunk j ^ (r mod 8): conflict-free) ->
+// tensor store.  The next box's TMEM load is in flight while the current one
+// is staged and stored; when this returns, every TMEM load of the tile is done.
+template <bool OB>
+__device__ __forceinline__ void proj_epilogue(const ProjParams& p, const CUtensorMap* pmap,
+                                              unsigned taddr, unsigned ebuf, int y0, int n0,
+                                              int c_lo, bool zero) {
+  constexpr int CB = OB ? 64 : 32;  // columns per 128-byte box row
+  const int lane = threadIdx.x & 31;
+  int nb = 0;  // boxes of this tile for this warp
+  while (nb * CB < 128 && n0 + c_lo + nb * CB < p.N) ++nb;
+  if (nb == 0) return;
+  unsigned cur[CB], nxt[CB];
+  tmem_ld_box_async<OB>(taddr + (unsigned)c_lo, cur);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll 1
+  for (int b = 0; b < nb; ++b) {
+    const int col = n0 + c_lo + b * CB;
+    if (zero) {
+#pragma unroll
+      for (int i = 0; i < CB; ++i) cur[i] = 0u;
+    }
+    if (p.bias) {
+      // bias is 16-byte aligned and N a multiple of 8: groups of 4 are whole
+#pragma unroll
+      for (int i = 0; i < CB; i += 4) {
+        if (col + i < p.N) {
+          const float4 bb = __ldg(reinterpret_cast<const float4*>(p.bias + col + i));
+          cur[i] = __float_as_uint(__uint_as_float(cur[i]) + bb.x);
+          cur[i + 1] = __float_as_uint(__uint_as_float(cur[i + 1]) + bb.y);
+          cur[i + 2] = __float_as_uint(__uint_as_float(cur[i + 2]) + bb.z);
+          cur[i + 3] = __float_as_uint(__uint_as_float(cur[i + 3]) + bb.w);
+        }
+      }
+    }
+    if (b + 1 < nb) tmem_ld_box_async<OB>(taddr + (unsigned)(c_lo + (b + 1) * CB), nxt);
+    // the previous tensor store has finished reading the staging box
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    __syncwarp();
+    const unsigned rowp = ebuf + (unsigned)lane * 128u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      unsigned w0, w1, w2, w3;
+      if constexpr (OB) {
+        __nv_bfloat162 t0 = __floats2bfloat162_rn(__uint_as_float(cur[8 * j]), __uint_as_float(cur[8 * j + 1]));
+        __nv_bfloat162 t1 = __floats2bfloat162_rn(__uint_as_float(cur[8 * j + 2]), __uint_as_float(cur[8 * j + 3]));
+        __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(cur[8 * j + 4]), __uint_as_float(cur[8 * j + 5]));
+        __nv_bfloat162 t3 = __floats2bfloat162_rn(__uint_as_float(cur[8 * j + 6]), __uint_as_float(cur[8 * j + 7]));
+        w0 = *reinterpret_cast<unsigned*>(&t0);
+        w1 = *reinterpret_cast<unsigned*>(&t1);
+        w2 = *reinterpret_cast<unsigned*>(&t2);
+        w3 = *reinterpret_cast<unsigned*>(&t3);
+      } else {
+        w0 = cur[4 * j];
+        w1 = cur[4 * j + 1];
+        w2 = cur[4 * j + 2];
+        w3 = cur[4 * j + 3];
+      }
+      const unsigned dst = rowp + ((unsigned)(j ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w0), "r"(w1),
+                   "r"(w2), "r"(w3)
+                   : "memory");
+    }
+    // make the generic-proxy writes visible to the tensor store, then issue it
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) tma_store_2d(pmap, ebuf, col, y0);
+    if (b + 1 < nb) {
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int i = 0; i < CB; ++i) cur[i] = nxt[i];
+    }
+  }
+}
+
+// Persistent: CTA c takes tiles c, c + grid, ... (row-block major, so CTAs
+// running at once share x row blocks and all of W in L2).  Warp 0 = TMA
+// producer, warp 1 = MMA issuer, warps 2-5 = epilogue; the shared-memory ring
+// runs on across tiles and the accumulator is double-buffered in TMEM (2 x 256
+// columns), so the epilogue of tile i overlaps the MMAs of tile i + 1.
+template <int ST, bool OB>
+__global__ void __launch_bounds__(kProjThreads, 1)
     pararnn_proj_kernel(const __grid_constant__ ProjParams p, const __grid_constant__ ProjMaps tm) {
   extern __shared__ __align__(1024) unsigned char dsmem[];
-  __shared__ unsigned long long s_full[ST], s_empty[ST], s_acc;
+  __shared__ unsigned long long s_full[ST], s_empty[ST], s_tfull[2], s_tempty[2];
   __shared__ unsigned s_tmem;
   __shared__ int s_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned sbase = (smem_u32(dsmem) + 1023u) & ~1023u;
-  const int nb = blockIdx.x % p.ntn, mb = blockIdx.x / p.ntn;
-  const int m0 = mb * kProjBM, n0 = nb * kProjBN;
   const int nk = (p.K + kProjBK - 1) / kProjBK;
+  const int ntiles = ((p.M + kProjBM - 1) / kProjBM) * p.ntn;
   const WaitCtx wctx{nullptr, p.status_dev, p.timeout_ns};
 
   if (threadIdx.x == 0) {
@@ -139,15 +269,18 @@ __global__ void __launch_bounds__(128, 1)
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 1);
     }
-    mbar_init(&s_acc, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&s_tfull[a], 1);
+      mbar_init(&s_tempty[a], 32 * kProjEpiWarps);  // every epilogue thread arrives
+    }
     s_fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 0) {  // the whole warp allocates the accumulator's 256 columns
+  if (warp == 0) {  // the whole warp allocates both accumulators (all 512 columns)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&s_tmem)),
-                 "r"(kProjBN)
+                 "r"(2 * kProjBN)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -156,97 +289,92 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const unsigned tmem = s_tmem;
 
-  if (warp == 0 && lane == 0) {
-    // ---- producer: k-blocks into the ring ---------------------------------
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % ST;
-      const unsigned ph = (unsigned)(kb / ST) & 1u;
-      // a fresh barrier passes a wait on parity 1: the first ST stages are free
-      if (!stage_wait(&s_empty[s], ph ^ 1u, wctx)) {
-        s_fail = 1;
-        break;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- producer: k-blocks of every tile into the ring -----------------------
+      unsigned it = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*(volatile int*)&s_fail; tile += gridDim.x) {
+        const int m0 = (tile / p.ntn) * kProjBM, n0 = (tile % p.ntn) * kProjBN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % ST;
+          const unsigned ph = (it / ST) & 1u;
+          // a fresh barrier passes a wait on parity 1: the first ST stages are free
+          if (!stage_wait(&s_empty[s], ph ^ 1u, wctx)) {
+            s_fail = 1;
+            break;
+          }
+          const unsigned a = sbase + s * kProjStageBytes;
+          mbar_expect_tx(&s_full[s], kProjStageBytes);
+          tma_load_2d_s(a, &tm.x, kb * kProjBK, m0, &s_full[s]);
+          tma_load_2d_s(a + kProjABytes, &tm.w, kb * kProjBK, n0, &s_full[s]);
+        }
       }
-      const unsigned a = sbase + s * kProjStageBytes;
-      mbar_expect_tx(&s_full[s], kProjStageBytes);
-      tma_load_2d_s(a, &tm.x, kb * kProjBK, m0, &s_full[s]);
-      tma_load_2d_s(a + kProjABytes, &tm.w, kb * kProjBK, n0, &s_full[s]);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer -----------------------------------------------------------
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % ST;
-      const unsigned ph = (unsigned)(kb / ST) & 1u;
-      if (!stage_wait(&s_full[s], ph, wctx)) {
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ---------------------------------------------------------------
+      unsigned it = 0, lt = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*(volatile int*)&s_fail; tile += gridDim.x, ++lt) {
+        const unsigned acc = lt & 1u, use = lt >> 1;
+        // the epilogue has drained this accumulator (fresh: passes)
+        if (!stage_wait(&s_tempty[acc], (use & 1u) ^ 1u, wctx)) {
+          s_fail = 1;
+          break;
+        }
+        tc_fence_after();
+        const unsigned d = tmem + acc * kProjBN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % ST;
+          const unsigned ph = (it / ST) & 1u;
+          if (!stage_wait(&s_full[s], ph, wctx)) {
+            s_fail = 1;
+            break;
+          }
+          tc_fence_after();
+          const unsigned a = sbase + s * kProjStageBytes;
+          const unsigned b = a + kProjABytes;
+#pragma unroll
+          for (int k = 0; k < kProjBK / 16; ++k)  // K = 16 per MMA: 32 bytes along the row
+            umma_f16_ss(d, umma_desc_sw128(a + 32u * k), umma_desc_sw128(b + 32u * k),
+                        kProjIdesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&s_empty[s]);  // the stage is free once these MMAs have read it
+        }
+        umma_commit(&s_tfull[acc]);  // the tile's accumulator is final
+      }
+    }
+  } else {
+    // ---- epilogue (warps 2-9: TMEM lane quarter = warp % 4, column half) -------
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const unsigned ebuf = sbase + ST * kProjStageBytes + (unsigned)(warp - 2) * kProjEpiBox;
+    unsigned lt = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+      const unsigned acc = lt & 1u, use = lt >> 1;
+      const bool ok = stage_wait(&s_tfull[acc], use & 1u, wctx);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ok) || *(volatile int*)&s_fail) {
         s_fail = 1;
         break;
       }
       tc_fence_after();
-      const unsigned a = sbase + s * kProjStageBytes;
-      const unsigned b = a + kProjABytes;
-#pragma unroll
-      for (int k = 0; k < kProjBK / 16; ++k)  // K = 16 per MMA: 32 bytes along the swizzled row
-        umma_f16_ss(tmem, umma_desc_sw128(a + 32u * k), umma_desc_sw128(b + 32u * k), kProjIdesc,
-                    (kb | k) != 0 ? 1u : 0u);
-      umma_commit(&s_empty[s]);  // the stage is free once these MMAs have read it
+      const int m0 = (tile / p.ntn) * kProjBM, n0 = (tile % p.ntn) * kProjBN;
+      proj_epilogue<OB>(p, &tm.p, tmem + acc * kProjBN + ((unsigned)(32 * q) << 16), ebuf,
+                    m0 + 32 * q, n0, half * 128, nk == 0);
+      tc_fence_before();
+      mbar_arrive(&s_tempty[acc]);
     }
-    umma_commit(&s_acc);  // the accumulator is final once every MMA has completed
-  }
-  __syncwarp();
-
-  // ---- epilogue: TMEM -> registers -> bias -> P ------------------------------------
-  const bool ok = stage_wait(&s_acc, 0u, wctx);
-  __syncwarp();
-  tc_fence_after();
-  const int row = m0 + warp * 32 + lane;
-  if (!ok || s_fail) {
-    if (lane == 0 && p.status_dev) atomicCAS(p.status_dev, 0, 4);
-  } else {
-#pragma unroll 1
-    for (int c0 = 0; c0 < kProjBN && n0 + c0 < p.N; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem + ((unsigned)(warp * 32) << 16) + (unsigned)c0, v);
-      if (nk == 0) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
-      }
-      const int col = n0 + c0;
-      if (p.bias) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] += col + i < p.N ? __ldg(p.bias + col + i) : 0.0f;
-      }
-      if (row < p.M) {
-        const size_t o = (size_t)row * p.N + col;
-        // N is a multiple of 8: the tile's tail is whole groups of 8 columns
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (col + 8 * h + 8 > p.N) break;
-          if (p.out_bf16) {
-            uint4 q;
-            __nv_bfloat162 t[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              t[i] = __floats2bfloat162_rn(v[8 * h + 2 * i], v[8 * h + 2 * i + 1]);
-            q.x = *reinterpret_cast<unsigned*>(&t[0]);
-            q.y = *reinterpret_cast<unsigned*>(&t[1]);
-            q.z = *reinterpret_cast<unsigned*>(&t[2]);
-            q.w = *reinterpret_cast<unsigned*>(&t[3]);
-            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o + 8 * h) = q;
-          } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o + 8 * h);
-            dst[0] = make_float4(v[8 * h], v[8 * h + 1], v[8 * h + 2], v[8 * h + 3]);
-            dst[1] = make_float4(v[8 * h + 4], v[8 * h + 5], v[8 * h + 6], v[8 * h + 7]);
-          }
-        }
-      }
-    }
+    // every tensor store of this warp has completed before the CTA exits
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0 && s_fail && p.status_dev) atomicCAS(p.status_dev, 0, 4);
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kProjBN)
+                 "r"(2 * kProjBN)
                  : "memory");
   }
 }

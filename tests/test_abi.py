@@ -122,6 +122,8 @@ def test_input_projection_host_validation(lib):
                                         None) == 1
     assert lib.pararnn_input_projection(vp(4100), fake, None, fake, 0, 16, 16, 64, None,
                                         None) == 1
+    assert lib.pararnn_input_projection(fake, fake, vp(4100), fake, 0, 16, 16, 64, None,
+                                        None) == 1
     # M = 0 or N = 0: nothing to do, nothing launched
     assert lib.pararnn_input_projection(fake, fake, None, fake, 0, 0, 16, 64, None, None) == 0
     assert lib.pararnn_input_projection(fake, fake, None, fake, 1, 16, 0, 64, None, None) == 0
