@@ -21,6 +21,10 @@ What each function computes, and the passage it follows:
 * ``gru_cell`` / ``lstm_cell``: one cell step and its Jacobian.
 * ``backward_gru`` / ``backward_lstm``: gradients of a loss through the solved
   trajectory by the adjoint (reverse-time, transposed bi-diagonal) recursion.
+* ``mhgru_cell`` / ``rollout_mhgru`` / ``newton_mhgru``: the multi-head GRU
+  whose recurrence is block-diagonal with dense 8x8 blocks (the dense-block
+  case the DEER summary's caveats price at O(n^3) per step), reducing to the
+  ParaGRU cell when every block is diagonal.
 * ``input_projection``: P = x W^T + bias, the projected gate inputs of the
   cells (ParaRNN TL;DR: dense weights act on the inputs, the recurrence keeps
   diagonal ones), as plain fp64 sums.
@@ -86,6 +90,11 @@ def _bind(lib):
                                         _i64, _i64, _i64]
     lib.oracle_backward_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
                                          _f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+    lib.oracle_mhgru_cell.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p]
+    lib.oracle_rollout_mhgru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+    lib.oracle_newton_mhgru.argtypes = [_f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_int,
+                                        _i64, _i64, _i64, _f64p, _f64p, _intp, _intp]
+    lib.oracle_newton_mhgru.restype = ctypes.c_int
     lib.oracle_input_projection.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_get_threads.restype = ctypes.c_int
@@ -291,3 +300,42 @@ def input_projection(x, W, bias=None):
     P = np.empty((M, N))
     _load().oracle_input_projection(_p(x2), _p(W), _p(bias), _p(P), M, N, K)
     return P.reshape(lead + (N,))
+
+
+def mhgru_cell(p, U, h):
+    """One multi-head GRU step of one head: p [3, 8] (z, r, c), U [3, 8, 8] (that
+    head's blocks), h [8] -> (h' [8], J = dh'/dh [8, 8])."""
+    p, U, h = _d(p).reshape(3, 8), _d(U).reshape(3, 8, 8), _d(h).reshape(8)
+    f = np.empty(8)
+    J = np.empty((8, 8))
+    _load().oracle_mhgru_cell(_p(p), _p(U), _p(h), _p(f), _p(J))
+    return f, J
+
+
+def rollout_mhgru(P, U, h0=None):
+    """Sequential multi-head GRU rollout.  P [B, L, 3, D], U [3, H, 8, 8], D = 8 H."""
+    P, U = _d(P), _d(U)
+    B, L, G, D = P.shape
+    H = U.shape[1]
+    assert G == 3 and U.shape == (3, H, 8, 8) and D == 8 * H
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    h = np.empty((B, L, D))
+    _load().oracle_rollout_mhgru(_p(P), _p(U), _p(h0), _p(h), B, L, H)
+    return h
+
+
+def newton_mhgru(P, U, h0=None, tol=1e-4, max_iters=32):
+    """Serial Newton for the multi-head GRU system from h^0 = 0, 8x8 block
+    bi-diagonal solve per head (see oracle.c)."""
+    P, U = _d(P), _d(U)
+    B, L, G, D = P.shape
+    H = U.shape[1]
+    assert G == 3 and U.shape == (3, H, 8, 8) and D == 8 * H
+    h0 = None if h0 is None else _d(h0).reshape(B, D)
+    h = np.empty((B, L, D))
+    rho = np.full(max_iters + 1, np.nan)
+    conv = ctypes.c_int()
+    nf = ctypes.c_int()
+    k = _load().oracle_newton_mhgru(_p(P), _p(U), _p(h0), float(tol), int(max_iters), B, L, H,
+                                    _p(h), _p(rho), ctypes.byref(conv), ctypes.byref(nf))
+    return NewtonResult(k, conv.value, nf.value, rho[: k + 1], None, h=h)

@@ -643,3 +643,168 @@ void oracle_input_projection(const double* x, const double* W, const double* bia
   proj_ctx c = {x, W, bias, P, N, K};
   for_channels(M, projection_row, &c);
 }
+
+/* ------------------------------------------------------------------------
+ * Multi-head GRU with dense 8x8 recurrence blocks (the "dense small-block"
+ * variant: DEER summary, caveats -- dense Jacobians cost O(n^3) per step; here
+ * n = 8 per head).  Channels d = 8 * head + i; per head, with U_g the head's
+ * 8x8 block of gate g (row i = output channel, column j = input channel):
+ *   z = sig(P_z + U_z h),  r = sig(P_r + U_r h),  c = tanh(P_c + r * (U_c h)),
+ *   h' = (1 - z) * h + z * c            (elementwise products)
+ * which is the ParaGRU cell when every U_g is diagonal.  Jacobian, row i:
+ *   dh'_i/dh_j = [i == j] (1 - z_i) + (c_i - h_i) z_i (1 - z_i) U_z[i][j]
+ *              + z_i (1 - c_i^2) (r_i U_c[i][j] + (U_c h)_i r_i (1 - r_i) U_r[i][j])
+ * P is [B, L, 3, D] (gates z, r, c), U is [3, H, 8, 8], D = 8 H.
+ * ---------------------------------------------------------------------- */
+#define NB 8
+
+void oracle_mhgru_cell(const double* p /* [3][8] */, const double* U /* [3][8][8] of one head */,
+                       const double* h, double* f, double* J /* [8][8] or NULL */) {
+  double uz[NB], ur[NB], uc[NB];
+  for (int i = 0; i < NB; ++i) {
+    uz[i] = ur[i] = uc[i] = 0.0;
+    for (int j = 0; j < NB; ++j) {
+      uz[i] += U[(0 * NB + i) * NB + j] * h[j];
+      ur[i] += U[(1 * NB + i) * NB + j] * h[j];
+      uc[i] += U[(2 * NB + i) * NB + j] * h[j];
+    }
+  }
+  for (int i = 0; i < NB; ++i) {
+    double z = sig(p[0 * NB + i] + uz[i]);
+    double r = sig(p[1 * NB + i] + ur[i]);
+    double c = tanh(p[2 * NB + i] + r * uc[i]);
+    f[i] = (1.0 - z) * h[i] + z * c;
+    if (J) {
+      double dz = (c - h[i]) * z * (1.0 - z);
+      double dc = z * (1.0 - c * c);
+      for (int j = 0; j < NB; ++j)
+        J[i * NB + j] = (i == j ? 1.0 - z : 0.0) + dz * U[(0 * NB + i) * NB + j] +
+                        dc * (r * U[(2 * NB + i) * NB + j] +
+                              uc[i] * r * (1.0 - r) * U[(1 * NB + i) * NB + j]);
+    }
+  }
+}
+
+typedef struct {
+  const double *P, *U, *h0;
+  double *h, *Jt, *rt, *cmax;
+  int64_t L, H;
+} mh_ctx;
+
+/* gates of head g at (b, t): p[gate * 8 + i] */
+static void mh_gates(const mh_ctx* x, int64_t bb, int64_t t, int64_t g, double* p) {
+  int64_t D = NB * x->H;
+  for (int k = 0; k < 3; ++k)
+    for (int i = 0; i < NB; ++i) p[k * NB + i] = x->P[IDXP(bb, t, k, g * NB + i, x->L, 3, D)];
+}
+
+static void mh_prev(const mh_ctx* x, int64_t bb, int64_t t, int64_t g, double* hp) {
+  int64_t D = NB * x->H;
+  for (int i = 0; i < NB; ++i)
+    hp[i] = (t == 0) ? (x->h0 ? x->h0[bb * D + g * NB + i] : 0.0)
+                     : x->h[IDX3(bb, t - 1, g * NB + i, x->L, D)];
+}
+
+static void rollout_mhgru_head(void* p, int64_t u) {
+  mh_ctx* x = (mh_ctx*)p;
+  int64_t bb = u / x->H, g = u % x->H, D = NB * x->H;
+  double hp[NB], f[NB], pg[3 * NB];
+  for (int64_t t = 0; t < x->L; ++t) {
+    mh_prev(x, bb, t, g, hp);
+    mh_gates(x, bb, t, g, pg);
+    oracle_mhgru_cell(pg, x->U + g * 3 * NB * NB, hp, f, NULL);
+    for (int i = 0; i < NB; ++i) x->h[IDX3(bb, t, g * NB + i, x->L, D)] = f[i];
+  }
+}
+
+/* U here is [3, H, 8, 8]; the cell wants one head's [3][8][8]: gather it. */
+static double* mh_heads(const double* U, int64_t H) {
+  double* Uh = (double*)malloc((size_t)H * 3 * NB * NB * sizeof(double));
+  for (int64_t g = 0; g < H; ++g)
+    for (int k = 0; k < 3; ++k)
+      for (int e = 0; e < NB * NB; ++e)
+        Uh[(g * 3 + k) * NB * NB + e] = U[((size_t)k * H + g) * NB * NB + e];
+  return Uh;
+}
+
+void oracle_rollout_mhgru(const double* P, const double* U, const double* h0, double* h,
+                          int64_t B, int64_t L, int64_t H) {
+  double* Uh = mh_heads(U, H);
+  mh_ctx x = {P, Uh, h0, h, NULL, NULL, NULL, L, H};
+  for_channels(B * H, rollout_mhgru_head, &x);
+  free(Uh);
+}
+
+static void newton_mhgru_residual_head(void* p, int64_t u) {
+  mh_ctx* x = (mh_ctx*)p;
+  int64_t bb = u / x->H, g = u % x->H, D = NB * x->H, L = x->L;
+  double hp[NB], f[NB], pg[3 * NB], m = 0.0;
+  for (int64_t t = 0; t < L; ++t) {
+    mh_prev(x, bb, t, g, hp);
+    mh_gates(x, bb, t, g, pg);
+    double* J = x->Jt + ((size_t)u * L + t) * NB * NB;
+    oracle_mhgru_cell(pg, x->U + g * 3 * NB * NB, hp, f, J);
+    for (int i = 0; i < NB; ++i) {
+      size_t k = IDX3(bb, t, g * NB + i, L, D);
+      x->rt[k] = f[i] - x->h[k];
+      double ar = fabs(x->rt[k]);
+      if (!(ar <= m)) m = ar; /* keeps a NaN */
+    }
+  }
+  x->cmax[u] = m;
+}
+
+static void newton_mhgru_solve_head(void* p, int64_t u) {
+  mh_ctx* x = (mh_ctx*)p;
+  int64_t bb = u / x->H, g = u % x->H, D = NB * x->H, L = x->L;
+  double delta[NB] = {0}, nd[NB];
+  for (int64_t t = 0; t < L; ++t) {
+    const double* J = x->Jt + ((size_t)u * L + t) * NB * NB;
+    for (int i = 0; i < NB; ++i) {
+      double s = x->rt[IDX3(bb, t, g * NB + i, L, D)];
+      for (int j = 0; j < NB; ++j) s += J[i * NB + j] * delta[j];
+      nd[i] = s;
+    }
+    for (int i = 0; i < NB; ++i) {
+      delta[i] = nd[i];
+      x->h[IDX3(bb, t, g * NB + i, L, D)] += delta[i];
+    }
+  }
+}
+
+/* Serial Newton as oracle_newton_gru, with 8x8 blocks: the linear solve is
+ * delta_t = J_t delta_{t-1} + r_t per head.  rho_hist has max_iters + 1 slots. */
+int oracle_newton_mhgru(const double* P, const double* U, const double* h0, double tol,
+                        int max_iters, int64_t B, int64_t L, int64_t H, double* h,
+                        double* rho_hist, int* converged, int* nonfinite) {
+  size_t N = (size_t)B * (size_t)L * (size_t)(NB * H);
+  double* Uh = mh_heads(U, H);
+  mh_ctx x = {P, Uh, h0, h, NULL, NULL, NULL, L, H};
+  x.Jt = (double*)malloc(N * NB * sizeof(double));
+  x.rt = (double*)malloc(N * sizeof(double));
+  x.cmax = (double*)malloc((size_t)(B * H) * sizeof(double));
+  int k;
+  *converged = 0;
+  *nonfinite = 0;
+  for (size_t i = 0; i < N; ++i) h[i] = 0.0;
+  for (k = 0;; ++k) {
+    for_channels(B * H, newton_mhgru_residual_head, &x);
+    double rho = reduce_rho(x.cmax, B * H, tol, k, NULL);
+    rho_hist[k] = rho;
+    if (!isfinite(rho)) {
+      *nonfinite = 1;
+      break;
+    }
+    if (rho <= tol) {
+      *converged = 1;
+      break;
+    }
+    if (k == max_iters) break;
+    for_channels(B * H, newton_mhgru_solve_head, &x);
+  }
+  free(x.Jt);
+  free(x.rt);
+  free(x.cmax);
+  free(Uh);
+  return k;
+}

@@ -23,6 +23,7 @@ deer     ParaGRU solve, fp32, DEER shape        16, 2^20, 1
 lm       ParaGRU solve, bf16 P, fp32 state      8, 8192, 4096
 proj     input projection x W^T (+bias), G=3    8, 4096, 1024, K = 1024
 proj_lm  input projection, LM width, G=3        8, 8192, 4096, K = 4096
+mhgru    multi-head GRU, 8x8 blocks, fp32       8, 4096, 1024 (128 heads)
 =======  =====================================  ==========================
 
 Distributions: projected gate inputs P ~ N(0, 1); diagonal recurrence weights
@@ -31,6 +32,8 @@ b ~ N(0, 1), h0 ~ N(0, 1).  Block scan: A entries ~ U(-0.5, 0.5), b ~ N(0, 1),
 x0 ~ N(0, 1).  Draw order: P (or A) first, then a (or b), then h0 (or x0).
 Backward passes: the forward workload's inputs, and upstream gradients
 dl/dh (and dl/dc) ~ N(0, 1) from their own generator.
+Multi-head GRU: U blocks ~ U(-0.3, 0.3) (so that each 8x8 block has norm
+below 1, like the diagonal a ~ U(-0.5, 0.5)).
 Input projection: x ~ N(0, 1) and W ~ N(0, 1/K), both rounded to bf16 once,
 bias ~ N(0, 0.1^2) fp32 (draw order x, W, bias), so that P = x W^T + bias has
 about the N(0, 1) spread of the solves' P.
@@ -49,6 +52,7 @@ WORKLOADS = {
     "lm": dict(op="gru", B=8, L=8192, D=4096, seed=5, bf16=True),
     "gru_bwd": dict(op="gru_bwd", B=8, L=4096, D=1024, seed=2, bf16=False),
     "lstm_bwd": dict(op="lstm_bwd", B=8, L=4096, D=1024, seed=3, bf16=False),
+    "mhgru": dict(op="mhgru", B=8, L=4096, D=1024, seed=8, bf16=False),
     "proj": dict(op="proj", B=8, L=4096, D=1024, K=1024, G=3, seed=6, bf16=False),
     "proj_lm": dict(op="proj", B=8, L=8192, D=4096, K=4096, G=3, seed=7, bf16=True),
 }
@@ -162,3 +166,14 @@ def projection_inputs(M, N, K, seed):
     w_bits, W = round_to_bf16(w32)
     bias = (_normal(rng, (N,)) * np.float32(0.1)).astype(np.float32)
     return dict(x=x, x_bits=x_bits, W=W, W_bits=w_bits, bias=bias)
+
+
+def mhgru_inputs(B, L, H, seed, u_scale=0.3, h0_normal=False):
+    """Multi-head GRU (dense 8x8 recurrence blocks): P [B, L, 3, 8H] ~ N(0, 1),
+    U [3, H, 8, 8] ~ U(-u_scale, u_scale), h0 zeros (or N(0, 1)).  Draw order P, U, h0."""
+    rng = _rng(seed)
+    D = 8 * H
+    P = _normal(rng, (B, L, 3, D))
+    U = _uniform(rng, -u_scale, u_scale, (3, H, 8, 8))
+    h0 = _normal(rng, (B, D)) if h0_normal else np.zeros((B, D), np.float32)
+    return dict(P=P, U=U, h0=h0)

@@ -46,6 +46,12 @@ MUTANTS = {
                                         "double dfdr = dfdu * w[2] * hp * r;"),
     "backward_lstm_untransposed_jacobian": ("mc = J[0] * lc + J[2] * lh;\n    mh = J[1] * lc + J[3] * lh;",
                                             "mc = J[0] * lc + J[1] * lh;\n    mh = J[2] * lc + J[3] * lh;"),
+    "mhgru_reset_gate_inside": ("double c = tanh(p[2 * NB + i] + r * uc[i]);",
+                                "double c = tanh(p[2 * NB + i] + uc[i]);"),
+    "mhgru_jacobian_drops_ur": ("uc[i] * r * (1.0 - r) * U[(1 * NB + i) * NB + j]);",
+                                "0.0 * U[(1 * NB + i) * NB + j]);"),
+    "mhgru_transposed_block": ("uz[i] += U[(0 * NB + i) * NB + j] * h[j];",
+                               "uz[i] += U[(0 * NB + j) * NB + i] * h[j];"),
     "projection_transposed_w": ("s += c->x[m * c->K + k] * c->W[n * c->K + k];",
                                 "s += c->x[m * c->K + k] * c->W[k * c->N + n];"),
     "projection_drops_bias": ("double s = c->bias ? c->bias[n] : 0.0;", "double s = 0.0;"),

@@ -586,3 +586,95 @@ def test_projection_matches_library_matmul(oracle):
     rng = np.random.default_rng(705)
     x, W, b = rng.standard_normal((33, 70)), rng.standard_normal((24, 70)), rng.standard_normal(24)
     assert np.allclose(oracle.input_projection(x, W, b), x @ W.T + b, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Multi-head GRU with dense 8x8 recurrence blocks
+# --------------------------------------------------------------------------
+def torch_mhgru_cell(U):
+    """GRUCell(3D -> D) whose hidden-to-hidden weights are block-diagonal with the
+    8x8 blocks of U [3, H, 8, 8]; x = [Pr, -Pz, Pc] as for ParaGRU (torch's z is
+    1 - z, so its z-row gets -U_z)."""
+    U = torch.as_tensor(np.asarray(U, np.float64))
+    H = U.shape[1]
+    D = 8 * H
+    bd = [torch.block_diag(*[U[g, k] for k in range(H)]) for g in range(3)]
+    cell = torch.nn.GRUCell(3 * D, D, bias=False).double()
+    with torch.no_grad():
+        cell.weight_ih.copy_(torch.eye(3 * D))
+        cell.weight_hh.copy_(torch.cat([bd[1], -bd[0], bd[2]]))
+    return cell
+
+
+def test_mhgru_cell_matches_torch_gru_cell(oracle):
+    rng = np.random.default_rng(720)
+    for _ in range(20):
+        U = rng.uniform(-0.8, 0.8, (3, 1, 8, 8))   # not symmetric: a transposed block fails
+        p = rng.standard_normal((3, 8)) * 2
+        h = rng.standard_normal(8)
+        f, J = oracle.mhgru_cell(p, U[:, 0], h)
+        cell = torch_mhgru_cell(U)
+        ht = torch.tensor(h[None, :], requires_grad=True)
+        out = torch_gru_step(cell, p[None], ht)
+        np.testing.assert_allclose(out.detach().numpy()[0], f, atol=1e-14, rtol=0)
+        Jt = torch.autograd.functional.jacobian(lambda x: torch_gru_step(cell, p[None], x), ht)
+        np.testing.assert_allclose(Jt.numpy().reshape(8, 8), J, atol=1e-12, rtol=0)
+
+
+def test_mhgru_rollout_matches_torch(oracle):
+    x = inputs.mhgru_inputs(2, 40, 3, seed=721, h0_normal=True)
+    cell = torch_mhgru_cell(x["U"])
+    h = torch.as_tensor(x["h0"].astype(np.float64))
+    ref = []
+    with torch.no_grad():
+        for t in range(40):
+            h = torch_gru_step(cell, x["P"][:, t], h)
+            ref.append(h)
+    ref = torch.stack(ref, 1).numpy()
+    np.testing.assert_allclose(oracle.rollout_mhgru(x["P"], x["U"], x["h0"]), ref, atol=1e-13,
+                               rtol=0)
+
+
+def test_mhgru_diagonal_blocks_are_paragru(oracle):
+    """With every block diagonal the cell, the rollout and Newton's iterates are
+    those of ParaGRU with a_g = the blocks' diagonals."""
+    x = inputs.gru_inputs(2, 60, 16, seed=722)
+    H = 2
+    U = np.zeros((3, H, 8, 8))
+    for g in range(3):
+        for k in range(H):
+            U[g, k] = np.diag(x["a"][g, 8 * k: 8 * k + 8])
+    np.testing.assert_allclose(oracle.rollout_mhgru(x["P"], U), oracle.rollout_gru(x["P"], x["a"]),
+                               atol=1e-14, rtol=0)
+    rm = oracle.newton_mhgru(x["P"], U)
+    rg = oracle.newton_gru(x["P"], x["a"])
+    assert rm.iterations == rg.iterations
+    np.testing.assert_allclose(rm.rho, rg.rho, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(rm.h, rg.h, atol=1e-14, rtol=0)
+
+
+def test_mhgru_newton_converges_to_rollout(oracle):
+    x = inputs.mhgru_inputs(2, 300, 2, seed=723, h0_normal=True)
+    res = oracle.newton_mhgru(x["P"], x["U"], x["h0"], tol=1e-12, max_iters=50)
+    assert res.converged
+    np.testing.assert_allclose(res.h, oracle.rollout_mhgru(x["P"], x["U"], x["h0"]), atol=1e-10,
+                               rtol=0)
+
+
+def test_mhgru_no_recurrence_single_iteration(oracle):
+    """U = 0: the gates do not depend on h, the step is affine in h, Newton is exact
+    after one update."""
+    x = inputs.mhgru_inputs(1, 100, 2, seed=724, h0_normal=True)
+    U = np.zeros_like(x["U"])
+    res = oracle.newton_mhgru(x["P"], U, x["h0"], tol=1e-12)
+    assert res.iterations == 1 and res.rho[1] < 1e-13
+
+
+def test_mhgru_prefix_exactness(oracle):
+    L = 6
+    x = inputs.mhgru_inputs(2, L, 2, seed=725, u_scale=0.6, h0_normal=True)
+    ref = oracle.rollout_mhgru(x["P"], x["U"], x["h0"])
+    for k in range(1, L + 1):
+        res = oracle.newton_mhgru(x["P"], x["U"], x["h0"], tol=0.0, max_iters=k)
+        assert res.iterations == k
+        np.testing.assert_allclose(res.h[:, :k], ref[:, :k], atol=1e-13, rtol=0)
