@@ -37,6 +37,10 @@ UNIT = "channel-steps/s"
 MUFU_PER_SM_PER_CLK = 16        # ex2 / rcp issue rate per SM per clock
 SMS = 148
 MUFU_PER_STEP = {"gru": 6, "lstm": 10}   # (ex2 + rcp) per sigmoid/tanh, per channel-step
+FMA_PER_SM_PER_CLK = 128        # fp32 FMA lanes per SM
+# multi-head GRU, per channel-step and Newton evaluation: gate matvecs 24 +
+# Jacobian 24 + b_t 8 + map composition (8x8 product + matvec) 72 = 128 FMA
+MHGRU_FMA_PER_STEP = 128
 
 
 def peaks():
@@ -200,6 +204,8 @@ def algorithmic_bytes(op, bf16, B, L, D, passes=1):
         return 32 * N
     if op == "proj":      # handled by projection_bytes (depends on K and G)
         raise ValueError("use projection_bytes for the input projection")
+    if op == "mhgru":     # one evaluation: read P, the iterate, write the iterate
+        return N * (12 + 4 + 4) * passes
     if op == "gru_bwd":   # read P, h_{t-1}, dl/dh; write dP
         return N * (3 * (2 if bf16 else 4) + 4 + 4 + 12)
     if op == "lstm_bwd":  # read P, (c, h)_{t-1}, dl/dc, dl/dh; write dP
@@ -301,6 +307,10 @@ class Case:
                 self.host["h"] = hs.cpu()
             G = 3 if cell == "gru" else 4
             self.out_shapes = [(B, L, G, D), (G, D), (B, D)] + ([(B, D)] if cell == "lstm" else [])
+        elif self.op == "mhgru":
+            x = inputs.mhgru_inputs(B, L, D // 8, seed)
+            self.host = {"P": torch.from_numpy(x["P"]), "U": torch.from_numpy(x["U"])}
+            self.out_shapes = [(B, L, D)]
         elif self.op in ("gru", "lstm"):
             x = (inputs.gru_inputs if self.op == "gru" else inputs.lstm_inputs)(B, L, D, seed,
                                                                                   self.bf16)
@@ -334,6 +344,9 @@ class Case:
         elif op == "lstm":
             pr.solve_lstm(d["P"], d["a"], d["c0"], d["h0"], self.tol, self.max_iters,
                           out=(outs[0], outs[1]), info=self.info_t)
+        elif op == "mhgru":
+            pr.solve_mhgru(d["P"], d["U"], None, self.tol, self.max_iters, out=outs[0],
+                           info=self.info_t)
         elif op == "proj":
             pr.input_projection(d["x"], d["W"], d["bias"], out=outs[0], out_dtype=self.out_dtype)
         elif op == "gru_bwd":
@@ -351,7 +364,7 @@ class Case:
         self.run(self.dev, self.outs)
 
     def solve_info(self):
-        if self.op in ("gru", "lstm"):
+        if self.op in ("gru", "lstm", "mhgru"):
             return self.pr.SolveInfo(self.info_t)
         return None
 
@@ -440,6 +453,18 @@ def run_ours(args, world, rank, local):
         else:
             roofline = dict(hbm)
             roofline["alu"] = {k: alu[k] for k in ("achieved", "peak", "unit", "frac")}
+    elif op == "mhgru":
+        ev_iters = (iters or 0) + 1
+        sm_mhz = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
+        flops = 2.0 * N * ev_iters * MHGRU_FMA_PER_STEP
+        fpeak = SMS * FMA_PER_SM_PER_CLK * 2 * sm_mhz * 1e6 / 1e12
+        ach = flops / (launch_ms * 1e-3) / 1e12
+        roofline = {"bound": "alu", "achieved": ach, "peak": fpeak,
+                    "unit": "TFLOP/s (fp32 FMA, CUDA cores)", "frac": ach / fpeak,
+                    "traffic": traffic, "flops_per_launch": flops,
+                    "peak_kind": "derived: 148 SMs x 128 FMA/clk x 2 x sampled SM clock",
+                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": hbm_frac}}
     elif op == "proj":
         ev_iters = None
         flops = 2.0 * (B * L) * (cs.G * D) * cs.K
@@ -461,7 +486,8 @@ def run_ours(args, world, rank, local):
                           "scan_block2": "pararnn scan (2x2)",
                           "gru_bwd": "pararnn backward kernel (GRU)",
                           "lstm_bwd": "pararnn backward kernel (LSTM)",
-                          "proj": "pararnn input projection (tcgen05)"}[op]
+                          "proj": "pararnn input projection (tcgen05)",
+                          "mhgru": "pararnn multi-head GRU Newton kernel (8x8 blocks)"}[op]
     roofline["launch_ms"] = launch_ms
     roofline["traffic_source"] = traffic_src
 
@@ -592,6 +618,7 @@ def run_ours(args, world, rank, local):
               "block2": "2x2 block affine scan fp32",
               "gru_bwd": "ParaGRU backward pass fp32",
               "lstm_bwd": "ParaLSTM backward pass fp32",
+              "mhgru": "multi-head GRU Newton solve fp32, dense 8x8 recurrence blocks",
               "proj": "input projection x W^T + bias, bf16 in, fp32 out (tcgen05)",
               "proj_lm": "input projection x W^T + bias, bf16 in, bf16 out (tcgen05)",
               }[args.workload]
@@ -602,7 +629,7 @@ def run_ours(args, world, rank, local):
                "parallelism": f"replicas x{world} (independent batches)",
                "l2": "inputs larger than L2 (%.0f MB per step), no flush needed" % (
                    sum(v.numel() * v.element_size() for v in cs.host.values()) / 1e6)}
-        if op in ("gru", "lstm"):
+        if op in ("gru", "lstm", "mhgru"):
             cfg.update({"tol": cs.tol, "max_iters": cs.max_iters, "newton_iterations": iters,
                         "sweeps": passes, "evaluated_iterations": ev_iters})
         line = {
@@ -647,6 +674,18 @@ def cpu_baseline(x, op, B, L, D, budget_s=15.0):
                 "kind": "oracle",
                 "sample": f"fp64 projection of {nrows} of {x['x'].shape[0]} rows "
                           f"(N={Nf}, K={Wd.shape[1]}; {dt:.1f} s)"}
+    if op == "mhgru":
+        # whole heads of one batch row, as many as fit the budget
+        t0 = time.perf_counter()
+        oracle.newton_mhgru(x["P"][:1, :, :, :8], x["U"][:, :1])
+        per_head = max(time.perf_counter() - t0, 1e-6)
+        nh = int(max(1, min(D // 8, budget_s / per_head)))
+        t0 = time.perf_counter()
+        res = oracle.newton_mhgru(x["P"][:1, :, :, :8 * nh], x["U"][:, :nh])
+        dt = time.perf_counter() - t0
+        return {"value": L * 8 * nh / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"serial fp64 Newton, B=1 x {nh} heads x L={L} "
+                          f"({res.iterations} iterations, {dt:.1f} s)"}
     if op in ("gru_bwd", "lstm_bwd"):
         nb = 1
         nd = min(D, 256)
@@ -738,6 +777,15 @@ def run_reference(args, world, rank, local):
                 return oracle.backward_lstm(Ps, as_, cc, hh, g[1], g[0])
         what = "adjoint (backward) recursion"
         x = None
+    elif op == "mhgru":
+        x = inputs.mhgru_inputs(B, L, D // 8, w["seed"])
+        nd = min(D, 32)
+        Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
+        Us = np.ascontiguousarray(x["U"][:, : nd // 8])
+
+        def step():
+            return oracle.newton_mhgru(Ps, Us)
+        what = "serial fp64 Newton (8x8 blocks)"
     elif op == "proj":
         Nf, K = w["G"] * D, w["K"]
         x = inputs.projection_inputs(B * L, Nf, K, w["seed"])
@@ -749,7 +797,7 @@ def run_reference(args, world, rank, local):
         what = f"fp64 input projection ({nrows} rows x N={Nf} x K={K})"
     else:
         x = inputs.workload_inputs(args.workload)  # the same draws as the GPU arm, then sliced
-    if op in ("gru_bwd", "lstm_bwd", "proj"):
+    if op in ("gru_bwd", "lstm_bwd", "proj", "mhgru"):
         pass
     elif op in ("gru", "lstm"):
         Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
@@ -801,7 +849,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gru_l",
                     choices=["gru_l", "lm", "deer", "gru_s", "lstm", "scan", "block2",
-                             "gru_bwd", "lstm_bwd", "proj", "proj_lm"])
+                             "gru_bwd", "lstm_bwd", "proj", "proj_lm", "mhgru"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-scan", action="store_true", help="skip the scan leg (gru_l)")

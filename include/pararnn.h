@@ -67,7 +67,8 @@ typedef enum {
   PARARNN_OP_GRU = 2,
   PARARNN_OP_LSTM = 3,
   PARARNN_OP_GRU_BACKWARD = 4,
-  PARARNN_OP_LSTM_BACKWARD = 5
+  PARARNN_OP_LSTM_BACKWARD = 5,
+  PARARNN_OP_MHGRU = 6
 } pararnn_op_t;
 
 /* Device-side outcome of a solve (caller-owned DEVICE memory, written by the
@@ -238,6 +239,25 @@ pararnn_status_t pararnn_rollout_gru(const void* P, pararnn_dtype_t p_dtype, con
 pararnn_status_t pararnn_rollout_lstm(const void* P, pararnn_dtype_t p_dtype, const float* a,
                                       const float* c0, const float* h0, float* c, float* h,
                                       int64_t B, int64_t L, int64_t D, void* stream);
+
+/* Newton solve of the multi-head GRU whose recurrence is block-diagonal with
+ * dense 8x8 blocks, one per head of 8 channels (the dense-block case that the
+ * DEER summary's caveats price at O(n^3) per step).  Per head, elementwise:
+ *   z = sig(P_z + U_z h), r = sig(P_r + U_r h), c = tanh(P_c + r (U_c h)),
+ *   h' = (1 - z) h + z c   -- the ParaGRU cell when every block is diagonal.
+ * Same method, stopping rule, info and status semantics as pararnn_solve_gru;
+ * each Newton step solves a block bi-diagonal system with dense 8x8 blocks.
+ *   P  : [B, L, 3, D] (z, r, c), fp32 or bf16, D = 8 H, 16-byte aligned;
+ *   U  : [3, H, 8, 8] fp32: gate, head, row (output channel), column (input);
+ *   h0 : [B, D] or NULL (= 0);  h : [B, L, D], 16-byte aligned: the iterate,
+ *        updated in place, and the result (must not overlap P, U or h0);
+ *   ws : pararnn_workspace_size(PARARNN_OP_MHGRU, B, L, 8 H, max_iters, opts).
+ * The kernel is cooperative (every CTA resident), one warp per (b, head). */
+pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p_dtype, const float* U,
+                                     const float* h0, float* h, int64_t B, int64_t L,
+                                     int64_t H, float tol, int32_t max_iters, void* ws,
+                                     size_t ws_bytes, pararnn_solve_info_t* info,
+                                     const pararnn_options_t* opts, void* stream);
 
 /* Input projection P = x W^T + bias on the tensor cores (tcgen05, bf16 inputs,
  * fp32 accumulation): the projected gate pre-activations that the cells take

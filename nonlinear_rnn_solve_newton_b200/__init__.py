@@ -36,6 +36,7 @@ library_path = os.path.join(_HERE, "libpararnn.so")
 
 OP_SCAN_DIAG, OP_SCAN_BLOCK2, OP_GRU, OP_LSTM = 0, 1, 2, 3
 OP_GRU_BACKWARD, OP_LSTM_BACKWARD = 4, 5
+OP_MHGRU = 6
 F32, BF16 = 0, 1
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA runtime error",
@@ -127,6 +128,10 @@ def load(build_if_missing: bool = True):
                                                       _i64, _i64, ctypes.c_float, ctypes.c_int32,
                                                       _vp, _vp, _vp]
             lib.pararnn_solve_gru_noalloc.restype = ctypes.c_int
+            lib.pararnn_solve_mhgru.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64, _i64,
+                                                _i64, ctypes.c_float, ctypes.c_int32, _vp,
+                                                ctypes.c_size_t, _vp, _vp, _vp]
+            lib.pararnn_solve_mhgru.restype = ctypes.c_int
             lib.pararnn_input_projection.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i64,
                                                      _i64, _i64, _vp, _vp]
             lib.pararnn_input_projection.restype = ctypes.c_int
@@ -302,6 +307,33 @@ def solve_gru(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
                                ctypes.byref(opts) if opts is not None else None,
                                _stream_handle(stream))
     _raise(st, "pararnn_solve_gru")
+    return h, SolveInfo(info)
+
+
+def solve_mhgru(P, U, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
+                opts: Options | None = None, stream=None):
+    """Multi-head GRU (dense 8x8 recurrence blocks) Newton solve.  P [B, L, 3, D]
+    (z, r, c), U [3, H, 8, 8] with D = 8 H -> (h [B, L, D], SolveInfo)."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 3 or U.dim() != 4 or tuple(U.shape[2:]) != (8, 8) or D != 8 * U.shape[1]:
+        raise ValueError("P must be [B, L, 3, 8 H] and U [3, H, 8, 8]")
+    H = U.shape[1]
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 3, D))
+    _check_dev("U", U, torch.float32, (3, H, 8, 8))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    h = torch.empty((B, L, D), dtype=torch.float32, device=P.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, L, D))
+    if info is None:
+        info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    n = workspace_size(OP_MHGRU, B, L, D, max_iters, opts)
+    ws = _workspace(n, P.device)
+    st = lib.pararnn_solve_mhgru(_ptr(P), dt, _ptr(U), _ptr(h0), _ptr(h), B, L, H, float(tol),
+                                 int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
+                                 ctypes.byref(opts) if opts is not None else None,
+                                 _stream_handle(stream))
+    _raise(st, "pararnn_solve_mhgru")
     return h, SolveInfo(info)
 
 

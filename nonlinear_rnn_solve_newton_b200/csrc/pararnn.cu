@@ -17,6 +17,7 @@
 #include "pararnn_bwd.cuh"
 #include "pararnn_bwd_walk.cuh"
 #include "pararnn_kernel.cuh"
+#include "pararnn_mhgru.cuh"
 #include "pararnn_proj.cuh"
 #include "pararnn_seq.cuh"
 #include "pararnn_walk.cuh"
@@ -680,6 +681,10 @@ const char* pararnn_status_string(pararnn_status_t s) {
 
 size_t pararnn_workspace_size(pararnn_op_t op, int64_t B, int64_t L, int64_t D, int32_t max_iters,
                               const pararnn_options_t* opts) {
+  if ((int)op == 6) {  // multi-head GRU: control block + one residual word per iteration
+    if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return 0;
+    return (sizeof(Ctrl) + 4 * (size_t)(max_iters + 1) + 255) / 256 * 256;
+  }
   if ((int)op < 0 || (int)op > 5) return 0;
   if (B == 0 || L == 0 || D == 0) return 256;
   Plan pl = make_plan((int)op, B, L, D, max_iters, opts);
@@ -1134,6 +1139,83 @@ extern "C" pararnn_status_t pararnn_input_projection(const void* x, const void* 
   const unsigned grid = (unsigned)(ntiles < resident ? ntiles : resident);
   void* args[] = {&pp, &tm};
   if (cudaLaunchKernel(fn, dim3(grid), dim3(kProjThreads), args, smem, st) != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  return PARARNN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Multi-head GRU (dense 8x8 blocks).
+// ---------------------------------------------------------------------------
+extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p_dtype,
+                                                const float* U, const float* h0, float* h,
+                                                int64_t B, int64_t L, int64_t H, float tol,
+                                                int32_t max_iters, void* ws, size_t ws_bytes,
+                                                pararnn_solve_info_t* info,
+                                                const pararnn_options_t* opts, void* stream) {
+  if (B < 0 || L < 0 || H < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!info || !aligned(info, 4)) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!(tol >= 0.0f)) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (p_dtype != PARARNN_F32 && p_dtype != PARARNN_BF16) return PARARNN_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (B == 0 || L == 0 || H == 0) {
+    empty_info_kernel<<<1, 1, 0, st>>>(info);
+    return cudaGetLastError() == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA;
+  }
+  if (!P || !U || !h) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!aligned(P, 16) || !aligned(U, 4) || !aligned(h, 16) || (h0 && !aligned(h0, 4)))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+  if (B * H > (1LL << 40) || L > (1LL << 40)) return PARARNN_ERR_INVALID_ARGUMENT;
+  const size_t need = pararnn_workspace_size(PARARNN_OP_MHGRU, B, L, 8 * H, max_iters, opts);
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return PARARNN_ERR_WORKSPACE;
+
+  const void* fn = p_dtype == PARARNN_BF16
+                       ? (const void*)pararnn_mhgru_kernel<__nv_bfloat16>
+                       : (const void*)pararnn_mhgru_kernel<float>;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_UNSUPPORTED;
+  }
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMhSmem) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  int resident = 0;
+  if (resident_ctas(fn, 32 * kMhWarps, kMhSmem, &resident) != cudaSuccess || resident <= 0) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  const long long units = B * H;
+  const long long want = (units + kMhWarps - 1) / kMhWarps;
+  const int grid = (int)(want < resident ? want : resident);
+
+  MhParams mp;
+  mp.P = P;
+  mp.U = U;
+  mp.h0 = h0;
+  mp.h = h;
+  mp.B = B;
+  mp.L = L;
+  mp.H = H;
+  mp.tol = tol;
+  mp.max_iters = max_iters;
+  mp.ctrl = static_cast<Ctrl*>(ws);
+  mp.rho_bits = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + sizeof(Ctrl));
+  mp.info = info;
+  mp.status_dev = nullptr;
+  mp.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? opts->wait_timeout_ns : 1000000000LL;
+  if (cudaMemsetAsync(ws, 0, need, st) != cudaSuccess) return PARARNN_ERR_CUDA;
+  // no update at all: the result is the initial iterate h^0 = 0
+  if (max_iters == 0 &&
+      cudaMemsetAsync(h, 0, sizeof(float) * (size_t)(B * L * 8 * H), st) != cudaSuccess)
+    return PARARNN_ERR_CUDA;
+  void* args[] = {&mp};
+  if (cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(32 * kMhWarps), args, kMhSmem, st) !=
+      cudaSuccess) {
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }

@@ -1,0 +1,130 @@
+"""Parity of the multi-head GRU Newton solve (dense 8x8 recurrence blocks) with
+the fp64 oracle, through the C ABI.
+
+Tolerance as for the diagonal solves: the trajectory within 1e-4 (max-abs) of
+the oracle's fp64 rollout once converged at tol = 1e-4; the iteration count
+within one of the oracle's serial Newton (rho_k near tol under fp32 rounding);
+an unconverged iterate h^k against the oracle's h^k within 1e-4.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pr():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import nonlinear_rnn_solve_newton_b200 as m
+
+    m.load()
+    return m
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+
+
+# (B, L, H): one chunk, a chunk boundary with a 1-step tail (chunk = 512 steps),
+# several chunks, one head, a single step, more sequences than one CTA holds
+SHAPES = [(2, 100, 2), (1, 513, 3), (2, 1500, 4), (3, 37, 1), (2, 1, 2), (4, 300, 9)]
+
+
+@pytest.mark.parametrize("h0_normal", [False, True])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_mhgru_matches_rollout(pr, shape, h0_normal):
+    B, L, H = shape
+    x = inputs.mhgru_inputs(B, L, H, seed=[800, B, L, H], h0_normal=h0_normal)
+    h, info = pr.solve_mhgru(dev(x["P"]), dev(x["U"]), dev(x["h0"]) if h0_normal else None)
+    torch.cuda.synchronize()
+    ref = oracle.rollout_mhgru(x["P"], x["U"], x["h0"])
+    res = oracle.newton_mhgru(x["P"], x["U"], x["h0"])
+    assert info.status == 0 and info.converged
+    assert abs(info.iterations - res.iterations) <= 1
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
+
+
+def test_mhgru_bf16_inputs(pr):
+    B, L, H = 2, 700, 3
+    x = inputs.mhgru_inputs(B, L, H, seed=801)
+    bits, vals = inputs.round_to_bf16(x["P"])
+    P16 = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    h, info = pr.solve_mhgru(P16, dev(x["U"]))
+    torch.cuda.synchronize()
+    assert info.converged
+    assert np.max(np.abs(h.cpu().numpy() - oracle.rollout_mhgru(vals, x["U"]))) <= 1e-4
+
+
+def test_mhgru_diagonal_blocks_match_paragru_solve(pr):
+    """Diagonal blocks: the multi-head solve and the ParaGRU solve agree."""
+    B, L, D = 2, 800, 32
+    x = inputs.gru_inputs(B, L, D, seed=802)
+    H = D // 8
+    U = np.zeros((3, H, 8, 8), np.float32)
+    for g in range(3):
+        for k in range(H):
+            U[g, k] = np.diag(x["a"][g, 8 * k: 8 * k + 8])
+    hm, im = pr.solve_mhgru(dev(x["P"]), dev(U))
+    hg, ig = pr.solve_gru(dev(x["P"]), dev(x["a"]))
+    torch.cuda.synchronize()
+    assert abs(im.iterations - ig.iterations) <= 1
+    assert np.max(np.abs(hm.cpu().numpy() - hg.cpu().numpy())) <= 1e-4
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_mhgru_unconverged_iterate(pr, k):
+    """tol = 0 and max_iters = k: the result is Newton's h^k."""
+    B, L, H = 2, 600, 2
+    x = inputs.mhgru_inputs(B, L, H, seed=[803, k], h0_normal=True)
+    h, info = pr.solve_mhgru(dev(x["P"]), dev(x["U"]), dev(x["h0"]), tol=0.0, max_iters=k)
+    torch.cuda.synchronize()
+    res = oracle.newton_mhgru(x["P"], x["U"], x["h0"], tol=0.0, max_iters=k)
+    assert info.iterations == k and not info.converged and info.updates == k
+    assert np.max(np.abs(h.cpu().numpy() - res.h)) <= 1e-4
+    np.testing.assert_allclose(info.rho[: k + 1], res.rho, rtol=1e-3, atol=1e-6)
+
+
+def test_mhgru_zero_iterations_returns_h0_iterate(pr):
+    x = inputs.mhgru_inputs(1, 50, 1, seed=804)
+    h, info = pr.solve_mhgru(dev(x["P"]), dev(x["U"]), max_iters=0)
+    torch.cuda.synchronize()
+    assert info.iterations == 0 and info.updates == 0
+    assert not h.cpu().numpy().any()
+
+
+def test_mhgru_nonfinite_reported(pr):
+    x = inputs.mhgru_inputs(1, 200, 2, seed=805)
+    x["P"][0, 77, 1, 3] = np.nan
+    h, info = pr.solve_mhgru(dev(x["P"]), dev(x["U"]))
+    torch.cuda.synchronize()
+    assert info.status == 5 and not info.converged
+
+
+def test_mhgru_empty(pr):
+    P = torch.empty((0, 10, 3, 16), device="cuda")
+    U = torch.zeros((3, 2, 8, 8), device="cuda")
+    h, info = pr.solve_mhgru(P, U)
+    torch.cuda.synchronize()
+    assert info.converged and info.iterations == 0
+
+
+def test_mhgru_full_size_sampled_heads(pr):
+    """The multi-head workload at full size (B = 8, L = 4096, 128 heads), a
+    sample of (batch row, head) sequences against the oracle's rollout."""
+    w = inputs.WORKLOADS["mhgru"]
+    B, L, D = w["B"], w["L"], w["D"]
+    H = D // 8
+    x = inputs.mhgru_inputs(B, L, H, seed=w["seed"])
+    h, info = pr.solve_mhgru(dev(x["P"]), dev(x["U"]))
+    torch.cuda.synchronize()
+    assert info.converged
+    hc = h.cpu().numpy()
+    rng = np.random.default_rng(806)
+    for b, g in zip(rng.integers(0, B, 6), rng.integers(0, H, 6)):
+        ref = oracle.rollout_mhgru(x["P"][b:b + 1, :, :, 8 * g: 8 * g + 8], x["U"][:, g:g + 1])
+        assert np.max(np.abs(hc[b:b + 1, :, 8 * g: 8 * g + 8] - ref)) <= 1e-4
