@@ -1174,6 +1174,8 @@ extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p
   const void* fn = p_dtype == PARARNN_BF16
                        ? (const void*)pararnn_mhgru_kernel<__nv_bfloat16>
                        : (const void*)pararnn_mhgru_kernel<float>;
+  const size_t kMhSmem = p_dtype == PARARNN_BF16 ? mh_smem_bytes<__nv_bfloat16>()
+                                                 : mh_smem_bytes<float>();
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();

@@ -23,36 +23,46 @@
 //   C. each lane recomputes its steps' maps and applies them from that state,
 //      writing h^{k+1} over h^k (the chunk's h^k was staged in shared memory
 //      first, so no lane reads an overwritten value).
-// The chunk's gate inputs are staged in shared memory too, by coalesced loads
-// that are all in flight at once, so neither phase waits on global memory.
+// The chunk's gates and h^k arrive by cp.async copies into one of two
+// shared-memory buffers while the previous chunk is being processed.
 #pragma once
 
 #include "pararnn_kernel.cuh"
+#include "pararnn_walk.cuh"
 
-// Steps per lane and sequences per CTA, measured on B200 at B=8, L=4096,
-// 128 heads (4 x 4 with staged gates: 4.1 ms; 8-16 steps: 4.8 ms; 32: 8.4 ms).
+// Steps per lane and sequences per CTA, measured on B200 at B=8, L=4096, 128
+// heads: 6 x 4, one buffer: 2.65 ms; 4 x 4: 3.2 ms; 8 x 4: 3.8 ms; two buffers
+// (3 x 4): 2.85 ms -- the second buffer costs more occupancy than it hides.
 #ifndef PARARNN_MH_STEPS
-#define PARARNN_MH_STEPS 4
+#define PARARNN_MH_STEPS 6
 #endif
 #ifndef PARARNN_MH_WARPS
 #define PARARNN_MH_WARPS 4
 #endif
-#ifndef PARARNN_MH_STAGE_P
-#define PARARNN_MH_STAGE_P 1
+// 1: the next chunk's copies are in flight while this one is processed (two
+// buffers per warp); 0: one buffer, filled at the start of each chunk.
+#ifndef PARARNN_MH_ASYNC
+#define PARARNN_MH_ASYNC 0
 #endif
 
 namespace pararnn {
 
-constexpr int kMhS = PARARNN_MH_STEPS;  // steps per lane per chunk
+constexpr int kMhS = PARARNN_MH_STEPS;      // steps per lane per chunk
 constexpr int kMhWarps = PARARNN_MH_WARPS;  // sequences (warps) per CTA
 constexpr int kMhT = 32 * kMhS;             // steps per chunk
-// dynamic shared memory per warp: h^k of the chunk ((T + 1) x 8) and its gates (T x 24)
-constexpr bool kMhStageP = PARARNN_MH_STAGE_P != 0;
-constexpr size_t kMhWarpFloats = (size_t)(kMhT + 1) * 8 + (kMhStageP ? (size_t)kMhT * 24 : 0);
-constexpr size_t kMhSmem = (size_t)kMhWarps * kMhWarpFloats * sizeof(float);
+constexpr int kMhHkFloats = (kMhT + 1) * 8;  // h^k of a chunk: row 0 = the step before it
+constexpr int kMhBufs = PARARNN_MH_ASYNC ? 2 : 1;
+
+// Dynamic shared memory per warp: one or two buffers of (h^k rows, gates of the chunk).
+template <typename PT> __host__ __device__ constexpr size_t mh_buf_bytes() {
+  return (size_t)kMhHkFloats * 4 + (size_t)kMhT * 24 * sizeof(PT);
+}
+template <typename PT> __host__ __device__ constexpr size_t mh_smem_bytes() {
+  return (size_t)kMhWarps * kMhBufs * mh_buf_bytes<PT>();
+}
 
 struct MhParams {
-  const void* P;       // [B, L, 3, D] (z, r, c), fp32 or bf16; D = 8 H
+  const void* P;       // [B, L, 3, D] (z, r, c), fp32 or bf16; D = 8 H; 16-byte aligned
   const float* U;      // [3, H, 8, 8]: gate, head, row (output), column (input)
   const float* h0;     // [B, D] or NULL (= 0)
   float* h;            // [B, L, D]: the iterate, updated in place; the result
@@ -66,17 +76,41 @@ struct MhParams {
   long long timeout_ns;
 };
 
-// Cell and Jacobian of one head at h (row-major J[i][j] = dh'_i / dh_j).
-__device__ __forceinline__ void mh_cell(const float* p, const float (*U)[8][8], const float* h,
-                                        float* f, float (*J)[8]) {
+// 16-byte asynchronous copy global -> shared; with valid == false it writes
+// zeros and reads nothing.
+__device__ __forceinline__ void cp_async16(unsigned dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Cell and Jacobian of one head at h (row-major J[i][j] = dh'_i / dh_j).  U is
+// the head's blocks in shared memory (16-byte aligned rows); each row of the
+// three blocks is read once, as float4, for both the product and the Jacobian.
+__device__ __forceinline__ void mh_cell(const float* p, const float* U, const float* h, float* f,
+                                        float (*J)[8]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
+    float u[3][8];
+#pragma unroll
+    for (int gt = 0; gt < 3; ++gt) {
+      const float4 a = reinterpret_cast<const float4*>(U + (gt * 8 + i) * 8)[0];
+      const float4 c = reinterpret_cast<const float4*>(U + (gt * 8 + i) * 8)[1];
+      u[gt][0] = a.x; u[gt][1] = a.y; u[gt][2] = a.z; u[gt][3] = a.w;
+      u[gt][4] = c.x; u[gt][5] = c.y; u[gt][6] = c.z; u[gt][7] = c.w;
+    }
     float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      uz = fmaf(U[0][i][j], h[j], uz);
-      ur = fmaf(U[1][i][j], h[j], ur);
-      uc = fmaf(U[2][i][j], h[j], uc);
+      uz = fmaf(u[0][j], h[j], uz);
+      ur = fmaf(u[1][j], h[j], ur);
+      uc = fmaf(u[2][j], h[j], uc);
     }
     const float z = sigm(p[i] + uz);
     const float r = sigm(p[8 + i] + ur);
@@ -87,75 +121,53 @@ __device__ __forceinline__ void mh_cell(const float* p, const float (*U)[8][8], 
     const float db = q * r;
     const float dc = q * uc * r * (1.0f - r);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      J[i][j] = fmaf(da, U[0][i][j], fmaf(db, U[2][i][j], dc * U[1][i][j]));
+    for (int j = 0; j < 8; ++j) J[i][j] = fmaf(da, u[0][j], fmaf(db, u[2][j], dc * u[1][j]));
     J[i][i] += 1.0f - z;
   }
 }
 
+// Issue the copies of chunk t0 into one buffer: h^k of steps t0 .. t0 + T - 1
+// into rows 1..T (zeros at k = 0, where h^0 = 0, and past L) and their gates.
 template <typename PT>
-__device__ __forceinline__ void mh_load_gates(const PT* P, long long row, long long D, int g,
-                                              float* p) {
-  const PT* q = P + row * 3 * D + 8 * g;
-#pragma unroll
-  for (int k = 0; k < 3; ++k)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) p[8 * k + i] = to_f(__ldg(q + k * D + i));
-}
-
-// Stage the gates of steps t0 .. t0 + T - 1 of head g, batch row b into
-// sp[s][24] (z, r, c x 8 channels); steps past L are zero.
-template <typename PT>
-__device__ __forceinline__ void mh_stage_gates(const PT* P, long long b, long long t0, long long L,
-                                               long long D, int g, float* sp, int lane) {
-  if constexpr (sizeof(PT) == 4) {
-    // 6 float4 per step (3 gates x 8 channels)
-    for (int e = lane; e < kMhT * 6; e += 32) {
-      const int s = e / 6, q = e - 6 * s;  // q: gate = q / 2, half = q % 2
-      const long long t = t0 + s;
-      float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      if (t < L)
-        v = __ldg(reinterpret_cast<const float4*>(P + ((b * L + t) * 3 + (q >> 1)) * D + 8 * g) +
-                  (q & 1));
-      reinterpret_cast<float4*>(sp)[e] = v;
-    }
-  } else {
-    // 3 x 16 bytes (8 bf16) per step
-    for (int e = lane; e < kMhT * 3; e += 32) {
-      const int s = e / 3, gate = e - 3 * s;
-      const long long t = t0 + s;
-      float f[8];
-      if (t < L) {
-        const uint4 v =
-            __ldg(reinterpret_cast<const uint4*>(P + ((b * L + t) * 3 + gate) * D + 8 * g));
-        const unsigned w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          f[2 * i] = __uint_as_float(w[i] << 16);
-          f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.0f;
-      }
-      float4* d = reinterpret_cast<float4*>(sp + 24 * s + 8 * gate);
-      d[0] = make_float4(f[0], f[1], f[2], f[3]);
-      d[1] = make_float4(f[4], f[5], f[6], f[7]);
-    }
+__device__ __forceinline__ void mh_issue_chunk(const MhParams& p, const PT* P, long long b, int g,
+                                               long long D, long long t0, int k, float* hkb,
+                                               PT* spb, int lane) {
+  for (int e = lane; e < kMhT * 2; e += 32) {
+    const int s = e >> 1, half = e & 1;
+    const long long t = t0 + s;
+    const bool valid = k > 0 && t < p.L;
+    const float* src = valid ? p.h + (b * p.L + t) * D + 8 * g + 4 * half : p.h;
+    cp_async16(smem_u32(hkb + 8 + 8 * s + 4 * half), src, valid);
   }
+  constexpr int per = 24 * (int)sizeof(PT) / 16;  // 16-byte pieces per step (6 or 3)
+  for (int e = lane; e < kMhT * per; e += 32) {
+    const int s = e / per, q = e - per * s;
+    const long long t = t0 + s;
+    const bool valid = t < p.L;
+    // piece q covers gate (q * 16 / sizeof(PT)) / 8, channels from (q * 16 / sizeof(PT)) % 8
+    const int first = q * 16 / (int)sizeof(PT);
+    const PT* src = valid ? P + ((b * p.L + t) * 3 + first / 8) * D + 8 * g + (first % 8) : P;
+    cp_async16(smem_u32(spb + 24 * s + first), src, valid);
+  }
+  cp_async_commit();
 }
 
 template <typename PT>
 __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const MhParams p) {
-  __shared__ float s_U[kMhWarps][3][8][8];
-  // per warp, h^k of the chunk: row 0 = the step before it, row s + 1 = step s
-  extern __shared__ float s_hk[];
+  __shared__ __align__(16) float s_U[kMhWarps][3 * 64];
+  extern __shared__ __align__(16) unsigned char s_dyn[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long D = 8 * p.H;
   const long long nunits = p.B * p.H;
   const WaitCtx wctx{p.ctrl, p.status_dev, p.timeout_ns};
-  const PT* P = static_cast<const PT*>(p.P);  // 16-byte aligned rows of 8 channels
+  const PT* P = static_cast<const PT*>(p.P);
+  unsigned char* wbase = s_dyn + (size_t)warp * kMhBufs * mh_buf_bytes<PT>();
+  // buffer j: h^k rows, then the gates
+  auto hkbuf = [&](int j) { return reinterpret_cast<float*>(wbase + j * mh_buf_bytes<PT>()); };
+  auto spbuf = [&](int j) {
+    return reinterpret_cast<PT*>(wbase + j * mh_buf_bytes<PT>() + kMhHkFloats * 4);
+  };
   int last = -1;  // last iteration whose global residual is complete
   bool stop = false;
 
@@ -167,24 +179,26 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
       const long long b = u / p.H;
       const int g = (int)(u - b * p.H);
       for (int e = lane; e < 192; e += 32)
-        (&s_U[warp][0][0][0])[e] = __ldg(p.U + ((long long)(e >> 6) * p.H + g) * 64 + (e & 63));
-      float x[8], hb[8];  // state entering the chunk: h^{k+1} and h^k
+        s_U[warp][e] = __ldg(p.U + ((long long)(e >> 6) * p.H + g) * 64 + (e & 63));
+      float x[8], hb[8];  // entering the chunk: h^{k+1} and h^k (h0 before the first)
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] = hb[i] = p.h0 ? __ldg(p.h0 + b * D + 8 * g + i) : 0.0f;
-      __syncwarp();
-      const float(*U)[8][8] = s_U[warp];
-      float* hk = s_hk + (size_t)warp * kMhWarpFloats;
-      float* sp = hk + (kMhT + 1) * 8;
+      const float* U = s_U[warp];
+      const int nch = (int)((p.L + kMhT - 1) / kMhT);
+      if (kMhBufs == 2) mh_issue_chunk<PT>(p, P, b, g, D, 0, k, hkbuf(0), spbuf(0), lane);
 
-      for (long long t0 = 0; t0 < p.L; t0 += kMhT) {
-        // ---- stage h^k of the chunk (zero at k = 0: h^0 = 0) --------------------
-        if (lane < 8) hk[lane] = hb[lane];
-        for (int e = lane; e < kMhT * 8; e += 32) {
-          const long long t = t0 + (e >> 3);
-          hk[8 + e] = (k > 0 && t < p.L) ? p.h[(b * p.L + t) * D + 8 * g + (e & 7)] : 0.0f;
-        }
-        if constexpr (kMhStageP) mh_stage_gates<PT>(P, b, t0, p.L, D, g, sp, lane);
+      for (int ci = 0; ci < nch; ++ci) {
+        const long long t0 = (long long)ci * kMhT;
+        const int cur = kMhBufs == 2 ? (ci & 1) : 0;
+        float* hk = hkbuf(cur);
+        const PT* sp = spbuf(cur);
+        if (kMhBufs == 1) mh_issue_chunk<PT>(p, P, b, g, D, t0, k, hk, spbuf(0), lane);
+        cp_async_wait_all();
         __syncwarp();
+        if (lane < 8) hk[lane] = hb[lane];  // row 0: h^k of the step before the chunk
+        __syncwarp();
+        if (kMhBufs == 2 && ci + 1 < nch)
+          mh_issue_chunk<PT>(p, P, b, g, D, t0 + kMhT, k, hkbuf(cur ^ 1), spbuf(cur ^ 1), lane);
 
         // ---- A: linearise this lane's steps, compose their maps ------------------
         const int s0 = lane * kMhS;
@@ -198,19 +212,14 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
         for (int s = 0; s < kMhS; ++s) {
           const long long t = t0 + s0 + s;
           if (t >= p.L) break;
-          float hp[8], hc[8], f[8], J[8][8];
+          float hp[8], hc[8], pg[24], f[8], J[8][8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             hp[i] = hk[(s0 + s) * 8 + i];
             hc[i] = hk[(s0 + s + 1) * 8 + i];
           }
-          float pg[24];
-          if constexpr (kMhStageP) {
 #pragma unroll
-            for (int i = 0; i < 24; ++i) pg[i] = sp[24 * (s0 + s) + i];
-          } else {
-            mh_load_gates<PT>(P, b * p.L + t, D, g, pg);
-          }
+          for (int i = 0; i < 24; ++i) pg[i] = to_f(sp[24 * (s0 + s) + i]);
           mh_cell(pg, U, hp, f, J);
           float bt[8];
 #pragma unroll
@@ -221,7 +230,7 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
             for (int j = 0; j < 8; ++j) s2 = fmaf(-J[i][j], hp[j], s2);
             bt[i] = s2;
           }
-          // (A, bv) <- (J A, J bv + bt)
+          // (A, bv) <- (J A, J bv + bt), column by column
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             float col[8];
@@ -272,16 +281,11 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
           for (int s = 0; s < kMhS; ++s) {
             const long long t = t0 + s0 + s;
             if (t >= p.L) break;
-            float hp[8], f[8], J[8][8];
+            float hp[8], pg[24], f[8], J[8][8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) hp[i] = hk[(s0 + s) * 8 + i];
-            float pg[24];
-            if constexpr (kMhStageP) {
 #pragma unroll
-              for (int i = 0; i < 24; ++i) pg[i] = sp[24 * (s0 + s) + i];
-            } else {
-              mh_load_gates<PT>(P, b * p.L + t, D, g, pg);
-            }
+            for (int i = 0; i < 24; ++i) pg[i] = to_f(sp[24 * (s0 + s) + i]);
             mh_cell(pg, U, hp, f, J);
             float y[8];
 #pragma unroll
@@ -303,9 +307,10 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) hb[i] = hk[kMhT * 8 + i];
-        __syncwarp();  // s_hk is restaged by the next chunk
+        __syncwarp();  // the buffer is refilled by a later chunk
       }
-      __syncwarp();  // s_U is reloaded by the next sequence
+      cp_async_wait_all();
+      __syncwarp();  // s_U and the buffers are reused by the next sequence
     }
 
     // ---- global residual of iteration k, then every CTA takes the same decision
