@@ -33,3 +33,30 @@ def test_traffic_record_is_tied_to_kernel_sources():
     assert d1 == bench.kernel_source_digest() and len(d1) == 64
     traffic, why = bench.recorded_traffic("no-such-workload")
     assert traffic is None
+
+
+def test_backward_and_projection_bytes():
+    N = 8 * 4096 * 1024
+    # backward: read P, the trajectory one step behind and dl/dh (and dl/dc); write dP
+    assert bench.algorithmic_bytes("gru_bwd", False, 8, 4096, 1024) == 32 * N
+    assert bench.algorithmic_bytes("lstm_bwd", False, 8, 4096, 1024) == 48 * N
+    # projection: x [M, K] and W [N, K] in bf16 once, the bias, P once
+    M, Nf, K = 8 * 4096, 3 * 1024, 1024
+    assert bench.projection_bytes(M, Nf, K, False) == 2 * M * K + 2 * Nf * K + 4 * Nf + 4 * M * Nf
+    assert bench.projection_bytes(M, Nf, K, True) == 2 * M * K + 2 * Nf * K + 4 * Nf + 2 * M * Nf
+    # multi-head solve: every Newton evaluation streams P and the iterate
+    assert bench.algorithmic_bytes("mhgru", False, 8, 4096, 1024, passes=4) == 4 * 20 * N
+
+
+def test_reference_arm_runs_every_new_workload(capsys):
+    """The oracle arm prints one JSON line for the projection and the multi-head
+    workloads (bounded samples; no GPU)."""
+    import argparse
+    import json
+
+    for wl in ("proj", "mhgru"):
+        args = argparse.Namespace(workload=wl, steps=1, warmup=1)
+        bench.run_reference(args, 1, 0, 0)
+        line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+        assert line["impl"] == "reference" and line["value"] > 0
+        assert line["e2e"]["h2d_bytes_per_step"] == 0
