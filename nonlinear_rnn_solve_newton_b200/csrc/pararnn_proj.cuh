@@ -380,3 +380,213 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 }
 
 }  // namespace pararnn
+
+// ===========================================================================
+// CTA-pair variant: a cluster of two CTAs computes 256 x 256 tiles with
+// tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads its own 128 rows of x and
+// its own 128 rows of W (half of N) per k-block -- 32 KB instead of 48 KB for
+// the same tensor work, so six stages fit and each SM pulls a third less from
+// L2.  No multicast load anywhere: each CTA copies only into its own shared
+// memory; the copies complete on the leader CTA's barrier (.cta_group::2).
+//   * leader (rank 0), warp 1: issues the MMAs (A from both CTAs' stages, B
+//     from both CTAs' stages, D rows 128 r .. 128 r + 127 in CTA r's TMEM) and
+//     commits them to the stage and accumulator barriers of both CTAs;
+//   * both CTAs: warp 0 produces, warps 2-9 drain their own TMEM; the leader's
+//     accumulator-free barrier counts the epilogue threads of both CTAs.
+// ===========================================================================
+namespace pararnn {
+
+constexpr unsigned kP2ABytes = kProjBM * kProjBK * 2;       // 128 rows of x
+constexpr unsigned kP2BBytes = (kProjBN / 2) * kProjBK * 2;  // 128 rows of W
+constexpr unsigned kP2StageBytes = kP2ABytes + kP2BBytes;
+// M = 256 (both CTAs), N = 256, fp32 accumulate, bf16 A/B, K-major
+constexpr unsigned kP2Idesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                              ((unsigned)(kProjBN >> 3) << 17) | ((unsigned)(256 >> 4) << 24);
+
+template <int ST> constexpr size_t proj2_smem_bytes() {
+  return (size_t)ST * kP2StageBytes + kProjEpiBytes + 1024;
+}
+
+__device__ __forceinline__ unsigned cluster_rank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of this CTA's shared variable at `local` in CTA `rank`
+__device__ __forceinline__ unsigned mapa_shared(unsigned local, unsigned rank) {
+  unsigned r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(unsigned dst, const CUtensorMap* map, int x, int y,
+                                                 unsigned bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<unsigned long long>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void umma_f16_ss_pair(unsigned tmem_d, unsigned long long da,
+                                                 unsigned long long db, unsigned idesc,
+                                                 unsigned accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at this offset in both CTAs of the pair when the
+// MMAs issued so far have completed.
+__device__ __forceinline__ void umma_commit_pair(unsigned long long* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], m;\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(unsigned bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
+template <int ST, bool OB>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
+    pararnn_proj2_kernel(const __grid_constant__ ProjParams p, const __grid_constant__ ProjMaps tm) {
+  extern __shared__ __align__(1024) unsigned char dsmem[];
+  __shared__ unsigned long long s_full[ST], s_empty[ST], s_tfull[2], s_tempty[2];
+  __shared__ unsigned s_tmem;
+  __shared__ int s_fail;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned rank = cluster_rank();
+  const unsigned sbase = (smem_u32(dsmem) + 1023u) & ~1023u;
+  const int nk = (p.K + kProjBK - 1) / kProjBK;
+  const int ntm = (p.M + 2 * kProjBM - 1) / (2 * kProjBM);
+  const int ntiles = ntm * p.ntn;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const WaitCtx wctx{nullptr, p.status_dev, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&s_tfull[a], 1);
+      mbar_init(&s_tempty[a], 2 * 32 * kProjEpiWarps);  // epilogue threads of both CTAs
+    }
+    s_fail = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {  // same warp in both CTAs: both accumulators of the pair
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem)),
+                 "r"(2 * kProjBN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  const unsigned tmem = s_tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- producer (both CTAs): this CTA's halves of each k-block ------------------
+      unsigned it = 0;
+      for (int tile = pair; tile < ntiles && !*(volatile int*)&s_fail; tile += npairs) {
+        const int m0 = (tile / p.ntn) * 2 * kProjBM + (int)rank * kProjBM;
+        const int n0 = (tile % p.ntn) * kProjBN + (int)rank * (kProjBN / 2);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % ST;
+          const unsigned ph = (it / ST) & 1u;
+          if (!stage_wait(&s_empty[s], ph ^ 1u, wctx)) {
+            s_fail = 1;
+            break;
+          }
+          // the leader's barrier expects both CTAs' bytes of this stage
+          if (rank == 0) mbar_expect_tx(&s_full[s], 2 * kP2StageBytes);
+          const unsigned bar = mapa_shared(smem_u32(&s_full[s]), 0);
+          const unsigned a = sbase + s * kP2StageBytes;
+          tma_load_2d_pair(a, &tm.x, kb * kProjBK, m0, bar);
+          tma_load_2d_pair(a + kP2ABytes, &tm.w, kb * kProjBK, n0, bar);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---- MMA issuer (leader CTA) ----------------------------------------------------
+      unsigned it = 0, lt = 0;
+      for (int tile = pair; tile < ntiles && !*(volatile int*)&s_fail; tile += npairs, ++lt) {
+        const unsigned acc = lt & 1u, use = lt >> 1;
+        if (!stage_wait(&s_tempty[acc], (use & 1u) ^ 1u, wctx)) {
+          s_fail = 1;
+          break;
+        }
+        tc_fence_after();
+        const unsigned d = tmem + acc * kProjBN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % ST;
+          const unsigned ph = (it / ST) & 1u;
+          if (!stage_wait(&s_full[s], ph, wctx)) {
+            s_fail = 1;
+            break;
+          }
+          tc_fence_after();
+          const unsigned a = sbase + s * kP2StageBytes;
+          const unsigned b = a + kP2ABytes;
+#pragma unroll
+          for (int k = 0; k < kProjBK / 16; ++k)
+            umma_f16_ss_pair(d, umma_desc_sw128(a + 32u * k), umma_desc_sw128(b + 32u * k),
+                             kP2Idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair(&s_empty[s]);  // frees stage s in both CTAs
+        }
+        umma_commit_pair(&s_tfull[acc]);  // both CTAs' accumulators are final
+      }
+    }
+  } else {
+    // ---- epilogue (both CTAs, own TMEM: rows m0 + 128 rank + 32 q + lane) -------------
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const unsigned ebuf = sbase + ST * kP2StageBytes + (unsigned)(warp - 2) * kProjEpiBox;
+    const unsigned tempty0 = mapa_shared(smem_u32(&s_tempty[0]), 0);
+    const unsigned tempty1 = mapa_shared(smem_u32(&s_tempty[1]), 0);
+    unsigned lt = 0;
+    for (int tile = pair; tile < ntiles; tile += npairs, ++lt) {
+      const unsigned acc = lt & 1u, use = lt >> 1;
+      const bool ok = stage_wait(&s_tfull[acc], use & 1u, wctx);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ok) || *(volatile int*)&s_fail) {
+        s_fail = 1;
+        break;
+      }
+      tc_fence_after();
+      const int m0 = (tile / p.ntn) * 2 * kProjBM + (int)rank * kProjBM;
+      const int n0 = (tile % p.ntn) * kProjBN;
+      proj_epilogue<OB>(p, &tm.p, tmem + acc * kProjBN + ((unsigned)(32 * q) << 16), ebuf,
+                        m0 + 32 * q, n0, half * 128, nk == 0);
+      tc_fence_before();
+      mbar_arrive_cluster(acc ? tempty1 : tempty0);
+    }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while its peer may still signal it
+  if (threadIdx.x == 0 && s_fail && p.status_dev) atomicCAS(p.status_dev, 0, 4);
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(2 * kProjBN)
+                 : "memory");
+  }
+}
+
+}  // namespace pararnn

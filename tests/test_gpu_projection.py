@@ -48,8 +48,9 @@ def check(P, x, W, b, out_bf16, rows=None):
     assert np.all(err <= tol), (float(err.max()), float((err / tol).max()))
 
 
+# K <= 2048 runs on CTA pairs, larger K on single CTAs: both kernels are covered
 SHAPES = [(128, 256, 64), (300, 264, 200), (1, 8, 8), (37, 40, 1024), (129, 512, 136),
-          (1000, 3072, 1024)]
+          (1000, 3072, 1024), (257, 384, 2056), (520, 264, 4096)]
 
 
 @pytest.mark.parametrize("out_bf16", [False, True])
