@@ -386,8 +386,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 // tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads its own 128 rows of x and
 // its own 128 rows of W (half of N) per k-block -- 32 KB instead of 48 KB for
 // the same tensor work, so six stages fit and each SM pulls a third less from
-// L2.  No multicast load anywhere: each CTA copies only into its own shared
-// memory; the copies complete on the leader CTA's barrier (.cta_group::2).
+// L2.  Each CTA copies only into its own shared memory (plain tensor copies);
+// the copies complete on the leader CTA's barrier (.cta_group::2).
 //   * leader (rank 0), warp 1: issues the MMAs (A from both CTAs' stages, B
 //     from both CTAs' stages, D rows 128 r .. 128 r + 127 in CTA r's TMEM) and
 //     commits them to the stage and accumulator barriers of both CTAs;
