@@ -115,7 +115,11 @@ typedef struct {
  *                iterations are evaluated per sweep.
  *  walk_warps  : warps per CTA in the walk regime with 32-channel tiles:
  *                0 = automatic (16 for the diagonal scan below 512 tiles,
- *                else 8), 8 or 16. */
+ *                else 8), 8 or 16.
+ *  walk_width  : channels per tile of the walk regime's tensor-copy walker for
+ *                the GRU / LSTM solves: 0 = automatic (8 when 32-channel tiles
+ *                would be fewer than 4 per SM -- finer tiles balance the SMs --
+ *                else 32), 8 or 32.  The scans always use 32. */
 typedef struct {
   int32_t iters_first;
   int32_t iters_next;
@@ -123,6 +127,8 @@ typedef struct {
   int64_t debug_stall_unit;
   int32_t regime;
   int32_t walk_warps;
+  int32_t walk_width;
+  int32_t reserved;
 } pararnn_options_t;
 
 /* Bytes of workspace the call with the same arguments needs. 0 on bad sizes. */

@@ -61,14 +61,15 @@ class Options(ctypes.Structure):
     """Tuning and test hooks (see pararnn_options_t)."""
     _fields_ = [("iters_first", ctypes.c_int32), ("iters_next", ctypes.c_int32),
                 ("wait_timeout_ns", ctypes.c_int64), ("debug_stall_unit", ctypes.c_int64),
-                ("regime", ctypes.c_int32), ("walk_warps", ctypes.c_int32)]
+                ("regime", ctypes.c_int32), ("walk_warps", ctypes.c_int32),
+                ("walk_width", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
     AUTO, LOOKBACK, WALK = 0, 1, 2
 
     def __init__(self, iters_first=0, iters_next=0, wait_timeout_ns=0, debug_stall_unit=-1,
-                 regime=0, walk_warps=0):
+                 regime=0, walk_warps=0, walk_width=0):
         super().__init__(iters_first, iters_next, wait_timeout_ns, debug_stall_unit, regime,
-                         walk_warps)
+                         walk_warps, walk_width, 0)
 
 
 INFO_BYTES = ctypes.sizeof(_Info)

@@ -84,6 +84,26 @@ constexpr int kMinBlocksSolve = PARARNN_MINB_SOLVE;
 constexpr int kWalkMinTiles = 200;
 // Below this many tiles the walker uses 16-warp CTAs.
 constexpr int kWalkWideTiles = 512;
+// Below this many 32-channel tiles (4 per SM on B200) the solves' walker uses
+// 8-channel tiles.
+constexpr int kWalkNarrowTiles = 4 * 148;
+// The GRU solve's walker on 8-channel tiles.  A warp holds 8 channels x 4
+// segments; with S steps per segment, segment k of a warp starts 3 * 8 * S * k
+// words (fp32) into the stage, so an odd S puts the four segments on different
+// shared-memory banks (S a multiple of 4 would make every read a 4-way
+// conflict), and NW x 4 x S must stay within TMA's 256 rows per box.
+// Measured on B200 (GRU, B=8, L=4096, D=1024): 4 warps x 13 steps 0.289 ms,
+// 4 x 15 0.293 ms, 8 x 7 0.312 ms, 8 x 5 0.342 ms; 32-channel tiles 0.311 ms.
+#ifndef PARARNN_NARROW_STEPS
+#define PARARNN_NARROW_STEPS 13
+#endif
+#ifndef PARARNN_NARROW_WARPS
+#define PARARNN_NARROW_WARPS 4
+#endif
+constexpr int kNarrowSteps = PARARNN_NARROW_STEPS;
+constexpr int kNarrowWarps = PARARNN_NARROW_WARPS;
+static_assert(kNarrowWarps * 4 * kNarrowSteps <= 256, "TMA box rows");
+
 
 constexpr int kStepsGruBwd = 8;
 constexpr int kStepsLstmBwd = 4;
@@ -147,8 +167,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
   bool walk = false;
-  int S_walk = 0;   // steps per thread of the TMA walk kernel (32-wide tiles)
+  int S_walk = 0;   // steps per thread of the TMA walk kernel
   int NW_walk = 8;  // warps per CTA of the TMA walk kernel
+  int CW_walk = 32; // channels per tile of the TMA walk kernel
   int op = 0, CW = 1, S = 1, T = 1, ntd = 0, ntiles = 0, nchunks = 0, nunits = 0;
   int m_first = 1, m_next = 1, mmax = 1, npasses = 1, max_iters = 0;
   size_t off_rho = 0, off_ticket = 0, off_rec = 0, zero_bytes = 0;
@@ -204,7 +225,19 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
     // B200); the solves and the 2x2 scan keep 8 warps.
     const bool wide = op == kScanDiag && ntiles < kWalkWideTiles;
     pl.NW_walk = (want == 8 || want == 16) ? want : (wide ? 16 : 8);
-    long long tw = (long long)pl.NW_walk * pl.S_walk;
+    // Tile width: 32-channel tiles leave the SMs unevenly loaded when there are
+    // few of them per SM (256 tiles on 148 SMs: 108 SMs hold two, 40 hold one);
+    // 8-channel tiles (a warp = 8 channels x 4 segments) cut the tail to < 2%.
+    const int ww = opts ? opts->walk_width : 0;
+    if (op == kGru)
+      pl.CW_walk = (ww == 8 || ww == 32) ? ww : (ntiles < kWalkNarrowTiles ? 8 : 32);
+    if (pl.CW_walk == 8) {
+      pl.S_walk = kNarrowSteps;
+      pl.NW_walk = kNarrowWarps;
+    }
+    const long long ntd_w = (D + pl.CW_walk - 1) / pl.CW_walk;
+    if (B * ntd_w > INT_MAX / 2) return pl;
+    long long tw = (long long)pl.NW_walk * (32 / pl.CW_walk) * pl.S_walk;
     long long nchunks_w = (L + tw - 1) / tw;
     if (nchunks_w > INT_MAX / 2) return pl;
   }
@@ -365,9 +398,9 @@ bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 // Tile-walking kernel with TMA staging (32-channel tiles).
 // ---------------------------------------------------------------------------
 
-template <int OP, typename PT, int S, int NW>
+template <int OP, typename PT, int S, int NW, int CW = 32>
 size_t walk_smem_bytes() {
-  constexpr unsigned b = Stage<OP, PT, NW * S>::kBytes;
+  constexpr unsigned b = Stage<OP, PT, NW * (32 / CW) * S, CW>::kBytes;
   return 2 * (size_t)((b + 1023u) / 1024u * 1024u) + 1024;  // + alignment slack
 }
 
@@ -383,7 +416,17 @@ const void* walk_kernel_nw(int nw, size_t* smem) {
   return (const void*)pararnn_walk_kernel<OP, PT, S, 8, MINB>;
 }
 
-const void* select_walk_kernel(int op, bool bf16, int nw, size_t* smem) {
+// The GRU walker on 8-channel tiles.
+template <typename PT, int MINB>
+const void* walk_kernel_narrow(size_t* smem) {
+  *smem = walk_smem_bytes<kGru, PT, kNarrowSteps, kNarrowWarps, 8>();
+  return (const void*)pararnn_walk_kernel<kGru, PT, kNarrowSteps, kNarrowWarps, MINB, 8>;
+}
+
+const void* select_walk_kernel(int op, bool bf16, int nw, int cw, size_t* smem) {
+  if (cw == 8 && op == kGru)
+    return bf16 ? walk_kernel_narrow<__nv_bfloat16, kWalkMinBlocks>(smem)
+                : walk_kernel_narrow<float, kWalkMinBlocksWide>(smem);
   switch (op) {
     case kScanDiag:
       return walk_kernel_nw<kScanDiag, float, kWalkStepsScanDiag, kWalkMinBlocks>(nw, smem);
@@ -444,9 +487,9 @@ bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, size_t
 
 // Tensor maps for the walk kernel, or false if the shapes or pointers do not
 // meet TMA's rules (16-byte aligned base, row pitch a multiple of 16 bytes).
-bool make_walk_maps(int op, bool bf16, const KParams& kp, int T, TmaMaps* tm) {
+bool make_walk_maps(int op, bool bf16, const KParams& kp, int T, int CW, TmaMaps* tm) {
   const long long B = kp.B, L = kp.L, D = kp.D;
-  if (D < 32 || B * L >= (1LL << 31)) return false;
+  if (D < CW || B * L >= (1LL << 31)) return false;
   const size_t es = bf16 ? 2 : 4;
   const CUtensorMapDataType dt =
       bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
@@ -456,7 +499,7 @@ bool make_walk_maps(int op, bool bf16, const KParams& kp, int T, TmaMaps* tm) {
     case kLstm: {
       const int G = op == kGru ? 3 : 4;
       if (!aligned(kp.in0, 16) || (D * (long long)es) % 16 != 0) return false;
-      return encode_map(&tm->in0, kp.in0, dt, es, D, G, rows, 32, T);
+      return encode_map(&tm->in0, kp.in0, dt, es, D, G, rows, (unsigned)CW, T);
     }
     case kScanDiag:
       if (!aligned(kp.in0, 16) || !aligned(kp.in1, 16) || (D * 4) % 16 != 0) return false;
@@ -537,14 +580,17 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
   // The TMA tile walker when the tiles are 32 wide and TMA's rules hold;
   // otherwise the general kernel (look-back or register-staged walk).
   TmaMaps tm;
+  const int tch_w = pl.NW_walk * (32 / pl.CW_walk) * pl.S_walk;  // steps per walker chunk
   const bool tma_walk = pl.walk && pl.CW == 32 && pl.S_walk > 0 &&
-                        make_walk_maps(pl.op, bf16, kp, pl.NW_walk * pl.S_walk, &tm);
+                        make_walk_maps(pl.op, bf16, kp, tch_w, pl.CW_walk, &tm);
   const void* fn;
   size_t dyn_smem = 0;
   int threads = kThreads;
   if (tma_walk) {
-    fn = select_walk_kernel(pl.op, bf16, pl.NW_walk, &dyn_smem);
-    kp.nchunks = (int)((kp.L + pl.NW_walk * pl.S_walk - 1) / (pl.NW_walk * pl.S_walk));
+    fn = select_walk_kernel(pl.op, bf16, pl.NW_walk, pl.CW_walk, &dyn_smem);
+    kp.nchunks = (int)((kp.L + tch_w - 1) / tch_w);
+    kp.ntd = (int)((kp.D + pl.CW_walk - 1) / pl.CW_walk);
+    kp.ntiles = (int)(kp.B * kp.ntd);
     threads = 32 * pl.NW_walk;
   } else {
     fn = select_kernel(pl.op, bf16, pl.walk, pl.CW);
@@ -565,7 +611,7 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }
-  const int nwork = pl.walk ? pl.ntiles : pl.nunits;
+  const int nwork = pl.walk ? kp.ntiles : pl.nunits;
   int grid = nwork < resident ? nwork : resident;
 
   if (cudaMemsetAsync(ws, 0, pl.zero_bytes, stream) != cudaSuccess) return PARARNN_ERR_CUDA;

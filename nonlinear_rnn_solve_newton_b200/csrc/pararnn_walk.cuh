@@ -69,39 +69,39 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// Shared-memory image of one time chunk, per op (32 channels wide).
-template <int OP, typename PT, int TCH> struct Stage;
-template <typename PT, int TCH> struct Stage<kGru, PT, TCH> {
-  static constexpr unsigned kBytes = TCH * 3 * 32 * sizeof(PT);
+// Shared-memory image of one time chunk, per op: [T][G][CW] for CW channels.
+template <int OP, typename PT, int TCH, int CW = 32> struct Stage;
+template <typename PT, int TCH, int CW> struct Stage<kGru, PT, TCH, CW> {
+  static constexpr unsigned kBytes = TCH * 3 * CW * sizeof(PT);
   __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
                                unsigned long long* bar) {
     mbar_expect_tx(bar, kBytes);
     tma_load_3d(s, &tm.in0, d0, 0, row, bar);
   }
   __device__ static void read(const unsigned char* s, int tl, int c, float* v) {
-    const PT* q = reinterpret_cast<const PT*>(s) + tl * 96 + c;
+    const PT* q = reinterpret_cast<const PT*>(s) + tl * 3 * CW + c;
     v[0] = to_f(q[0]);
-    v[1] = to_f(q[32]);
-    v[2] = to_f(q[64]);
+    v[1] = to_f(q[CW]);
+    v[2] = to_f(q[2 * CW]);
   }
 };
-template <typename PT, int TCH> struct Stage<kLstm, PT, TCH> {
-  static constexpr unsigned kBytes = TCH * 4 * 32 * sizeof(PT);
+template <typename PT, int TCH, int CW> struct Stage<kLstm, PT, TCH, CW> {
+  static constexpr unsigned kBytes = TCH * 4 * CW * sizeof(PT);
   __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
                                unsigned long long* bar) {
     mbar_expect_tx(bar, kBytes);
     tma_load_3d(s, &tm.in0, d0, 0, row, bar);
   }
   __device__ static void read(const unsigned char* s, int tl, int c, float* v) {
-    const PT* q = reinterpret_cast<const PT*>(s) + tl * 128 + c;
+    const PT* q = reinterpret_cast<const PT*>(s) + tl * 4 * CW + c;
     v[0] = to_f(q[0]);
-    v[1] = to_f(q[32]);
-    v[2] = to_f(q[64]);
-    v[3] = to_f(q[96]);
+    v[1] = to_f(q[CW]);
+    v[2] = to_f(q[2 * CW]);
+    v[3] = to_f(q[3 * CW]);
   }
 };
-template <typename PT, int TCH> struct Stage<kScanDiag, PT, TCH> {
-  static constexpr unsigned kHalf = TCH * 32 * 4;
+template <typename PT, int TCH, int CW> struct Stage<kScanDiag, PT, TCH, CW> {
+  static constexpr unsigned kHalf = TCH * CW * 4;
   static constexpr unsigned kBytes = 2 * kHalf;
   __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
                                unsigned long long* bar) {
@@ -110,11 +110,12 @@ template <typename PT, int TCH> struct Stage<kScanDiag, PT, TCH> {
     tma_load_2d(s + kHalf, &tm.in1, d0, row, bar);
   }
   __device__ static void read(const unsigned char* s, int tl, int c, float* v) {
-    v[0] = reinterpret_cast<const float*>(s)[tl * 32 + c];
-    v[1] = reinterpret_cast<const float*>(s + kHalf)[tl * 32 + c];
+    v[0] = reinterpret_cast<const float*>(s)[tl * CW + c];
+    v[1] = reinterpret_cast<const float*>(s + kHalf)[tl * CW + c];
   }
 };
-template <typename PT, int TCH> struct Stage<kScanBlock2, PT, TCH> {
+template <typename PT, int TCH, int CW> struct Stage<kScanBlock2, PT, TCH, CW> {
+  static_assert(CW == 32, "the 2x2 scan walker stages 32-channel tiles");
   static constexpr unsigned kA = TCH * 32 * 16;
   static constexpr unsigned kBytes = kA + TCH * 32 * 8;
   __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
@@ -159,16 +160,18 @@ __device__ __forceinline__ void drain_stages(unsigned long long* bars, unsigned 
     if (pending & (1u << st)) stage_wait(&bars[st], (phase >> st) & 1u, wl);
 }
 
-template <int OP, typename PT, int S, int NW, int MINB>
+template <int OP, typename PT, int S, int NW, int MINB, int CW = 32>
 __global__ void __launch_bounds__(NW * 32, MINB)
     pararnn_walk_kernel(const __grid_constant__ KParams p, const __grid_constant__ TmaMaps tm) {
   using T_ = OpT<OP>;
   constexpr int NS = T_::NS;
   constexpr int NI = T_::NI;
   constexpr bool NEWTON = T_::newton;
-  constexpr int CW = 32;
-  constexpr int TCH = NW * S;  // steps per chunk (one segment of S steps per warp)
-  using St = Stage<OP, PT, TCH>;
+  static_assert(CW == 32 || CW == 16 || CW == 8, "tile width");
+  constexpr int SPL = 32 / CW;       // segments per warp (lane = channel + CW * segment)
+  constexpr int NSEG = NW * SPL;     // segments per chunk, S steps each
+  constexpr int TCH = NSEG * S;      // steps per chunk
+  using St = Stage<OP, PT, TCH, CW>;
   constexpr unsigned kStageBytes = (St::kBytes + 1023u) / 1024u * 1024u;
   constexpr int WM = kMaxWalkIters;
 
@@ -185,8 +188,10 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int c = lane;
-  const int seg = warp;
+  const int c = lane % CW;        // channel within the tile
+  const int sub = lane / CW;      // segment within the warp
+  const int seg = warp * SPL + sub;
+  const bool last_in_warp = sub == SPL - 1;
 
   if (tid == 0) {
     mbar_init(&s_bar[0], 1);
@@ -278,7 +283,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
             } else if (cvalid && t0 - 1 < p.L) {
               IO<OP, PT>::load_state(p, (b * p.L + t0 - 1) * p.D + d, xb.x);
             }
-            if (seg == NW - 1) s_pend[j & 1][c] = x[S - 1];
+            if (seg == NSEG - 1) s_pend[j & 1][c] = x[S - 1];
           }
         }
 
@@ -347,14 +352,25 @@ __global__ void __launch_bounds__(NW * 32, MINB)
           // cannot overtake a slow warp's reads) and applies the prefix to the
           // state carried in from the previous chunk at this iteration.
           const int buf = kk & 1;
-          s_wagg[buf][warp][c] = agg;
+          // segments of this warp: inclusive scan over the lanes of each channel
+          Map<NS> wincl = agg, wexcl = map_identity<NS>();
+          if constexpr (SPL > 1) {
+#pragma unroll
+            for (int off = CW; off < 32; off <<= 1) {
+              const Map<NS> o = shfl_up_map(wincl, off);
+              if (lane >= off) wincl = compose(wincl, o);
+            }
+            const Map<NS> e = shfl_up_map(wincl, CW);
+            if (sub > 0) wexcl = e;
+          }
+          if (last_in_warp) s_wagg[buf][warp][c] = wincl;
           __syncthreads();
           Map<NS> pre = map_identity<NS>();
 #pragma unroll 4
           for (int w2 = 0; w2 < warp; ++w2) pre = compose(s_wagg[buf][w2][c], pre);
           const Vec<NS> carry = (j == 0) ? x0v : s_inc[(j - 1) & 1][kk][c];
-          const Vec<NS> xin = apply(pre, carry);
-          if (warp == NW - 1) s_inc[j & 1][kk][c] = apply(agg, xin);
+          const Vec<NS> xin = apply(wexcl, apply(pre, carry));
+          if (warp == NW - 1 && last_in_warp) s_inc[j & 1][kk][c] = apply(agg, xin);
           Vec<NS> xr = xin;
 #pragma unroll
           for (int s = 0; s < S; ++s) {

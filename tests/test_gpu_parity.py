@@ -304,3 +304,59 @@ def test_walk_regime_unconverged_iterate(pr):
     orc = oracle.newton_gru(x["P"], x["a"], tol=0.0, max_iters=3)
     assert not info.converged and info.iterations == 3 and info.updates == 3
     assert np.max(np.abs(h.cpu().numpy() - orc.h)) <= 1e-5
+
+
+# --------------------------------------------------------------------------
+# The tensor-copy walker on 8- and 32-channel tiles (a warp = 8 channels x 4
+# time segments, or 32 channels x 1): same results.  Shapes with D a multiple
+# of 8 that is not of 32, a ragged last tile (D = 36), L not a multiple of the
+# chunk, and bf16 gates.
+# --------------------------------------------------------------------------
+WIDTH_SHAPES = [(2, 1500, 64), (3, 700, 40), (1, 2100, 36), (2, 513, 96)]
+
+
+@pytest.mark.parametrize("width", [8, 32])
+@pytest.mark.parametrize("shape", WIDTH_SHAPES)
+def test_walk_widths_gru(pr, shape, width):
+    B, L, D = shape
+    if width == 32 and D < 32:
+        pytest.skip("32-channel tiles need D >= 32")
+    x = inputs.gru_inputs(B, L, D, seed=[510, B, L, D], h0_normal=True)
+    o = pr.Options(regime=2, walk_width=width)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), dev(x["h0"]), opts=o)
+    torch.cuda.synchronize()
+    ref = oracle.rollout_gru(x["P"], x["a"], x["h0"])
+    assert info.converged
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
+    orc = oracle.newton_gru(x["P"], x["a"], x["h0"], tol=1e-4, max_iters=32)
+    assert abs(info.iterations - orc.iterations) <= 1
+
+
+@pytest.mark.parametrize("width", [8, 32])
+@pytest.mark.parametrize("shape", WIDTH_SHAPES)
+def test_walk_widths_lstm_bf16(pr, shape, width):
+    B, L, D = shape
+    if width == 32 and D < 32:
+        pytest.skip("32-channel tiles need D >= 32")
+    x = inputs.lstm_inputs(B, L, D, seed=[511, B, L, D], bf16=True)
+    P16 = torch.from_numpy(x["P_bits"].view(np.int16)).cuda().view(torch.bfloat16)
+    o = pr.Options(regime=2, walk_width=width)
+    c, h, info = pr.solve_lstm(P16, dev(x["a"]), opts=o)
+    torch.cuda.synchronize()
+    rc, rh = oracle.rollout_lstm(x["P"], x["a"])
+    assert info.converged
+    assert np.max(np.abs(h.cpu().numpy() - rh)) <= SOLVE_ATOL
+    assert np.max(np.abs(c.cpu().numpy() - rc)) <= SOLVE_ATOL
+
+
+def test_walk_width_unconverged_iterate(pr):
+    """8-channel walker, several sweeps (2 then 1 iterations), tol = 0: h^3 exactly."""
+    B, L, D = 2, 1100, 48
+    x = inputs.gru_inputs(B, L, D, seed=512, h0_normal=True)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), dev(x["h0"]), tol=0.0, max_iters=3,
+                           opts=pr.Options(regime=2, iters_first=2, iters_next=1,
+                                           walk_width=8))
+    torch.cuda.synchronize()
+    orc = oracle.newton_gru(x["P"], x["a"], x["h0"], tol=0.0, max_iters=3)
+    assert not info.converged and info.iterations == 3 and info.updates == 3
+    assert np.max(np.abs(h.cpu().numpy() - orc.h)) <= 1e-5
