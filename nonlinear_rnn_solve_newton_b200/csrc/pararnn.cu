@@ -87,11 +87,12 @@ constexpr int kWalkWideTiles = 512;
 // Below this many 32-channel tiles (4 per SM on B200) the solves' walker uses
 // 8-channel tiles.
 constexpr int kWalkNarrowTiles = 4 * 148;
-// The GRU solve's walker on 8-channel tiles.  A warp holds 8 channels x 4
-// segments; with S steps per segment, segment k of a warp starts 3 * 8 * S * k
-// words (fp32) into the stage, so an odd S puts the four segments on different
-// shared-memory banks (S a multiple of 4 would make every read a 4-way
-// conflict), and NW x 4 x S must stay within TMA's 256 rows per box.
+// The solves' walker on 8-channel tiles.  A warp holds 8 channels x 4
+// segments; with S steps per segment, segment k of a warp starts 24 S k words
+// (GRU, fp32 rows of 3 gates) or 8 S k words (LSTM gate planes) into the stage,
+// so an odd S puts the four segments on different shared-memory banks (S a
+// multiple of 4 would make every read a 4-way conflict), and NW x 4 x S must
+// stay within TMA's 256 rows per box.
 // Measured on B200 (GRU, B=8, L=4096, D=1024): 4 warps x 13 steps 0.289 ms,
 // 4 x 15 0.293 ms, 8 x 7 0.312 ms, 8 x 5 0.342 ms; 32-channel tiles 0.311 ms.
 #ifndef PARARNN_NARROW_STEPS
@@ -229,7 +230,7 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
     // few of them per SM (256 tiles on 148 SMs: 108 SMs hold two, 40 hold one);
     // 8-channel tiles (a warp = 8 channels x 4 segments) cut the tail to < 2%.
     const int ww = opts ? opts->walk_width : 0;
-    if (op == kGru)
+    if (is_newton(op))
       pl.CW_walk = (ww == 8 || ww == 32) ? ww : (ntiles < kWalkNarrowTiles ? 8 : 32);
     if (pl.CW_walk == 8) {
       pl.S_walk = kNarrowSteps;
@@ -416,17 +417,20 @@ const void* walk_kernel_nw(int nw, size_t* smem) {
   return (const void*)pararnn_walk_kernel<OP, PT, S, 8, MINB>;
 }
 
-// The GRU walker on 8-channel tiles.
-template <typename PT, int MINB>
+// The solves' walker on 8-channel tiles.
+template <int OP, typename PT, int MINB>
 const void* walk_kernel_narrow(size_t* smem) {
-  *smem = walk_smem_bytes<kGru, PT, kNarrowSteps, kNarrowWarps, 8>();
-  return (const void*)pararnn_walk_kernel<kGru, PT, kNarrowSteps, kNarrowWarps, MINB, 8>;
+  *smem = walk_smem_bytes<OP, PT, kNarrowSteps, kNarrowWarps, 8>();
+  return (const void*)pararnn_walk_kernel<OP, PT, kNarrowSteps, kNarrowWarps, MINB, 8>;
 }
 
 const void* select_walk_kernel(int op, bool bf16, int nw, int cw, size_t* smem) {
   if (cw == 8 && op == kGru)
-    return bf16 ? walk_kernel_narrow<__nv_bfloat16, kWalkMinBlocks>(smem)
-                : walk_kernel_narrow<float, kWalkMinBlocksWide>(smem);
+    return bf16 ? walk_kernel_narrow<kGru, __nv_bfloat16, kWalkMinBlocks>(smem)
+                : walk_kernel_narrow<kGru, float, kWalkMinBlocksWide>(smem);
+  if (cw == 8 && op == kLstm)
+    return bf16 ? walk_kernel_narrow<kLstm, __nv_bfloat16, kWalkMinBlocksWide>(smem)
+                : walk_kernel_narrow<kLstm, float, kWalkMinBlocksWide>(smem);
   switch (op) {
     case kScanDiag:
       return walk_kernel_nw<kScanDiag, float, kWalkStepsScanDiag, kWalkMinBlocks>(nw, smem);
@@ -462,7 +466,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // Row-major tensor [outer][mid][inner] (mid = 1 for 2-D), TMA box = inner x mid x rows.
 bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, size_t esize,
                 unsigned long long inner, unsigned long long mid, unsigned long long outer,
-                unsigned box_inner, unsigned box_rows) {
+                unsigned box_inner, unsigned box_rows, unsigned box_mid = 0) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return false;
   CUresult r;
@@ -470,7 +474,7 @@ bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, size_t
   if (mid > 1) {
     const cuuint64_t dims[3] = {inner, mid, outer};
     const cuuint64_t strides[2] = {inner * esize, inner * mid * esize};
-    const cuuint32_t box[3] = {box_inner, (cuuint32_t)mid, box_rows};
+    const cuuint32_t box[3] = {box_inner, box_mid ? box_mid : (cuuint32_t)mid, box_rows};
     r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -499,7 +503,9 @@ bool make_walk_maps(int op, bool bf16, const KParams& kp, int T, int CW, TmaMaps
     case kLstm: {
       const int G = op == kGru ? 3 : 4;
       if (!aligned(kp.in0, 16) || (D * (long long)es) % 16 != 0) return false;
-      return encode_map(&tm->in0, kp.in0, dt, es, D, G, rows, (unsigned)CW, T);
+      // 8-channel LSTM tiles are staged one gate plane per copy
+      const unsigned box_mid = (op == kLstm && CW == 8) ? 1u : 0u;
+      return encode_map(&tm->in0, kp.in0, dt, es, D, G, rows, (unsigned)CW, T, box_mid);
     }
     case kScanDiag:
       if (!aligned(kp.in0, 16) || !aligned(kp.in1, 16) || (D * 4) % 16 != 0) return false;

@@ -85,6 +85,26 @@ template <typename PT, int TCH, int CW> struct Stage<kGru, PT, TCH, CW> {
     v[2] = to_f(q[2 * CW]);
   }
 };
+// 8-channel LSTM tiles: one plane per gate, [G][T][8] (four tensor copies of
+// 8 channels x 1 gate x T rows).  Rows of 8 channels put a warp's four time
+// segments on different shared-memory banks when the steps per segment are
+// odd; one [T][G][8] image would give rows of 32 words, a 4-way conflict.
+template <typename PT, int TCH> struct Stage<kLstm, PT, TCH, 8> {
+  static constexpr unsigned kPlane = TCH * 8 * sizeof(PT);
+  static_assert(kPlane % 128 == 0, "gate planes stay 128-byte aligned");
+  static constexpr unsigned kBytes = 4 * kPlane;
+  __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
+                               unsigned long long* bar) {
+    mbar_expect_tx(bar, kBytes);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) tma_load_3d(s + g * kPlane, &tm.in0, d0, g, row, bar);
+  }
+  __device__ static void read(const unsigned char* s, int tl, int c, float* v) {
+    const PT* q = reinterpret_cast<const PT*>(s) + tl * 8 + c;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) v[g] = to_f(q[g * (TCH * 8)]);
+  }
+};
 template <typename PT, int TCH, int CW> struct Stage<kLstm, PT, TCH, CW> {
   static constexpr unsigned kBytes = TCH * 4 * CW * sizeof(PT);
   __device__ static void issue(unsigned char* s, const TmaMaps& tm, int d0, int row,
