@@ -13,6 +13,13 @@ Entry points (same names as the C ABI, without the ``pararnn_`` prefix):
 * ``solve_gru(P, a, h0=None, tol=1e-4, max_iters=32)``   ParaGRU Newton solve
 * ``solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32)``  ParaLSTM Newton solve
 * ``solve_gru_backward`` / ``solve_lstm_backward``  gradients through the solution
+* ``solve_mhgru(P, U, h0=None)``     multi-head GRU, dense 8x8 recurrence blocks
+* ``input_projection(x, W, bias=None)``  P = x W^T + bias on the tensor cores
+* ``step_gru`` / ``step_lstm``      one decode step;  ``rollout_gru`` / ``rollout_lstm``
+  the sequential application on the GPU
+
+The workspace the solves and scans need comes from torch's allocator and is
+reused between calls on the same thread, device and stream.
 """
 from __future__ import annotations
 
@@ -25,8 +32,8 @@ import torch
 from . import build as _build
 
 __all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc",
-           "solve_gru_backward", "solve_lstm_backward", "step_gru", "step_lstm",
-           "rollout_gru", "rollout_lstm",
+           "solve_gru_backward", "solve_lstm_backward", "solve_mhgru", "input_projection",
+           "step_gru", "step_lstm", "rollout_gru", "rollout_lstm",
            "workspace_size",
            "SolveInfo", "Options", "PararnnError", "library_path", "load", "MAX_ITERS"]
 
@@ -176,15 +183,20 @@ def _stream_handle(stream):
 _ws_cache = threading.local()
 
 
-def _workspace(nbytes, device):
-    """Workspace from torch's allocator, reused between calls on the same thread and device."""
+def _workspace(nbytes, device, stream=None):
+    """Workspace from torch's allocator, reused between calls on the same thread,
+    device and stream (calls on one stream run in order, so they can share it;
+    calls on different streams get their own)."""
     cache = getattr(_ws_cache, "bufs", None)
     if cache is None:
         cache = _ws_cache.bufs = {}
-    key = (device.index if device.index is not None else torch.cuda.current_device())
+    dev = device.index if device.index is not None else torch.cuda.current_device()
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    key = (dev, s.cuda_stream)
     buf = cache.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        with torch.cuda.stream(s):
+            buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
         cache[key] = buf
     return buf
 
@@ -251,7 +263,7 @@ def scan_diag(A, b, h0=None, out=None, status=None, opts: Options | None = None,
     h = torch.empty_like(A) if out is None else out
     _check_dev("out", h, torch.float32, (B, L, D))
     n = workspace_size(OP_SCAN_DIAG, B, L, D, 0, opts)
-    ws = _workspace(n, A.device)
+    ws = _workspace(n, A.device, stream)
     st = lib.pararnn_scan_diag(_ptr(A), _ptr(b), _ptr(h0), _ptr(h), B, L, D, _ptr(ws), ws.numel(),
                                _ptr(status), ctypes.byref(opts) if opts is not None else None,
                                _stream_handle(stream))
@@ -269,7 +281,7 @@ def scan_block2(A, b, x0=None, out=None, status=None, opts: Options | None = Non
     x = torch.empty_like(b) if out is None else out
     _check_dev("out", x, torch.float32, (B, L, D, 2))
     n = workspace_size(OP_SCAN_BLOCK2, B, L, D, 0, opts)
-    ws = _workspace(n, A.device)
+    ws = _workspace(n, A.device, stream)
     st = lib.pararnn_scan_block2(_ptr(A), _ptr(b), _ptr(x0), _ptr(x), B, L, D, _ptr(ws),
                                  ws.numel(), _ptr(status),
                                  ctypes.byref(opts) if opts is not None else None,
@@ -302,7 +314,7 @@ def solve_gru(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
     n = workspace_size(OP_GRU, B, L, D, max_iters, opts)
-    ws = _workspace(n, P.device)
+    ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D, float(tol),
                                int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
                                ctypes.byref(opts) if opts is not None else None,
@@ -329,7 +341,7 @@ def solve_mhgru(P, U, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
     n = workspace_size(OP_MHGRU, B, L, D, max_iters, opts)
-    ws = _workspace(n, P.device)
+    ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_mhgru(_ptr(P), dt, _ptr(U), _ptr(h0), _ptr(h), B, L, H, float(tol),
                                  int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
                                  ctypes.byref(opts) if opts is not None else None,
@@ -360,7 +372,7 @@ def solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32, out=None, info=No
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
     n = workspace_size(OP_LSTM, B, L, D, max_iters, opts)
-    ws = _workspace(n, P.device)
+    ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_lstm(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h), B, L,
                                 D, float(tol), int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
                                 ctypes.byref(opts) if opts is not None else None,
@@ -425,7 +437,7 @@ def solve_gru_backward(P, a, h, dh, h0=None, out=None, status=None,
     _check_dev("da", da, torch.float32, (3, D))
     _check_dev("dh0", dh0, torch.float32, (B, D))
     n = workspace_size(OP_GRU_BACKWARD, B, L, D, 0, opts)
-    ws = _workspace(n, P.device)
+    ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_gru_backward(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), _ptr(dh),
                                         _ptr(dP), _ptr(da), _ptr(dh0), B, L, D, _ptr(ws),
                                         ws.numel(), _ptr(status),
@@ -458,7 +470,7 @@ def solve_lstm_backward(P, a, c, h, dc, dh, c0=None, h0=None, out=None, status=N
     else:
         dP, da, dc0, dh0 = out
     n = workspace_size(OP_LSTM_BACKWARD, B, L, D, 0, opts)
-    ws = _workspace(n, P.device)
+    ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_lstm_backward(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c),
                                          _ptr(h), _ptr(dc), _ptr(dh), _ptr(dP), _ptr(da),
                                          _ptr(dc0), _ptr(dh0), B, L, D, _ptr(ws), ws.numel(),

@@ -360,3 +360,22 @@ def test_walk_width_unconverged_iterate(pr):
     orc = oracle.newton_gru(x["P"], x["a"], x["h0"], tol=0.0, max_iters=3)
     assert not info.converged and info.iterations == 3 and info.updates == 3
     assert np.max(np.abs(h.cpu().numpy() - orc.h)) <= 1e-5
+
+
+def test_concurrent_solves_on_two_streams(pr):
+    """Solves issued on two streams at once each get their own cached workspace:
+    both results match the oracle."""
+    B, L, D = 4, 2000, 64
+    xs = [inputs.gru_inputs(B, L, D, seed=[520, i]) for i in range(2)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    Ps = [dev(x["P"]) for x in xs]
+    As = [dev(x["a"]) for x in xs]
+    torch.cuda.synchronize()
+    outs = []
+    for i in range(2):
+        with torch.cuda.stream(streams[i]):
+            outs.append(pr.solve_gru(Ps[i], As[i], stream=streams[i]))
+    torch.cuda.synchronize()
+    for (h, info), x in zip(outs, xs):
+        assert info.converged
+        assert np.max(np.abs(h.cpu().numpy() - oracle.rollout_gru(x["P"], x["a"]))) <= SOLVE_ATOL
