@@ -402,6 +402,26 @@ def run_ours(args, world, rank, local):
     iters = info.iterations if info else None
     passes = info.passes if info else 1
 
+    # ---- optional: the step as a CUDA graph (removes the per-call host cost
+    # that dominates latency-bound workloads; the graph holds the same launches)
+    graph = None
+    use_graph = args.graph if args.graph is not None else args.workload == "gru_s"
+    if use_graph:
+        gs = torch.cuda.Stream(device)
+        gs.wait_stream(stream)
+        with torch.cuda.stream(gs):
+            cs.step()
+        stream.wait_stream(gs)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gs):
+            cs.step()
+        torch.cuda.synchronize()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+    run_step = graph.replay if graph is not None else cs.step
+
     # ---- timed region: exactly K steps ---------------------------------------
     K = args.steps
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
@@ -410,7 +430,7 @@ def run_ours(args, world, rank, local):
     with ClockSampler(local) as clk:
         evs[0].record(stream)
         for i in range(K):
-            cs.step()
+            run_step()
             evs[i + 1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -660,6 +680,7 @@ def run_ours(args, world, rank, local):
         if op == "proj":
             wlname += f" K={cs.K} G={cs.G} (M={B * L}, N={cs.G * D})"
         cfg = {"workload": wlname, "B": B, "L": L, "D": D,
+               "launch": "CUDA graph replay" if graph is not None else "direct calls",
                "parallelism": f"replicas x{world} (independent batches)",
                "l2": "inputs larger than L2 (%.0f MB per step), no flush needed" % (
                    sum(v.numel() * v.element_size() for v in cs.host.values()) / 1e6)}
@@ -890,6 +911,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--no-sequential", action="store_true",
                     help="skip the sequential-application context timings")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=None,
+                    help="time the step as CUDA graph replays (default for gru_s)")
+    ap.add_argument("--no-graph", dest="graph", action="store_false")
     ap.add_argument("--warmup-seconds", type=float, default=0.5,
                     help="keep warming up until this much time has passed (after W steps)")
     args = ap.parse_args()

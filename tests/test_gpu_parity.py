@@ -379,3 +379,33 @@ def test_concurrent_solves_on_two_streams(pr):
     for (h, info), x in zip(outs, xs):
         assert info.converged
         assert np.max(np.abs(h.cpu().numpy() - oracle.rollout_gru(x["P"], x["a"]))) <= SOLVE_ATOL
+
+
+def test_solve_replays_from_a_cuda_graph(pr):
+    """A solve (workspace zeroing + cooperative launch) can be captured into a
+    CUDA graph and replayed: the replays give the direct call's result, also
+    after the inputs are overwritten in place."""
+    B, L, D = 2, 512, 16
+    x1 = inputs.gru_inputs(B, L, D, seed=530)
+    x2 = inputs.gru_inputs(B, L, D, seed=531)
+    P, a = dev(x1["P"]), dev(x1["a"])
+    h = torch.empty((B, L, D), device="cuda")
+    info_t = torch.empty(pr.INFO_BYTES // 4, dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):                   # warm-up outside the capture
+            pr.solve_gru(P, a, out=h, info=info_t, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        pr.solve_gru(P, a, out=h, info=info_t, stream=s)
+    for x in (x1, x2):
+        P.copy_(dev(x["P"]))
+        a.copy_(dev(x["a"]))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = oracle.rollout_gru(x["P"], x["a"])
+        assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
+        assert pr.SolveInfo(info_t).converged
