@@ -256,7 +256,7 @@ def recorded_traffic(workload):
 # workloads: device inputs, one step, host copies for the end-to-end leg
 # ---------------------------------------------------------------------------
 class Case:
-    def __init__(self, name, rank, device):
+    def __init__(self, name, rank, device, seq_len=None):
         import torch
 
         import nonlinear_rnn_solve_newton_b200 as pr
@@ -264,12 +264,18 @@ class Case:
         self.pr = pr
         self.name = name
         w = dict(inputs.WORKLOADS[name])
+        base_seed = w["seed"]
+        if seq_len is not None:
+            # the sequence-length sweep: the same draws as tests.inputs.workload_inputs(name, L)
+            w["L"] = int(seq_len)
+            base_seed = [w["seed"], int(seq_len)]
         self.w = w
         self.op, self.B, self.L, self.D, self.bf16 = w["op"], w["B"], w["L"], w["D"], w["bf16"]
         self.N = self.B * self.L * self.D
         self.device = device
         self.tol, self.max_iters = 1e-4, 32
-        seed = w["seed"] if rank == 0 else [w["seed"], 1000 + rank]
+        seed = base_seed if rank == 0 else [base_seed, 1000 + rank] if not isinstance(
+            base_seed, list) else base_seed + [1000 + rank]
         B, L, D = self.B, self.L, self.D
         self.out_dtype = None
         if self.op == "proj":
@@ -381,7 +387,7 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     maybe_init_pg(world, "nccl")
     pr.load()
-    cs = Case(args.workload, rank, device)
+    cs = Case(args.workload, rank, device, args.seq_len)
     op, B, L, D, bf16, N = cs.op, cs.B, cs.L, cs.D, cs.bf16, cs.N
     stream = torch.cuda.current_stream()
 
@@ -405,7 +411,10 @@ def run_ours(args, world, rank, local):
     # ---- optional: the step as a CUDA graph (removes the per-call host cost
     # that dominates latency-bound workloads; the graph holds the same launches)
     graph = None
-    use_graph = args.graph if args.graph is not None else args.workload == "gru_s"
+    # (default: the small and the short-sequence workloads, where host-side call
+    # cost is a visible part of a step)
+    use_graph = (args.graph if args.graph is not None
+                 else args.workload == "gru_s" or (args.seq_len is not None and args.seq_len <= 1024))
     if use_graph:
         gs = torch.cuda.Stream(device)
         gs.wait_stream(stream)
@@ -911,6 +920,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--no-sequential", action="store_true",
                     help="skip the sequential-application context timings")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override L (the sequence-length sweep, e.g. 64 .. 16384 for gru_l)")
     ap.add_argument("--graph", dest="graph", action="store_true", default=None,
                     help="time the step as CUDA graph replays (default for gru_s)")
     ap.add_argument("--no-graph", dest="graph", action="store_false")
