@@ -85,8 +85,18 @@ constexpr int kWalkMinTiles = 200;
 // Below this many tiles the walker uses 16-warp CTAs.
 constexpr int kWalkWideTiles = 512;
 // Below this many 32-channel tiles (4 per SM on B200) the solves' walker uses
-// 8-channel tiles.
+// 8-channel tiles, provided each tile is long enough for the better balance to
+// outweigh the fixed cost of four times as many tiles (pipeline fill, the first
+// stage's copy latency).  Measured on B200, GRU B=8 D=1024 with CUDA-graph
+// replay, 8- vs 32-channel tiles: L=64 37 vs 21 us, 512 65 vs 51 us, 1024 99 vs
+// 92 us, 1536 132 vs 128 us, 2048 164 vs 165 us, 3072 222 vs 238 us, 4096 289
+// vs 311 us; the LSTM crosses over at the same length (1536: 289 vs 288 us,
+// 2048: 358 vs 378 us).
 constexpr int kWalkNarrowTiles = 4 * 148;
+#ifndef PARARNN_NARROW_MIN_LEN
+#define PARARNN_NARROW_MIN_LEN 2048
+#endif
+constexpr long long kWalkNarrowMinLen = PARARNN_NARROW_MIN_LEN;
 // The solves' walker on 8-channel tiles.  A warp holds 8 channels x 4
 // segments; with S steps per segment, segment k of a warp starts 24 S k words
 // (GRU, fp32 rows of 3 gates) or 8 S k words (LSTM gate planes) into the stage,
@@ -231,7 +241,8 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
     // 8-channel tiles (a warp = 8 channels x 4 segments) cut the tail to < 2%.
     const int ww = opts ? opts->walk_width : 0;
     if (is_newton(op))
-      pl.CW_walk = (ww == 8 || ww == 32) ? ww : (ntiles < kWalkNarrowTiles ? 8 : 32);
+      pl.CW_walk = (ww == 8 || ww == 32) ? ww
+                   : (ntiles < kWalkNarrowTiles && L >= kWalkNarrowMinLen ? 8 : 32);
     if (pl.CW_walk == 8) {
       pl.S_walk = kNarrowSteps;
       pl.NW_walk = kNarrowWarps;
