@@ -67,6 +67,13 @@ namespace {
 #ifndef PARARNN_WALK_MINB_WIDE
 #define PARARNN_WALK_MINB_WIDE 2
 #endif
+// the same for the GRU solve's 32-channel walker, fp32 and bf16 gates
+#ifndef PARARNN_WALK_MINB_GRU_F32
+#define PARARNN_WALK_MINB_GRU_F32 PARARNN_WALK_MINB_WIDE
+#endif
+#ifndef PARARNN_WALK_MINB_GRU_BF16
+#define PARARNN_WALK_MINB_GRU_BF16 PARARNN_WALK_MINB
+#endif
 constexpr int kWalkStepsGru = PARARNN_WALK_STEPS_GRU;
 constexpr int kWalkStepsLstm = PARARNN_WALK_STEPS_LSTM;
 constexpr int kWalkStepsScanDiag = PARARNN_WALK_STEPS_SCAN_DIAG;
@@ -112,6 +119,24 @@ constexpr long long kWalkNarrowMinLen = PARARNN_NARROW_MIN_LEN;
 #define PARARNN_NARROW_WARPS 4
 #endif
 constexpr int kNarrowSteps = PARARNN_NARROW_STEPS;
+// Resident-CTA targets (launch bounds) of the 8-channel walker.  Measured on
+// B200 (B=8, L=4096, D=1024): the fp32 GRU walker at a target of 2 takes 108
+// registers (4 CTAs per SM) and 288 us, at 4 it takes 96 (5 CTAs, the shared-
+// memory limit) and 263 us, at 5 it takes 80 (still 5 CTAs) and 277 us; the
+// LSTM walker at 2 takes 166 registers (3 CTAs) and 658 us, at 3 156 (3 CTAs)
+// and 695 us, at 4 128 with spills (4 CTAs) and 690 us.
+#ifndef PARARNN_NARROW_MINB_GRU
+#define PARARNN_NARROW_MINB_GRU 4
+#endif
+#ifndef PARARNN_NARROW_MINB_GRU_BF16
+#define PARARNN_NARROW_MINB_GRU_BF16 3
+#endif
+#ifndef PARARNN_NARROW_MINB_LSTM
+#define PARARNN_NARROW_MINB_LSTM 2
+#endif
+constexpr int kNarrowMinBlocksGru = PARARNN_NARROW_MINB_GRU;
+constexpr int kNarrowMinBlocksGruBf16 = PARARNN_NARROW_MINB_GRU_BF16;
+constexpr int kNarrowMinBlocksLstm = PARARNN_NARROW_MINB_LSTM;
 constexpr int kNarrowWarps = PARARNN_NARROW_WARPS;
 static_assert(kNarrowWarps * 4 * kNarrowSteps <= 256, "TMA box rows");
 
@@ -437,19 +462,20 @@ const void* walk_kernel_narrow(size_t* smem) {
 
 const void* select_walk_kernel(int op, bool bf16, int nw, int cw, size_t* smem) {
   if (cw == 8 && op == kGru)
-    return bf16 ? walk_kernel_narrow<kGru, __nv_bfloat16, kWalkMinBlocks>(smem)
-                : walk_kernel_narrow<kGru, float, kWalkMinBlocksWide>(smem);
+    return bf16 ? walk_kernel_narrow<kGru, __nv_bfloat16, kNarrowMinBlocksGruBf16>(smem)
+                : walk_kernel_narrow<kGru, float, kNarrowMinBlocksGru>(smem);
   if (cw == 8 && op == kLstm)
-    return bf16 ? walk_kernel_narrow<kLstm, __nv_bfloat16, kWalkMinBlocksWide>(smem)
-                : walk_kernel_narrow<kLstm, float, kWalkMinBlocksWide>(smem);
+    return bf16 ? walk_kernel_narrow<kLstm, __nv_bfloat16, kNarrowMinBlocksLstm>(smem)
+                : walk_kernel_narrow<kLstm, float, kNarrowMinBlocksLstm>(smem);
   switch (op) {
     case kScanDiag:
       return walk_kernel_nw<kScanDiag, float, kWalkStepsScanDiag, kWalkMinBlocks>(nw, smem);
     case kScanBlock2:
       return walk_kernel_nw<kScanBlock2, float, kWalkStepsScanBlock2, kWalkMinBlocks>(nw, smem);
     case kGru:
-      return bf16 ? walk_kernel_nw<kGru, __nv_bfloat16, kWalkStepsGru, kWalkMinBlocks>(nw, smem)
-                  : walk_kernel_nw<kGru, float, kWalkStepsGru, kWalkMinBlocksWide>(nw, smem);
+      return bf16 ? walk_kernel_nw<kGru, __nv_bfloat16, kWalkStepsGru, PARARNN_WALK_MINB_GRU_BF16>(
+                        nw, smem)
+                  : walk_kernel_nw<kGru, float, kWalkStepsGru, PARARNN_WALK_MINB_GRU_F32>(nw, smem);
     default:
       return bf16
                  ? walk_kernel_nw<kLstm, __nv_bfloat16, kWalkStepsLstm, kWalkMinBlocksWide>(nw, smem)

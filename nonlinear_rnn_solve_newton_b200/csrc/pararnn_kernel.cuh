@@ -291,6 +291,10 @@ __device__ __forceinline__ float max_abs_nan(float m, float r) {
   return y;
 }
 
+// s (1 - s), the logistic derivative, as s - s^2 in one fused multiply-add
+// (measured on B200: 1-2% off the GRU and LSTM solves against s * (1 - s)).
+__device__ __forceinline__ float dsig(float s) { return fmaf(-s, s, s); }
+
 // ParaGRU: h' = (1-z) h + z c; returns f and dh'/dh.
 __device__ __forceinline__ void gru_cell(const float* p, const float* w, float h, float& f,
                                          float& J) {
@@ -300,8 +304,8 @@ __device__ __forceinline__ void gru_cell(const float* p, const float* w, float h
   float c = tanh_f(fmaf(w[2], rh, p[2]));
   float cmh = c - h;
   f = fmaf(z, cmh, h);
-  float dz = z * (1.0f - z) * w[0];
-  float dr = r * (1.0f - r) * w[1];
+  float dz = dsig(z) * w[0];
+  float dr = dsig(r) * w[1];
   float du = w[2] * fmaf(h, dr, r);
   float dc = fmaf(-c, c, 1.0f) * du;
   J = fmaf(cmh, dz, 1.0f - z) + z * dc;
@@ -318,10 +322,10 @@ __device__ __forceinline__ void lstm_cell(const float* p, const float* w, float 
   float tc = tanh_f(cn);
   fc = cn;
   fh = og * tc;
-  float di = ig * (1.0f - ig) * w[0];
-  float df = fg * (1.0f - fg) * w[1];
+  float di = dsig(ig) * w[0];
+  float df = dsig(fg) * w[1];
   float dg = fmaf(-gg, gg, 1.0f) * w[2];
-  float dov = og * (1.0f - og) * w[3];
+  float dov = dsig(og) * w[3];
   float dcn_dh = fmaf(df, c, fmaf(di, gg, ig * dg));
   float odtc = og * fmaf(-tc, tc, 1.0f);
   J[0][0] = fg;
