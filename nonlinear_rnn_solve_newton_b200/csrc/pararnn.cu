@@ -501,9 +501,11 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Row-major tensor [outer][mid][inner] (mid = 1 for 2-D), TMA box = inner x mid x rows.
+// promo: the L2 promotion of the copies' DRAM reads.
 bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, size_t esize,
                 unsigned long long inner, unsigned long long mid, unsigned long long outer,
-                unsigned box_inner, unsigned box_rows, unsigned box_mid = 0) {
+                unsigned box_inner, unsigned box_rows, unsigned box_mid = 0,
+                CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return false;
   CUresult r;
@@ -514,14 +516,14 @@ bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, size_t
     const cuuint32_t box[3] = {box_inner, box_mid ? box_mid : (cuuint32_t)mid, box_rows};
     r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else {
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {inner * esize};
     const cuuint32_t box[2] = {box_inner, box_rows};
     r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
   return r == CUDA_SUCCESS;
 }
@@ -542,7 +544,15 @@ bool make_walk_maps(int op, bool bf16, const KParams& kp, int T, int CW, TmaMaps
       if (!aligned(kp.in0, 16) || (D * (long long)es) % 16 != 0) return false;
       // 8-channel LSTM tiles are staged one gate plane per copy
       const unsigned box_mid = (op == kLstm && CW == 8) ? 1u : 0u;
-      return encode_map(&tm->in0, kp.in0, dt, es, D, G, rows, (unsigned)CW, T, box_mid);
+      // An 8-channel tile reads 32-byte row pieces.  With 256-byte promotion the
+      // other seven tiles of each promoted block must use it before it leaves L2,
+      // and at 5 CTAs per SM many do not: measured on B200 (GRU, B=8, L=4096,
+      // D=1024, ncu) DRAM reads of 752 MB for 403 MB of gates, against 544 MB
+      // with 64-byte promotion (663 MB at 128, 692 MB with none), all at the same
+      // solve time; the LSTM 615 -> 573 MB for 537 MB of gates.
+      const CUtensorMapL2promotion promo =
+          CW == 8 ? CU_TENSOR_MAP_L2_PROMOTION_L2_64B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+      return encode_map(&tm->in0, kp.in0, dt, es, D, G, rows, (unsigned)CW, T, box_mid, promo);
     }
     case kScanDiag:
       if (!aligned(kp.in0, 16) || !aligned(kp.in1, 16) || (D * 4) % 16 != 0) return false;
