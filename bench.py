@@ -436,8 +436,8 @@ def run_ours(args, world, rank, local):
     # ---- timed region: exactly K steps ---------------------------------------
     K = args.steps
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
-    # The clock sampler starts (NVML queries, its thread) before the bracket:
-    # started inside it, it delayed the first launch by ~0.14 ms on B200.
+    # The clock sampler (NVML queries, its thread) starts before the bracket,
+    # so its start-up is not timed.
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
