@@ -90,6 +90,9 @@ _i64 = ctypes.c_int64
 def load(build_if_missing: bool = True):
     """Load libpararnn.so (building it in-tree with nvcc if it is missing or stale)."""
     global _lib
+    lib = _lib
+    if lib is not None:  # loaded: no lock on the per-call path
+        return lib
     with _lock:
         if _lib is None:
             if build_if_missing and _build.needs_build():
@@ -146,16 +149,30 @@ def load(build_if_missing: bool = True):
             lib.pararnn_status_string.argtypes = [ctypes.c_int]
             lib.pararnn_status_string.restype = ctypes.c_char_p
             lib.pararnn_version.restype = ctypes.c_int32
+            _ws_sizes.clear()  # sizes are the loaded library's answers
             _lib = lib
     return _lib
 
 
+_ws_sizes = {}
+
+
 def workspace_size(op: int, B: int, L: int, D: int, max_iters: int = 0, opts: Options | None = None):
-    n = load().pararnn_workspace_size(int(op), int(B), int(L), int(D), int(max_iters),
-                                      ctypes.byref(opts) if opts is not None else None)
-    if n == 0:
-        raise PararnnError(1, "workspace_size")
-    return int(n)
+    """Workspace bytes of a call: the library's answer, remembered per distinct
+    argument tuple (options included) until another library is loaded."""
+    lib = load()
+    key = (int(op), int(B), int(L), int(D), int(max_iters), None if opts is None else bytes(opts))
+    n = _ws_sizes.get(key)
+    if n is None:
+        n = lib.pararnn_workspace_size(int(op), int(B), int(L), int(D), int(max_iters),
+                                       ctypes.byref(opts) if opts is not None else None)
+        if n == 0:
+            raise PararnnError(1, "workspace_size")
+        n = int(n)
+        if len(_ws_sizes) > 4096:
+            _ws_sizes.clear()
+        _ws_sizes[key] = n
+    return n
 
 
 def _ptr(t):

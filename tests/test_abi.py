@@ -140,3 +140,20 @@ def test_binding_refuses_cpu_tensors():
     P = torch.zeros(1, 4, 3, 2, dtype=torch.float32)
     with pytest.raises(ValueError, match="CUDA"):
         pr.solve_gru(P, torch.zeros(3, 2, dtype=torch.float32))
+
+
+def test_workspace_size_remembered_per_argument_tuple():
+    """The binding remembers sizes per (op, B, L, D, max_iters, options bytes):
+    changing an Options object in place must give the size of its new value."""
+    import nonlinear_rnn_solve_newton_b200 as pr
+
+    o = pr.Options(regime=1)
+    lookback = pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32, o)
+    assert pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32, o) == lookback
+    o.regime = 2
+    walk = pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 32, o)
+    assert walk == pr.load().pararnn_workspace_size(pr.OP_GRU, 8, 4096, 1024, 32,
+                                                     ctypes.byref(pr.Options(regime=2)))
+    assert walk != lookback
+    with pytest.raises(pr.PararnnError):
+        pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 500, o)
