@@ -59,6 +59,23 @@ MUTANTS = {
                                  "for (int64_t k = 1; k < c->K; ++k) s +="),
     "backward_gru_forward_time": ("double lam = x->gh[IDX3(bb, t, d, L, D)] + lam_next;",
                                   "double lam = x->gh[IDX3(bb, t, d, L, D)];"),
+    "rho_max_over_first_channel_only": (
+        "  for (int64_t c = 0; c < n; ++c) {\n    if (!(cmax[c] <= rho)) rho = cmax[c];",
+        "  for (int64_t c = 0; c < 1; ++c) {\n    if (!(cmax[c] <= rho)) rho = cmax[c];"),
+    "rho_drops_nan": ("if (!(cmax[c] <= rho)) rho = cmax[c];", "if (cmax[c] > rho) rho = cmax[c];"),
+    "scan_diag_ignores_h0": ("  double x = c->x0 ? c->x0[bb * c->D + d] : 0.0;", "  double x = 0.0;"),
+    "lstm_rollout_ignores_c0": ("double sc = x->c0 ? x->c0[bb * D + d] : 0.0;", "double sc = 0.0;"),
+    "newton_lstm_ignores_c0": (
+        "  double m = 0.0;\n  for (int64_t t = 0; t < L; ++t) {\n    double cp, hp;\n    if (t == 0) {\n"
+        "      cp = x->c0 ? x->c0[bb * D + d] : 0.0;",
+        "  double m = 0.0;\n  for (int64_t t = 0; t < L; ++t) {\n    double cp, hp;\n    if (t == 0) {\n"
+        "      cp = 0.0;"),
+    "backward_gru_da_z_without_h": ("da[0] += lam * dfdz * hp;", "da[0] += lam * dfdz;"),
+    "backward_lstm_dh0_from_c": ("if (x->dh0) x->dh0[bb * D + d] = mh;",
+                                 "if (x->dh0) x->dh0[bb * D + d] = mc;"),
+    "backward_lstm_da_without_h": ("      da[g] += v * hp;", "      da[g] += v;"),
+    "mhgru_ignores_h0": ("hp[i] = (t == 0) ? (x->h0 ? x->h0[bb * D + g * NB + i] : 0.0)",
+                         "hp[i] = (t == 0) ? 0.0"),
 }
 
 
