@@ -817,10 +817,33 @@ def cpu_baseline(x, op, B, L, D, budget_s=15.0):
     else:
         oracle.rollout_lstm(Ps, as_)
     dtr = time.perf_counter() - t1
+    # the same two programs on one host thread, on the first channels of the
+    # sample (about 3 s of single-threaded work, estimated from the calibration)
+    n1 = int(max(1, min(ndd, 3.0 / max(per_chan * cores, 1e-9))))
+    P1, a1 = Ps[:1, :, :, :n1], as_[:, :n1]
+    oracle.set_threads(1)
+    try:
+        t2 = time.perf_counter()
+        if op == "gru":
+            oracle.newton_gru(P1, a1, tol=1e-4, max_iters=32)
+        else:
+            oracle.newton_lstm(P1, a1, tol=1e-4, max_iters=32)
+        dt1 = time.perf_counter() - t2
+        t3 = time.perf_counter()
+        if op == "gru":
+            oracle.rollout_gru(P1, a1)
+        else:
+            oracle.rollout_lstm(P1, a1)
+        dtr1 = time.perf_counter() - t3
+    finally:
+        oracle.set_threads(0)
     return {"value": steps / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"serial fp64 Newton on B={nb} x D={ndd} channels x L={L} "
                       f"({steps} channel-steps, {res.iterations} iterations, {dt:.1f} s)",
-            "rollout_channel_steps_per_s": steps / dtr}
+            "rollout_channel_steps_per_s": steps / dtr,
+            "single_thread": {"newton_channel_steps_per_s": n1 * L / dt1,
+                              "rollout_channel_steps_per_s": n1 * L / dtr1,
+                              "sample": f"{n1} channels x L={L} on one host thread"}}
 
 
 # ---------------------------------------------------------------------------

@@ -60,3 +60,18 @@ def test_reference_arm_runs_every_new_workload(capsys):
         line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
         assert line["impl"] == "reference" and line["value"] > 0
         assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_cpu_baseline_reports_threaded_and_single_thread():
+    """The CPU leg times the oracle's Newton and rollout on the host cores and
+    on one thread (a small GRU case, CPU only)."""
+    import bench
+    import oracle
+    from tests import inputs
+
+    x = inputs.gru_inputs(1, 64, 8, seed=5)
+    out = bench.cpu_baseline(x, "gru", 1, 64, 8, budget_s=0.05)
+    assert out["kind"] == "oracle" and out["cores"] >= 1 and out["value"] > 0
+    st = out["single_thread"]
+    assert st["newton_channel_steps_per_s"] > 0 and st["rollout_channel_steps_per_s"] > 0
+    assert oracle.get_threads() == out["cores"]   # the thread count is restored
