@@ -246,6 +246,45 @@ def test_gru_jacobian_finite_difference(oracle):
         assert abs((fp - fm) / (2 * e) - J) < 1e-8 * max(1, abs(J))
 
 
+def test_lstm_jacobian_finite_difference(oracle):
+    """Central differences of the oracle's own LSTM step in c and in h agree with
+    all four entries of its analytic Jacobian (row-major d(c', h')/d(c, h))."""
+    rng = np.random.default_rng(16)
+    e = 1e-5
+    for _ in range(30):
+        p = rng.standard_normal(4)
+        w = rng.uniform(-0.5, 0.5, 4)
+        c, h = rng.standard_normal(2)
+        _, _, J = oracle.lstm_cell(p, w, c, h)
+        J = np.asarray(J).reshape(2, 2)
+        cp, hp_, _ = oracle.lstm_cell(p, w, c + e, h)
+        cm, hm, _ = oracle.lstm_cell(p, w, c - e, h)
+        dc = np.array([(cp - cm) / (2 * e), (hp_ - hm) / (2 * e)])   # column d/dc
+        cp, hp_, _ = oracle.lstm_cell(p, w, c, h + e)
+        cm, hm, _ = oracle.lstm_cell(p, w, c, h - e)
+        dh = np.array([(cp - cm) / (2 * e), (hp_ - hm) / (2 * e)])   # column d/dh
+        fd = np.stack([dc, dh], axis=1)
+        np.testing.assert_allclose(fd, J, atol=1e-8, rtol=1e-8)
+
+
+def test_mhgru_jacobian_finite_difference(oracle):
+    """Central differences of the oracle's own multi-head step, one input channel
+    at a time, agree with its 8x8 Jacobian's columns."""
+    rng = np.random.default_rng(17)
+    e = 1e-5
+    for _ in range(10):
+        U = rng.uniform(-0.6, 0.6, (3, 8, 8))
+        p = rng.standard_normal((3, 8))
+        h = rng.standard_normal(8)
+        _, J = oracle.mhgru_cell(p, U, h)
+        for j in range(8):
+            dh = np.zeros(8)
+            dh[j] = e
+            fp, _ = oracle.mhgru_cell(p, U, h + dh)
+            fm, _ = oracle.mhgru_cell(p, U, h - dh)
+            np.testing.assert_allclose((fp - fm) / (2 * e), J[:, j], atol=1e-8, rtol=1e-8)
+
+
 # --------------------------------------------------------------------------
 # Rollouts against the library cells
 # --------------------------------------------------------------------------
