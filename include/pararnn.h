@@ -118,8 +118,9 @@ typedef struct {
  *                else 8), 8 or 16.
  *  walk_width  : channels per tile of the walk regime's tensor-copy walker for
  *                the GRU / LSTM solves: 0 = automatic (8 when 32-channel tiles
- *                would be fewer than 4 per SM -- finer tiles balance the SMs --
- *                else 32), 8 or 32.  The scans always use 32. */
+ *                would be fewer than 4 per SM and L >= 2048 -- finer tiles
+ *                balance the SMs once sequences are long enough to repay their
+ *                start-up -- else 32), 8 or 32.  The scans always use 32. */
 typedef struct {
   int32_t iters_first;
   int32_t iters_next;
