@@ -377,6 +377,27 @@ class Case:
         return None
 
 
+def workload_name(name, B, L, D, K=None, G=None):
+    """The `config.workload` string of a workload (the same in both arms)."""
+    wl = {"gru_l": "ParaGRU Newton solve fp32",
+          "lm": "ParaGRU Newton solve, bf16 P, fp32 state",
+          "deer": "ParaGRU Newton solve fp32 (DEER shape)",
+          "gru_s": "ParaGRU Newton solve fp32 (small)",
+          "lstm": "ParaLSTM Newton solve fp32",
+          "scan": "diagonal affine scan fp32",
+          "block2": "2x2 block affine scan fp32",
+          "gru_bwd": "ParaGRU backward pass fp32",
+          "lstm_bwd": "ParaLSTM backward pass fp32",
+          "mhgru": "multi-head GRU Newton solve fp32, dense 8x8 recurrence blocks",
+          "proj": "input projection x W^T + bias, bf16 in, fp32 out (tcgen05)",
+          "proj_lm": "input projection x W^T + bias, bf16 in, bf16 out (tcgen05)",
+          }[name]
+    out = f"{wl} B={B} L={L} D={D}"
+    if K is not None:
+        out += f" K={K} G={G} (M={B * L}, N={G * D})"
+    return out
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -687,22 +708,8 @@ def run_ours(args, world, rank, local):
         cpu = cpu_baseline(cs.x, op, B, L, D, budget_s=args.cpu_seconds)
 
     if rank == 0:
-        wl = {"gru_l": "ParaGRU Newton solve fp32",
-              "lm": "ParaGRU Newton solve, bf16 P, fp32 state",
-              "deer": "ParaGRU Newton solve fp32 (DEER shape)",
-              "gru_s": "ParaGRU Newton solve fp32 (small)",
-              "lstm": "ParaLSTM Newton solve fp32",
-              "scan": "diagonal affine scan fp32",
-              "block2": "2x2 block affine scan fp32",
-              "gru_bwd": "ParaGRU backward pass fp32",
-              "lstm_bwd": "ParaLSTM backward pass fp32",
-              "mhgru": "multi-head GRU Newton solve fp32, dense 8x8 recurrence blocks",
-              "proj": "input projection x W^T + bias, bf16 in, fp32 out (tcgen05)",
-              "proj_lm": "input projection x W^T + bias, bf16 in, bf16 out (tcgen05)",
-              }[args.workload]
-        wlname = f"{wl} B={B} L={L} D={D}"
-        if op == "proj":
-            wlname += f" K={cs.K} G={cs.G} (M={B * L}, N={cs.G * D})"
+        wlname = workload_name(args.workload, B, L, D, cs.K if op == "proj" else None,
+                               cs.G if op == "proj" else None)
         cfg = {"workload": wlname, "B": B, "L": L, "D": D,
                "launch": "CUDA graph replay" if graph is not None else "direct calls",
                "parallelism": f"replicas x{world} (independent batches)",
@@ -933,9 +940,12 @@ def run_reference(args, world, rank, local):
             "steps": args.steps, "warmup": max(args.warmup, 1), "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded numpy)",
-            "config": {"workload": (f"oracle {what} from the {args.workload} workload" if op == "proj"
-                                    else f"oracle {what}, sample of B=1 x D={nd} x L={L} "
-                                         f"from the {args.workload} workload (B={B}, D={D})")},
+            "config": {"workload": workload_name(args.workload, B, L, D,
+                                                 w.get("K") if op == "proj" else None,
+                                                 w.get("G") if op == "proj" else None),
+                       "B": B, "L": L, "D": D, "parallelism": "rank 0 only, host cores",
+                       "sample": (f"oracle {what}" if op == "proj"
+                                  else f"oracle {what} on B=1 x D={nd} x L={L} per step")},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": (what if op == "proj" else f"B=1, D={nd}, L={L} per step")},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -54,12 +54,19 @@ def test_reference_arm_runs_every_new_workload(capsys):
     import argparse
     import json
 
-    for wl in ("proj", "mhgru"):
+    from tests import inputs
+
+    for wl in ("proj", "mhgru", "gru_l"):
         args = argparse.Namespace(workload=wl, steps=1, warmup=1)
         bench.run_reference(args, 1, 0, 0)
         line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
         assert line["impl"] == "reference" and line["value"] > 0
         assert line["e2e"]["h2d_bytes_per_step"] == 0
+        # the same config.workload as our arm's line for this workload
+        w = inputs.WORKLOADS[wl]
+        assert line["config"]["workload"] == bench.workload_name(
+            wl, w["B"], w["L"], w["D"], w.get("K"), w.get("G"))
+        assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
 
 
 def test_cpu_baseline_reports_threaded_and_single_thread():
