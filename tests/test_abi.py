@@ -129,6 +129,64 @@ def test_input_projection_host_validation(lib):
     assert lib.pararnn_input_projection(fake, fake, None, fake, 1, 16, 0, 64, None, None) == 0
 
 
+def test_other_entry_points_validate_on_the_host(lib):
+    """The backward passes, decode steps, rollouts, the multi-head solve and the
+    allocation-free solve reject bad arguments before any CUDA call."""
+    vp = ctypes.c_void_p
+    fake, info, ws = vp(4096), vp(8192), vp(1 << 20)
+    f1e4 = ctypes.c_float(1e-4)
+    # GRU backward: (P, dtype, a, h0, h, dh, dP, da, dh0, B, L, D, ws, ws_bytes, status, opts, s)
+    gb = lib.pararnn_solve_gru_backward
+    assert gb(fake, 0, fake, None, fake, fake, fake, fake, None, -1, 8, 4, ws, 1 << 20, None, None,
+              None) == 1
+    assert gb(fake, 7, fake, None, fake, fake, fake, fake, None, 2, 8, 4, ws, 1 << 20, None, None,
+              None) == 1
+    assert gb(None, 0, fake, None, fake, fake, fake, fake, None, 2, 8, 4, ws, 1 << 20, None, None,
+              None) == 1
+    assert gb(fake, 0, fake, None, fake, None, fake, fake, None, 2, 8, 4, ws, 1 << 20, None, None,
+              None) == 1                                   # no upstream gradient
+    assert gb(fake, 0, vp(4098), None, fake, fake, fake, fake, None, 2, 8, 4, ws, 1 << 20, None,
+              None, None) == 1                             # misaligned fp32 weights
+    assert gb(vp(4097), 1, fake, None, fake, fake, fake, fake, None, 2, 8, 4, ws, 1 << 20, None,
+              None, None) == 1                             # misaligned bf16 P
+    # LSTM backward: neither dc nor dh given, or c missing
+    lb = lib.pararnn_solve_lstm_backward
+    assert lb(fake, 0, fake, None, None, fake, fake, None, None, fake, fake, None, None, 2, 8, 4,
+              ws, 1 << 20, None, None, None) == 1
+    assert lb(fake, 0, fake, None, None, None, fake, fake, fake, fake, fake, None, None, 2, 8, 4,
+              ws, 1 << 20, None, None, None) == 1
+    # decode steps and rollouts
+    assert lib.pararnn_step_gru(fake, 0, fake, None, fake, -1, 4, None) == 1
+    assert lib.pararnn_step_gru(fake, 3, fake, None, fake, 2, 4, None) == 1
+    assert lib.pararnn_step_gru(None, 0, fake, None, fake, 2, 4, None) == 1
+    assert lib.pararnn_step_gru(fake, 0, fake, None, fake, 0, 4, None) == 0   # nothing to do
+    assert lib.pararnn_step_lstm(fake, 0, fake, None, None, fake, None, 2, 4, None) == 1
+    assert lib.pararnn_rollout_gru(fake, 0, fake, vp(4098), fake, 2, 8, 4, None) == 1
+    assert lib.pararnn_rollout_gru(fake, 0, fake, None, fake, 2, 0, 4, None) == 0
+    assert lib.pararnn_rollout_lstm(fake, 0, fake, None, None, fake, None, 2, 8, 4, None) == 1
+    # multi-head solve: (P, dtype, U, h0, h, B, L, H, tol, max_iters, ws, ws_bytes, info, opts, s)
+    mh = lib.pararnn_solve_mhgru
+    assert mh(fake, 0, fake, None, fake, -1, 8, 2, f1e4, 4, ws, 1 << 20, info, None, None) == 1
+    assert mh(fake, 0, fake, None, fake, 2, 8, 2, f1e4, 4, ws, 1 << 20, None, None, None) == 1
+    assert mh(fake, 0, fake, None, fake, 2, 8, 2, f1e4, 200, ws, 1 << 20, info, None, None) == 1
+    assert mh(fake, 0, fake, None, fake, 2, 8, 2, ctypes.c_float(float("nan")), 4, ws, 1 << 20,
+              info, None, None) == 1
+    assert mh(fake, 5, fake, None, fake, 2, 8, 2, f1e4, 4, ws, 1 << 20, info, None, None) == 1
+    assert mh(None, 0, fake, None, fake, 2, 8, 2, f1e4, 4, ws, 1 << 20, info, None, None) == 1
+    assert mh(vp(4100), 0, fake, None, fake, 2, 8, 2, f1e4, 4, ws, 1 << 20, info, None,
+              None) == 1                                   # P must be 16-byte aligned
+    assert mh(fake, 0, fake, None, fake, 2, 8, 2, f1e4, 4, ws, 16, info, None, None) == 6
+    assert mh(fake, 0, fake, None, fake, 2, 8, 2, f1e4, 4, None, 1 << 20, info, None, None) == 6
+    # allocation-free solve: negative sizes, and a problem beyond its fixed scratch
+    na = lib.pararnn_solve_gru_noalloc
+    assert na(fake, 0, fake, None, fake, -1, 8, 4, f1e4, 4, info, None, None) == 1
+    import nonlinear_rnn_solve_newton_b200 as pr
+
+    o = ctypes.byref(pr.Options(regime=pr.Options.LOOKBACK, iters_first=8))
+    assert lib.pararnn_workspace_size(2, 64, 1 << 16, 1024, 32, o) > pr.NOALLOC_SCRATCH_BYTES
+    assert na(fake, 0, fake, None, fake, 64, 1 << 16, 1024, f1e4, 32, info, o, None) == 6
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
 
