@@ -279,6 +279,7 @@ def scan_diag(A, b, h0=None, out=None, status=None, opts: Options | None = None,
     _check_dev("h0", h0, torch.float32, (B, D))
     h = torch.empty_like(A) if out is None else out
     _check_dev("out", h, torch.float32, (B, L, D))
+    _check_dev("status", status, torch.int32, (1,))
     n = workspace_size(OP_SCAN_DIAG, B, L, D, 0, opts)
     ws = _workspace(n, A.device, stream)
     st = lib.pararnn_scan_diag(_ptr(A), _ptr(b), _ptr(h0), _ptr(h), B, L, D, _ptr(ws), ws.numel(),
@@ -297,6 +298,7 @@ def scan_block2(A, b, x0=None, out=None, status=None, opts: Options | None = Non
     _check_dev("x0", x0, torch.float32, (B, D, 2))
     x = torch.empty_like(b) if out is None else out
     _check_dev("out", x, torch.float32, (B, L, D, 2))
+    _check_dev("status", status, torch.int32, (1,))
     n = workspace_size(OP_SCAN_BLOCK2, B, L, D, 0, opts)
     ws = _workspace(n, A.device, stream)
     st = lib.pararnn_scan_block2(_ptr(A), _ptr(b), _ptr(x0), _ptr(x), B, L, D, _ptr(ws),
@@ -330,6 +332,7 @@ def solve_gru(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
     _check_dev("out", h, torch.float32, (B, L, D))
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
     n = workspace_size(OP_GRU, B, L, D, max_iters, opts)
     ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D, float(tol),
@@ -357,6 +360,7 @@ def solve_mhgru(P, U, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
     _check_dev("out", h, torch.float32, (B, L, D))
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
     n = workspace_size(OP_MHGRU, B, L, D, max_iters, opts)
     ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_mhgru(_ptr(P), dt, _ptr(U), _ptr(h0), _ptr(h), B, L, H, float(tol),
@@ -388,6 +392,7 @@ def solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32, out=None, info=No
     _check_dev("h", h, torch.float32, (B, L, D))
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
     n = workspace_size(OP_LSTM, B, L, D, max_iters, opts)
     ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_lstm(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h), B, L,
@@ -421,6 +426,7 @@ def solve_gru_noalloc(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None
     _check_dev("out", h, torch.float32, (B, L, D))
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
     st = lib.pararnn_solve_gru_noalloc(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D,
                                        float(tol), int(max_iters), _ptr(info),
                                        ctypes.byref(opts) if opts is not None else None,
@@ -453,6 +459,7 @@ def solve_gru_backward(P, a, h, dh, h0=None, out=None, status=None,
     _check_dev("dP", dP, torch.float32, (B, L, 3, D))
     _check_dev("da", da, torch.float32, (3, D))
     _check_dev("dh0", dh0, torch.float32, (B, D))
+    _check_dev("status", status, torch.int32, (1,))
     n = workspace_size(OP_GRU_BACKWARD, B, L, D, 0, opts)
     ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_gru_backward(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), _ptr(dh),
@@ -486,6 +493,11 @@ def solve_lstm_backward(P, a, c, h, dc, dh, c0=None, h0=None, out=None, status=N
         dh0 = torch.empty((B, D), dtype=torch.float32, device=P.device)
     else:
         dP, da, dc0, dh0 = out
+    _check_dev("dP", dP, torch.float32, (B, L, 4, D))
+    _check_dev("da", da, torch.float32, (4, D))
+    _check_dev("dc0", dc0, torch.float32, (B, D))
+    _check_dev("dh0", dh0, torch.float32, (B, D))
+    _check_dev("status", status, torch.int32, (1,))
     n = workspace_size(OP_LSTM_BACKWARD, B, L, D, 0, opts)
     ws = _workspace(n, P.device, stream)
     st = lib.pararnn_solve_lstm_backward(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c),
