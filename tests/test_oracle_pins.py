@@ -709,6 +709,23 @@ def test_mhgru_no_recurrence_single_iteration(oracle):
     assert res.iterations == 1 and res.rho[1] < 1e-13
 
 
+def test_mhgru_newton_quadratic_convergence(oracle):
+    """Newton on the dense-block system converges quadratically too (measured
+    rho_{k+1} / rho_k^2 <= 0.22 at these seeds); a wrong or missing term of the
+    8x8 Jacobian degrades it to linear convergence."""
+    for seed, u_scale in ((726, 0.3), (728, 0.6)):
+        x = inputs.mhgru_inputs(2, 256, 2, seed=seed, u_scale=u_scale)
+        res = oracle.newton_mhgru(x["P"], x["U"], tol=1e-13, max_iters=30)
+        assert res.converged
+        rho = res.rho
+        checked = 0
+        for k in range(len(rho) - 1):
+            if 1e-9 < rho[k] < 0.05:
+                assert rho[k + 1] <= 50.0 * rho[k] ** 2, (k, rho)
+                checked += 1
+        assert checked >= 1
+
+
 def test_mhgru_prefix_exactness(oracle):
     L = 6
     x = inputs.mhgru_inputs(2, L, 2, seed=725, u_scale=0.6, h0_normal=True)
