@@ -1,14 +1,15 @@
 #!/usr/bin/env python
 """Benchmark of the ParaGRU Newton solve (and the diagonal affine scan) on B200.
 
-One step = one complete Newton solve, all iterations, of the ParaGRU layer
-B=8, L=4096, D=1024 in fp32 (P ~ N(0,1), a ~ U(-0.5,0.5), h0 = 0, tol 1e-4,
-max 32 iterations) -- the workload shape of the diagonal-scan configuration,
-whose Newton solve is its headline metric.  The same run times the diagonal
-affine scan at that shape (the scan HBM GB/s half of the metric).
+One step = one complete Newton solve, all iterations, of the LM-width ParaGRU
+layer: B=8, L=8192, D=4096, bf16 projected gate inputs P ~ N(0,1), fp32 state,
+Jacobians and scan, a ~ U(-0.5,0.5), h0 = 0, tol 1e-4, max 32 iterations.  The
+same run times the diagonal affine scan at that width (B=8, L=8192, D=4096,
+fp32: the scan HBM GB/s half of the metric) and, as extra keys, the fp32 solve
+and scan at B=8, L=4096, D=1024.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gru_l|lm|deer|gru_s|lstm]
+                    [--workload lm|gru_l|deer|gru_s|lstm|...]
 
 Under torchrun (N > 1) every rank solves its own independent batch (weak
 scaling, no data-path collective); the time is the max over ranks.  Rank 0
@@ -34,10 +35,8 @@ from tests import inputs  # noqa: E402  (seeded synthetic inputs only)
 
 METRIC = "Newton-solve channel-steps/sec (B*L*D) and scan HBM GB/s, % of B200 HBM peak"
 UNIT = "channel-steps/s"
-MUFU_PER_SM_PER_CLK = 16        # ex2 / rcp issue rate per SM per clock
 SMS = 148
 MUFU_PER_STEP = {"gru": 6, "lstm": 10}   # (ex2 + rcp) per sigmoid/tanh, per channel-step
-FMA_PER_SM_PER_CLK = 128        # fp32 FMA lanes per SM
 # multi-head GRU, per channel-step and Newton evaluation: gate matvecs 24 +
 # Jacobian 24 + b_t 8 + map composition (8x8 product + matvec) 72 = 128 FMA
 MHGRU_FMA_PER_STEP = 128
@@ -50,6 +49,45 @@ def peaks():
         return float(j["hbm_gbs"]), "measured", j
     except Exception:
         return 6650.0, "fallback", {}
+
+
+def measure_pipe_peak(pr, pipe, device, local, target_ms=150.0):
+    """Measured peak of one functional-unit pipe on this GPU: the library's
+    throughput probe (ex2 + rcp for the special-function pipe, fp32 FMA)
+    timed with CUDA events over about `target_ms`, with the SM clock sampled
+    meanwhile.  Returns the rate per SM per clock, so that a kernel timed at
+    another clock is compared with the peak at its own clock."""
+    import torch
+
+    sink = torch.zeros(1, device=device)
+    stream = torch.cuda.current_stream(device)
+    iters = 64
+    for _ in range(2):                      # warm-up
+        pr.probe_rate(pipe, iters, sink)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    pr.probe_rate(pipe, iters, sink)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    one = max(e0.elapsed_time(e1), 1e-3)
+    iters = int(max(64, min(1 << 20, iters * 2.0 / one)))    # ~2 ms per launch
+    n = int(max(4, target_ms / 2.0))
+    pr.probe_rate(pipe, iters, sink)
+    torch.cuda.synchronize()
+    with ClockSampler(local, period_s=0.002) as clk:
+        e0.record(stream)
+        ops = sum(pr.probe_rate(pipe, iters, sink) for _ in range(n))
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    c = clk.summary()
+    nsm = torch.cuda.get_device_properties(device).multi_processor_count
+    mhz = c.get("sm_mhz") or 1965.0
+    rate = ops / (ms * 1e-3)
+    return {"ops_per_s": rate, "per_sm_per_clk": rate / (nsm * mhz * 1e6), "sm_mhz": mhz,
+            "sms": nsm, "ms": ms, "launches": n, "clock_reasons": c.get("reasons"),
+            "clock_source": c.get("source")}
 
 
 # ---------------------------------------------------------------------------
@@ -385,6 +423,7 @@ def workload_name(name, B, L, D, K=None, G=None):
           "gru_s": "ParaGRU Newton solve fp32 (small)",
           "lstm": "ParaLSTM Newton solve fp32",
           "scan": "diagonal affine scan fp32",
+          "scan_lm": "diagonal affine scan fp32 (LM width)",
           "block2": "2x2 block affine scan fp32",
           "gru_bwd": "ParaGRU backward pass fp32",
           "lstm_bwd": "ParaLSTM backward pass fp32",
@@ -396,6 +435,48 @@ def workload_name(name, B, L, D, K=None, G=None):
     if K is not None:
         out += f" K={K} G={G} (M={B * L}, N={G * D})"
     return out
+
+
+# the diagonal scan timed beside each solve workload (the scan half of the metric)
+SCAN_LEG = {"lm": "scan_lm", "gru_l": "scan"}
+
+
+def time_leg(name, K, W, warm_s, world, rank, device, stream):
+    """A second workload of the run, timed like the main step: at least W
+    untimed steps (and `warm_s` seconds), then K steps between CUDA events on
+    the launching stream, max over ranks.  Returns (case, ms per step)."""
+    import torch
+
+    cs = Case(name, rank, device)
+    n_w = 0
+    t_w = time.perf_counter()
+    while n_w < max(W, 3) or time.perf_counter() - t_w < warm_s:
+        cs.step()
+        n_w += 1
+        if n_w % 8 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(K):
+        cs.step()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    return cs, max_over_ranks(ev[0].elapsed_time(ev[1]) / K, world, device)
+
+
+def scan_summary(sc, ms, world, hbm_peak):
+    """The scan leg's line: its 12 algorithmic bytes per channel-step against
+    the measured HBM copy bandwidth and against 8 TB/s."""
+    sbytes = algorithmic_bytes("scan_diag", False, sc.B, sc.L, sc.D)
+    sgbs = sbytes / (ms * 1e-3) / 1e9
+    st, ssrc = recorded_traffic(sc.name)
+    return {"workload": workload_name(sc.name, sc.B, sc.L, sc.D), "ms": ms,
+            "channel_steps_per_s": world * sc.N / (ms * 1e-3), "achieved_gbs": sgbs,
+            "algorithmic_bytes": sbytes, "frac_of_measured_hbm": sgbs / hbm_peak,
+            "frac_of_8tbs": sgbs / 8000.0, "traffic": st, "traffic_source": ssrc}
 
 
 # ---------------------------------------------------------------------------
@@ -414,15 +495,21 @@ def run_ours(args, world, rank, local):
     op, B, L, D, bf16, N = cs.op, cs.B, cs.L, cs.D, cs.bf16, cs.N
     stream = torch.cuda.current_stream()
 
-    # Warm-up: at least W steps (and at least 3), continued until the GPU has
-    # run the workload for --warmup-seconds so clocks and memory have settled;
-    # the count actually run is reported as "warmup".
+    # Warm-up: W untimed steps (at least 3), reported as "warmup".  Then more
+    # untimed steps until the GPU has run the workload for --warmup-seconds, so
+    # that clocks and memory have settled; those are reported separately as
+    # "warmup_settle" (they only lengthen the untimed part of the run).
     W = 0
-    t_w = time.perf_counter()
-    while W < max(args.warmup, 3) or time.perf_counter() - t_w < args.warmup_seconds:
+    while W < max(args.warmup, 3):
         cs.step()
         W += 1
-        if W % 8 == 0 or W >= max(args.warmup, 3):
+    torch.cuda.synchronize()
+    settle = 0
+    t_w = time.perf_counter()
+    while time.perf_counter() - t_w < args.warmup_seconds:
+        cs.step()
+        settle += 1
+        if settle % 8 == 0:
             torch.cuda.synchronize()
     torch.cuda.synchronize()
     info = cs.solve_info()
@@ -456,13 +543,13 @@ def run_ours(args, world, rank, local):
 
     # One untimed pass shaped like the timed loop (back-to-back steps, events on
     # the stream); counted as warm-up.  The first such pass of a process ran its
-    # first step ~0.07 ms slower than later ones on B200.
+    # first step ~0.07 ms slower than later ones on B200.  Counted in warmup_settle.
     pre = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     pre[0].record(stream)
     for i in range(3):
         run_step()
         pre[i + 1].record(stream)
-        W += 1
+        settle += 1
     torch.cuda.synchronize()
 
     # ---- timed region: exactly K steps ---------------------------------------
@@ -494,6 +581,7 @@ def run_ours(args, world, rank, local):
     achieved_gbs = bytes_launch / (launch_ms * 1e-3) / 1e9
     hbm_frac = achieved_gbs / hbm_peak
     traffic, traffic_src = recorded_traffic(args.workload)
+    mufu_probe = None
     hbm = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
            "frac": hbm_frac, "traffic": traffic, "peak_kind": peak_kind,
            "algorithmic_bytes_per_launch": bytes_launch}
@@ -505,12 +593,15 @@ def run_ours(args, world, rank, local):
             ev_iters = 1  # the backward evaluates each step once
         mufu_ops = N * ev_iters * MUFU_PER_STEP[op[:4].rstrip("_")]
         sm_mhz = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
-        mufu_peak = SMS * MUFU_PER_SM_PER_CLK * sm_mhz * 1e6
+        probe = mufu_probe = measure_pipe_peak(pr, pr.PROBE_MUFU, device, local)
+        mufu_peak = probe["per_sm_per_clk"] * probe["sms"] * sm_mhz * 1e6
         alu = {"bound": "alu", "achieved": mufu_ops / (launch_ms * 1e-3) / 1e12,
                "peak": mufu_peak / 1e12, "unit": "Tops/s (MUFU ex2+rcp)",
                "frac": mufu_ops / (launch_ms * 1e-3) / mufu_peak, "traffic": traffic,
-               "peak_kind": "derived: 148 SMs x 16 MUFU/clk x sampled SM clock",
-               "mufu_ops_per_launch": mufu_ops}
+               "peak_kind": ("measured: ex2+rcp throughput probe, %.2f ops per SM per clock "
+                             "at %.0f MHz, scaled to the timed region's SM clock"
+                             % (probe["per_sm_per_clk"], probe["sm_mhz"])),
+               "peak_probe": probe, "mufu_ops_per_launch": mufu_ops}
         if alu["frac"] >= hbm_frac:
             roofline = dict(alu)
             roofline["hbm"] = {k: hbm[k] for k in ("achieved", "peak", "unit", "frac",
@@ -522,12 +613,16 @@ def run_ours(args, world, rank, local):
         ev_iters = (iters or 0) + 1
         sm_mhz = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
         flops = 2.0 * N * ev_iters * MHGRU_FMA_PER_STEP
-        fpeak = SMS * FMA_PER_SM_PER_CLK * 2 * sm_mhz * 1e6 / 1e12
+        probe = measure_pipe_peak(pr, pr.PROBE_FMA, device, local)
+        fpeak = probe["per_sm_per_clk"] * probe["sms"] * 2 * sm_mhz * 1e6 / 1e12
         ach = flops / (launch_ms * 1e-3) / 1e12
         roofline = {"bound": "alu", "achieved": ach, "peak": fpeak,
                     "unit": "TFLOP/s (fp32 FMA, CUDA cores)", "frac": ach / fpeak,
                     "traffic": traffic, "flops_per_launch": flops,
-                    "peak_kind": "derived: 148 SMs x 128 FMA/clk x 2 x sampled SM clock",
+                    "peak_kind": ("measured: fp32 FMA throughput probe, %.1f FMA per SM per "
+                                  "clock at %.0f MHz, scaled to the timed region's SM clock"
+                                  % (probe["per_sm_per_clk"], probe["sm_mhz"])),
+                    "peak_probe": probe,
                     "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                             "frac": hbm_frac}}
     elif op == "proj":
@@ -556,31 +651,39 @@ def run_ours(args, world, rank, local):
     roofline["launch_ms"] = launch_ms
     roofline["traffic_source"] = traffic_src
 
-    # ---- the diagonal scan at the same shape (the scan half of the metric) ---
+    # ---- the diagonal scan at the same width (the scan half of the metric) --
     scan = None
-    if args.workload == "gru_l" and not args.no_scan:
-        sc = Case("scan", rank, device)
-        t_w = time.perf_counter()
-        n_w = 0
-        while n_w < W or time.perf_counter() - t_w < args.warmup_seconds:
-            sc.step()
-            n_w += 1
-            torch.cuda.synchronize()
-        sev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        barrier(world)
-        sev[0].record(stream)
-        for _ in range(K):
-            sc.step()
-        sev[1].record(stream)
-        torch.cuda.synchronize()
-        sms = max_over_ranks(sev[0].elapsed_time(sev[1]) / K, world, device)
-        sbytes = algorithmic_bytes("scan_diag", False, sc.B, sc.L, sc.D)
-        sgbs = sbytes / (sms * 1e-3) / 1e9
-        st, ssrc = recorded_traffic("scan")
-        scan = {"workload": f"diagonal scan fp32 B={sc.B} L={sc.L} D={sc.D}", "ms": sms,
-                "channel_steps_per_s": world * sc.N / (sms * 1e-3), "achieved_gbs": sgbs,
-                "algorithmic_bytes": sbytes, "frac_of_measured_hbm": sgbs / hbm_peak,
-                "frac_of_8tbs": sgbs / 8000.0, "traffic": st, "traffic_source": ssrc}
+    scan_name = SCAN_LEG.get(args.workload)
+    if scan_name and not args.no_scan:
+        sc, sms = time_leg(scan_name, K, W, args.warmup_seconds, world, rank, device, stream)
+        scan = scan_summary(sc, sms, world, hbm_peak)
+        del sc
+
+    # ---- extra keys: the fp32 solve and scan at B=8, L=4096, D=1024 ----------
+    extra = None
+    if args.workload == "lm" and not args.no_extra:
+        g, gms = time_leg("gru_l", K, W, args.warmup_seconds, world, rank, device, stream)
+        ginfo = g.solve_info()
+        gpasses = ginfo.passes
+        gev = evaluated_iterations(gpasses, g.max_iters)
+        gmufu = g.N * gev * MUFU_PER_STEP["gru"]
+        gbytes = algorithmic_bytes("gru", False, g.B, g.L, g.D, gpasses)
+        gsm = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
+        if mufu_probe is None:
+            mufu_probe = measure_pipe_peak(pr, pr.PROBE_MUFU, device, local)
+        gpeak = mufu_probe["per_sm_per_clk"] * mufu_probe["sms"] * gsm * 1e6
+        gtr, gtsrc = recorded_traffic("gru_l")
+        extra = {"workload": workload_name("gru_l", g.B, g.L, g.D), "ms": gms,
+                 "channel_steps_per_s": world * g.N / (gms * 1e-3),
+                 "newton_iterations": ginfo.iterations, "sweeps": gpasses,
+                 "evaluated_iterations": gev,
+                 "mufu_frac": gmufu / (gms * 1e-3) / gpeak,
+                 "hbm_gbs": gbytes / (gms * 1e-3) / 1e9,
+                 "hbm_frac": gbytes / (gms * 1e-3) / 1e9 / hbm_peak,
+                 "traffic": gtr, "traffic_source": gtsrc}
+        del g
+        sc, sms = time_leg("scan", K, W, args.warmup_seconds, world, rank, device, stream)
+        extra["scan"] = scan_summary(sc, sms, world, hbm_peak)
         del sc
 
     # ---- context: sequential application on the same GPU ---------------------
@@ -720,14 +823,18 @@ def run_ours(args, world, rank, local):
                         "sweeps": passes, "evaluated_iterations": ev_iters})
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": ms, "higher_is_better": True,
+            "warmup": W,
+            "warmup_settle": {"steps": settle, "seconds": args.warmup_seconds,
+                              "why": "extra untimed steps until the GPU has run the workload "
+                                     "this long, so clocks and memory have settled"},
+            "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": ("bf16-in/f32-acc" if op == "proj" else
                       "f32" if not bf16 else "bf16-in/f32"),
             "data": "synthetic (seeded numpy; see tests/inputs.py)",
             "config": cfg, "roofline": roofline, "clocks": clocks, "e2e": e2e,
             "gpu_launches": K, "scan": scan, "cpu_baseline": cpu,
-            "sequential_gpu": sequential,
+            "sequential_gpu": sequential, "gru_l": extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -959,12 +1066,15 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="gru_l",
-                    choices=["gru_l", "lm", "deer", "gru_s", "lstm", "scan", "block2",
+    ap.add_argument("--workload", default="lm",
+                    choices=["lm", "gru_l", "deer", "gru_s", "lstm", "scan", "scan_lm", "block2",
                              "gru_bwd", "lstm_bwd", "proj", "proj_lm", "mhgru"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
-    ap.add_argument("--no-scan", action="store_true", help="skip the scan leg (gru_l)")
+    ap.add_argument("--no-scan", action="store_true", help="skip the scan leg (lm, gru_l)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the extra keys of the lm workload (solve and scan at "
+                         "B=8 L=4096 D=1024)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--no-sequential", action="store_true",
                     help="skip the sequential-application context timings")

@@ -103,10 +103,12 @@ typedef struct {
  *                (0 = 4 for GRU, 5 for LSTM).
  *  iters_next  : Newton iterations per later sweep (0 = 2).
  *  wait_timeout_ns : bound on every device-side wait (0 = 1e9, i.e. 1 s).
- *  debug_stall_unit: test hook, -1 = off.  The work unit with this index
- *                 never publishes its look-back status, so the units after it
- *                 run their bounded waits out; the call must then report
- *                 PARARNN_ERR_DEVICE_TIMEOUT (look-back regime only).
+ *  debug_stall_unit: FOR TESTS ONLY -- leave at -1 (off) in any other use.
+ *                 The work unit with this index never publishes its look-back
+ *                 status, so the units after it run their bounded waits out;
+ *                 the call must then report PARARNN_ERR_DEVICE_TIMEOUT
+ *                 (look-back regime only).  It exists so that the test suite
+ *                 can check the bounded waits without faulting a GPU.
  *  regime      : how the time chunks of a channel tile are chained.
  *                0 = automatic; 1 = look-back (chunks of a tile on different
  *                CTAs, chained through global memory); 2 = walk (one CTA walks
@@ -306,7 +308,10 @@ pararnn_status_t pararnn_input_projection(const void* x, const void* W, const fl
  *    cleared on the stream at every call.
  *  - The first call on a device looks up the array's device address with that
  *    device current (a one-time set-up per device); make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address belongs to the device's context:
+ *    after cudaDeviceReset the next call finds a new context (by the driver's
+ *    context id) and looks the address up again, so it is never stale; that
+ *    call, too, should come before any capture.
  *  - Every call on a device shares the one array, which keeps what the last
  *    call left: calls whose kernels may overlap on the GPU (different streams
  *    without ordering, several host threads) race on it and must be
@@ -317,6 +322,25 @@ pararnn_status_t pararnn_solve_gru_noalloc(const void* P, pararnn_dtype_t p_dtyp
                                            int64_t D, float tol, int32_t max_iters,
                                            pararnn_solve_info_t* info,
                                            const pararnn_options_t* opts, void* stream);
+
+/* Throughput probe: a measurement aid with no counterpart in the pages.  It
+ * enqueues on `stream` one launch of a kernel that keeps one functional-unit
+ * pipe of every SM busy (many independent dependency chains per thread, all
+ * CTAs resident) and stores in *ops (host memory) the number of operations
+ * that launch performs.  Timing the launch with events gives the measured
+ * peak that a kernel bound by that pipe is reported against:
+ *  pipe 0: the special-function pipe, as one base-2 exponential and one
+ *          reciprocal per step (ex2.approx + rcp.approx, the pair each
+ *          sigmoid and tanh of the ParaGRU / ParaLSTM cells takes);
+ *          *ops counts both.
+ *  pipe 1: fp32 fused multiply-add; *ops counts FMAs (2 flops each).
+ * iters (> 0) sets the launch's length: 32 * iters chain steps per thread.
+ * sink: device memory of at least 4 bytes; it is written only if the chains
+ * hit a value they never reach (so the work cannot be optimised away).
+ * Errors: PARARNN_ERR_INVALID_ARGUMENT (pipe, iters, NULL pointers),
+ * PARARNN_ERR_UNSUPPORTED (not sm_100a), PARARNN_ERR_CUDA (launch). */
+pararnn_status_t pararnn_probe_rate(int32_t pipe, int32_t iters, float* sink, int64_t* ops,
+                                    void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* pararnn_status_string(pararnn_status_t status);

@@ -34,7 +34,7 @@ from . import build as _build
 __all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc",
            "solve_gru_backward", "solve_lstm_backward", "solve_mhgru", "input_projection",
            "step_gru", "step_lstm", "rollout_gru", "rollout_lstm",
-           "workspace_size",
+           "workspace_size", "probe_rate", "PROBE_MUFU", "PROBE_FMA",
            "SolveInfo", "Options", "PararnnError", "library_path", "load", "MAX_ITERS"]
 
 MAX_ITERS = 127
@@ -146,6 +146,8 @@ def load(build_if_missing: bool = True):
             lib.pararnn_input_projection.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i64,
                                                      _i64, _i64, _vp, _vp]
             lib.pararnn_input_projection.restype = ctypes.c_int
+            lib.pararnn_probe_rate.argtypes = [ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp]
+            lib.pararnn_probe_rate.restype = ctypes.c_int
             lib.pararnn_status_string.argtypes = [ctypes.c_int]
             lib.pararnn_status_string.restype = ctypes.c_char_p
             lib.pararnn_version.restype = ctypes.c_int32
@@ -192,8 +194,42 @@ def _check_dev(name, t, dtype, shape):
         raise ValueError(f"{name} must be contiguous")
 
 
-def _stream_handle(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
+def _one_device(**named):
+    """The one CUDA device every given tensor lives on.  The library resolves
+    the launch (stream, scratch, occupancy) against the current device, so
+    tensors on a device other than the one the call runs on, or on several
+    devices, are refused here."""
+    dev = None
+    first = None
+    for name, t in named.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+        if dev is None:
+            dev, first = t.device, name
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device} but {first} is on {dev}: "
+                             "all arguments of a call must be on one device")
+    if dev is None:
+        raise ValueError("no tensor argument")
+    return dev
+
+
+def _device_guard(dev):
+    """Makes `dev` the current device for the duration of one library call."""
+    return torch.cuda.device(dev)
+
+
+def _stream_handle(stream, dev=None):
+    """The stream a call is enqueued on: the given one (which must belong to
+    the tensors' device) or that device's current stream."""
+    if stream is None:
+        s = torch.cuda.current_stream(dev)
+    else:
+        s = stream
+        if dev is not None and s.device != dev:
+            raise ValueError(f"stream is on {s.device} but the tensors are on {dev}")
     return ctypes.c_void_p(s.cuda_stream)
 
 
@@ -280,11 +316,14 @@ def scan_diag(A, b, h0=None, out=None, status=None, opts: Options | None = None,
     h = torch.empty_like(A) if out is None else out
     _check_dev("out", h, torch.float32, (B, L, D))
     _check_dev("status", status, torch.int32, (1,))
+    dev = _one_device(A=A, b=b, h0=h0, out=h, status=status)
     n = workspace_size(OP_SCAN_DIAG, B, L, D, 0, opts)
-    ws = _workspace(n, A.device, stream)
-    st = lib.pararnn_scan_diag(_ptr(A), _ptr(b), _ptr(h0), _ptr(h), B, L, D, _ptr(ws), ws.numel(),
-                               _ptr(status), ctypes.byref(opts) if opts is not None else None,
-                               _stream_handle(stream))
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_scan_diag(_ptr(A), _ptr(b), _ptr(h0), _ptr(h), B, L, D, _ptr(ws),
+                                   ws.numel(), _ptr(status),
+                                   ctypes.byref(opts) if opts is not None else None,
+                                   _stream_handle(stream, dev))
     _raise(st, "pararnn_scan_diag")
     return h
 
@@ -299,12 +338,14 @@ def scan_block2(A, b, x0=None, out=None, status=None, opts: Options | None = Non
     x = torch.empty_like(b) if out is None else out
     _check_dev("out", x, torch.float32, (B, L, D, 2))
     _check_dev("status", status, torch.int32, (1,))
+    dev = _one_device(A=A, b=b, x0=x0, out=x, status=status)
     n = workspace_size(OP_SCAN_BLOCK2, B, L, D, 0, opts)
-    ws = _workspace(n, A.device, stream)
-    st = lib.pararnn_scan_block2(_ptr(A), _ptr(b), _ptr(x0), _ptr(x), B, L, D, _ptr(ws),
-                                 ws.numel(), _ptr(status),
-                                 ctypes.byref(opts) if opts is not None else None,
-                                 _stream_handle(stream))
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_scan_block2(_ptr(A), _ptr(b), _ptr(x0), _ptr(x), B, L, D, _ptr(ws),
+                                     ws.numel(), _ptr(status),
+                                     ctypes.byref(opts) if opts is not None else None,
+                                     _stream_handle(stream, dev))
     _raise(st, "pararnn_scan_block2")
     return x
 
@@ -333,12 +374,14 @@ def solve_gru(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
     _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
+    dev = _one_device(P=P, a=a, h0=h0, out=h, info=info)
     n = workspace_size(OP_GRU, B, L, D, max_iters, opts)
-    ws = _workspace(n, P.device, stream)
-    st = lib.pararnn_solve_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D, float(tol),
-                               int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
-                               ctypes.byref(opts) if opts is not None else None,
-                               _stream_handle(stream))
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_solve_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D, float(tol),
+                                   int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
+                                   ctypes.byref(opts) if opts is not None else None,
+                                   _stream_handle(stream, dev))
     _raise(st, "pararnn_solve_gru")
     return h, SolveInfo(info)
 
@@ -361,12 +404,14 @@ def solve_mhgru(P, U, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
     _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
+    dev = _one_device(P=P, U=U, h0=h0, out=h, info=info)
     n = workspace_size(OP_MHGRU, B, L, D, max_iters, opts)
-    ws = _workspace(n, P.device, stream)
-    st = lib.pararnn_solve_mhgru(_ptr(P), dt, _ptr(U), _ptr(h0), _ptr(h), B, L, H, float(tol),
-                                 int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
-                                 ctypes.byref(opts) if opts is not None else None,
-                                 _stream_handle(stream))
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_solve_mhgru(_ptr(P), dt, _ptr(U), _ptr(h0), _ptr(h), B, L, H,
+                                     float(tol), int(max_iters), _ptr(ws), ws.numel(),
+                                     _ptr(info), ctypes.byref(opts) if opts is not None else None,
+                                     _stream_handle(stream, dev))
     _raise(st, "pararnn_solve_mhgru")
     return h, SolveInfo(info)
 
@@ -393,12 +438,14 @@ def solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32, out=None, info=No
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
     _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
+    dev = _one_device(P=P, a=a, c0=c0, h0=h0, c=c, h=h, info=info)
     n = workspace_size(OP_LSTM, B, L, D, max_iters, opts)
-    ws = _workspace(n, P.device, stream)
-    st = lib.pararnn_solve_lstm(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h), B, L,
-                                D, float(tol), int(max_iters), _ptr(ws), ws.numel(), _ptr(info),
-                                ctypes.byref(opts) if opts is not None else None,
-                                _stream_handle(stream))
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_solve_lstm(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h),
+                                    B, L, D, float(tol), int(max_iters), _ptr(ws), ws.numel(),
+                                    _ptr(info), ctypes.byref(opts) if opts is not None else None,
+                                    _stream_handle(stream, dev))
     _raise(st, "pararnn_solve_lstm")
     return c, h, SolveInfo(info)
 
@@ -427,10 +474,12 @@ def solve_gru_noalloc(P, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None
     if info is None:
         info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
     _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
-    st = lib.pararnn_solve_gru_noalloc(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D,
-                                       float(tol), int(max_iters), _ptr(info),
-                                       ctypes.byref(opts) if opts is not None else None,
-                                       _stream_handle(stream))
+    dev = _one_device(P=P, a=a, h0=h0, out=h, info=info)
+    with _device_guard(dev):
+        st = lib.pararnn_solve_gru_noalloc(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D,
+                                           float(tol), int(max_iters), _ptr(info),
+                                           ctypes.byref(opts) if opts is not None else None,
+                                           _stream_handle(stream, dev))
     _raise(st, "pararnn_solve_gru_noalloc")
     return h, SolveInfo(info)
 
@@ -460,13 +509,15 @@ def solve_gru_backward(P, a, h, dh, h0=None, out=None, status=None,
     _check_dev("da", da, torch.float32, (3, D))
     _check_dev("dh0", dh0, torch.float32, (B, D))
     _check_dev("status", status, torch.int32, (1,))
+    dev = _one_device(P=P, a=a, h0=h0, h=h, dh=dh, dP=dP, da=da, dh0=dh0, status=status)
     n = workspace_size(OP_GRU_BACKWARD, B, L, D, 0, opts)
-    ws = _workspace(n, P.device, stream)
-    st = lib.pararnn_solve_gru_backward(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), _ptr(dh),
-                                        _ptr(dP), _ptr(da), _ptr(dh0), B, L, D, _ptr(ws),
-                                        ws.numel(), _ptr(status),
-                                        ctypes.byref(opts) if opts is not None else None,
-                                        _stream_handle(stream))
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_solve_gru_backward(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), _ptr(dh),
+                                            _ptr(dP), _ptr(da), _ptr(dh0), B, L, D, _ptr(ws),
+                                            ws.numel(), _ptr(status),
+                                            ctypes.byref(opts) if opts is not None else None,
+                                            _stream_handle(stream, dev))
     _raise(st, "pararnn_solve_gru_backward")
     return dP, da, dh0
 
@@ -498,14 +549,17 @@ def solve_lstm_backward(P, a, c, h, dc, dh, c0=None, h0=None, out=None, status=N
     _check_dev("dc0", dc0, torch.float32, (B, D))
     _check_dev("dh0", dh0, torch.float32, (B, D))
     _check_dev("status", status, torch.int32, (1,))
+    dev = _one_device(P=P, a=a, c0=c0, h0=h0, c=c, h=h, dc=dc, dh=dh, dP=dP, da=da, dc0=dc0,
+                      dh0=dh0, status=status)
     n = workspace_size(OP_LSTM_BACKWARD, B, L, D, 0, opts)
-    ws = _workspace(n, P.device, stream)
-    st = lib.pararnn_solve_lstm_backward(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c),
-                                         _ptr(h), _ptr(dc), _ptr(dh), _ptr(dP), _ptr(da),
-                                         _ptr(dc0), _ptr(dh0), B, L, D, _ptr(ws), ws.numel(),
-                                         _ptr(status),
-                                         ctypes.byref(opts) if opts is not None else None,
-                                         _stream_handle(stream))
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_solve_lstm_backward(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c),
+                                             _ptr(h), _ptr(dc), _ptr(dh), _ptr(dP), _ptr(da),
+                                             _ptr(dc0), _ptr(dh0), B, L, D, _ptr(ws), ws.numel(),
+                                             _ptr(status),
+                                             ctypes.byref(opts) if opts is not None else None,
+                                             _stream_handle(stream, dev))
     _raise(st, "pararnn_solve_lstm_backward")
     return dP, da, dc0, dh0
 
@@ -522,8 +576,11 @@ def step_gru(P, a, h_prev=None, out=None, stream=None):
     _check_dev("h_prev", h_prev, torch.float32, (B, D))
     h = torch.empty((B, D), dtype=torch.float32, device=P.device) if out is None else out
     _check_dev("out", h, torch.float32, (B, D))
-    _raise(lib.pararnn_step_gru(_ptr(P), dt, _ptr(a), _ptr(h_prev), _ptr(h), B, D,
-                                _stream_handle(stream)), "pararnn_step_gru")
+    dev = _one_device(P=P, a=a, h_prev=h_prev, out=h)
+    with _device_guard(dev):
+        st = lib.pararnn_step_gru(_ptr(P), dt, _ptr(a), _ptr(h_prev), _ptr(h), B, D,
+                                  _stream_handle(stream, dev))
+    _raise(st, "pararnn_step_gru")
     return h
 
 
@@ -553,9 +610,11 @@ def input_projection(x, W, bias=None, out=None, out_dtype=torch.float32, status=
     _check_dev("out", P, out_dtype, lead + (N,))
     _check_dev("status", status, torch.int32, (1,))
     dt = BF16 if out_dtype == torch.bfloat16 else F32
-    _raise(lib.pararnn_input_projection(_ptr(x), _ptr(W), _ptr(bias), _ptr(P), dt, M, N, K,
-                                        _ptr(status), _stream_handle(stream)),
-           "pararnn_input_projection")
+    dev = _one_device(x=x, W=W, bias=bias, out=P, status=status)
+    with _device_guard(dev):
+        st = lib.pararnn_input_projection(_ptr(x), _ptr(W), _ptr(bias), _ptr(P), dt, M, N, K,
+                                          _ptr(status), _stream_handle(stream, dev))
+    _raise(st, "pararnn_input_projection")
     return P
 
 
@@ -575,8 +634,13 @@ def step_lstm(P, a, c_prev=None, h_prev=None, out=None, stream=None):
         h = torch.empty((B, D), dtype=torch.float32, device=P.device)
     else:
         c, h = out
-    _raise(lib.pararnn_step_lstm(_ptr(P), dt, _ptr(a), _ptr(c_prev), _ptr(h_prev), _ptr(c),
-                                 _ptr(h), B, D, _stream_handle(stream)), "pararnn_step_lstm")
+    _check_dev("c", c, torch.float32, (B, D))
+    _check_dev("h", h, torch.float32, (B, D))
+    dev = _one_device(P=P, a=a, c_prev=c_prev, h_prev=h_prev, c=c, h=h)
+    with _device_guard(dev):
+        st = lib.pararnn_step_lstm(_ptr(P), dt, _ptr(a), _ptr(c_prev), _ptr(h_prev), _ptr(c),
+                                   _ptr(h), B, D, _stream_handle(stream, dev))
+    _raise(st, "pararnn_step_lstm")
     return c, h
 
 
@@ -592,8 +656,11 @@ def rollout_gru(P, a, h0=None, out=None, stream=None):
     _check_dev("h0", h0, torch.float32, (B, D))
     h = torch.empty((B, L, D), dtype=torch.float32, device=P.device) if out is None else out
     _check_dev("out", h, torch.float32, (B, L, D))
-    _raise(lib.pararnn_rollout_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D,
-                                   _stream_handle(stream)), "pararnn_rollout_gru")
+    dev = _one_device(P=P, a=a, h0=h0, out=h)
+    with _device_guard(dev):
+        st = lib.pararnn_rollout_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D,
+                                     _stream_handle(stream, dev))
+    _raise(st, "pararnn_rollout_gru")
     return h
 
 
@@ -613,6 +680,29 @@ def rollout_lstm(P, a, c0=None, h0=None, out=None, stream=None):
         h = torch.empty((B, L, D), dtype=torch.float32, device=P.device)
     else:
         c, h = out
-    _raise(lib.pararnn_rollout_lstm(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h),
-                                    B, L, D, _stream_handle(stream)), "pararnn_rollout_lstm")
+    _check_dev("c", c, torch.float32, (B, L, D))
+    _check_dev("h", h, torch.float32, (B, L, D))
+    dev = _one_device(P=P, a=a, c0=c0, h0=h0, c=c, h=h)
+    with _device_guard(dev):
+        st = lib.pararnn_rollout_lstm(_ptr(P), dt, _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h),
+                                      B, L, D, _stream_handle(stream, dev))
+    _raise(st, "pararnn_rollout_lstm")
     return c, h
+
+
+PROBE_MUFU, PROBE_FMA = 0, 1
+
+
+def probe_rate(pipe, iters, sink, stream=None):
+    """Enqueue one throughput-probe launch (``pararnn_probe_rate``) and return
+    the number of operations it performs: ex2 + rcp for ``PROBE_MUFU``, FMAs
+    for ``PROBE_FMA``.  ``sink`` is a device tensor of at least 4 bytes."""
+    lib = load()
+    if not sink.is_cuda or sink.numel() * sink.element_size() < 4:
+        raise ValueError("sink must be a CUDA tensor of at least 4 bytes")
+    ops = ctypes.c_int64(0)
+    with _device_guard(sink.device):
+        st = lib.pararnn_probe_rate(int(pipe), int(iters), _ptr(sink), ctypes.byref(ops),
+                                    _stream_handle(stream, sink.device))
+    _raise(st, "pararnn_probe_rate")
+    return int(ops.value)

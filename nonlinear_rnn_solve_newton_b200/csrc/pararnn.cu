@@ -18,6 +18,7 @@
 #include "pararnn_bwd_walk.cuh"
 #include "pararnn_kernel.cuh"
 #include "pararnn_mhgru.cuh"
+#include "pararnn_probe.cuh"
 #include "pararnn_proj.cuh"
 #include "pararnn_seq.cuh"
 #include "pararnn_walk.cuh"
@@ -913,11 +914,44 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[PARARNN_NOALLOC
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoallocSlot {
+  void* ptr;                 // device address of the array in that context
+  unsigned long long ctx_id; // the driver's unique id of the context it was resolved in
+};
+NoallocSlot g_noalloc[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device.  Resolved once per
-// device, on the first call made with that device current; the name of the
-// array is only a host-side stand-in and must never be handed to a kernel.
+// The driver's id of the calling thread's current context (0 if there is none
+// or the driver does not offer the query).  Ids are never reused, so a context
+// created after cudaDeviceReset has a new one even if its handle repeats.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+    cudaGetLastError();
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device.  The name of the
+// array is only a host-side stand-in and must never be handed to a kernel: the
+// address is looked up with the device current, on the first call on that
+// device, and again whenever the device's context has changed since (a
+// cudaDeviceReset ends the context the cached address belonged to).
 pararnn_status_t noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -925,15 +959,19 @@ pararnn_status_t noalloc_scratch(void** out) {
     return PARARNN_ERR_CUDA;
   }
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocSlot& slot = g_noalloc[dev];
+  const unsigned long long id = current_context_id();
+  if (!slot.ptr || id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
       return PARARNN_ERR_CUDA;
     }
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    // the lookup made the device's primary context current if none was
+    slot.ctx_id = id != 0 ? id : current_context_id();
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return PARARNN_OK;
 }
 
@@ -1361,5 +1399,36 @@ extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }
+  return PARARNN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Throughput probes (measured peaks for the rooflines).
+// ---------------------------------------------------------------------------
+extern "C" pararnn_status_t pararnn_probe_rate(int32_t pipe, int32_t iters, float* sink,
+                                               int64_t* ops, void* stream) {
+  using namespace pararnn;
+  if ((pipe != 0 && pipe != 1) || iters <= 0 || !sink || !ops)
+    return PARARNN_ERR_INVALID_ARGUMENT;
+  const void* fn = pipe == 0 ? (const void*)pararnn_probe_kernel<0>
+                             : (const void*)pararnn_probe_kernel<1>;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_UNSUPPORTED;
+  }
+  int total = 0;
+  if (resident_ctas(fn, kProbeThreads, 0, &total) != cudaSuccess || total <= 0) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (pipe == 0)
+    pararnn_probe_kernel<0><<<total, kProbeThreads, 0, st>>>(iters, sink);
+  else
+    pararnn_probe_kernel<1><<<total, kProbeThreads, 0, st>>>(iters, sink);
+  if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
+  const int64_t per_step = pipe == 0 ? 2 : 1;
+  *ops = (int64_t)total * kProbeThreads * (int64_t)iters * kProbeUnroll * kProbeChains * per_step;
   return PARARNN_OK;
 }

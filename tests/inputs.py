@@ -21,6 +21,7 @@ lstm_bwd ParaLSTM backward pass, fp32          8, 4096, 1024
 lstm     ParaLSTM solve, fp32 (+ block scan)    8, 4096, 1024
 deer     ParaGRU solve, fp32, DEER shape        16, 2^20, 1
 lm       ParaGRU solve, bf16 P, fp32 state      8, 8192, 4096
+scan_lm  diagonal affine scan, fp32, LM width   8, 8192, 4096
 proj     input projection x W^T (+bias), G=3    8, 4096, 1024, K = 1024
 proj_lm  input projection, LM width, G=3        8, 8192, 4096, K = 4096
 mhgru    multi-head GRU, 8x8 blocks, fp32       8, 4096, 1024 (128 heads)
@@ -50,6 +51,7 @@ WORKLOADS = {
     "block2": dict(op="scan_block2", B=8, L=4096, D=1024, seed=3, bf16=False),
     "deer": dict(op="gru", B=16, L=1 << 20, D=1, seed=4, bf16=False),
     "lm": dict(op="gru", B=8, L=8192, D=4096, seed=5, bf16=True),
+    "scan_lm": dict(op="scan_diag", B=8, L=8192, D=4096, seed=9, bf16=False),
     "gru_bwd": dict(op="gru_bwd", B=8, L=4096, D=1024, seed=2, bf16=False),
     "lstm_bwd": dict(op="lstm_bwd", B=8, L=4096, D=1024, seed=3, bf16=False),
     "mhgru": dict(op="mhgru", B=8, L=4096, D=1024, seed=8, bf16=False),

@@ -51,6 +51,23 @@ def test_info_struct_layout():
     assert pr.INFO_BYTES == 4 * (6 + 1 + 128)
 
 
+def _header_define(name):
+    m = re.search(r"#define\s+" + name + r"\s+\(?\s*(\d+)u?\s*(?:<<\s*(\d+))?\s*\)?",
+                  open(HEADER).read())
+    assert m, name
+    v = int(m.group(1))
+    return v << int(m.group(2)) if m.group(2) else v
+
+
+def test_binding_constants_match_the_header():
+    # the binding keeps its own copies of these limits; a stale copy would let
+    # the binding accept what the library rejects (or the reverse)
+    import nonlinear_rnn_solve_newton_b200 as pr
+
+    assert pr.NOALLOC_SCRATCH_BYTES == _header_define("PARARNN_NOALLOC_SCRATCH_BYTES")
+    assert pr.MAX_ITERS == _header_define("PARARNN_MAX_ITERS")
+
+
 def test_workspace_size_host_only():
     import nonlinear_rnn_solve_newton_b200 as pr
 
@@ -215,3 +232,18 @@ def test_workspace_size_remembered_per_argument_tuple():
     assert walk != lookback
     with pytest.raises(pr.PararnnError):
         pr.workspace_size(pr.OP_GRU, 8, 4096, 1024, 500, o)
+
+
+def test_probe_rate_host_validation(lib):
+    """The throughput probe refuses a bad pipe, a non-positive length and NULL
+    pointers on the host, before any CUDA call."""
+    ops = ctypes.c_int64(-1)
+    fake = ctypes.c_void_p(0x1000)
+    for pipe, iters, sink, out in ((2, 10, fake, ctypes.byref(ops)),
+                                   (-1, 10, fake, ctypes.byref(ops)),
+                                   (0, 0, fake, ctypes.byref(ops)),
+                                   (1, -5, fake, ctypes.byref(ops)),
+                                   (0, 10, None, ctypes.byref(ops)),
+                                   (0, 10, fake, None)):
+        assert lib.pararnn_probe_rate(pipe, iters, sink, out, None) == 1
+    assert ops.value == -1

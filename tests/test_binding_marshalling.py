@@ -8,6 +8,9 @@ requirement of the argument checks is lifted for the test; dtype, shape and
 contiguity are still checked.  The real library, its kernels and the
 no-CPU-path guarantee are tested elsewhere (tests/test_abi.py, the GPU suites).
 """
+import contextlib
+from types import SimpleNamespace
+
 import pytest
 import torch
 
@@ -43,7 +46,9 @@ def fake(monkeypatch):
     monkeypatch.setattr(pr, "_check_dev", _check_host)
     monkeypatch.setattr(pr, "_workspace",
                         lambda n, device, stream=None: torch.empty(n, dtype=torch.uint8))
-    monkeypatch.setattr(pr, "_stream_handle", lambda s: None)
+    monkeypatch.setattr(pr, "_stream_handle", lambda s, dev=None: None)
+    monkeypatch.setattr(pr, "_one_device", lambda **named: torch.device("cpu"))
+    monkeypatch.setattr(pr, "_device_guard", lambda dev: contextlib.nullcontext())
     pr._ws_sizes.clear()
     yield lib
     pr._ws_sizes.clear()   # sizes from the stand-in must not outlive the test
@@ -134,3 +139,34 @@ def test_outputs_status_and_info_are_checked_before_the_call(fake):
         with pytest.raises((ValueError, TypeError)):
             call()
         assert [c for c in fake.calls if c != "pararnn_workspace_size"] == [], i
+
+
+def _on(dev):
+    """A stand-in for a CUDA tensor on `dev` (only what the device check reads)."""
+    return SimpleNamespace(is_cuda=dev is not None,
+                           device=torch.device("cuda", dev) if dev is not None else
+                           torch.device("cpu"))
+
+
+def test_one_device_accepts_one_device_and_skips_absent_arguments():
+    assert pr._one_device(P=_on(1), a=_on(1), h0=None, out=_on(1)) == torch.device("cuda", 1)
+
+
+def test_one_device_refuses_mixed_devices():
+    # the C library launches on the current device: a tensor on another GPU
+    # would be read through peer memory or fault, so the binding refuses it
+    with pytest.raises(ValueError, match="one device"):
+        pr._one_device(P=_on(1), a=_on(0))
+    with pytest.raises(ValueError, match="one device"):
+        pr._one_device(P=_on(0), a=_on(0), info=_on(1))
+
+
+def test_one_device_refuses_host_tensors():
+    with pytest.raises(ValueError, match="CUDA"):
+        pr._one_device(P=_on(0), a=_on(None))
+
+
+def test_stream_of_another_device_is_refused():
+    s = SimpleNamespace(device=torch.device("cuda", 1), cuda_stream=0)
+    with pytest.raises(ValueError, match="stream"):
+        pr._stream_handle(s, torch.device("cuda", 0))
