@@ -542,8 +542,8 @@ def run_ours(args, world, rank, local):
     run_step = graph.replay if graph is not None else cs.step
 
     # One untimed pass shaped like the timed loop (back-to-back steps, events on
-    # the stream); counted as warm-up.  The first such pass of a process ran its
-    # first step ~0.07 ms slower than later ones on B200.  Counted in warmup_settle.
+    # the stream), counted in warmup_settle.  The first such pass of a process
+    # ran its first step ~0.07 ms slower than later ones on B200.
     pre = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     pre[0].record(stream)
     for i in range(3):
