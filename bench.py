@@ -241,7 +241,7 @@ def algorithmic_bytes(op, bf16, B, L, D, passes=1):
         return 12 * N
     if op == "scan_block2":
         return 32 * N
-    if op == "proj":      # handled by projection_bytes (depends on K and G)
+    if op in ("proj", "proj_solve"):  # handled by projection_bytes (depends on K and G)
         raise ValueError("use projection_bytes for the input projection")
     if op == "mhgru":     # one evaluation: read P, the iterate, write the iterate
         return N * (12 + 4 + 4) * passes
@@ -331,6 +331,16 @@ class Case:
                 "bias": torch.from_numpy(x["bias"])}
             self.out_dtype = torch.bfloat16 if self.bf16 else torch.float32
             self.out_shapes = [(B, L, Nf)]
+        elif self.op == "proj_solve":
+            # x [B, L, K] and W [3 D, K] (bf16) -> the ParaGRU solve, P kept on chip
+            self.K, self.G = w["K"], 3
+            x = inputs.projected_gru_inputs(B, L, D, self.K, seed)
+            self.host = {
+                "x": torch.from_numpy(x["x_bits"].view(np.int16)).view(torch.bfloat16),
+                "W": torch.from_numpy(x["W_bits"].view(np.int16)).view(torch.bfloat16),
+                "bias": torch.from_numpy(x["bias"]), "a": torch.from_numpy(x["a"]),
+                "h0": torch.from_numpy(x["h0"])}
+            self.out_shapes = [(B, L, D)]
         elif self.op in ("gru_bwd", "lstm_bwd"):
             # the backward pass differentiates the forward solution: solve once here
             cell = self.op[:-4]
@@ -395,6 +405,9 @@ class Case:
                            info=self.info_t)
         elif op == "proj":
             pr.input_projection(d["x"], d["W"], d["bias"], out=outs[0], out_dtype=self.out_dtype)
+        elif op == "proj_solve":
+            pr.solve_gru_projected(d["x"], d["W"], d["bias"], d["a"], d["h0"], self.tol,
+                                   self.max_iters, out=outs[0], info=self.info_t)
         elif op == "gru_bwd":
             pr.solve_gru_backward(d["P"], d["a"], d["h"], d["gh"], d["h0"],
                                   out=(outs[0], outs[1], outs[2]))
@@ -410,7 +423,7 @@ class Case:
         self.run(self.dev, self.outs)
 
     def solve_info(self):
-        if self.op in ("gru", "lstm", "mhgru"):
+        if self.op in ("gru", "lstm", "mhgru", "proj_solve"):
             return self.pr.SolveInfo(self.info_t)
         return None
 
@@ -430,6 +443,8 @@ def workload_name(name, B, L, D, K=None, G=None):
           "mhgru": "multi-head GRU Newton solve fp32, dense 8x8 recurrence blocks",
           "proj": "input projection x W^T + bias, bf16 in, fp32 out (tcgen05)",
           "proj_lm": "input projection x W^T + bias, bf16 in, bf16 out (tcgen05)",
+          "proj_solve": "ParaGRU layer from its inputs: projection x W^T + bias (tcgen05, "
+                        "bf16 in, fp32 P kept on chip) fused with the Newton solve",
           }[name]
     out = f"{wl} B={B} L={L} D={D}"
     if K is not None:
@@ -576,8 +591,13 @@ def run_ours(args, world, rank, local):
     # (they also hold the ~2 us zeroing of the workspace control block).
     launch_ms = statistics.mean(per_step)
     hbm_peak, peak_kind, pk = peaks()
-    bytes_launch = (projection_bytes(B * L, cs.G * D, cs.K, bf16) if op == "proj"
-                    else algorithmic_bytes(op, bf16, B, L, D, passes))
+    if op == "proj":
+        bytes_launch = projection_bytes(B * L, cs.G * D, cs.K, bf16)
+    elif op == "proj_solve":
+        # x and W once per sweep, the bias, the trajectory written once; no P
+        bytes_launch = passes * (2 * B * L * cs.K + 2 * 3 * D * cs.K) + 4 * 3 * D + 4 * B * L * D
+    else:
+        bytes_launch = algorithmic_bytes(op, bf16, B, L, D, passes)
     achieved_gbs = bytes_launch / (launch_ms * 1e-3) / 1e9
     hbm_frac = achieved_gbs / hbm_peak
     traffic, traffic_src = recorded_traffic(args.workload)
@@ -625,6 +645,27 @@ def run_ours(args, world, rank, local):
                     "peak_probe": probe,
                     "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                             "frac": hbm_frac}}
+    elif op == "proj_solve":
+        ev_iters = evaluated_iterations(passes, cs.max_iters)
+        flops = 2.0 * (B * L) * (3 * D) * cs.K * passes
+        tf_peak = pk.get("bf16_tflops")
+        tf_kind = "measured burst (cuBLAS bf16 GEMM, MEASURED_PEAKS)"
+        if not tf_peak:
+            tf_peak, tf_kind = 1590.0, "fallback"
+        tflops = flops / (launch_ms * 1e-3) / 1e12
+        sm_mhz = clocks.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
+        probe = mufu_probe = measure_pipe_peak(pr, pr.PROBE_MUFU, device, local)
+        mufu_ops = N * ev_iters * MUFU_PER_STEP["gru"]
+        mufu_peak = probe["per_sm_per_clk"] * probe["sms"] * sm_mhz * 1e6
+        roofline = {"bound": "tensor", "achieved": tflops, "peak": tf_peak, "unit": "TFLOP/s",
+                    "frac": tflops / tf_peak, "traffic": traffic, "peak_kind": tf_kind,
+                    "flops_per_launch": flops,
+                    "alu": {"achieved": mufu_ops / (launch_ms * 1e-3) / 1e12,
+                            "peak": mufu_peak / 1e12, "unit": "Tops/s (MUFU ex2+rcp)",
+                            "frac": mufu_ops / (launch_ms * 1e-3) / mufu_peak,
+                            "peak_kind": "measured: ex2+rcp throughput probe"},
+                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": hbm_frac, "algorithmic_bytes_per_launch": bytes_launch}}
     elif op == "proj":
         ev_iters = None
         flops = 2.0 * (B * L) * (cs.G * D) * cs.K
@@ -647,6 +688,8 @@ def run_ours(args, world, rank, local):
                           "gru_bwd": "pararnn backward kernel (GRU)",
                           "lstm_bwd": "pararnn backward kernel (LSTM)",
                           "proj": "pararnn input projection (tcgen05)",
+                          "proj_solve": "pararnn projection fused with the GRU Newton walk "
+                                        "(tcgen05 + CUDA cores)",
                           "mhgru": "pararnn multi-head GRU Newton kernel (8x8 blocks)"}[op]
     roofline["launch_ms"] = launch_ms
     roofline["traffic_source"] = traffic_src
@@ -658,6 +701,34 @@ def run_ours(args, world, rank, local):
         sc, sms = time_leg(scan_name, K, W, args.warmup_seconds, world, rank, device, stream)
         scan = scan_summary(sc, sms, world, hbm_peak)
         del sc
+
+    # ---- the fused layer against the unfused pair (P through HBM) ------------
+    unfused = None
+    if op == "proj_solve" and not args.no_extra:
+        d = cs.dev
+        Pbuf = torch.empty((B, L, 3 * D), dtype=torch.bfloat16, device=device)
+        hbuf = torch.empty((B, L, D), dtype=torch.float32, device=device)
+
+        def pair():
+            pr.input_projection(d["x"], d["W"], d["bias"], out=Pbuf, out_dtype=torch.bfloat16)
+            pr.solve_gru(Pbuf.view(B, L, 3, D), d["a"], d["h0"], cs.tol, cs.max_iters,
+                         out=hbuf, info=cs.info_t)
+        for _ in range(max(W, 3)):
+            pair()
+        torch.cuda.synchronize()
+        pev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        barrier(world)
+        pev[0].record(stream)
+        for _ in range(K):
+            pair()
+        pev[1].record(stream)
+        torch.cuda.synchronize()
+        pms = max_over_ranks(pev[0].elapsed_time(pev[1]) / K, world, device)
+        unfused = {"what": "pararnn_input_projection (bf16 P to HBM) then pararnn_solve_gru "
+                           "(bf16 P read back), same inputs", "ms": pms,
+                   "fused_speedup": pms / ms,
+                   "max_abs_diff_vs_fused": float(torch.max(torch.abs(hbuf - cs.outs[0])).item())}
+        del Pbuf, hbuf
 
     # ---- extra keys: the fp32 solve and scan at B=8, L=4096, D=1024 ----------
     extra = None
@@ -811,14 +882,17 @@ def run_ours(args, world, rank, local):
         cpu = cpu_baseline(cs.x, op, B, L, D, budget_s=args.cpu_seconds)
 
     if rank == 0:
-        wlname = workload_name(args.workload, B, L, D, cs.K if op == "proj" else None,
-                               cs.G if op == "proj" else None)
+        kg = op in ("proj", "proj_solve")
+        wlname = workload_name(args.workload, B, L, D, cs.K if kg else None,
+                               cs.G if kg else None)
         cfg = {"workload": wlname, "B": B, "L": L, "D": D,
                "launch": "CUDA graph replay" if graph is not None else "direct calls",
                "parallelism": f"replicas x{world} (independent batches)",
                "l2": "inputs larger than L2 (%.0f MB per step), no flush needed" % (
                    sum(v.numel() * v.element_size() for v in cs.host.values()) / 1e6)}
-        if op in ("gru", "lstm", "mhgru"):
+        if op == "proj_solve":
+            cfg.update({"K": cs.K})
+        if op in ("gru", "lstm", "mhgru", "proj_solve"):
             cfg.update({"tol": cs.tol, "max_iters": cs.max_iters, "newton_iterations": iters,
                         "sweeps": passes, "evaluated_iterations": ev_iters})
         line = {
@@ -829,12 +903,12 @@ def run_ours(args, world, rank, local):
                                      "this long, so clocks and memory have settled"},
             "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": ("bf16-in/f32-acc" if op == "proj" else
+            "dtype": ("bf16-in/f32-acc" if op in ("proj", "proj_solve") else
                       "f32" if not bf16 else "bf16-in/f32"),
             "data": "synthetic (seeded numpy; see tests/inputs.py)",
             "config": cfg, "roofline": roofline, "clocks": clocks, "e2e": e2e,
             "gpu_launches": K, "scan": scan, "cpu_baseline": cpu,
-            "sequential_gpu": sequential, "gru_l": extra,
+            "sequential_gpu": sequential, "gru_l": extra, "unfused_pair": unfused,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -867,6 +941,27 @@ def cpu_baseline(x, op, B, L, D, budget_s=15.0):
                 "kind": "oracle",
                 "sample": f"fp64 projection of {nrows} of {x['x'].shape[0]} rows "
                           f"(N={Nf}, K={Wd.shape[1]}; {dt:.1f} s)"}
+    if op == "proj_solve":
+        # one batch row, as many channels as fit the budget: the fp64 projection
+        # of those channels' three gate rows, then the serial fp64 Newton solve
+        Bx, Lx, Kx = x["x"].shape
+        Dx = x["a"].shape[1]
+
+        def sample(nd):
+            rows = np.concatenate([np.arange(nd), Dx + np.arange(nd), 2 * Dx + np.arange(nd)])
+            Pc = oracle.input_projection(x["x"][0], x["W"][rows], x["bias"][rows])
+            Pc = Pc.reshape(1, Lx, 3, nd)
+            return oracle.newton_gru(Pc, x["a"][:, :nd], tol=1e-4, max_iters=32)
+        t0 = time.perf_counter()
+        sample(4)
+        per = max((time.perf_counter() - t0) / 4, 1e-6)
+        nd = int(max(4, min(Dx, budget_s / per)))
+        t0 = time.perf_counter()
+        res = sample(nd)
+        dt = time.perf_counter() - t0
+        return {"value": Lx * nd / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"fp64 projection (K={Kx}) + serial fp64 Newton, B=1 x D={nd} x "
+                          f"L={Lx} ({res.iterations} iterations, {dt:.1f} s)"}
     if op == "mhgru":
         # whole heads of one batch row, as many as fit the budget
         t0 = time.perf_counter()
@@ -1002,6 +1097,18 @@ def run_reference(args, world, rank, local):
         def step():
             return oracle.newton_mhgru(Ps, Us)
         what = "serial fp64 Newton (8x8 blocks)"
+    elif op == "proj_solve":
+        K = w["K"]
+        x = inputs.projected_gru_inputs(B, L, D, K, w["seed"])
+        nd = min(D, 16)
+        rows = np.concatenate([np.arange(nd), D + np.arange(nd), 2 * D + np.arange(nd)])
+        xs, Ws, bs = x["x"][0], np.ascontiguousarray(x["W"][rows]), x["bias"][rows]
+        as_ = np.ascontiguousarray(x["a"][:, :nd])
+
+        def step():
+            Pc = oracle.input_projection(xs, Ws, bs).reshape(1, L, 3, nd)
+            return oracle.newton_gru(Pc, as_, tol=1e-4, max_iters=32)
+        what = f"fp64 projection (K={K}) + serial fp64 Newton"
     elif op == "proj":
         Nf, K = w["G"] * D, w["K"]
         x = inputs.projection_inputs(B * L, Nf, K, w["seed"])
@@ -1013,7 +1120,7 @@ def run_reference(args, world, rank, local):
         what = f"fp64 input projection ({nrows} rows x N={Nf} x K={K})"
     else:
         x = inputs.workload_inputs(args.workload)  # the same draws as the GPU arm, then sliced
-    if op in ("gru_bwd", "lstm_bwd", "proj", "mhgru"):
+    if op in ("gru_bwd", "lstm_bwd", "proj", "mhgru", "proj_solve"):
         pass
     elif op in ("gru", "lstm"):
         Ps = np.ascontiguousarray(x["P"][:1, :, :, :nd])
@@ -1048,8 +1155,10 @@ def run_reference(args, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded numpy)",
             "config": {"workload": workload_name(args.workload, B, L, D,
-                                                 w.get("K") if op == "proj" else None,
-                                                 w.get("G") if op == "proj" else None),
+                                                 w.get("K") if op in ("proj", "proj_solve")
+                                                 else None,
+                                                 w.get("G") if op in ("proj", "proj_solve")
+                                                 else None),
                        "B": B, "L": L, "D": D, "parallelism": "rank 0 only, host cores",
                        "sample": (f"oracle {what}" if op == "proj"
                                   else f"oracle {what} on B=1 x D={nd} x L={L} per step")},
@@ -1068,7 +1177,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="lm",
                     choices=["lm", "gru_l", "deer", "gru_s", "lstm", "scan", "scan_lm", "block2",
-                             "gru_bwd", "lstm_bwd", "proj", "proj_lm", "mhgru"])
+                             "gru_bwd", "lstm_bwd", "proj", "proj_lm", "proj_solve", "mhgru"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-scan", action="store_true", help="skip the scan leg (lm, gru_l)")

@@ -68,7 +68,8 @@ typedef enum {
   PARARNN_OP_LSTM = 3,
   PARARNN_OP_GRU_BACKWARD = 4,
   PARARNN_OP_LSTM_BACKWARD = 5,
-  PARARNN_OP_MHGRU = 6
+  PARARNN_OP_MHGRU = 6,
+  PARARNN_OP_GRU_PROJECTED = 7
 } pararnn_op_t;
 
 /* Device-side outcome of a solve (caller-owned DEVICE memory, written by the
@@ -287,6 +288,33 @@ pararnn_status_t pararnn_input_projection(const void* x, const void* W, const fl
                                           void* P, pararnn_dtype_t p_dtype, int64_t M,
                                           int64_t N, int64_t K, int32_t* status_dev,
                                           void* stream);
+
+/* ParaGRU layer from its inputs: the input projection P = x W^T + bias fused
+ * with the Newton solve, so that P is never written to HBM (ParaRNN, TL;DR and
+ * Abstract: dense weights act on the inputs of an LM layer, the recurrence
+ * keeps diagonal ones).  The result is the one of pararnn_input_projection
+ * with fp32 P followed by pararnn_solve_gru on that P, up to the order of
+ * floating-point rounding.
+ *  x    : [B, L, K] bf16 (row b L + t = input at step t + 1 of batch row b),
+ *         16-byte aligned.
+ *  W    : [3 D, K] bf16, the nn.Linear layout: rows 0..D-1 give the z gate,
+ *         D..2D-1 the r gate, 2D..3D-1 the c gate; 16-byte aligned.
+ *  bias : [3 D] fp32 or NULL (zero), same row order.
+ *  a, h0, h, tol, max_iters, info, opts: as in pararnn_solve_gru (h0 [B, D]
+ *         or NULL, h [B, L, D] fp32 output, info device memory).
+ *  ws   : workspace of pararnn_workspace_size(PARARNN_OP_GRU_PROJECTED, ...)
+ *         bytes (a few hundred; zeroed by the call), 256-byte aligned.
+ * The projection runs on the tensor cores (bf16 operands, fp32 accumulation);
+ * each chunk of P stays in TMEM and shared memory.  A solve that needs more
+ * than one sweep of the default 4 Newton iterations recomputes the projection
+ * for each later sweep.  Requirements: K > 0 and K % 8 == 0, B L < 2^31;
+ * otherwise PARARNN_ERR_INVALID_ARGUMENT.  Needs sm_100a. */
+pararnn_status_t pararnn_solve_gru_projected(const void* x, const void* W, const float* bias,
+                                             const float* a, const float* h0, float* h,
+                                             int64_t B, int64_t L, int64_t D, int64_t K,
+                                             float tol, int32_t max_iters, void* ws,
+                                             size_t ws_bytes, pararnn_solve_info_t* info,
+                                             const pararnn_options_t* opts, void* stream);
 
 /* Allocation-free variant of pararnn_solve_gru (the pages have no counterpart:
  * this is an interface convenience of this library).

@@ -15,6 +15,8 @@ Entry points (same names as the C ABI, without the ``pararnn_`` prefix):
 * ``solve_gru_backward`` / ``solve_lstm_backward``  gradients through the solution
 * ``solve_mhgru(P, U, h0=None)``     multi-head GRU, dense 8x8 recurrence blocks
 * ``input_projection(x, W, bias=None)``  P = x W^T + bias on the tensor cores
+* ``solve_gru_projected(x, W, bias, a, h0=None)``  the projection fused with the
+  ParaGRU Newton solve (P never reaches HBM)
 * ``step_gru`` / ``step_lstm``      one decode step;  ``rollout_gru`` / ``rollout_lstm``
   the sequential application on the GPU
 
@@ -31,7 +33,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc",
+__all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc", "solve_gru_projected",
            "solve_gru_backward", "solve_lstm_backward", "solve_mhgru", "input_projection",
            "step_gru", "step_lstm", "rollout_gru", "rollout_lstm",
            "workspace_size", "probe_rate", "PROBE_MUFU", "PROBE_FMA",
@@ -44,6 +46,7 @@ library_path = os.path.join(_HERE, "libpararnn.so")
 OP_SCAN_DIAG, OP_SCAN_BLOCK2, OP_GRU, OP_LSTM = 0, 1, 2, 3
 OP_GRU_BACKWARD, OP_LSTM_BACKWARD = 4, 5
 OP_MHGRU = 6
+OP_GRU_PROJECTED = 7
 F32, BF16 = 0, 1
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA runtime error",
@@ -146,6 +149,11 @@ def load(build_if_missing: bool = True):
             lib.pararnn_input_projection.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i64,
                                                      _i64, _i64, _vp, _vp]
             lib.pararnn_input_projection.restype = ctypes.c_int
+            lib.pararnn_solve_gru_projected.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                                        _i64, _i64, ctypes.c_float,
+                                                        ctypes.c_int32, _vp, ctypes.c_size_t,
+                                                        _vp, _vp, _vp]
+            lib.pararnn_solve_gru_projected.restype = ctypes.c_int
             lib.pararnn_probe_rate.argtypes = [ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp]
             lib.pararnn_probe_rate.restype = ctypes.c_int
             lib.pararnn_status_string.argtypes = [ctypes.c_int]
@@ -448,6 +456,41 @@ def solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32, out=None, info=No
                                     _stream_handle(stream, dev))
     _raise(st, "pararnn_solve_lstm")
     return c, h, SolveInfo(info)
+
+
+def solve_gru_projected(x, W, bias, a, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
+                        opts: Options | None = None, stream=None):
+    """ParaGRU layer from its inputs: P = x W^T + bias on the tensor cores, fused
+    with the Newton solve so that P never reaches HBM.  x [B, L, K] bf16, W
+    [3 D, K] bf16 (rows z, r, c), bias [3 D] fp32 or None, a [3, D] ->
+    (h [B, L, D], SolveInfo)."""
+    lib = load()
+    if x.dim() != 3 or W.dim() != 2 or x.shape[-1] != W.shape[1] or W.shape[0] % 3 != 0:
+        raise ValueError(f"x [B, L, K] and W [3 D, K] do not match: {tuple(x.shape)}, "
+                         f"{tuple(W.shape)}")
+    B, L, K = x.shape
+    D = W.shape[0] // 3
+    _check_dev("x", x, torch.bfloat16, (B, L, K))
+    _check_dev("W", W, torch.bfloat16, (3 * D, K))
+    _check_dev("bias", bias, torch.float32, (3 * D,))
+    _check_dev("a", a, torch.float32, (3, D))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    h = torch.empty((B, L, D), dtype=torch.float32, device=x.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, L, D))
+    if info is None:
+        info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=x.device)
+    _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
+    dev = _one_device(x=x, W=W, bias=bias, a=a, h0=h0, out=h, info=info)
+    n = workspace_size(OP_GRU_PROJECTED, B, L, D, max_iters, opts)
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_solve_gru_projected(_ptr(x), _ptr(W), _ptr(bias), _ptr(a), _ptr(h0),
+                                             _ptr(h), B, L, D, K, float(tol), int(max_iters),
+                                             _ptr(ws), ws.numel(), _ptr(info),
+                                             ctypes.byref(opts) if opts is not None else None,
+                                             _stream_handle(stream, dev))
+    _raise(st, "pararnn_solve_gru_projected")
+    return h, SolveInfo(info)
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20

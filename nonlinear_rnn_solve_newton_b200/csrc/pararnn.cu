@@ -20,6 +20,7 @@
 #include "pararnn_mhgru.cuh"
 #include "pararnn_probe.cuh"
 #include "pararnn_proj.cuh"
+#include "pararnn_projsolve.cuh"
 #include "pararnn_seq.cuh"
 #include "pararnn_walk.cuh"
 
@@ -785,6 +786,10 @@ size_t pararnn_workspace_size(pararnn_op_t op, int64_t B, int64_t L, int64_t D, 
     if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return 0;
     return (sizeof(Ctrl) + 4 * (size_t)(max_iters + 1) + 255) / 256 * 256;
   }
+  if ((int)op == 7) {  // projected GRU solve: control block, residuals, no look-back records
+    if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return 0;
+    return (sizeof(Ctrl) + 4 * (size_t)(max_iters + 1) + 255) / 256 * 256;
+  }
   if ((int)op < 0 || (int)op > 5) return 0;
   if (B == 0 || L == 0 || D == 0) return 256;
   Plan pl = make_plan((int)op, B, L, D, max_iters, opts);
@@ -1430,5 +1435,118 @@ extern "C" pararnn_status_t pararnn_probe_rate(int32_t pipe, int32_t iters, floa
   if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
   const int64_t per_step = pipe == 0 ? 2 : 1;
   *ops = (int64_t)total * kProbeThreads * (int64_t)iters * kProbeUnroll * kProbeChains * per_step;
+  return PARARNN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Projected ParaGRU solve: input projection on the tensor cores fused with the
+// Newton walk (P never reaches HBM).
+// ---------------------------------------------------------------------------
+namespace pararnn {
+namespace {
+
+#ifndef PARARNN_PS_STAGES
+#define PARARNN_PS_STAGES 5
+#endif
+constexpr int kPsStages = PARARNN_PS_STAGES;
+
+// W [3 D, K] bf16 viewed as 3 gate blocks of D rows: {K, D, 3}, box {64, 32, 3},
+// 128-byte swizzle (the box lands as 96 consecutive swizzled 128-byte rows).
+bool encode_map_w3(CUtensorMap* m, const void* W, unsigned long long K, unsigned long long D) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {K, D, 3};
+  const cuuint64_t strides[2] = {K * 2, D * K * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)kPsCW, 3};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(W), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace pararnn
+
+extern "C" pararnn_status_t pararnn_solve_gru_projected(
+    const void* x, const void* W, const float* bias, const float* a, const float* h0, float* h,
+    int64_t B, int64_t L, int64_t D, int64_t K, float tol, int32_t max_iters, void* ws,
+    size_t ws_bytes, pararnn_solve_info_t* info, const pararnn_options_t* opts, void* stream) {
+  using namespace pararnn;
+  if (B < 0 || L < 0 || D < 0 || K < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!info || !aligned(info, 4)) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!(tol >= 0.0f)) return PARARNN_ERR_INVALID_ARGUMENT;  // rejects NaN too
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (B == 0 || L == 0 || D == 0) {
+    empty_info_kernel<<<1, 1, 0, st>>>(info);
+    return cudaGetLastError() == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA;
+  }
+  if (!x || !W || !a || !h) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (K == 0 || K % 8 != 0 || K >= (1LL << 31) || B * L >= (1LL << 31) || D >= (1LL << 30))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+  if (!aligned(x, 16) || !aligned(W, 16) || (bias && !aligned(bias, 4)) || !aligned(a, 4) ||
+      (h0 && !aligned(h0, 4)) || !aligned(h, 4))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+  const size_t need = pararnn_workspace_size((pararnn_op_t)7, B, L, D, max_iters, opts);
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return PARARNN_ERR_WORKSPACE;
+
+  PsMaps tm;
+  if (!encode_map_sw128(&tm.x, x, (unsigned long long)K, (unsigned long long)(B * L), kPsBM) ||
+      !encode_map_w3(&tm.w, W, (unsigned long long)K, (unsigned long long)D))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+
+  PsParams pp;
+  pp.bias = bias;
+  pp.w = a;
+  pp.h0 = h0;
+  pp.h = h;
+  pp.B = B;
+  pp.L = L;
+  pp.D = D;
+  pp.K = (int)K;
+  pp.ntd = (int)((D + kPsCW - 1) / kPsCW);
+  pp.nitems = (int)(B * pp.ntd);
+  pp.nchunks = (int)((L + kPsBM - 1) / kPsBM);
+  pp.tol = tol;
+  pp.max_iters = max_iters;
+  int mf = (opts && opts->iters_first > 0) ? opts->iters_first : 4;
+  int mn = (opts && opts->iters_next > 0) ? opts->iters_next : 2;
+  if (mf > kMaxWalkIters) mf = kMaxWalkIters;
+  if (mn > kMaxWalkIters) mn = kMaxWalkIters;
+  pp.m_first = mf;
+  pp.m_next = mn;
+  pp.ctrl = static_cast<Ctrl*>(ws);
+  pp.rho_bits = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + sizeof(Ctrl));
+  pp.info = info;
+  pp.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? opts->wait_timeout_ns : 1000000000LL;
+  if (B * (long long)pp.ntd >= (1LL << 31) || L / kPsBM >= (1LL << 30))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+
+  const void* fn = (const void*)pararnn_projsolve_kernel<kPsStages>;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_UNSUPPORTED;
+  }
+  const size_t smem = ps_smem_bytes<kPsStages>();
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  int resident = 0;
+  if (resident_ctas(fn, kPsThreads, smem, &resident) != cudaSuccess || resident <= 0) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
+  const int grid = pp.nitems < resident ? pp.nitems : resident;
+  if (cudaMemsetAsync(ws, 0, need, st) != cudaSuccess) return PARARNN_ERR_CUDA;
+  void* args[] = {&pp, &tm};
+  // sweeps are separated by a grid barrier: every CTA must be resident
+  if (cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kPsThreads), args, smem, st) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return PARARNN_ERR_CUDA;
+  }
   return PARARNN_OK;
 }

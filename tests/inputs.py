@@ -24,6 +24,7 @@ lm       ParaGRU solve, bf16 P, fp32 state      8, 8192, 4096
 scan_lm  diagonal affine scan, fp32, LM width   8, 8192, 4096
 proj     input projection x W^T (+bias), G=3    8, 4096, 1024, K = 1024
 proj_lm  input projection, LM width, G=3        8, 8192, 4096, K = 4096
+proj_solve projection fused with the GRU solve   8, 8192, 4096, K = 4096
 mhgru    multi-head GRU, 8x8 blocks, fp32       8, 4096, 1024 (128 heads)
 =======  =====================================  ==========================
 
@@ -57,6 +58,7 @@ WORKLOADS = {
     "mhgru": dict(op="mhgru", B=8, L=4096, D=1024, seed=8, bf16=False),
     "proj": dict(op="proj", B=8, L=4096, D=1024, K=1024, G=3, seed=6, bf16=False),
     "proj_lm": dict(op="proj", B=8, L=8192, D=4096, K=4096, G=3, seed=7, bf16=True),
+    "proj_solve": dict(op="proj_solve", B=8, L=8192, D=4096, K=4096, G=3, seed=10, bf16=True),
 }
 
 L_SWEEP = [1 << e for e in range(6, 15)]
@@ -168,6 +170,22 @@ def projection_inputs(M, N, K, seed):
     w_bits, W = round_to_bf16(w32)
     bias = (_normal(rng, (N,)) * np.float32(0.1)).astype(np.float32)
     return dict(x=x, x_bits=x_bits, W=W, W_bits=w_bits, bias=bias)
+
+
+def projected_gru_inputs(B, L, D, K, seed, h0_normal=False):
+    """A ParaGRU layer from its inputs: x [B, L, K] and W [3 D, K] as bf16 (bits
+    and values), bias [3 D] (as projection_inputs with M = B L, N = 3 D), then
+    a [3, D] ~ U(-0.5, 0.5) and h0 [B, D] (zeros, or N(0, 1)).  Draw order x, W,
+    bias, a, h0."""
+    rng = _rng(seed)
+    x_bits, x = round_to_bf16(_normal(rng, (B * L, K)))
+    w32 = (_normal(rng, (3 * D, K)) * np.float32(1.0 / np.sqrt(max(K, 1)))).astype(np.float32)
+    w_bits, W = round_to_bf16(w32)
+    bias = (_normal(rng, (3 * D,)) * np.float32(0.1)).astype(np.float32)
+    a = _uniform(rng, -0.5, 0.5, (3, D))
+    h0 = _normal(rng, (B, D)) if h0_normal else np.zeros((B, D), np.float32)
+    return dict(x=x.reshape(B, L, K), x_bits=x_bits.reshape(B, L, K), W=W, W_bits=w_bits,
+                bias=bias, a=a, h0=h0)
 
 
 def mhgru_inputs(B, L, H, seed, u_scale=0.3, h0_normal=False):

@@ -82,3 +82,14 @@ def test_cpu_baseline_reports_threaded_and_single_thread():
     st = out["single_thread"]
     assert st["newton_channel_steps_per_s"] > 0 and st["rollout_channel_steps_per_s"] > 0
     assert oracle.get_threads() == out["cores"]   # the thread count is restored
+
+
+def test_cpu_baseline_projected_solve():
+    """The CPU leg of the fused projection + solve workload: the oracle's fp64
+    projection of a channel sample followed by its serial Newton (small case)."""
+    from tests import inputs
+
+    x = inputs.projected_gru_inputs(1, 64, 16, 32, seed=6)
+    out = bench.cpu_baseline(x, "proj_solve", 1, 64, 16, budget_s=0.05)
+    assert out["kind"] == "oracle" and out["value"] > 0 and out["cores"] >= 1
+    assert "projection" in out["sample"]

@@ -94,6 +94,10 @@ def test_every_entry_point_reaches_its_c_function(fake):
         ("pararnn_step_lstm", lambda: pr.step_lstm(z(B, 4, D), z(4, D), z(B, D), z(B, D))),
         ("pararnn_rollout_gru", lambda: pr.rollout_gru(z(B, L, 3, D), z(3, D), z(B, D))),
         ("pararnn_rollout_lstm", lambda: pr.rollout_lstm(z(B, L, 4, D), z(4, D))),
+        ("pararnn_solve_gru_projected",
+         lambda: pr.solve_gru_projected(z(B, L, K, dtype=torch.bfloat16),
+                                        z(3 * D, K, dtype=torch.bfloat16), z(3 * D), z(3, D),
+                                        z(B, D), info=info_t())),
         ("pararnn_input_projection",
          lambda: pr.input_projection(z(B, L, K, dtype=torch.bfloat16),
                                      z(3 * D, K, dtype=torch.bfloat16), z(3 * D),
