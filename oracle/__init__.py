@@ -91,9 +91,9 @@ def _bind(lib):
     lib.oracle_backward_lstm.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
                                          _f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
     lib.oracle_mhgru_cell.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p]
-    lib.oracle_rollout_mhgru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
+    lib.oracle_rollout_mhgru.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64, _intp]
     lib.oracle_newton_mhgru.argtypes = [_f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_int,
-                                        _i64, _i64, _i64, _f64p, _f64p, _intp, _intp]
+                                        _i64, _i64, _i64, _f64p, _f64p, _intp, _intp, _intp]
     lib.oracle_newton_mhgru.restype = ctypes.c_int
     lib.oracle_input_projection.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64]
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
@@ -312,21 +312,31 @@ def mhgru_cell(p, U, h):
     return f, J
 
 
-def rollout_mhgru(P, U, h0=None):
-    """Sequential multi-head GRU rollout.  P [B, L, 3, D], U [3, H, 8, 8], D = 8 H."""
+def _strides(strides, H):
+    if strides is None:
+        return None, None
+    st = np.ascontiguousarray(strides, dtype=np.int32).reshape(H)
+    assert np.all(st >= 1), "strides must be >= 1"
+    return st, st.ctypes.data_as(_intp)
+
+
+def rollout_mhgru(P, U, h0=None, strides=None):
+    """Sequential multi-head GRU rollout.  P [B, L, 3, D], U [3, H, 8, 8], D = 8 H;
+    strides [H] (optional): head g recurs on h_{t - strides[g]}."""
     P, U = _d(P), _d(U)
     B, L, G, D = P.shape
     H = U.shape[1]
     assert G == 3 and U.shape == (3, H, 8, 8) and D == 8 * H
     h0 = None if h0 is None else _d(h0).reshape(B, D)
     h = np.empty((B, L, D))
-    _load().oracle_rollout_mhgru(_p(P), _p(U), _p(h0), _p(h), B, L, H)
+    keep, sp = _strides(strides, H)
+    _load().oracle_rollout_mhgru(_p(P), _p(U), _p(h0), _p(h), B, L, H, sp)
     return h
 
 
-def newton_mhgru(P, U, h0=None, tol=1e-4, max_iters=32):
+def newton_mhgru(P, U, h0=None, tol=1e-4, max_iters=32, strides=None):
     """Serial Newton for the multi-head GRU system from h^0 = 0, 8x8 block
-    bi-diagonal solve per head (see oracle.c)."""
+    bi-diagonal solve per head (see oracle.c); strides as in rollout_mhgru."""
     P, U = _d(P), _d(U)
     B, L, G, D = P.shape
     H = U.shape[1]
@@ -336,6 +346,7 @@ def newton_mhgru(P, U, h0=None, tol=1e-4, max_iters=32):
     rho = np.full(max_iters + 1, np.nan)
     conv = ctypes.c_int()
     nf = ctypes.c_int()
+    keep, sp = _strides(strides, H)
     k = _load().oracle_newton_mhgru(_p(P), _p(U), _p(h0), float(tol), int(max_iters), B, L, H,
-                                    _p(h), _p(rho), ctypes.byref(conv), ctypes.byref(nf))
+                                    _p(h), _p(rho), ctypes.byref(conv), ctypes.byref(nf), sp)
     return NewtonResult(k, conv.value, nf.value, rho[: k + 1], None, h=h)

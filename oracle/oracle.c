@@ -655,6 +655,11 @@ void oracle_input_projection(const double* x, const double* W, const double* bia
  *   dh'_i/dh_j = [i == j] (1 - z_i) + (c_i - h_i) z_i (1 - z_i) U_z[i][j]
  *              + z_i (1 - c_i^2) (r_i U_c[i][j] + (U_c h)_i r_i (1 - r_i) U_r[i][j])
  * P is [B, L, 3, D] (gates z, r, c), U is [3, H, 8, 8], D = 8 H.
+ *
+ * Time strides (DEER summary, caveats paragraph: heads of 8 channels with
+ * exponentially increasing strides, i.e. shorter effective sequences): head g
+ * may recur at stride s_g >= 1, h_t = f(h_{t - s_g}, P_t), with h_{t - s_g} = h0
+ * for t < s_g.  strides == NULL means s_g = 1 for every head.
  * ---------------------------------------------------------------------- */
 #define NB 8
 
@@ -689,7 +694,11 @@ typedef struct {
   const double *P, *U, *h0;
   double *h, *Jt, *rt, *cmax;
   int64_t L, H;
+  const int32_t* stride; /* [H] or NULL (all 1) */
+  double* dt;            /* Newton step delta, [B, L, D] */
 } mh_ctx;
+
+static int64_t mh_stride(const mh_ctx* x, int64_t g) { return x->stride ? x->stride[g] : 1; }
 
 /* gates of head g at (b, t): p[gate * 8 + i] */
 static void mh_gates(const mh_ctx* x, int64_t bb, int64_t t, int64_t g, double* p) {
@@ -698,11 +707,12 @@ static void mh_gates(const mh_ctx* x, int64_t bb, int64_t t, int64_t g, double* 
     for (int i = 0; i < NB; ++i) p[k * NB + i] = x->P[IDXP(bb, t, k, g * NB + i, x->L, 3, D)];
 }
 
+/* the state the step at t recurs on: h_{t - s_g}, or h0 before the sequence */
 static void mh_prev(const mh_ctx* x, int64_t bb, int64_t t, int64_t g, double* hp) {
-  int64_t D = NB * x->H;
+  int64_t D = NB * x->H, tp = t - mh_stride(x, g);
   for (int i = 0; i < NB; ++i)
-    hp[i] = (t == 0) ? (x->h0 ? x->h0[bb * D + g * NB + i] : 0.0)
-                     : x->h[IDX3(bb, t - 1, g * NB + i, x->L, D)];
+    hp[i] = (tp < 0) ? (x->h0 ? x->h0[bb * D + g * NB + i] : 0.0)
+                     : x->h[IDX3(bb, tp, g * NB + i, x->L, D)];
 }
 
 static void rollout_mhgru_head(void* p, int64_t u) {
@@ -728,9 +738,9 @@ static double* mh_heads(const double* U, int64_t H) {
 }
 
 void oracle_rollout_mhgru(const double* P, const double* U, const double* h0, double* h,
-                          int64_t B, int64_t L, int64_t H) {
+                          int64_t B, int64_t L, int64_t H, const int32_t* strides) {
   double* Uh = mh_heads(U, H);
-  mh_ctx x = {P, Uh, h0, h, NULL, NULL, NULL, L, H};
+  mh_ctx x = {P, Uh, h0, h, NULL, NULL, NULL, L, H, strides, NULL};
   for_channels(B * H, rollout_mhgru_head, &x);
   free(Uh);
 }
@@ -756,30 +766,37 @@ static void newton_mhgru_residual_head(void* p, int64_t u) {
 
 static void newton_mhgru_solve_head(void* p, int64_t u) {
   mh_ctx* x = (mh_ctx*)p;
-  int64_t bb = u / x->H, g = u % x->H, D = NB * x->H, L = x->L;
-  double delta[NB] = {0}, nd[NB];
+  int64_t bb = u / x->H, g = u % x->H, D = NB * x->H, L = x->L, st = mh_stride(x, g);
   for (int64_t t = 0; t < L; ++t) {
+    /* delta_t = J_t delta_{t - s} + r_t, with delta = 0 before the sequence */
     const double* J = x->Jt + ((size_t)u * L + t) * NB * NB;
+    double prev[NB], nd[NB];
+    for (int j = 0; j < NB; ++j)
+      prev[j] = (t - st < 0) ? 0.0 : x->dt[IDX3(bb, t - st, g * NB + j, L, D)];
     for (int i = 0; i < NB; ++i) {
       double s = x->rt[IDX3(bb, t, g * NB + i, L, D)];
-      for (int j = 0; j < NB; ++j) s += J[i * NB + j] * delta[j];
+      for (int j = 0; j < NB; ++j) s += J[i * NB + j] * prev[j];
       nd[i] = s;
     }
-    for (int i = 0; i < NB; ++i) {
-      delta[i] = nd[i];
-      x->h[IDX3(bb, t, g * NB + i, L, D)] += delta[i];
-    }
+    for (int i = 0; i < NB; ++i) x->dt[IDX3(bb, t, g * NB + i, L, D)] = nd[i];
   }
+  /* the update, once every delta of the head is known */
+  for (int64_t t = 0; t < L; ++t)
+    for (int i = 0; i < NB; ++i)
+      x->h[IDX3(bb, t, g * NB + i, L, D)] += x->dt[IDX3(bb, t, g * NB + i, L, D)];
 }
 
 /* Serial Newton as oracle_newton_gru, with 8x8 blocks: the linear solve is
- * delta_t = J_t delta_{t-1} + r_t per head.  rho_hist has max_iters + 1 slots. */
+ * delta_t = J_t delta_{t-s} + r_t per head (s = the head's stride, 1 by
+ * default).  rho_hist has max_iters + 1 slots. */
 int oracle_newton_mhgru(const double* P, const double* U, const double* h0, double tol,
                         int max_iters, int64_t B, int64_t L, int64_t H, double* h,
-                        double* rho_hist, int* converged, int* nonfinite) {
+                        double* rho_hist, int* converged, int* nonfinite,
+                        const int32_t* strides) {
   size_t N = (size_t)B * (size_t)L * (size_t)(NB * H);
   double* Uh = mh_heads(U, H);
-  mh_ctx x = {P, Uh, h0, h, NULL, NULL, NULL, L, H};
+  mh_ctx x = {P, Uh, h0, h, NULL, NULL, NULL, L, H, strides, NULL};
+  x.dt = (double*)malloc(N * sizeof(double));
   x.Jt = (double*)malloc(N * NB * sizeof(double));
   x.rt = (double*)malloc(N * sizeof(double));
   x.cmax = (double*)malloc((size_t)(B * H) * sizeof(double));
@@ -805,6 +822,7 @@ int oracle_newton_mhgru(const double* P, const double* U, const double* h0, doub
   free(x.Jt);
   free(x.rt);
   free(x.cmax);
+  free(x.dt);
   free(Uh);
   return k;
 }

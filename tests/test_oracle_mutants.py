@@ -74,8 +74,13 @@ MUTANTS = {
     "backward_lstm_dh0_from_c": ("if (x->dh0) x->dh0[bb * D + d] = mh;",
                                  "if (x->dh0) x->dh0[bb * D + d] = mc;"),
     "backward_lstm_da_without_h": ("      da[g] += v * hp;", "      da[g] += v;"),
-    "mhgru_ignores_h0": ("hp[i] = (t == 0) ? (x->h0 ? x->h0[bb * D + g * NB + i] : 0.0)",
-                         "hp[i] = (t == 0) ? 0.0"),
+    "mhgru_ignores_h0": ("hp[i] = (tp < 0) ? (x->h0 ? x->h0[bb * D + g * NB + i] : 0.0)",
+                         "hp[i] = (tp < 0) ? 0.0"),
+    "mhgru_stride_ignored": ("int64_t D = NB * x->H, tp = t - mh_stride(x, g);",
+                             "int64_t D = NB * x->H, tp = t - 1;"),
+    "mhgru_newton_delta_lag_one": (
+        "prev[j] = (t - st < 0) ? 0.0 : x->dt[IDX3(bb, t - st, g * NB + j, L, D)];",
+        "prev[j] = (t - 1 < 0) ? 0.0 : x->dt[IDX3(bb, t - 1, g * NB + j, L, D)];"),
 }
 
 

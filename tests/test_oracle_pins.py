@@ -734,3 +734,61 @@ def test_mhgru_prefix_exactness(oracle):
         res = oracle.newton_mhgru(x["P"], x["U"], x["h0"], tol=0.0, max_iters=k)
         assert res.iterations == k
         np.testing.assert_allclose(res.h[:, :k], ref[:, :k], atol=1e-13, rtol=0)
+
+
+# --------------------------------------------------------------------------
+# Multi-head GRU with per-head time strides (DEER summary, caveats: heads with
+# exponentially increasing strides): head g recurs on h_{t - s_g}
+# --------------------------------------------------------------------------
+def test_mhgru_strided_rollout_matches_torch(oracle):
+    """A plain loop over torch's GRUCell in which each head reads its own lag."""
+    B, L, H = 2, 37, 3
+    strides = np.array([1, 2, 5], np.int32)
+    x = inputs.mhgru_inputs(B, L, H, seed=724, h0_normal=True)
+    cell = torch_mhgru_cell(x["U"])
+    hist = []
+    h0 = torch.as_tensor(x["h0"].astype(np.float64))
+    with torch.no_grad():
+        for t in range(L):
+            # the state each head recurs on, assembled head by head
+            prev = torch.cat([(hist[t - s] if t - s >= 0 else h0)[:, 8 * g:8 * g + 8]
+                              for g, s in enumerate(strides)], 1)
+            hist.append(torch_gru_step(cell, x["P"][:, t], prev))
+    ref = torch.stack(hist, 1).numpy()
+    got = oracle.rollout_mhgru(x["P"], x["U"], x["h0"], strides=strides)
+    np.testing.assert_allclose(got, ref, atol=1e-13, rtol=0)
+
+
+def test_mhgru_strided_head_is_interleaved_stride_one_sequences(oracle):
+    """A head at stride s is s independent stride-1 sequences (t = r, r + s, ...):
+    de-interleaving by slicing and solving each at stride 1 gives the same values."""
+    B, L, H = 2, 50, 4
+    strides = np.array([1, 3, 4, 7], np.int32)
+    x = inputs.mhgru_inputs(B, L, H, seed=725, h0_normal=True)
+    got = oracle.rollout_mhgru(x["P"], x["U"], x["h0"], strides=strides)
+    for g, s in enumerate(strides):
+        for r in range(s):
+            sub = oracle.rollout_mhgru(x["P"][:, r::s, :, 8 * g:8 * g + 8], x["U"][:, g:g + 1],
+                                       x["h0"][:, 8 * g:8 * g + 8])
+            np.testing.assert_allclose(got[:, r::s, 8 * g:8 * g + 8], sub, atol=1e-14, rtol=0)
+    # and the Newton solve at those strides reaches the same trajectory
+    res = oracle.newton_mhgru(x["P"], x["U"], x["h0"], tol=1e-12, max_iters=50, strides=strides)
+    assert res.converged
+    np.testing.assert_allclose(res.h, got, atol=1e-10, rtol=0)
+
+
+def test_mhgru_strides_beyond_the_sequence_are_one_explicit_step(oracle):
+    """With every stride >= L each step depends on h0 only: the system is explicit,
+    Newton is exact after one update, and h_t = cell(P_t, h0)."""
+    B, L, H = 2, 9, 2
+    x = inputs.mhgru_inputs(B, L, H, seed=726, h0_normal=True)
+    strides = np.array([L, L + 5], np.int32)
+    got = oracle.rollout_mhgru(x["P"], x["U"], x["h0"], strides=strides)
+    for b in range(B):
+        for t in range(L):
+            for g in range(H):
+                f, _ = oracle.mhgru_cell(x["P"][b, t][:, 8 * g:8 * g + 8], x["U"][:, g],
+                                         x["h0"][b, 8 * g:8 * g + 8])
+                np.testing.assert_allclose(got[b, t, 8 * g:8 * g + 8], f, atol=1e-15, rtol=0)
+    res = oracle.newton_mhgru(x["P"], x["U"], x["h0"], tol=1e-12, max_iters=5, strides=strides)
+    assert res.converged and res.iterations == 1
