@@ -69,7 +69,8 @@ typedef enum {
   PARARNN_OP_GRU_BACKWARD = 4,
   PARARNN_OP_LSTM_BACKWARD = 5,
   PARARNN_OP_MHGRU = 6,
-  PARARNN_OP_GRU_PROJECTED = 7
+  PARARNN_OP_GRU_PROJECTED = 7,
+  PARARNN_OP_MHGRU_STRIDED = 8
 } pararnn_op_t;
 
 /* Device-side outcome of a solve (caller-owned DEVICE memory, written by the
@@ -268,6 +269,28 @@ pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p_dtype, con
                                      int64_t H, float tol, int32_t max_iters, void* ws,
                                      size_t ws_bytes, pararnn_solve_info_t* info,
                                      const pararnn_options_t* opts, void* stream);
+
+/* The multi-head GRU with a time stride per head (DEER summary, caveats
+ * paragraph: heads of 8 channels with exponentially increasing strides, i.e.
+ * shorter effective sequences).  Head g recurs on h_{t - s_g}:
+ *   h_t[head g] = cell_g(P_t, h_{t - s_g}[head g]),   h_{t - s_g} = h0 for t < s_g,
+ * so a head at stride s is s independent interleaved sequences (t = r, r + s,
+ * ...), each of about L / s steps; the Newton solve, its stopping rule and its
+ * outputs are otherwise those of pararnn_solve_mhgru (which is this call with
+ * every stride 1).
+ *  strides : [H] int32 in DEVICE memory, each >= 1 (a stride of L or more makes
+ *            every step of the head depend on h0 only).  A stride below 1 is
+ *            found on the device: the call then does no work and info.status
+ *            reads PARARNN_ERR_INVALID_ARGUMENT.  NULL is rejected.
+ *  ws      : pararnn_workspace_size(PARARNN_OP_MHGRU_STRIDED, B, L, 8 H, max_iters,
+ *            opts) bytes (it also holds the heads' stride offsets).
+ * Requires H L < 2^31; other arguments and errors as pararnn_solve_mhgru. */
+pararnn_status_t pararnn_solve_mhgru_strided(const void* P, pararnn_dtype_t p_dtype,
+                                             const float* U, const int32_t* strides,
+                                             const float* h0, float* h, int64_t B, int64_t L,
+                                             int64_t H, float tol, int32_t max_iters, void* ws,
+                                             size_t ws_bytes, pararnn_solve_info_t* info,
+                                             const pararnn_options_t* opts, void* stream);
 
 /* Input projection P = x W^T + bias on the tensor cores (tcgen05, bf16 inputs,
  * fp32 accumulation): the projected gate pre-activations that the cells take

@@ -14,6 +14,7 @@ Entry points (same names as the C ABI, without the ``pararnn_`` prefix):
 * ``solve_lstm(P, a, c0=None, h0=None, tol=1e-4, max_iters=32)``  ParaLSTM Newton solve
 * ``solve_gru_backward`` / ``solve_lstm_backward``  gradients through the solution
 * ``solve_mhgru(P, U, h0=None)``     multi-head GRU, dense 8x8 recurrence blocks
+* ``solve_mhgru_strided(P, U, strides, h0=None)``  the same with a time stride per head
 * ``input_projection(x, W, bias=None)``  P = x W^T + bias on the tensor cores
 * ``solve_gru_projected(x, W, bias, a, h0=None)``  the projection fused with the
   ParaGRU Newton solve (P never reaches HBM)
@@ -33,7 +34,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc", "solve_gru_projected",
+__all__ = ["scan_diag", "scan_block2", "solve_gru", "solve_lstm", "solve_gru_noalloc", "solve_gru_projected", "solve_mhgru_strided",
            "solve_gru_backward", "solve_lstm_backward", "solve_mhgru", "input_projection",
            "step_gru", "step_lstm", "rollout_gru", "rollout_lstm",
            "workspace_size", "probe_rate", "PROBE_MUFU", "PROBE_FMA",
@@ -47,6 +48,7 @@ OP_SCAN_DIAG, OP_SCAN_BLOCK2, OP_GRU, OP_LSTM = 0, 1, 2, 3
 OP_GRU_BACKWARD, OP_LSTM_BACKWARD = 4, 5
 OP_MHGRU = 6
 OP_GRU_PROJECTED = 7
+OP_MHGRU_STRIDED = 8
 F32, BF16 = 0, 1
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA runtime error",
@@ -146,6 +148,11 @@ def load(build_if_missing: bool = True):
                                                 _i64, ctypes.c_float, ctypes.c_int32, _vp,
                                                 ctypes.c_size_t, _vp, _vp, _vp]
             lib.pararnn_solve_mhgru.restype = ctypes.c_int
+            lib.pararnn_solve_mhgru_strided.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp,
+                                                        _i64, _i64, _i64, ctypes.c_float,
+                                                        ctypes.c_int32, _vp, ctypes.c_size_t,
+                                                        _vp, _vp, _vp]
+            lib.pararnn_solve_mhgru_strided.restype = ctypes.c_int
             lib.pararnn_input_projection.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i64,
                                                      _i64, _i64, _vp, _vp]
             lib.pararnn_input_projection.restype = ctypes.c_int
@@ -421,6 +428,39 @@ def solve_mhgru(P, U, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
                                      _ptr(info), ctypes.byref(opts) if opts is not None else None,
                                      _stream_handle(stream, dev))
     _raise(st, "pararnn_solve_mhgru")
+    return h, SolveInfo(info)
+
+
+def solve_mhgru_strided(P, U, strides, h0=None, tol=1e-4, max_iters=32, out=None, info=None,
+                        opts: Options | None = None, stream=None):
+    """Multi-head GRU with a time stride per head: head g recurs on h_{t - strides[g]}.
+    P [B, L, 3, D] (z, r, c), U [3, H, 8, 8], strides [H] int32 (device, each >= 1)
+    -> (h [B, L, D], SolveInfo)."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 3 or U.dim() != 4 or tuple(U.shape[2:]) != (8, 8) or D != 8 * U.shape[1]:
+        raise ValueError("P must be [B, L, 3, 8 H] and U [3, H, 8, 8]")
+    H = U.shape[1]
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 3, D))
+    _check_dev("U", U, torch.float32, (3, H, 8, 8))
+    _check_dev("strides", strides, torch.int32, (H,))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    h = torch.empty((B, L, D), dtype=torch.float32, device=P.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, L, D))
+    if info is None:
+        info = torch.empty(INFO_BYTES // 4, dtype=torch.int32, device=P.device)
+    _check_dev("info", info, torch.int32, (INFO_BYTES // 4,))
+    dev = _one_device(P=P, U=U, strides=strides, h0=h0, out=h, info=info)
+    n = workspace_size(OP_MHGRU_STRIDED, B, L, D, max_iters, opts)
+    ws = _workspace(n, dev, stream)
+    with _device_guard(dev):
+        st = lib.pararnn_solve_mhgru_strided(_ptr(P), dt, _ptr(U), _ptr(strides), _ptr(h0),
+                                             _ptr(h), B, L, H, float(tol), int(max_iters),
+                                             _ptr(ws), ws.numel(), _ptr(info),
+                                             ctypes.byref(opts) if opts is not None else None,
+                                             _stream_handle(stream, dev))
+    _raise(st, "pararnn_solve_mhgru_strided")
     return h, SolveInfo(info)
 
 

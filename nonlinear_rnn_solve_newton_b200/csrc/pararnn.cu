@@ -786,6 +786,11 @@ size_t pararnn_workspace_size(pararnn_op_t op, int64_t B, int64_t L, int64_t D, 
     if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return 0;
     return (sizeof(Ctrl) + 4 * (size_t)(max_iters + 1) + 255) / 256 * 256;
   }
+  if ((int)op == 8) {  // strided multi-head GRU: + the heads' stride offsets (H = D / 8)
+    if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS || D < 0 || D % 8 != 0) return 0;
+    const size_t base = (sizeof(Ctrl) + 4 * (size_t)(max_iters + 1) + 255) / 256 * 256;
+    return base + (4 * (size_t)(D / 8 + 2) + 255) / 256 * 256;
+  }
   if ((int)op == 7) {  // projected GRU solve: control block, residuals, no look-back records
     if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return 0;
     return (sizeof(Ctrl) + 4 * (size_t)(max_iters + 1) + 255) / 256 * 256;
@@ -1331,12 +1336,52 @@ extern "C" pararnn_status_t pararnn_input_projection(const void* x, const void* 
 // ---------------------------------------------------------------------------
 // Multi-head GRU (dense 8x8 blocks).
 // ---------------------------------------------------------------------------
-extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p_dtype,
-                                                const float* U, const float* h0, float* h,
-                                                int64_t B, int64_t L, int64_t H, float tol,
-                                                int32_t max_iters, void* ws, size_t ws_bytes,
-                                                pararnn_solve_info_t* info,
-                                                const pararnn_options_t* opts, void* stream) {
+namespace pararnn {
+namespace {
+
+// Prefix offsets of the heads' strides (each capped at L: a stride of L or more
+// makes every step depend on h0 alone) for the multi-head kernel's work units:
+// offs[g] = sum of the capped strides before head g, offs[H] = their total,
+// offs[H + 1] = 1 if some stride is below 1.  One warp.
+__global__ void mh_stride_offsets_kernel(const int32_t* strides, int* offs, long long H,
+                                         long long L) {
+  const int lane = threadIdx.x;
+  const long long per = (H + 31) / 32;
+  const long long g0 = lane * per;
+  const long long g1 = g0 + per < H ? g0 + per : H;
+  long long sum = 0;
+  int bad = 0;
+  for (long long g = g0; g < g1; ++g) {
+    const long long sg = strides[g];
+    if (sg < 1) bad = 1;
+    sum += sg < 1 ? 1 : (sg < L ? sg : L);
+  }
+  long long incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  long long acc = incl - sum;
+  for (long long g = g0; g < g1; ++g) {
+    offs[g] = (int)acc;
+    const long long sg = strides[g];
+    acc += sg < 1 ? 1 : (sg < L ? sg : L);
+  }
+  if (lane == 31) offs[H] = (int)incl;
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) offs[H + 1] = bad;
+}
+
+size_t mh_offsets_at(int32_t max_iters) {
+  return (sizeof(Ctrl) + 4 * (size_t)(max_iters + 1) + 255) / 256 * 256;
+}
+
+pararnn_status_t mhgru_common(const void* P, pararnn_dtype_t p_dtype, const float* U,
+                              const int32_t* strides, const float* h0, float* h, int64_t B,
+                              int64_t L, int64_t H, float tol, int32_t max_iters, void* ws,
+                              size_t ws_bytes, pararnn_solve_info_t* info,
+                              const pararnn_options_t* opts, void* stream) {
   if (B < 0 || L < 0 || H < 0) return PARARNN_ERR_INVALID_ARGUMENT;
   if (!info || !aligned(info, 4)) return PARARNN_ERR_INVALID_ARGUMENT;
   if (max_iters < 0 || max_iters > PARARNN_MAX_ITERS) return PARARNN_ERR_INVALID_ARGUMENT;
@@ -1351,7 +1396,10 @@ extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p
   if (!aligned(P, 16) || !aligned(U, 4) || !aligned(h, 16) || (h0 && !aligned(h0, 4)))
     return PARARNN_ERR_INVALID_ARGUMENT;
   if (B * H > (1LL << 40) || L > (1LL << 40)) return PARARNN_ERR_INVALID_ARGUMENT;
-  const size_t need = pararnn_workspace_size(PARARNN_OP_MHGRU, B, L, 8 * H, max_iters, opts);
+  // with strides, the work units of a batch row (sum of the capped strides) stay below 2^31
+  if (strides && (!aligned(strides, 4) || H * L >= (1LL << 31))) return PARARNN_ERR_INVALID_ARGUMENT;
+  const size_t need = pararnn_workspace_size(
+      strides ? PARARNN_OP_MHGRU_STRIDED : PARARNN_OP_MHGRU, B, L, 8 * H, max_iters, opts);
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return PARARNN_ERR_WORKSPACE;
 
   const void* fn = p_dtype == PARARNN_BF16
@@ -1374,9 +1422,10 @@ extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }
+  // with strides the unit count is known on the device only: every resident CTA runs
   const long long units = B * H;
   const long long want = (units + kMhWarps - 1) / kMhWarps;
-  const int grid = (int)(want < resident ? want : resident);
+  const int grid = strides ? resident : (int)(want < resident ? want : resident);
 
   MhParams mp;
   mp.P = P;
@@ -1390,10 +1439,17 @@ extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p
   mp.max_iters = max_iters;
   mp.ctrl = static_cast<Ctrl*>(ws);
   mp.rho_bits = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + sizeof(Ctrl));
+  int* offs = strides ? reinterpret_cast<int*>(static_cast<char*>(ws) + mh_offsets_at(max_iters))
+                      : nullptr;
+  mp.offs = offs;
   mp.info = info;
   mp.status_dev = nullptr;
   mp.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? opts->wait_timeout_ns : 1000000000LL;
   if (cudaMemsetAsync(ws, 0, need, st) != cudaSuccess) return PARARNN_ERR_CUDA;
+  if (strides) {
+    mh_stride_offsets_kernel<<<1, 32, 0, st>>>(strides, offs, H, L);
+    if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
+  }
   // no update at all: the result is the initial iterate h^0 = 0
   if (max_iters == 0 &&
       cudaMemsetAsync(h, 0, sizeof(float) * (size_t)(B * L * 8 * H), st) != cudaSuccess)
@@ -1405,6 +1461,29 @@ extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p
     return PARARNN_ERR_CUDA;
   }
   return PARARNN_OK;
+}
+
+}  // namespace
+}  // namespace pararnn
+
+extern "C" pararnn_status_t pararnn_solve_mhgru(const void* P, pararnn_dtype_t p_dtype,
+                                                const float* U, const float* h0, float* h,
+                                                int64_t B, int64_t L, int64_t H, float tol,
+                                                int32_t max_iters, void* ws, size_t ws_bytes,
+                                                pararnn_solve_info_t* info,
+                                                const pararnn_options_t* opts, void* stream) {
+  return pararnn::mhgru_common(P, p_dtype, U, nullptr, h0, h, B, L, H, tol, max_iters, ws,
+                               ws_bytes, info, opts, stream);
+}
+
+extern "C" pararnn_status_t pararnn_solve_mhgru_strided(
+    const void* P, pararnn_dtype_t p_dtype, const float* U, const int32_t* strides,
+    const float* h0, float* h, int64_t B, int64_t L, int64_t H, float tol, int32_t max_iters,
+    void* ws, size_t ws_bytes, pararnn_solve_info_t* info, const pararnn_options_t* opts,
+    void* stream) {
+  if (!strides && B > 0 && L > 0 && H > 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  return pararnn::mhgru_common(P, p_dtype, U, strides, h0, h, B, L, H, tol, max_iters, ws,
+                               ws_bytes, info, opts, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -25,6 +25,13 @@
 //      first, so no lane reads an overwritten value).
 // The chunk's gates and h^k arrive by cp.async copies into one of two
 // shared-memory buffers while the previous chunk is being processed.
+//
+// Time strides (DEER summary, caveats paragraph: heads with exponentially
+// increasing strides, i.e. shorter effective sequences): head g may recur at
+// stride s_g, h_t = f(h_{t - s_g}, P_t).  Such a head is s_g independent
+// sequences t = r, r + s_g, r + 2 s_g, ... (r < s_g), each solved exactly like a
+// stride-1 sequence; a work unit is then (batch row, head, residue r), and the
+// unit's positions k = 0, 1, ... address time step r + k s_g in memory.
 #pragma once
 
 #include "pararnn_kernel.cuh"
@@ -62,6 +69,9 @@ template <typename PT> __host__ __device__ constexpr size_t mh_smem_bytes() {
 }
 
 struct MhParams {
+  const int* offs;     // NULL (every stride 1) or [H + 2]: offs[g] = sum of the
+                       // heads' strides (each capped at L) before head g,
+                       // offs[H] = their total, offs[H + 1] = 1 if a stride was < 1
   const void* P;       // [B, L, 3, D] (z, r, c), fp32 or bf16; D = 8 H; 16-byte aligned
   const float* U;      // [3, H, 8, 8]: gate, head, row (output), column (input)
   const float* h0;     // [B, D] or NULL (= 0)
@@ -128,25 +138,29 @@ __device__ __forceinline__ void mh_cell(const float* p, const float* U, const fl
 
 // Issue the copies of chunk t0 into one buffer: h^k of steps t0 .. t0 + T - 1
 // into rows 1..T (zeros at k = 0, where h^0 = 0, and past L) and their gates.
+// Positions t0 .. t0 + T - 1 of a unit whose sequence has n positions; position
+// k is time step r + k st in memory (r = 0, st = 1 without strides).
 template <typename PT>
 __device__ __forceinline__ void mh_issue_chunk(const MhParams& p, const PT* P, long long b, int g,
                                                long long D, long long t0, int k, float* hkb,
-                                               PT* spb, int lane) {
+                                               PT* spb, int lane, long long r, long long st,
+                                               long long n) {
   for (int e = lane; e < kMhT * 2; e += 32) {
     const int s = e >> 1, half = e & 1;
     const long long t = t0 + s;
-    const bool valid = k > 0 && t < p.L;
-    const float* src = valid ? p.h + (b * p.L + t) * D + 8 * g + 4 * half : p.h;
+    const bool valid = k > 0 && t < n;
+    const float* src = valid ? p.h + (b * p.L + r + t * st) * D + 8 * g + 4 * half : p.h;
     cp_async16(smem_u32(hkb + 8 + 8 * s + 4 * half), src, valid);
   }
   constexpr int per = 24 * (int)sizeof(PT) / 16;  // 16-byte pieces per step (6 or 3)
   for (int e = lane; e < kMhT * per; e += 32) {
     const int s = e / per, q = e - per * s;
     const long long t = t0 + s;
-    const bool valid = t < p.L;
+    const bool valid = t < n;
     // piece q covers gate (q * 16 / sizeof(PT)) / 8, channels from (q * 16 / sizeof(PT)) % 8
     const int first = q * 16 / (int)sizeof(PT);
-    const PT* src = valid ? P + ((b * p.L + t) * 3 + first / 8) * D + 8 * g + (first % 8) : P;
+    const PT* src =
+        valid ? P + ((b * p.L + r + t * st) * 3 + first / 8) * D + 8 * g + (first % 8) : P;
     cp_async16(smem_u32(spb + 24 * s + first), src, valid);
   }
   cp_async_commit();
@@ -159,7 +173,11 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long D = 8 * p.H;
-  const long long nunits = p.B * p.H;
+  // work units: (batch row, head) sequences, or (batch row, head, residue) with strides
+  const bool strided = p.offs != nullptr;
+  const long long per_row = strided ? (long long)p.offs[p.H] : p.H;
+  const bool bad_strides = strided && p.offs[p.H + 1] != 0;
+  const long long nunits = bad_strides ? 0 : p.B * per_row;
   const WaitCtx wctx{p.ctrl, p.status_dev, p.timeout_ns};
   const PT* P = static_cast<const PT*>(p.P);
   unsigned char* wbase = s_dyn + (size_t)warp * kMhBufs * mh_buf_bytes<PT>();
@@ -176,29 +194,45 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
     float rmax = 0.0f;
     for (long long u = (long long)blockIdx.x * kMhWarps + warp; u < nunits;
          u += (long long)gridDim.x * kMhWarps) {
-      const long long b = u / p.H;
-      const int g = (int)(u - b * p.H);
+      const long long b = u / per_row;
+      const long long rem = u - b * per_row;
+      int g = (int)rem;
+      long long r = 0, st = 1, n = p.L;
+      if (strided) {  // the head whose residues hold rem: the last g with offs[g] <= rem
+        int lo = 0, hi = (int)p.H - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if ((long long)p.offs[mid] <= rem) lo = mid; else hi = mid - 1;
+        }
+        g = lo;
+        st = (long long)p.offs[g + 1] - p.offs[g];
+        r = rem - p.offs[g];
+        n = (p.L - r + st - 1) / st;
+      }
       for (int e = lane; e < 192; e += 32)
         s_U[warp][e] = __ldg(p.U + ((long long)(e >> 6) * p.H + g) * 64 + (e & 63));
       float x[8], hb[8];  // entering the chunk: h^{k+1} and h^k (h0 before the first)
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] = hb[i] = p.h0 ? __ldg(p.h0 + b * D + 8 * g + i) : 0.0f;
       const float* U = s_U[warp];
-      const int nch = (int)((p.L + kMhT - 1) / kMhT);
-      if (kMhBufs == 2) mh_issue_chunk<PT>(p, P, b, g, D, 0, k, hkbuf(0), spbuf(0), lane);
+      const int nch = (int)((n + kMhT - 1) / kMhT);
+      if (kMhBufs == 2)
+        mh_issue_chunk<PT>(p, P, b, g, D, 0, k, hkbuf(0), spbuf(0), lane, r, st, n);
 
       for (int ci = 0; ci < nch; ++ci) {
         const long long t0 = (long long)ci * kMhT;
         const int cur = kMhBufs == 2 ? (ci & 1) : 0;
         float* hk = hkbuf(cur);
         const PT* sp = spbuf(cur);
-        if (kMhBufs == 1) mh_issue_chunk<PT>(p, P, b, g, D, t0, k, hk, spbuf(0), lane);
+        if (kMhBufs == 1)
+          mh_issue_chunk<PT>(p, P, b, g, D, t0, k, hk, spbuf(0), lane, r, st, n);
         cp_async_wait_all();
         __syncwarp();
         if (lane < 8) hk[lane] = hb[lane];  // row 0: h^k of the step before the chunk
         __syncwarp();
         if (kMhBufs == 2 && ci + 1 < nch)
-          mh_issue_chunk<PT>(p, P, b, g, D, t0 + kMhT, k, hkbuf(cur ^ 1), spbuf(cur ^ 1), lane);
+          mh_issue_chunk<PT>(p, P, b, g, D, t0 + kMhT, k, hkbuf(cur ^ 1), spbuf(cur ^ 1), lane,
+                             r, st, n);
 
         // ---- A: linearise this lane's steps, compose their maps ------------------
         const int s0 = lane * kMhS;
@@ -211,7 +245,7 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
         }
         for (int s = 0; s < kMhS; ++s) {
           const long long t = t0 + s0 + s;
-          if (t >= p.L) break;
+          if (t >= n) break;
           float hp[8], hc[8], pg[24], f[8], J[8][8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -280,7 +314,7 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
           // ---- C: recompute and apply this lane's steps, write h^{k+1} ----------
           for (int s = 0; s < kMhS; ++s) {
             const long long t = t0 + s0 + s;
-            if (t >= p.L) break;
+            if (t >= n) break;
             float hp[8], pg[24], f[8], J[8][8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) hp[i] = hk[(s0 + s) * 8 + i];
@@ -295,7 +329,7 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
               for (int j = 0; j < 8; ++j) s2 = fmaf(J[i][j], xin[j] - hp[j], s2);
               y[i] = s2;
             }
-            float4* dst = reinterpret_cast<float4*>(p.h + (b * p.L + t) * D + 8 * g);
+            float4* dst = reinterpret_cast<float4*>(p.h + (b * p.L + r + t * st) * D + 8 * g);
             dst[0] = make_float4(y[0], y[1], y[2], y[3]);
             dst[1] = make_float4(y[4], y[5], y[6], y[7]);
 #pragma unroll
@@ -335,6 +369,7 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
     Info* info = reinterpret_cast<Info*>(p.info);
     __threadfence();
     unsigned status = ld_volatile(&p.ctrl->status);
+    if (bad_strides) status = 1u;  // PARARNN_ERR_INVALID_ARGUMENT: a stride below 1
     int iters = last, conv = 0, nonfinite = 0;
     float maxres = 0.0f;
     for (int kk = 0; kk <= p.max_iters; ++kk) {

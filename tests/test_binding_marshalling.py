@@ -83,6 +83,9 @@ def test_every_entry_point_reaches_its_c_function(fake):
         ("pararnn_solve_lstm", lambda: pr.solve_lstm(z(B, L, 4, D), z(4, D), z(B, D), z(B, D))),
         ("pararnn_solve_gru_noalloc", lambda: pr.solve_gru_noalloc(z(B, L, 3, D), z(3, D))),
         ("pararnn_solve_mhgru", lambda: pr.solve_mhgru(z(B, L, 3, D), z(3, D // 8, 8, 8))),
+        ("pararnn_solve_mhgru_strided",
+         lambda: pr.solve_mhgru_strided(z(B, L, 3, D), z(3, D // 8, 8, 8),
+                                        z(D // 8, dtype=torch.int32))),
         ("pararnn_solve_gru_backward",
          lambda: pr.solve_gru_backward(z(B, L, 3, D), z(3, D), z(B, L, D), z(B, L, D), z(B, D),
                                        status=status_t())),

@@ -128,3 +128,79 @@ def test_mhgru_full_size_every_head(pr):
     assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
     orc = oracle.newton_mhgru(x["P"], x["U"])
     assert orc.converged and abs(info.iterations - orc.iterations) <= 1
+
+
+# --------------------------------------------------------------------------
+# Per-head time strides (DEER summary, caveats: heads with exponentially
+# increasing strides): head g recurs on h_{t - s_g}
+# --------------------------------------------------------------------------
+def sdev(strides):
+    return torch.from_numpy(np.ascontiguousarray(strides, dtype=np.int32)).cuda()
+
+
+# (B, L, strides): exponentially increasing strides; strides past the sequence
+# end; stride 1 everywhere (= the unstrided solve); a long sequence whose
+# residue sequences span several chunks; more units than one CTA holds
+STRIDED = [(2, 300, [1, 2, 4, 8]), (1, 50, [1, 64, 3]), (2, 400, [1, 1, 1]),
+           (1, 4000, [1, 2, 4, 8, 16, 32, 64, 128]), (4, 257, [1, 3, 5, 7, 2])]
+
+
+@pytest.mark.parametrize("h0_normal", [False, True])
+@pytest.mark.parametrize("B,L,strides", STRIDED)
+def test_mhgru_strided_matches_oracle(pr, B, L, strides, h0_normal):
+    H = len(strides)
+    x = inputs.mhgru_inputs(B, L, H, seed=[810, B, L, H], h0_normal=h0_normal)
+    h0 = dev(x["h0"]) if h0_normal else None
+    h, info = pr.solve_mhgru_strided(dev(x["P"]), dev(x["U"]), sdev(strides), h0)
+    torch.cuda.synchronize()
+    st = np.asarray(strides, np.int32)
+    ref = oracle.rollout_mhgru(x["P"], x["U"], x["h0"], strides=st)
+    res = oracle.newton_mhgru(x["P"], x["U"], x["h0"], strides=st)
+    assert info.status == 0 and info.converged
+    assert abs(info.iterations - res.iterations) <= 1
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
+
+
+def test_mhgru_strided_all_ones_is_the_unstrided_solve(pr):
+    x = inputs.mhgru_inputs(2, 700, 4, seed=811, h0_normal=True)
+    P, U, h0 = dev(x["P"]), dev(x["U"]), dev(x["h0"])
+    h1, i1 = pr.solve_mhgru(P, U, h0)
+    h2, i2 = pr.solve_mhgru_strided(P, U, sdev([1, 1, 1, 1]), h0)
+    torch.cuda.synchronize()
+    assert i1.iterations == i2.iterations
+    assert float(torch.max(torch.abs(h1 - h2)).item()) == 0.0
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_mhgru_strided_unconverged_iterate(pr, k):
+    B, L, strides = 2, 200, [1, 4, 9]
+    x = inputs.mhgru_inputs(B, L, len(strides), seed=812, h0_normal=True)
+    st = np.asarray(strides, np.int32)
+    h, info = pr.solve_mhgru_strided(dev(x["P"]), dev(x["U"]), sdev(st), dev(x["h0"]), tol=0.0,
+                                     max_iters=k)
+    torch.cuda.synchronize()
+    res = oracle.newton_mhgru(x["P"], x["U"], x["h0"], tol=0.0, max_iters=k, strides=st)
+    assert info.status == 0 and not info.converged and info.iterations == k
+    assert np.max(np.abs(h.cpu().numpy() - res.h)) <= 1e-4
+
+
+def test_mhgru_stride_below_one_is_reported(pr):
+    x = inputs.mhgru_inputs(1, 50, 3, seed=813)
+    h, info = pr.solve_mhgru_strided(dev(x["P"]), dev(x["U"]), sdev([1, 0, 2]))
+    torch.cuda.synchronize()
+    assert info.status == 1 and not info.converged
+
+
+def test_mhgru_strided_full_size_exponential_strides(pr):
+    """The multi-head workload's full size (B = 8, L = 4096, 128 heads) with
+    strides 2^(g mod 8): every sequence against the oracle's strided rollout."""
+    w = inputs.WORKLOADS["mhgru"]
+    B, L, D = w["B"], w["L"], w["D"]
+    H = D // 8
+    x = inputs.mhgru_inputs(B, L, H, seed=w["seed"])
+    st = (2 ** (np.arange(H) % 8)).astype(np.int32)
+    h, info = pr.solve_mhgru_strided(dev(x["P"]), dev(x["U"]), sdev(st))
+    torch.cuda.synchronize()
+    assert info.converged
+    ref = oracle.rollout_mhgru(x["P"], x["U"], strides=st)
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
