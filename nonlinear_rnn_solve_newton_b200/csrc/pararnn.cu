@@ -18,6 +18,7 @@
 #include "pararnn_bwd_walk.cuh"
 #include "pararnn_kernel.cuh"
 #include "pararnn_mhgru.cuh"
+#include "pararnn_mhgru2.cuh"
 #include "pararnn_probe.cuh"
 #include "pararnn_proj.cuh"
 #include "pararnn_projsolve.cuh"
@@ -1414,11 +1415,20 @@ pararnn_status_t mhgru_common(const void* P, pararnn_dtype_t p_dtype, const floa
       strides ? PARARNN_OP_MHGRU_STRIDED : PARARNN_OP_MHGRU, B, L, 8 * H, max_iters, opts);
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return PARARNN_ERR_WORKSPACE;
 
-  const void* fn = p_dtype == PARARNN_BF16
-                       ? (const void*)pararnn_mhgru_kernel<__nv_bfloat16>
-                       : (const void*)pararnn_mhgru_kernel<float>;
-  const size_t kMhSmem = p_dtype == PARARNN_BF16 ? mh_smem_bytes<__nv_bfloat16>()
-                                                 : mh_smem_bytes<float>();
+  // Layout: 8 lanes per head and time segment, a CTA per sequence (default), or
+  // one lane per segment holding whole 8x8 maps, a warp per sequence (regime 1).
+  const bool lane_maps = opts && opts->regime == 1;
+  const bool bf = p_dtype == PARARNN_BF16;
+  const void* fn =
+      lane_maps ? (bf ? (const void*)pararnn_mhgru_kernel<__nv_bfloat16>
+                      : (const void*)pararnn_mhgru_kernel<float>)
+                : (bf ? (const void*)pararnn_mhgru2_kernel<__nv_bfloat16>
+                      : (const void*)pararnn_mhgru2_kernel<float>);
+  const size_t kMhSmem =
+      lane_maps ? (bf ? mh_smem_bytes<__nv_bfloat16>() : mh_smem_bytes<float>())
+                : (bf ? sizeof(Mh2Smem<__nv_bfloat16>) : sizeof(Mh2Smem<float>));
+  const int mh_threads = lane_maps ? 32 * kMhWarps : kMh2Threads;
+  const int units_per_cta = lane_maps ? kMhWarps : 1;
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
@@ -1430,13 +1440,13 @@ pararnn_status_t mhgru_common(const void* P, pararnn_dtype_t p_dtype, const floa
     return PARARNN_ERR_CUDA;
   }
   int resident = 0;
-  if (resident_ctas(fn, 32 * kMhWarps, kMhSmem, &resident) != cudaSuccess || resident <= 0) {
+  if (resident_ctas(fn, mh_threads, kMhSmem, &resident) != cudaSuccess || resident <= 0) {
     cudaGetLastError();
     return PARARNN_ERR_CUDA;
   }
   // with strides the unit count is known on the device only: every resident CTA runs
   const long long units = B * H;
-  const long long want = (units + kMhWarps - 1) / kMhWarps;
+  const long long want = (units + units_per_cta - 1) / units_per_cta;
   const int grid = strides ? resident : (int)(want < resident ? want : resident);
 
   MhParams mp;
@@ -1467,7 +1477,7 @@ pararnn_status_t mhgru_common(const void* P, pararnn_dtype_t p_dtype, const floa
       cudaMemsetAsync(h, 0, sizeof(float) * (size_t)(B * L * 8 * H), st) != cudaSuccess)
     return PARARNN_ERR_CUDA;
   void* args[] = {&mp};
-  if (cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(32 * kMhWarps), args, kMhSmem, st) !=
+  if (cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(mh_threads), args, kMhSmem, st) !=
       cudaSuccess) {
     cudaGetLastError();
     return PARARNN_ERR_CUDA;

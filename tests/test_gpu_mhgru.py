@@ -35,12 +35,19 @@ def dev(x):
 SHAPES = [(2, 100, 2), (1, 513, 3), (2, 1500, 4), (3, 37, 1), (2, 1, 2), (4, 300, 9)]
 
 
+# the two layouts: 8 lanes per head and time segment (default), one lane per
+# segment holding whole 8x8 maps (regime 1)
+LAYOUTS = [0, 1]
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
 @pytest.mark.parametrize("h0_normal", [False, True])
 @pytest.mark.parametrize("shape", SHAPES)
-def test_mhgru_matches_rollout(pr, shape, h0_normal):
+def test_mhgru_matches_rollout(pr, shape, h0_normal, layout):
     B, L, H = shape
     x = inputs.mhgru_inputs(B, L, H, seed=[800, B, L, H], h0_normal=h0_normal)
-    h, info = pr.solve_mhgru(dev(x["P"]), dev(x["U"]), dev(x["h0"]) if h0_normal else None)
+    h, info = pr.solve_mhgru(dev(x["P"]), dev(x["U"]), dev(x["h0"]) if h0_normal else None,
+                             opts=pr.Options(regime=layout))
     torch.cuda.synchronize()
     ref = oracle.rollout_mhgru(x["P"], x["U"], x["h0"])
     res = oracle.newton_mhgru(x["P"], x["U"], x["h0"])
@@ -145,13 +152,15 @@ STRIDED = [(2, 300, [1, 2, 4, 8]), (1, 50, [1, 64, 3]), (2, 400, [1, 1, 1]),
            (1, 4000, [1, 2, 4, 8, 16, 32, 64, 128]), (4, 257, [1, 3, 5, 7, 2])]
 
 
+@pytest.mark.parametrize("layout", LAYOUTS)
 @pytest.mark.parametrize("h0_normal", [False, True])
 @pytest.mark.parametrize("B,L,strides", STRIDED)
-def test_mhgru_strided_matches_oracle(pr, B, L, strides, h0_normal):
+def test_mhgru_strided_matches_oracle(pr, B, L, strides, h0_normal, layout):
     H = len(strides)
     x = inputs.mhgru_inputs(B, L, H, seed=[810, B, L, H], h0_normal=h0_normal)
     h0 = dev(x["h0"]) if h0_normal else None
-    h, info = pr.solve_mhgru_strided(dev(x["P"]), dev(x["U"]), sdev(strides), h0)
+    h, info = pr.solve_mhgru_strided(dev(x["P"]), dev(x["U"]), sdev(strides), h0,
+                                     opts=pr.Options(regime=layout))
     torch.cuda.synchronize()
     st = np.asarray(strides, np.int32)
     ref = oracle.rollout_mhgru(x["P"], x["U"], x["h0"], strides=st)
