@@ -111,7 +111,10 @@ typedef struct {
  *                 the call must then report PARARNN_ERR_DEVICE_TIMEOUT
  *                 (look-back regime only).  It exists so that the test suite
  *                 can check the bounded waits without faulting a GPU.
- *  regime      : how the time chunks of a channel tile are chained.
+ *  regime      : how the time chunks of a channel tile are chained.  (For the
+ *                multi-head solves: 1 = one lane per time segment holding
+ *                whole 8x8 maps, 2 = 8 lanes per head and segment, 0 = the
+ *                first without strides, the second with them.)
  *                0 = automatic; 1 = look-back (chunks of a tile on different
  *                CTAs, chained through global memory); 2 = walk (one CTA walks
  *                a tile's chunks in order, no traffic between CTAs).  Both give
