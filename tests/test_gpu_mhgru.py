@@ -170,14 +170,20 @@ def test_mhgru_strided_matches_oracle(pr, B, L, strides, h0_normal, layout):
     assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
 
 
-def test_mhgru_strided_all_ones_is_the_unstrided_solve(pr):
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_mhgru_strided_all_ones_is_the_unstrided_solve(pr, layout):
+    """Within one layout, strides of 1 give the unstrided solve bit for bit; the
+    automatic choice (which differs with and without strides) agrees to rounding."""
     x = inputs.mhgru_inputs(2, 700, 4, seed=811, h0_normal=True)
     P, U, h0 = dev(x["P"]), dev(x["U"]), dev(x["h0"])
-    h1, i1 = pr.solve_mhgru(P, U, h0)
-    h2, i2 = pr.solve_mhgru_strided(P, U, sdev([1, 1, 1, 1]), h0)
+    o = pr.Options(regime=layout)
+    h1, i1 = pr.solve_mhgru(P, U, h0, opts=o)
+    h2, i2 = pr.solve_mhgru_strided(P, U, sdev([1, 1, 1, 1]), h0, opts=o)
+    h3, i3 = pr.solve_mhgru_strided(P, U, sdev([1, 1, 1, 1]), h0)
     torch.cuda.synchronize()
-    assert i1.iterations == i2.iterations
+    assert i1.iterations == i2.iterations == i3.iterations
     assert float(torch.max(torch.abs(h1 - h2)).item()) == 0.0
+    assert float(torch.max(torch.abs(h1 - h3)).item()) <= 1e-5
 
 
 @pytest.mark.parametrize("k", [1, 2])

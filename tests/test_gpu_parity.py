@@ -409,3 +409,58 @@ def test_solve_replays_from_a_cuda_graph(pr):
         ref = oracle.rollout_gru(x["P"], x["a"])
         assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
         assert pr.SolveInfo(info_t).converged
+
+
+# --------------------------------------------------------------------------
+# The GRU walker with two channels per thread (packed fp32x2 arithmetic), used
+# on 32-channel tiles with 8-warp CTAs when D is even: bf16 and fp32 gates, an
+# unconverged iterate, agreement with the one-channel-per-thread walker (forced
+# by 16-warp CTAs), and an odd D (which takes the one-channel walker).
+# --------------------------------------------------------------------------
+PAIR_SHAPES = [(4, 1000, 128), (2, 333, 64), (1, 2100, 36)]
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+@pytest.mark.parametrize("shape", PAIR_SHAPES)
+def test_walk_pairs_gru(pr, shape, bf16):
+    B, L, D = shape
+    x = inputs.gru_inputs(B, L, D, seed=[520, B, L, D], bf16=bf16, h0_normal=True)
+    P = (torch.from_numpy(x["P_bits"].view(np.int16)).cuda().view(torch.bfloat16) if bf16
+         else dev(x["P"]))
+    o = pr.Options(regime=2, walk_width=32)
+    h, info = pr.solve_gru(P, dev(x["a"]), dev(x["h0"]), opts=o)
+    h1, info1 = pr.solve_gru(P, dev(x["a"]), dev(x["h0"]),
+                             opts=pr.Options(regime=2, walk_width=32, walk_warps=16))
+    torch.cuda.synchronize()
+    ref = oracle.rollout_gru(x["P"], x["a"], x["h0"])
+    assert info.status == 0 and info.converged
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
+    orc = oracle.newton_gru(x["P"], x["a"], x["h0"], tol=1e-4, max_iters=32)
+    assert abs(info.iterations - orc.iterations) <= 1
+    assert info1.converged and info1.iterations == info.iterations
+    assert float(torch.max(torch.abs(h - h1)).item()) <= 1e-5
+
+
+def test_walk_pairs_unconverged_iterate(pr):
+    """tol = 0, max_iters = 3, two iterations per sweep: h^3 of the serial Newton."""
+    B, L, D = 2, 900, 64
+    x = inputs.gru_inputs(B, L, D, seed=521, h0_normal=True)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), dev(x["h0"]), tol=0.0, max_iters=3,
+                           opts=pr.Options(regime=2, walk_width=32, iters_first=2,
+                                           iters_next=1))
+    torch.cuda.synchronize()
+    orc = oracle.newton_gru(x["P"], x["a"], x["h0"], tol=0.0, max_iters=3)
+    assert not info.converged and info.iterations == 3 and info.updates == 3
+    assert np.max(np.abs(h.cpu().numpy() - orc.h)) <= 1e-5
+    np.testing.assert_allclose(info.rho[:4], orc.rho, rtol=1e-4, atol=1e-6)
+
+
+def test_walk_pairs_odd_width_falls_back(pr):
+    B, L, D = 2, 777, 33
+    x = inputs.gru_inputs(B, L, D, seed=522, h0_normal=True)
+    h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), dev(x["h0"]),
+                           opts=pr.Options(regime=2, walk_width=32))
+    torch.cuda.synchronize()
+    assert info.converged
+    ref = oracle.rollout_gru(x["P"], x["a"], x["h0"])
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= SOLVE_ATOL
