@@ -24,7 +24,6 @@
 #include "pararnn_projsolve.cuh"
 #include "pararnn_seq.cuh"
 #include "pararnn_walk.cuh"
-#include "pararnn_walk2.cuh"
 
 namespace pararnn {
 namespace {
@@ -147,28 +146,6 @@ constexpr int kNarrowSteps = PARARNN_NARROW_STEPS;
 #ifndef PARARNN_NARROW_MINB_LSTM
 #define PARARNN_NARROW_MINB_LSTM 2
 #endif
-// The GRU solve's 32-channel walker with two channels per thread in packed fp32x2
-// arithmetic (pararnn_walk2.cuh): steps per segment (odd, so that the warp's two
-// segments read different shared-memory banks) and the resident-CTA target.
-#ifndef PARARNN_PAIR_STEPS
-#define PARARNN_PAIR_STEPS 7
-#endif
-#ifndef PARARNN_PAIR_MINB
-#define PARARNN_PAIR_MINB 3
-#endif
-#ifndef PARARNN_PAIR_WALK
-#define PARARNN_PAIR_WALK 1
-#endif
-constexpr int kPairSteps = PARARNN_PAIR_STEPS;
-// The same on 8-channel tiles: 4 warps, a warp = 4 channel pairs x 8 segments.
-#ifndef PARARNN_PAIR8_STEPS
-#define PARARNN_PAIR8_STEPS 7
-#endif
-#ifndef PARARNN_PAIR8_MINB
-#define PARARNN_PAIR8_MINB 4
-#endif
-constexpr int kPair8Steps = PARARNN_PAIR8_STEPS;
-static_assert(4 * 8 * kPair8Steps <= 256, "TMA box rows");
 constexpr int kNarrowMinBlocksGru = PARARNN_NARROW_MINB_GRU;
 constexpr int kNarrowMinBlocksGruBf16 = PARARNN_NARROW_MINB_GRU_BF16;
 constexpr int kNarrowMinBlocksLstm = PARARNN_NARROW_MINB_LSTM;
@@ -479,15 +456,6 @@ size_t walk_smem_bytes() {
   return 2 * (size_t)((b + 1023u) / 1024u * 1024u) + 1024;  // + alignment slack
 }
 
-// The paired GRU walker: 8 warps x 2 segments x kPairSteps steps per chunk on
-// 32-channel tiles, 4 warps x 8 segments x kPair8Steps on 8-channel tiles.
-template <typename PT, int CW = 32>
-size_t pair_walk_smem_bytes() {
-  constexpr unsigned b = CW == 32 ? Stage<kGru, PT, 8 * 2 * kPairSteps, 32>::kBytes
-                                  : Stage<kGru, PT, 4 * 8 * kPair8Steps, 8>::kBytes;
-  return 2 * (size_t)((b + 1023u) / 1024u * 1024u) + 1024;  // + alignment slack
-}
-
 // Warps per CTA of the walker: 8, or 16 when the tiles are too few to fill the
 // SMs with 8-warp CTAs (more warps per tile then hide more latency).
 template <int OP, typename PT, int S, int MINB>
@@ -678,49 +646,15 @@ pararnn_status_t launch(const Plan& pl, KParams& kp, bool bf16, void* ws, size_t
   kp.stall_unit = opts ? opts->debug_stall_unit : -1;
 
   // The TMA tile walker when the tiles are 32 wide and TMA's rules hold;
-  // otherwise the general kernel (look-back or register-staged walk).  The GRU
-  // solve on 32-channel tiles takes two channels per thread (packed fp32x2) when
-  // D is even and the state arrays are 8-byte aligned.
+  // otherwise the general kernel (look-back or register-staged walk).
   TmaMaps tm;
-  const bool pair_ok = PARARNN_PAIR_WALK && pl.op == kGru && pl.walk && pl.CW == 32 &&
-                       pl.S_walk > 0 && kp.D % 2 == 0 && aligned(kp.out0, 8) &&
-                       (!kp.x0a || aligned(kp.x0a, 8));
-  const bool pairs = pair_ok && pl.CW_walk == 32 && pl.NW_walk == 8;
-  const bool pairs8 = pair_ok && pl.CW_walk == 8;
-  const int tch_w = pairs    ? 8 * 2 * kPairSteps
-                    : pairs8 ? 4 * 8 * kPair8Steps
-                             : pl.NW_walk * (32 / pl.CW_walk) * pl.S_walk;  // steps per chunk
+  const int tch_w = pl.NW_walk * (32 / pl.CW_walk) * pl.S_walk;  // steps per walker chunk
   const bool tma_walk = pl.walk && pl.CW == 32 && pl.S_walk > 0 &&
                         make_walk_maps(pl.op, bf16, kp, tch_w, pl.CW_walk, &tm);
   const void* fn;
   size_t dyn_smem = 0;
   int threads = kThreads;
-  if (tma_walk && pairs) {
-    if (bf16) {
-      fn = (const void*)pararnn_walk_gru2_kernel<__nv_bfloat16, kPairSteps, 8, PARARNN_PAIR_MINB>;
-      dyn_smem = pair_walk_smem_bytes<__nv_bfloat16>();
-    } else {
-      fn = (const void*)pararnn_walk_gru2_kernel<float, kPairSteps, 8, PARARNN_PAIR_MINB>;
-      dyn_smem = pair_walk_smem_bytes<float>();
-    }
-    kp.nchunks = (int)((kp.L + tch_w - 1) / tch_w);
-    kp.ntd = (int)((kp.D + 31) / 32);
-    kp.ntiles = (int)(kp.B * kp.ntd);
-    threads = 32 * 8;
-  } else if (tma_walk && pairs8) {
-    if (bf16) {
-      fn = (const void*)
-          pararnn_walk_gru2_kernel<__nv_bfloat16, kPair8Steps, 4, PARARNN_PAIR8_MINB, 8>;
-      dyn_smem = pair_walk_smem_bytes<__nv_bfloat16, 8>();
-    } else {
-      fn = (const void*)pararnn_walk_gru2_kernel<float, kPair8Steps, 4, PARARNN_PAIR8_MINB, 8>;
-      dyn_smem = pair_walk_smem_bytes<float, 8>();
-    }
-    kp.nchunks = (int)((kp.L + tch_w - 1) / tch_w);
-    kp.ntd = (int)((kp.D + 7) / 8);
-    kp.ntiles = (int)(kp.B * kp.ntd);
-    threads = 32 * 4;
-  } else if (tma_walk) {
+  if (tma_walk) {
     fn = select_walk_kernel(pl.op, bf16, pl.NW_walk, pl.CW_walk, &dyn_smem);
     kp.nchunks = (int)((kp.L + tch_w - 1) / tch_w);
     kp.ntd = (int)((kp.D + pl.CW_walk - 1) / pl.CW_walk);

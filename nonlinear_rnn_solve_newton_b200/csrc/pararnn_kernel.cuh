@@ -858,11 +858,6 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
   constexpr int NSEG = kThreads / CW;
   constexpr int TCH = NSEG * S;  // steps per chunk
   constexpr int WM = WALK ? kMaxWalkIters : 1;
-  // Above 16 steps per thread the inputs are not held in registers across the
-  // sweep's iterations: each iteration loads a step's inputs where it uses them
-  // (L1/L2-resident after the first), which leaves the registers to the iterate
-  // and the step maps.
-  constexpr bool kReload = S > 16;
 
   __shared__ Map<NS> s_wagg[kWarps][CW];
   __shared__ Vec<NS> s_carry[CW];
@@ -929,9 +924,8 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
         // (D == 1 and aligned: the S steps are one contiguous block)
         bool blk = false;
         if constexpr (CW == 1) blk = p.vec1 && cvalid && t0 + S <= p.L;
-        float vin[kReload ? 1 : S][NI];
-        if constexpr (kReload) {
-        } else if (blk) {
+        float vin[S][NI];
+        if (blk) {
           if constexpr (CW == 1) Block1<OP, PT, S>::load_in(p, b, t0, vin);
         } else {
 #pragma unroll
@@ -1010,19 +1004,11 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
           for (int s = 0; s < S; ++s) {
             const bool v = cvalid && (t0 + s) < p.L;
             if (v) {
-              float vr[NI];
-              const float* vs = vr;
-              if constexpr (kReload) {
-                const long long t = t0 + s;
-                IO<OP, PT>::load_in(p, (b * p.L + t) * p.D + d, b, t, d, vr);
-              } else {
-                vs = vin[s];
-              }
               if constexpr (NEWTON) {
-                mp[s] = newton_step<OP>(vs, wv, xp, x[s], rmax);
+                mp[s] = newton_step<OP>(vin[s], wv, xp, x[s], rmax);
                 xp = x[s];
               } else {
-                mp[s] = StepMap<OP>::from_inputs(vs);
+                mp[s] = StepMap<OP>::from_inputs(vin[s]);
               }
             } else {
               mp[s] = map_identity<NS>();

@@ -412,17 +412,16 @@ def test_solve_replays_from_a_cuda_graph(pr):
 
 
 # --------------------------------------------------------------------------
-# The GRU walker with two channels per thread (packed fp32x2 arithmetic), used
-# on 32-channel tiles with 8-warp CTAs when D is even: bf16 and fp32 gates, an
-# unconverged iterate, agreement with the one-channel-per-thread walker (forced
-# by 16-warp CTAs), and an odd D (which takes the one-channel walker).
+# The GRU walker on 32-channel tiles: bf16 and fp32 gates, an unconverged
+# iterate, agreement between 8- and 16-warp CTAs (different chunk splits, the
+# same answer to rounding), and an odd D.
 # --------------------------------------------------------------------------
-PAIR_SHAPES = [(4, 1000, 128), (2, 333, 64), (1, 2100, 36)]
+WALK32_SHAPES = [(4, 1000, 128), (2, 333, 64), (1, 2100, 36)]
 
 
 @pytest.mark.parametrize("bf16", [False, True])
-@pytest.mark.parametrize("shape", PAIR_SHAPES)
-def test_walk_pairs_gru(pr, shape, bf16):
+@pytest.mark.parametrize("shape", WALK32_SHAPES)
+def test_walk32_gru(pr, shape, bf16):
     B, L, D = shape
     x = inputs.gru_inputs(B, L, D, seed=[520, B, L, D], bf16=bf16, h0_normal=True)
     P = (torch.from_numpy(x["P_bits"].view(np.int16)).cuda().view(torch.bfloat16) if bf16
@@ -441,7 +440,7 @@ def test_walk_pairs_gru(pr, shape, bf16):
     assert float(torch.max(torch.abs(h - h1)).item()) <= 1e-5
 
 
-def test_walk_pairs_unconverged_iterate(pr):
+def test_walk32_unconverged_iterate(pr):
     """tol = 0, max_iters = 3, two iterations per sweep: h^3 of the serial Newton."""
     B, L, D = 2, 900, 64
     x = inputs.gru_inputs(B, L, D, seed=521, h0_normal=True)
@@ -455,7 +454,7 @@ def test_walk_pairs_unconverged_iterate(pr):
     np.testing.assert_allclose(info.rho[:4], orc.rho, rtol=1e-4, atol=1e-6)
 
 
-def test_walk_pairs_odd_width_falls_back(pr):
+def test_walk32_odd_width(pr):
     B, L, D = 2, 777, 33
     x = inputs.gru_inputs(B, L, D, seed=522, h0_normal=True)
     h, info = pr.solve_gru(dev(x["P"]), dev(x["a"]), dev(x["h0"]),
