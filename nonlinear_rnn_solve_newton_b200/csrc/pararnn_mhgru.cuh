@@ -57,12 +57,57 @@ namespace pararnn {
 constexpr int kMhS = PARARNN_MH_STEPS;      // steps per lane per chunk
 constexpr int kMhWarps = PARARNN_MH_WARPS;  // sequences (warps) per CTA
 constexpr int kMhT = 32 * kMhS;             // steps per chunk
-constexpr int kMhHkFloats = (kMhT + 1) * 8;  // h^k of a chunk: row 0 = the step before it
 constexpr int kMhBufs = PARARNN_MH_ASYNC ? 2 : 1;
+
+// Staged rows are grouped by lane (a lane's S consecutive steps), with 16 bytes
+// of padding after each lane's block.  Lanes read their own rows at the same
+// time; without the pad the lane blocks would sit 48 (h^k) or 144 (gates) words
+// apart, always on the same two banks (a 16-way conflict).  With it a 16-byte
+// read by 8 lanes hits 8 different bank groups.
+constexpr int kMhHkLane = kMhS * 8 + 4;          // floats per lane block of h^k rows
+template <typename PT> __host__ __device__ constexpr int mh_gate_lane() {
+  return kMhS * 24 + 16 / (int)sizeof(PT);      // elements per lane block of gate rows
+}
+constexpr int kMhHkFloats = 8 + 32 * kMhHkLane;  // + the step before the chunk (first 8)
+// h^k row of chunk position t (-1 = the step before the chunk); gate row of t
+__host__ __device__ constexpr int mh_hk(int t) {
+  return t < 0 ? 0 : 8 + (t / kMhS) * kMhHkLane + (t % kMhS) * 8;
+}
+template <typename PT> __host__ __device__ constexpr int mh_gate(int t) {
+  return (t / kMhS) * mh_gate_lane<PT>() + (t % kMhS) * 24;
+}
+static_assert((kMhHkFloats * 4) % 16 == 0 && (kMhHkLane * 4) % 16 == 0, "16-byte rows");
 
 // Dynamic shared memory per warp: one or two buffers of (h^k rows, gates of the chunk).
 template <typename PT> __host__ __device__ constexpr size_t mh_buf_bytes() {
-  return (size_t)kMhHkFloats * 4 + (size_t)kMhT * 24 * sizeof(PT);
+  return (size_t)kMhHkFloats * 4 + (size_t)32 * mh_gate_lane<PT>() * sizeof(PT);
+}
+
+// 8 h^k values and 24 gate values of one step as 16-byte shared-memory reads.
+__device__ __forceinline__ void mh_ld8(const float* src, float* v) {
+  const float4 a = reinterpret_cast<const float4*>(src)[0];
+  const float4 c = reinterpret_cast<const float4*>(src)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+}
+__device__ __forceinline__ void mh_ld_gates(const float* src, float* v) {
+#pragma unroll
+  for (int q = 0; q < 6; ++q) {
+    const float4 a = reinterpret_cast<const float4*>(src)[q];
+    v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+  }
+}
+__device__ __forceinline__ void mh_ld_gates(const __nv_bfloat16* src, float* v) {
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    const uint4 a = reinterpret_cast<const uint4*>(src)[q];
+    const unsigned w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * q + 2 * e] = __uint_as_float(w[e] << 16);
+      v[8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+  }
 }
 template <typename PT> __host__ __device__ constexpr size_t mh_smem_bytes() {
   return (size_t)kMhWarps * kMhBufs * mh_buf_bytes<PT>();
@@ -150,7 +195,7 @@ __device__ __forceinline__ void mh_issue_chunk(const MhParams& p, const PT* P, l
     const long long t = t0 + s;
     const bool valid = k > 0 && t < n;
     const float* src = valid ? p.h + (b * p.L + r + t * st) * D + 8 * g + 4 * half : p.h;
-    cp_async16(smem_u32(hkb + 8 + 8 * s + 4 * half), src, valid);
+    cp_async16(smem_u32(hkb + mh_hk(s) + 4 * half), src, valid);
   }
   constexpr int per = 24 * (int)sizeof(PT) / 16;  // 16-byte pieces per step (6 or 3)
   for (int e = lane; e < kMhT * per; e += 32) {
@@ -161,7 +206,7 @@ __device__ __forceinline__ void mh_issue_chunk(const MhParams& p, const PT* P, l
     const int first = q * 16 / (int)sizeof(PT);
     const PT* src =
         valid ? P + ((b * p.L + r + t * st) * 3 + first / 8) * D + 8 * g + (first % 8) : P;
-    cp_async16(smem_u32(spb + 24 * s + first), src, valid);
+    cp_async16(smem_u32(spb + mh_gate<PT>(s) + first), src, valid);
   }
   cp_async_commit();
 }
@@ -247,13 +292,9 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
           const long long t = t0 + s0 + s;
           if (t >= n) break;
           float hp[8], hc[8], pg[24], f[8], J[8][8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            hp[i] = hk[(s0 + s) * 8 + i];
-            hc[i] = hk[(s0 + s + 1) * 8 + i];
-          }
-#pragma unroll
-          for (int i = 0; i < 24; ++i) pg[i] = to_f(sp[24 * (s0 + s) + i]);
+          mh_ld8(hk + mh_hk(s0 + s - 1), hp);
+          mh_ld8(hk + mh_hk(s0 + s), hc);
+          mh_ld_gates(sp + mh_gate<PT>(s0 + s), pg);
           mh_cell(pg, U, hp, f, J);
           float bt[8];
 #pragma unroll
@@ -316,10 +357,8 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
             const long long t = t0 + s0 + s;
             if (t >= n) break;
             float hp[8], pg[24], f[8], J[8][8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) hp[i] = hk[(s0 + s) * 8 + i];
-#pragma unroll
-            for (int i = 0; i < 24; ++i) pg[i] = to_f(sp[24 * (s0 + s) + i]);
+            mh_ld8(hk + mh_hk(s0 + s - 1), hp);
+            mh_ld_gates(sp + mh_gate<PT>(s0 + s), pg);
             mh_cell(pg, U, hp, f, J);
             float y[8];
 #pragma unroll
@@ -340,7 +379,7 @@ __global__ void __launch_bounds__(32 * kMhWarps, 1) pararnn_mhgru_kernel(const M
           for (int i = 0; i < 8; ++i) x[i] = __shfl_sync(0xffffffffu, xin[i], 31);
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) hb[i] = hk[kMhT * 8 + i];
+        for (int i = 0; i < 8; ++i) hb[i] = hk[mh_hk(kMhT - 1) + i];
         __syncwarp();  // the buffer is refilled by a later chunk
       }
       cp_async_wait_all();
