@@ -122,7 +122,7 @@ typedef struct {
  *                iterations are evaluated per sweep.
  *  walk_warps  : warps per CTA in the walk regime with 32-channel tiles:
  *                0 = automatic (16 for the diagonal scan below 512 tiles,
- *                else 8), 8 or 16.
+ *                else 8), 4, 8 or 16.
  *  walk_width  : channels per tile of the walk regime's tensor-copy walker for
  *                the GRU / LSTM solves: 0 = automatic (8 when 32-channel tiles
  *                would be fewer than 4 per SM and L >= 2048 -- finer tiles

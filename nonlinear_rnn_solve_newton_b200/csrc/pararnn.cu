@@ -272,7 +272,7 @@ Plan make_plan(int op, long long B, long long L, long long D, int max_iters,
     // 16-warp CTAs only help the diagonal scan when tiles are few (measured on
     // B200); the solves and the 2x2 scan keep 8 warps.
     const bool wide = op == kScanDiag && ntiles < kWalkWideTiles;
-    pl.NW_walk = (want == 8 || want == 16) ? want : (wide ? 16 : 8);
+    pl.NW_walk = (want == 4 || want == 8 || want == 16) ? want : (wide ? 16 : 8);
     // Tile width: 32-channel tiles leave the SMs unevenly loaded when there are
     // few of them per SM (256 tiles on 148 SMs: 108 SMs hold two, 40 hold one);
     // 8-channel tiles (a warp = 8 channels x 4 segments) cut the tail to < 2%.
@@ -463,6 +463,10 @@ const void* walk_kernel_nw(int nw, size_t* smem) {
   if (nw == 16) {
     *smem = walk_smem_bytes<OP, PT, S, 16>();
     return (const void*)pararnn_walk_kernel<OP, PT, S, 16, (MINB + 1) / 2>;
+  }
+  if (nw == 4) {
+    *smem = walk_smem_bytes<OP, PT, S, 4>();
+    return (const void*)pararnn_walk_kernel<OP, PT, S, 4, 2 * MINB>;
   }
   *smem = walk_smem_bytes<OP, PT, S, 8>();
   return (const void*)pararnn_walk_kernel<OP, PT, S, 8, MINB>;
