@@ -74,8 +74,8 @@ template <> struct OpT<kLstm> {
 // Workspace control block (zeroed by the host before each launch).
 // ---------------------------------------------------------------------------
 struct Ctrl {
-  unsigned bar_count;
-  unsigned bar_gen;
+  unsigned bar_count;  // grid-barrier arrivals (only grows: (g + 1) x grid after barrier g)
+  unsigned bar_gen;    // grid barriers completed
   unsigned abort;
   unsigned status;
   unsigned pad[12];
@@ -492,25 +492,42 @@ __device__ __forceinline__ bool window_lookback(const unsigned long long* rec_ba
   }
 }
 
-// Grid-wide barrier (all CTAs are co-resident: cooperative launch).  Bounded;
-// returns false if the kernel is aborting.
+// Global stop rule after a sweep of m iterations from k0: stop at the first
+// iterate whose residual is within tol, on a non-finite residual, or once the
+// iteration limit is reached.  The m loads are independent.
+__device__ __forceinline__ int sweep_stops(const unsigned* rho_bits, int k0, int m, int max_iters,
+                                           float tol) {
+  int done = k0 + m > max_iters ? 1 : 0;
+  for (int kk = 0; kk < m; ++kk) {
+    const float r = __uint_as_float(ld_volatile(&rho_bits[k0 + kk]));
+    if (!(r <= 3.0e38f) || r <= tol) done = 1;
+  }
+  return done;
+}
+
+// Grid-wide barrier (all CTAs are co-resident: cooperative launch).  The
+// arrival counter only grows: every CTA arrives once per barrier and none can
+// arrive at the next one before this one completes, so an arrival's count tells
+// which barrier it belongs to (count / gridDim.x) and the last arrival of
+// barrier g releases it by publishing g + 1.  Nothing is read before arriving
+// and nothing is reset, so a barrier costs one atomic round trip plus the
+// release.  Bounded; returns false if the kernel is aborting or the wait ran
+// out.  The signature stays one small struct: the callers' hot loops compile as
+// if the call were not there.
 __device__ __noinline__ bool grid_barrier(WaitCtx p) {
   __shared__ int s_ok;
-  __threadfence();
+  __threadfence();  // every thread: its iterate and residuals before the CTA arrives
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    unsigned gen = ld_acquire(&p.ctrl->bar_gen);
-    __threadfence();
-    unsigned arrived = atomicAdd(&p.ctrl->bar_count, 1u);
-    if (arrived == gridDim.x - 1) {
-      atomicExch(&p.ctrl->bar_count, 0u);
-      __threadfence();
-      st_release(&p.ctrl->bar_gen, gen + 1u);
+    const unsigned arrived = atomicAdd(&p.ctrl->bar_count, 1u);
+    const unsigned next = arrived / gridDim.x + 1u;
+    if (arrived == next * gridDim.x - 1u) {
+      st_release(&p.ctrl->bar_gen, next);
     } else {
-      unsigned long long t0 = globaltimer();
+      const unsigned long long t0 = globaltimer();
       unsigned ns = 32;
-      while (ld_acquire(&p.ctrl->bar_gen) == gen) {
+      while (ld_acquire(&p.ctrl->bar_gen) < next) {
         if (ld_volatile(&p.ctrl->abort) != 0u) {
           ok = 0;
           break;
@@ -521,14 +538,60 @@ __device__ __noinline__ bool grid_barrier(WaitCtx p) {
           break;
         }
         __nanosleep(ns);
-        if (ns < 1024) ns <<= 1;
+        if (ns < 256) ns <<= 1;
       }
     }
-    if (ld_volatile(&p.ctrl->abort) != 0u) ok = 0;
     s_ok = ok;
   }
   __syncthreads();
   return s_ok != 0;
+}
+
+// The solve's report (pararnn_solve_info_t), written by one thread once every
+// CTA has finished: residuals rho_0..rho_last (zero after), the iteration count
+// (the first iterate within tol, or the first non-finite residual, else the
+// last evaluated), convergence and status.  `extra_status` replaces a zero
+// status (e.g. a wait that ran out in this thread's own CTA).
+__device__ __noinline__ void write_solve_info(void* info_ptr, Ctrl* ctrl,
+                                                 const unsigned* rho_bits, int last, int passes,
+                                                 int max_iters, float tol, unsigned extra_status) {
+  struct Info {
+    int iterations, converged, status, updates, passes, reserved;
+    float max_residual;
+    float rho[128];
+  };
+  Info* info = reinterpret_cast<Info*>(info_ptr);
+  __threadfence();
+  unsigned status = ld_volatile(&ctrl->status);
+  if (status == 0u) status = extra_status;
+  int iters = max_iters, conv = 0, nonfinite = 0;
+  bool found = false;
+  float maxres = 0.0f;
+  for (int k = 0; k <= max_iters; ++k) {
+    const float r = k <= last ? __uint_as_float(ld_volatile(&rho_bits[k])) : 0.0f;
+    info->rho[k] = r;
+    if (k > last) continue;
+    const bool bad = !(r <= 3.0e38f);
+    if (bad) nonfinite = 1;
+    if (!found) {
+      iters = k;
+      maxres = r;
+      if (bad) {
+        found = true;
+      } else if (r <= tol) {
+        conv = 1;
+        found = true;
+      }
+    }
+  }
+  if (status == 0u && nonfinite) status = 5u;
+  info->iterations = iters;
+  info->converged = (status == 0u) ? conv : 0;
+  info->status = (int)status;
+  info->updates = last < max_iters ? last + 1 : max_iters;
+  info->passes = passes;
+  info->reserved = 0;
+  info->max_residual = maxres;
 }
 
 // Iterations evaluated in sweep q that starts at iteration k0.
@@ -881,7 +944,6 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
   int q = 0;
   if (tid == 0) {
     s_abort = 0;
-    s_done = 0;
   }
   __syncthreads();
 
@@ -1161,25 +1223,13 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
     if constexpr (!NEWTON) {
       break;
     } else {
+      // every CTA takes the same decision from the same global residuals
       if (!grid_barrier(wctx)) {
         if (tid == 0) s_abort = 1;
         __syncthreads();
         break;
       }
-      // every CTA takes the same decision from the same global residuals
-      if (tid == 0) {
-        int done = 0;
-        for (int kk = 0; kk < m; ++kk) {
-          float r = __uint_as_float(ld_volatile(&p.rho_bits[k0 + kk]));
-          if (!(r <= 3.0e38f)) {  // NaN or Inf
-            done = 1;
-            break;
-          }
-          if (r <= p.tol) done = 1;
-        }
-        if (k0 + m > p.max_iters) done = 1;
-        s_done = done;
-      }
+      if (tid == 0) s_done = sweep_stops(p.rho_bits, k0, m, p.max_iters, p.tol);
       __syncthreads();
       if (s_done) break;
       k0 += m;
@@ -1188,43 +1238,10 @@ __global__ void __launch_bounds__(kThreads, MINB) pararnn_kernel(const KParams p
 
   // ---- report ---------------------------------------------------------------
   if constexpr (NEWTON) {
-    if (blockIdx.x == 0 && tid == 0) {
-      struct Info {
-        int iterations, converged, status, updates, passes, reserved;
-        float max_residual;
-        float rho[128];
-      };
-      Info* info = reinterpret_cast<Info*>(p.info);
-      __threadfence();
-      unsigned status = ld_volatile(&p.ctrl->status);
-      const int last = k0 + sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) - 1;
-      int iters = p.max_iters, conv = 0, nonfinite = 0;
-      float maxres = 0.0f;
-      for (int k = 0; k <= last && k <= p.max_iters; ++k) {
-        float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
-        info->rho[k] = r;
-        if (!(r <= 3.0e38f)) nonfinite = 1;
-      }
-      for (int k = 0; k <= last && k <= p.max_iters; ++k) {
-        float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
-        iters = k;
-        maxres = r;
-        if (!(r <= 3.0e38f)) break;
-        if (r <= p.tol) {
-          conv = 1;
-          break;
-        }
-      }
-      for (int k = last + 1; k <= p.max_iters; ++k) info->rho[k] = 0.0f;
-      if (status == 0u && nonfinite) status = 5u;
-      info->iterations = iters;
-      info->converged = (status == 0u) ? conv : 0;
-      info->status = (int)status;
-      info->updates = last < p.max_iters ? last + 1 : p.max_iters;
-      info->passes = q + 1;
-      info->reserved = 0;
-      info->max_residual = maxres;
-    }
+    if (blockIdx.x == 0 && tid == 0)
+      write_solve_info(p.info, p.ctrl, p.rho_bits,
+                       k0 + sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) - 1, q + 1,
+                       p.max_iters, p.tol, 0u);
   }
   // scans: a device-side error was written to status_dev by raise_error()
 }

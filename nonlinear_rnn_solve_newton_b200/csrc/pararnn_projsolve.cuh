@@ -6,20 +6,24 @@
 // only diagonal weights in the recurrence (TL;DR, Abstract).  Run as two calls,
 // the projection writes P [B, L, 3, D] to HBM and the Newton solve reads it
 // back.  Here a CTA owns a work item = (batch row b, 32 consecutive channels)
-// and walks its time chunks of 128 steps in order:
+// and walks its time chunks of 128 steps in order.  Items are numbered channel
+// group first (item = g B + b), so the CTAs running at once are the batch rows
+// of a few channel groups: they share those groups' rows of W in L2, and x is
+// streamed once per wave of items:
 //   * warp 0, one thread: TMA copies of each chunk's 64-deep k-blocks of x
 //     (rows b*L + t0 .. + 127) and of the item's W rows -- the z, r and c
 //     blocks of its 32 channels, one 3-D box -- into a ring of stages;
 //   * warp 1, one thread: tcgen05.mma with M = 128 steps, N = 96 (3 gates x 32
 //     channels), bf16 operands, fp32 accumulation, into one of two TMEM
 //     accumulators;
-//   * warps 2-9 (the walker): read the chunk's accumulator (a thread = one time
-//     step), add the bias and lay the chunk out in shared memory as
+//   * the walker warps (16 by default, warps 2-17): read the chunk's accumulator
+//     (a thread = one time step, a warp = a quarter of the steps x a share of the
+//     96 columns), add the bias and lay the chunk out in shared memory as
 //     [step][gate][channel] fp32, free the accumulator, and run the sweep's m
 //     Newton iterations on the chunk exactly as the tensor-copy walker does
-//     (a thread = one channel x 16 steps: cell, Jacobian and residual, serial
-//     composition, cross-warp combine, the carry of the previous chunk at the
-//     same iteration kept in shared memory).
+//     (a thread = one channel x 128 / warps steps: cell, Jacobian and residual,
+//     serial composition, cross-warp combine, the carry of the previous chunk at
+//     the same iteration kept in shared memory).
 // The MMAs of chunk j + 1 run on the tensor cores while the walker iterates on
 // chunk j on the CUDA cores.  A later sweep -- needed only when the first sweep's
 // m iterations do not converge -- recomputes the projection.  Every wait is
@@ -39,9 +43,16 @@ namespace pararnn {
 constexpr int kPsCW = 32;                         // channels per work item
 constexpr int kPsN = 3 * kPsCW;                   // accumulator columns: gates z, r, c
 constexpr int kPsBM = 128;                        // time steps per chunk (TMEM lanes)
-constexpr int kPsWalkWarps = 8;                   // walker warps = time segments
+#ifndef PARARNN_PS_WALK_WARPS
+#define PARARNN_PS_WALK_WARPS 16
+#endif
+constexpr int kPsWalkWarps = PARARNN_PS_WALK_WARPS;  // walker warps = time segments
 constexpr int kPsS = kPsBM / kPsWalkWarps;        // steps per walker thread
 constexpr int kPsThreads = 32 * (2 + kPsWalkWarps);
+constexpr int kPsParts = kPsWalkWarps / 4;        // walker warps per TMEM lane quarter
+constexpr int kPsCols = kPsN / kPsParts;          // accumulator columns one walker warp drains
+static_assert(kPsWalkWarps == 8 || kPsWalkWarps == 16, "walker warps");
+static_assert(kPsCols % 8 == 0, "columns are drained 8 at a time");
 constexpr unsigned kPsABytes = kPsBM * kProjBK * 2;         // x k-block: 128 rows x 128 B
 constexpr unsigned kPsBBytes = kPsN * kProjBK * 2;          // W k-block: 96 rows x 128 B
 constexpr unsigned kPsStageBytes = kPsABytes + kPsBBytes;   // 28 KB, a multiple of 1024
@@ -92,9 +103,9 @@ __device__ __forceinline__ void tma_load_3d_s(unsigned dst, const CUtensorMap* m
       : "memory");
 }
 
-// Named barrier of the 8 walker warps (barrier 0 stays __syncthreads).
+// Named barrier of the walker warps (barrier 0 stays __syncthreads).
 __device__ __forceinline__ void ps_walker_sync() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kPsWalkWarps) : "memory");
 }
 // The same barrier, returning whether `ok` held for every walker thread.
 __device__ __forceinline__ bool ps_walker_all(bool ok) {
@@ -102,10 +113,10 @@ __device__ __forceinline__ bool ps_walker_all(bool ok) {
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 256, p;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(ok ? 1u : 0u)
+      : "r"(ok ? 1u : 0u), "n"(32 * kPsWalkWarps)
       : "memory");
   return r != 0u;
 }
@@ -178,8 +189,8 @@ __global__ void __launch_bounds__(kPsThreads, 1)
       if (lane == 0) {
         // ---- producer: x and W k-blocks of every chunk of every item ------------
         for (int it = blockIdx.x; it < p.nitems; it += gridDim.x) {
-          const long long b = it / p.ntd;
-          const int g = it - (int)b * p.ntd;
+          const int g = it / (int)p.B;
+          const long long b = it - (long long)g * p.B;
           for (int j = 0; j < p.nchunks; ++j) {
             const int row = (int)(b * p.L) + j * kPsBM;
             for (int kb = 0; kb < nk; ++kb, ++pit) {
@@ -235,15 +246,15 @@ __global__ void __launch_bounds__(kPsThreads, 1)
         s_mma_uses = mit;
       }
     } else {
-      // ---- the walker (warps 2-9) -----------------------------------------------------
-      const int tw = threadIdx.x - 64;  // 0 .. 255
+      // ---- the walker (warps 2 .. 1 + kPsWalkWarps) ------------------------------------
+      const int tw = threadIdx.x - 64;  // 0 .. 32 kPsWalkWarps - 1
       const int ww = warp - 2;          // time segment of the chunk
       const int c = lane;               // channel within the item
       const int quarter = warp & 3;     // the TMEM lanes (time steps) this warp may read
-      const int half = ww >> 2;         // its 48 of the 96 accumulator columns
+      const int part = ww >> 2;         // its kPsCols of the 96 accumulator columns
       for (int it = blockIdx.x; it < p.nitems && !aborted; it += gridDim.x) {
-        const long long b = it / p.ntd;
-        const int g = it - (int)b * p.ntd;
+        const int g = it / (int)p.B;
+        const long long b = it - (long long)g * p.B;
         const long long d = (long long)g * CW + c;
         const bool cvalid = d < p.D;
         const long long bd = b * p.D + d;
@@ -276,26 +287,21 @@ __global__ void __launch_bounds__(kPsThreads, 1)
           ++wlt;
           tc_fence_after();
           {
-            const unsigned taddr =
-                tmem + acc * kPsAccCols + ((unsigned)(32 * quarter) << 16) + 48u * half;
-            unsigned r[48];
-#define PARARNN_PS_LD16(OFF, R)                                                                 \
-  asm volatile(                                                                                 \
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "   \
-      "%11, %12, %13, %14, %15}, [%16];"                                                        \
-      : "=r"(R[0]), "=r"(R[1]), "=r"(R[2]), "=r"(R[3]), "=r"(R[4]), "=r"(R[5]), "=r"(R[6]),     \
-        "=r"(R[7]), "=r"(R[8]), "=r"(R[9]), "=r"(R[10]), "=r"(R[11]), "=r"(R[12]), "=r"(R[13]), \
-        "=r"(R[14]), "=r"(R[15])                                                                \
-      : "r"(taddr + (OFF)))
-            PARARNN_PS_LD16(0u, (r + 0));
-            PARARNN_PS_LD16(16u, (r + 16));
-            PARARNN_PS_LD16(32u, (r + 32));
-#undef PARARNN_PS_LD16
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            float* dst = Ps + (32 * quarter + lane) * kPsRow + 48 * half;
-            const float* bsrc = s_bias + 48 * half;
+            const unsigned taddr = tmem + acc * kPsAccCols + ((unsigned)(32 * quarter) << 16) +
+                                   (unsigned)(kPsCols * part);
+            unsigned r[kPsCols];
 #pragma unroll
-            for (int i = 0; i < 48; i += 4) {
+            for (int i = 0; i < kPsCols; i += 8)
+              asm volatile(
+                  "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                  : "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]),
+                    "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+                  : "r"(taddr + (unsigned)i));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            float* dst = Ps + (32 * quarter + lane) * kPsRow + kPsCols * part;
+            const float* bsrc = s_bias + kPsCols * part;
+#pragma unroll
+            for (int i = 0; i < kPsCols; i += 4) {
               const float4 bb = *reinterpret_cast<const float4*>(bsrc + i);
               *reinterpret_cast<float4*>(dst + i) =
                   make_float4(__uint_as_float(r[i]) + bb.x, __uint_as_float(r[i + 1]) + bb.y,
@@ -408,19 +414,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
       aborted = true;
       break;
     }
-    if (threadIdx.x == 0) {
-      int done = 0;
-      for (int kk = 0; kk < m; ++kk) {
-        const float r = __uint_as_float(ld_volatile(&p.rho_bits[k0 + kk]));
-        if (!(r <= 3.0e38f)) {
-          done = 1;
-          break;
-        }
-        if (r <= p.tol) done = 1;
-      }
-      if (k0 + m > p.max_iters) done = 1;
-      s_flag = done;
-    }
+    if (threadIdx.x == 0) s_flag = sweep_stops(p.rho_bits, k0, m, p.max_iters, p.tol);
     __syncthreads();
     if (s_flag) break;
     k0 += m;
@@ -449,44 +443,10 @@ __global__ void __launch_bounds__(kPsThreads, 1)
                  : "memory");
   }
 
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    struct Info {
-      int iterations, converged, status, updates, passes, reserved;
-      float max_residual;
-      float rho[128];
-    };
-    Info* info = reinterpret_cast<Info*>(p.info);
-    __threadfence();
-    unsigned status = ld_volatile(&p.ctrl->status);
-    if (status == 0u && aborted) status = 4u;
-    const int last = k0 + sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) - 1;
-    int iters = p.max_iters, conv = 0, nonfinite = 0;
-    float maxres = 0.0f;
-    for (int k = 0; k <= last && k <= p.max_iters; ++k) {
-      const float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
-      info->rho[k] = r;
-      if (!(r <= 3.0e38f)) nonfinite = 1;
-    }
-    for (int k = 0; k <= last && k <= p.max_iters; ++k) {
-      const float r = __uint_as_float(ld_volatile(&p.rho_bits[k]));
-      iters = k;
-      maxres = r;
-      if (!(r <= 3.0e38f)) break;
-      if (r <= p.tol) {
-        conv = 1;
-        break;
-      }
-    }
-    for (int k = last + 1; k <= p.max_iters; ++k) info->rho[k] = 0.0f;
-    if (status == 0u && nonfinite) status = 5u;
-    info->iterations = iters;
-    info->converged = (status == 0u) ? conv : 0;
-    info->status = (int)status;
-    info->updates = last < p.max_iters ? last + 1 : p.max_iters;
-    info->passes = q + 1;
-    info->reserved = 0;
-    info->max_residual = maxres;
-  }
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    write_solve_info(p.info, p.ctrl, p.rho_bits,
+                     k0 + sweep_len(q, k0, p.m_first, p.m_next, p.max_iters) - 1, q + 1,
+                     p.max_iters, p.tol, aborted ? 4u : 0u);
 }
 
 }  // namespace pararnn
