@@ -289,7 +289,13 @@ def recorded_traffic(workload):
     # each capture carries the digest of the sources it was taken on
     if k.get("source_sha256", rec.get("source_sha256")) != kernel_source_digest():
         return None, "kernels changed since the capture"
-    return int(k["dram_bytes_per_launch"]), "ncu " + k.get("capture", "")
+    # a capture of a shorter sequence, scaled to the full launch by the
+    # channel-steps it processes (the walker's traffic grows with L)
+    scale = float(k.get("scale", 1))
+    src = "ncu " + k.get("capture", "")
+    if scale != 1:
+        src += f", x {scale:g} to the full length"
+    return int(round(k["dram_bytes_per_launch"] * scale)), src
 
 
 # ---------------------------------------------------------------------------

@@ -35,6 +35,28 @@ def test_traffic_record_is_tied_to_kernel_sources():
     assert traffic is None
 
 
+def test_traffic_record_scaling(tmp_path, monkeypatch):
+    """A capture of a shorter sequence is scaled to the full launch; a record
+    taken on other sources is refused."""
+    import json
+
+    (tmp_path / "profiles").mkdir()
+    digest = bench.kernel_source_digest()
+    rec = {"kernels": {
+        "short": {"dram_bytes_per_launch": 1000, "scale": 8, "capture": "L=1024",
+                  "source_sha256": digest},
+        "full": {"dram_bytes_per_launch": 1234, "capture": "full", "source_sha256": digest},
+        "stale": {"dram_bytes_per_launch": 1, "source_sha256": "0" * 64}}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda: digest)
+    t, src = bench.recorded_traffic("short")
+    assert t == 8000 and "x 8" in src
+    assert bench.recorded_traffic("full")[0] == 1234
+    t, why = bench.recorded_traffic("stale")
+    assert t is None and "changed" in why
+
+
 def test_backward_and_projection_bytes():
     N = 8 * 4096 * 1024
     # backward: read P, the trajectory one step behind and dl/dh (and dl/dc); write dP
