@@ -768,6 +768,28 @@ def run_ours(args, world, rank, local):
     # application: one launch per time step.  Also timed: the one-thread-per-
     # channel rollout, whose time is L x the cell's dependency chain.)
     sequential = None
+    if op == "mhgru" and not args.no_sequential:
+        # the multi-head cell applied in order (8 lanes per head): the DEER
+        # summary's caveat is that dense blocks make each Newton step O(n^3)
+        try:
+            d = cs.dev
+            hroll = torch.empty((B, L, D), dtype=torch.float32, device=device)
+            for _ in range(2):
+                pr.rollout_mhgru(d["P"], d["U"], out=hroll)
+            torch.cuda.synchronize()
+            qev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            Kq = max(1, min(K, 5))
+            qev[0].record(stream)
+            for _ in range(Kq):
+                pr.rollout_mhgru(d["P"], d["U"], out=hroll)
+            qev[1].record(stream)
+            torch.cuda.synchronize()
+            roll_ms = qev[0].elapsed_time(qev[1]) / Kq
+            sequential = {"rollout_8_lanes_per_head_ms": roll_ms,
+                          "newton_speedup_vs_rollout": roll_ms / ms}
+            del hroll
+        except Exception as e:  # context only; never fails the benchmark
+            sequential = {"error": str(e)[:200]}
     if op in ("gru", "lstm") and not args.no_sequential:
         try:
             seq_fn = pr.rollout_gru if op == "gru" else pr.rollout_lstm

@@ -295,6 +295,29 @@ pararnn_status_t pararnn_solve_mhgru_strided(const void* P, pararnn_dtype_t p_dt
                                              size_t ws_bytes, pararnn_solve_info_t* info,
                                              const pararnn_options_t* opts, void* stream);
 
+/* Sequential application of the multi-head GRU on the GPU: each (batch row,
+ * head) sequence walks t = 1..L in order, 8 lanes per sequence (lane i =
+ * channel i of the head, the head's state exchanged by shuffles each step).
+ * The baseline the Newton solve of the same system is compared with (the DEER
+ * summary's caveat: dense blocks make each Newton step O(n^3) per step, while
+ * the sequential cell is O(n^2)).  Arguments and layouts as pararnn_solve_mhgru
+ * (every head at stride 1) without tol, max_iters, workspace or info; P needs
+ * only its element alignment.  Requires 8 B H <= 2^31.  Errors:
+ * PARARNN_ERR_INVALID_ARGUMENT (bad sizes, dtype, NULL or misaligned
+ * pointers), PARARNN_ERR_CUDA (launch failure).  B, L or H = 0: no work. */
+pararnn_status_t pararnn_rollout_mhgru(const void* P, pararnn_dtype_t p_dtype, const float* U,
+                                       const float* h0, float* h, int64_t B, int64_t L,
+                                       int64_t H, void* stream);
+
+/* One multi-head GRU step for every (batch row, head): h_next = f(h_prev, P),
+ * the decode step of the multi-head cell.  P : [B, 3, D] (z, r, c) for one time
+ * step, fp32 or bf16, D = 8 H; U : [3, H, 8, 8]; h_prev : [B, D] or NULL (= 0);
+ * h_next : [B, D] (must not overlap h_prev).  Errors as pararnn_rollout_mhgru
+ * (it is that call with L = 1). */
+pararnn_status_t pararnn_step_mhgru(const void* P, pararnn_dtype_t p_dtype, const float* U,
+                                    const float* h_prev, float* h_next, int64_t B, int64_t H,
+                                    void* stream);
+
 /* Input projection P = x W^T + bias on the tensor cores (tcgen05, bf16 inputs,
  * fp32 accumulation): the projected gate pre-activations that the cells take
  * as inputs (ParaRNN TL;DR: the recurrence keeps only diagonal weights, the

@@ -140,6 +140,11 @@ def load(build_if_missing: bool = True):
             lib.pararnn_rollout_lstm.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i64,
                                                  _i64, _i64, _vp]
             lib.pararnn_rollout_lstm.restype = ctypes.c_int
+            lib.pararnn_rollout_mhgru.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64, _i64,
+                                                  _i64, _vp]
+            lib.pararnn_rollout_mhgru.restype = ctypes.c_int
+            lib.pararnn_step_mhgru.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _vp]
+            lib.pararnn_step_mhgru.restype = ctypes.c_int
             lib.pararnn_solve_gru_noalloc.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _i64,
                                                       _i64, _i64, ctypes.c_float, ctypes.c_int32,
                                                       _vp, _vp, _vp]
@@ -667,6 +672,28 @@ def step_gru(P, a, h_prev=None, out=None, stream=None):
     return h
 
 
+def step_mhgru(P, U, h_prev=None, out=None, stream=None):
+    """One multi-head GRU step (decode): P [B, 3, D] (z, r, c), U [3, H, 8, 8],
+    D = 8 H -> h_next [B, D]."""
+    lib = load()
+    B, G, D = P.shape
+    if G != 3 or U.dim() != 4 or tuple(U.shape[2:]) != (8, 8) or D != 8 * U.shape[1]:
+        raise ValueError("P must be [B, 3, 8 H] and U [3, H, 8, 8]")
+    H = U.shape[1]
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, 3, D))
+    _check_dev("U", U, torch.float32, (3, H, 8, 8))
+    _check_dev("h_prev", h_prev, torch.float32, (B, D))
+    h = torch.empty((B, D), dtype=torch.float32, device=P.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, D))
+    dev = _one_device(P=P, U=U, h_prev=h_prev, out=h)
+    with _device_guard(dev):
+        st = lib.pararnn_step_mhgru(_ptr(P), dt, _ptr(U), _ptr(h_prev), _ptr(h), B, H,
+                                    _stream_handle(stream, dev))
+    _raise(st, "pararnn_step_mhgru")
+    return h
+
+
 def input_projection(x, W, bias=None, out=None, out_dtype=torch.float32, status=None,
                      stream=None):
     """P = x W^T + bias on the tensor cores: x [..., K] bf16, W [N, K] bf16,
@@ -744,6 +771,28 @@ def rollout_gru(P, a, h0=None, out=None, stream=None):
         st = lib.pararnn_rollout_gru(_ptr(P), dt, _ptr(a), _ptr(h0), _ptr(h), B, L, D,
                                      _stream_handle(stream, dev))
     _raise(st, "pararnn_rollout_gru")
+    return h
+
+
+def rollout_mhgru(P, U, h0=None, out=None, stream=None):
+    """Sequential multi-head GRU application on the GPU (8 lanes per head
+    sequence).  P [B, L, 3, D] (z, r, c), U [3, H, 8, 8], D = 8 H -> h [B, L, D]."""
+    lib = load()
+    B, L, G, D = P.shape
+    if G != 3 or U.dim() != 4 or tuple(U.shape[2:]) != (8, 8) or D != 8 * U.shape[1]:
+        raise ValueError("P must be [B, L, 3, 8 H] and U [3, H, 8, 8]")
+    H = U.shape[1]
+    dt = _p_dtype(P)
+    _check_dev("P", P, P.dtype, (B, L, 3, D))
+    _check_dev("U", U, torch.float32, (3, H, 8, 8))
+    _check_dev("h0", h0, torch.float32, (B, D))
+    h = torch.empty((B, L, D), dtype=torch.float32, device=P.device) if out is None else out
+    _check_dev("out", h, torch.float32, (B, L, D))
+    dev = _one_device(P=P, U=U, h0=h0, out=h)
+    with _device_guard(dev):
+        st = lib.pararnn_rollout_mhgru(_ptr(P), dt, _ptr(U), _ptr(h0), _ptr(h), B, L, H,
+                                       _stream_handle(stream, dev))
+    _raise(st, "pararnn_rollout_mhgru")
     return h
 
 

@@ -1179,6 +1179,37 @@ extern "C" pararnn_status_t pararnn_rollout_lstm(const void* P, pararnn_dtype_t 
   return seq_common(true, kLstm, P, p_dtype, a, c0, h0, c, h, B, L, D, stream);
 }
 
+extern "C" pararnn_status_t pararnn_rollout_mhgru(const void* P, pararnn_dtype_t p_dtype,
+                                                  const float* U, const float* h0, float* h,
+                                                  int64_t B, int64_t L, int64_t H, void* stream) {
+  using namespace pararnn;
+  if (B < 0 || L < 0 || H < 0) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (p_dtype != PARARNN_F32 && p_dtype != PARARNN_BF16) return PARARNN_ERR_INVALID_ARGUMENT;
+  if (B == 0 || L == 0 || H == 0) return PARARNN_OK;
+  if (!P || !U || !h) return PARARNN_ERR_INVALID_ARGUMENT;
+  const size_t esz = p_dtype == PARARNN_BF16 ? 2 : 4;
+  if (!aligned(P, esz) || !aligned(U, 4) || (h0 && !aligned(h0, 4)) || !aligned(h, 4))
+    return PARARNN_ERR_INVALID_ARGUMENT;
+  if (B * H > (1LL << 31) / 8 || H > (1LL << 27)) return PARARNN_ERR_INVALID_ARGUMENT;
+  MhSeqParams sp = {P, U, h0, h, B, L, H};
+  const int threads = 64;  // 8 sequences per CTA
+  const unsigned blocks = (unsigned)((B * H * 8 + threads - 1) / threads);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p_dtype == PARARNN_BF16)
+    pararnn_rollout_mhgru_kernel<__nv_bfloat16, 8><<<blocks, threads, 0, st>>>(sp);
+  else
+    pararnn_rollout_mhgru_kernel<float, 8><<<blocks, threads, 0, st>>>(sp);
+  return cudaGetLastError() == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+// One decode step of the multi-head GRU is its rollout over one time step.
+extern "C" pararnn_status_t pararnn_step_mhgru(const void* P, pararnn_dtype_t p_dtype,
+                                               const float* U, const float* h_prev,
+                                               float* h_next, int64_t B, int64_t H,
+                                               void* stream) {
+  return pararnn_rollout_mhgru(P, p_dtype, U, h_prev, h_next, B, 1, H, stream);
+}
+
 // ---------------------------------------------------------------------------
 // Input projection P = x W^T + bias (tcgen05 tensor cores).
 // ---------------------------------------------------------------------------

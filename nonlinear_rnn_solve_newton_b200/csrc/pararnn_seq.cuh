@@ -108,4 +108,73 @@ __global__ void __launch_bounds__(128) pararnn_rollout_kernel(const SeqParams p)
   }
 }
 
+// Multi-head GRU (dense 8x8 blocks per head of 8 channels) applied in order:
+// 8 lanes per (batch row, head) sequence, lane i = channel i of the head.  Per
+// step the head's state is gathered from the group by shuffles, lane i forms
+// row i of U_z h, U_r h and U_c h, and
+//   z = sig(P_z + U_z h), r = sig(P_r + U_r h), c = tanh(P_c + r (U_c h)),
+//   h' = (1 - z) h + z c.
+// A ring of the next R steps' inputs stays in flight, as in the rollout above.
+struct MhSeqParams {
+  const void* P;   // [B, L, 3, D], D = 8 H
+  const float* U;  // [3, H, 8, 8]: gate, head, row, column
+  const float* h0; // [B, D] or NULL
+  float* h;        // [B, L, D]
+  long long B, L, H;
+};
+
+template <typename PT, int R>
+__global__ void __launch_bounds__(64) pararnn_rollout_mhgru_kernel(const MhSeqParams p) {
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const long long seq = gid >> 3;  // (batch row, head); the 8 lanes of a group agree
+  if (seq >= p.B * p.H) return;
+  const int i = threadIdx.x & 7;
+  const unsigned gmask = 0xffu << (threadIdx.x & 24);
+  const long long b = seq / p.H, g = seq - b * p.H;
+  const long long D = 8 * p.H;
+  float uz[8], ur[8], uc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uz[j] = __ldg(p.U + ((0 * p.H + g) * 8 + i) * 8 + j);
+    ur[j] = __ldg(p.U + ((1 * p.H + g) * 8 + i) * 8 + j);
+    uc[j] = __ldg(p.U + ((2 * p.H + g) * 8 + i) * 8 + j);
+  }
+  const long long ch = b * D + 8 * g + i;
+  float h = p.h0 ? __ldg(p.h0 + ch) : 0.0f;
+  const PT* P = reinterpret_cast<const PT*>(p.P) + b * p.L * 3 * D + 8 * g + i;
+  const long long step = 3 * D;
+  float* out = p.h + b * p.L * D + 8 * g + i;
+  float ring[R][3];
+#pragma unroll
+  for (int s = 0; s < R; ++s)
+#pragma unroll
+    for (int q = 0; q < 3; ++q) ring[s][q] = s < p.L ? to_f(__ldg(P + s * step + q * D)) : 0.0f;
+  for (long long t0 = 0; t0 < p.L; t0 += R) {
+#pragma unroll
+    for (int s = 0; s < R; ++s) {
+      const long long t = t0 + s;
+      if (t < p.L) {
+        const float pz = ring[s][0], pr = ring[s][1], pc = ring[s][2];
+        if (t + R < p.L) {
+#pragma unroll
+          for (int q = 0; q < 3; ++q) ring[s][q] = to_f(__ldg(P + (t + R) * step + q * D));
+        }
+        float az = pz, ar = pr, ac = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float hj = __shfl_sync(gmask, h, j, 8);
+          az = fmaf(uz[j], hj, az);
+          ar = fmaf(ur[j], hj, ar);
+          ac = fmaf(uc[j], hj, ac);
+        }
+        const float z = sigm(az);
+        const float r = sigm(ar);
+        const float c = tanh_f(fmaf(r, ac, pc));
+        h = fmaf(z, c - h, h);
+        __stcs(out + t * D, h);
+      }
+    }
+  }
+}
+
 }  // namespace pararnn

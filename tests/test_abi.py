@@ -181,6 +181,19 @@ def test_other_entry_points_validate_on_the_host(lib):
     assert lib.pararnn_rollout_gru(fake, 0, fake, vp(4098), fake, 2, 8, 4, None) == 1
     assert lib.pararnn_rollout_gru(fake, 0, fake, None, fake, 2, 0, 4, None) == 0
     assert lib.pararnn_rollout_lstm(fake, 0, fake, None, None, fake, None, 2, 8, 4, None) == 1
+    # multi-head rollout: (P, dtype, U, h0, h, B, L, H, stream)
+    mr = lib.pararnn_rollout_mhgru
+    assert mr(fake, 0, fake, None, fake, -1, 8, 2, None) == 1          # negative size
+    assert mr(fake, 3, fake, None, fake, 2, 8, 2, None) == 1           # unknown dtype
+    assert mr(None, 0, fake, None, fake, 2, 8, 2, None) == 1           # P missing
+    assert mr(fake, 0, None, None, fake, 2, 8, 2, None) == 1           # U missing
+    assert mr(vp(4098), 0, fake, None, fake, 2, 8, 2, None) == 1       # fp32 P misaligned
+    assert mr(fake, 0, fake, vp(4098), fake, 2, 8, 2, None) == 1       # h0 misaligned
+    assert mr(fake, 0, fake, None, fake, 2, 0, 2, None) == 0           # nothing to do
+    sm = lib.pararnn_step_mhgru  # (P, dtype, U, h_prev, h_next, B, H, stream)
+    assert sm(fake, 0, fake, None, fake, -1, 2, None) == 1
+    assert sm(fake, 0, None, None, fake, 2, 2, None) == 1
+    assert sm(fake, 0, fake, None, fake, 0, 2, None) == 0
     # multi-head solve: (P, dtype, U, h0, h, B, L, H, tol, max_iters, ws, ws_bytes, info, opts, s)
     mh = lib.pararnn_solve_mhgru
     assert mh(fake, 0, fake, None, fake, -1, 8, 2, f1e4, 4, ws, 1 << 20, info, None, None) == 1

@@ -97,6 +97,8 @@ def test_every_entry_point_reaches_its_c_function(fake):
         ("pararnn_step_lstm", lambda: pr.step_lstm(z(B, 4, D), z(4, D), z(B, D), z(B, D))),
         ("pararnn_rollout_gru", lambda: pr.rollout_gru(z(B, L, 3, D), z(3, D), z(B, D))),
         ("pararnn_rollout_lstm", lambda: pr.rollout_lstm(z(B, L, 4, D), z(4, D))),
+        ("pararnn_rollout_mhgru", lambda: pr.rollout_mhgru(z(B, L, 3, D), z(3, D // 8, 8, 8))),
+        ("pararnn_step_mhgru", lambda: pr.step_mhgru(z(B, 3, D), z(3, D // 8, 8, 8), z(B, D))),
         ("pararnn_solve_gru_projected",
          lambda: pr.solve_gru_projected(z(B, L, K, dtype=torch.bfloat16),
                                         z(3 * D, K, dtype=torch.bfloat16), z(3 * D), z(3, D),

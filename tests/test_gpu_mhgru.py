@@ -219,3 +219,64 @@ def test_mhgru_strided_full_size_exponential_strides(pr):
     assert info.converged
     ref = oracle.rollout_mhgru(x["P"], x["U"], strides=st)
     assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
+
+
+@pytest.mark.parametrize("shape", [(2, 100, 2), (1, 1, 1), (3, 517, 5), (1, 3000, 16)])
+def test_rollout_mhgru_matches_oracle(pr, shape):
+    """The sequential multi-head application (8 lanes per head) against the
+    oracle's fp64 rollout."""
+    B, L, H = shape
+    x = inputs.mhgru_inputs(B, L, H, seed=[820, B, L, H], h0_normal=True)
+    h = pr.rollout_mhgru(dev(x["P"]), dev(x["U"]), dev(x["h0"]))
+    torch.cuda.synchronize()
+    ref = oracle.rollout_mhgru(x["P"], x["U"], x["h0"])
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
+
+
+def test_rollout_mhgru_bf16_and_zero_state(pr):
+    B, L, H = 2, 700, 3
+    x = inputs.mhgru_inputs(B, L, H, seed=821)
+    bits, vals = inputs.round_to_bf16(x["P"])
+    P16 = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    h = pr.rollout_mhgru(P16, dev(x["U"]))
+    torch.cuda.synchronize()
+    assert np.max(np.abs(h.cpu().numpy() - oracle.rollout_mhgru(vals, x["U"]))) <= 1e-4
+
+
+def test_rollout_mhgru_full_size_equals_newton(pr):
+    """The multi-head workload's full size: every sequence of the rollout against
+    the oracle, and the Newton solve against the rollout."""
+    w = inputs.WORKLOADS["mhgru"]
+    B, L, D = w["B"], w["L"], w["D"]
+    H = D // 8
+    x = inputs.mhgru_inputs(B, L, H, seed=w["seed"])
+    P, U = dev(x["P"]), dev(x["U"])
+    roll = pr.rollout_mhgru(P, U)
+    h, info = pr.solve_mhgru(P, U)
+    torch.cuda.synchronize()
+    assert info.converged
+    ref = oracle.rollout_mhgru(x["P"], x["U"])
+    r = roll.cpu().numpy()
+    assert np.max(np.abs(r - ref)) <= 1e-4
+    assert np.max(np.abs(h.cpu().numpy() - r)) <= 1e-4
+
+
+def test_step_mhgru_matches_oracle_cell_and_rollout(pr):
+    """One decode step per head equals the oracle's cell; L steps equal the rollout."""
+    B, L, H = 3, 40, 5
+    x = inputs.mhgru_inputs(B, L, H, seed=822, h0_normal=True)
+    P, U, h0 = dev(x["P"]), dev(x["U"]), dev(x["h0"])
+    h1 = pr.step_mhgru(P[:, 0].contiguous(), U, h0)
+    torch.cuda.synchronize()
+    for b in range(B):
+        for g in range(H):
+            f, _ = oracle.mhgru_cell(x["P"][b, 0, :, 8 * g:8 * g + 8], x["U"][:, g],
+                                     x["h0"][b, 8 * g:8 * g + 8])
+            assert np.max(np.abs(h1[b, 8 * g:8 * g + 8].cpu().numpy() - f)) <= 2e-6
+    hs, prev = [], h0
+    for t in range(L):
+        prev = pr.step_mhgru(P[:, t].contiguous(), U, prev)
+        hs.append(prev)
+    roll = pr.rollout_mhgru(P, U, h0)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.stack(hs, 1), roll)
