@@ -1121,6 +1121,22 @@ static pararnn_status_t seq_common(bool rollout, int op, const void* P, pararnn_
   if (rollout) {
     const int threads = 128;
     const unsigned blocks = (unsigned)((n + threads - 1) / threads);
+    // inputs staged through shared memory when each warp's channels are one
+    // contiguous row segment (D % 32 == 0) and the rows are 16-byte aligned
+    if (D % 32 == 0 && aligned(P, 16)) {
+      if (op == kGru) {
+        if (bf16)
+          pararnn_rollout_staged_kernel<kGru, __nv_bfloat16, 16><<<blocks, threads, 0, st>>>(sp);
+        else
+          pararnn_rollout_staged_kernel<kGru, float, 16><<<blocks, threads, 0, st>>>(sp);
+      } else {
+        if (bf16)
+          pararnn_rollout_staged_kernel<kLstm, __nv_bfloat16, 8><<<blocks, threads, 0, st>>>(sp);
+        else
+          pararnn_rollout_staged_kernel<kLstm, float, 8><<<blocks, threads, 0, st>>>(sp);
+      }
+      return cudaGetLastError() == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA;
+    }
     if (op == kGru) {
       if (bf16)
         pararnn_rollout_kernel<kGru, __nv_bfloat16, 16><<<blocks, threads, 0, st>>>(sp);
@@ -1195,10 +1211,20 @@ extern "C" pararnn_status_t pararnn_rollout_mhgru(const void* P, pararnn_dtype_t
   const int threads = 64;  // 8 sequences per CTA
   const unsigned blocks = (unsigned)((B * H * 8 + threads - 1) / threads);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (p_dtype == PARARNN_BF16)
-    pararnn_rollout_mhgru_kernel<__nv_bfloat16, 8><<<blocks, threads, 0, st>>>(sp);
-  else
-    pararnn_rollout_mhgru_kernel<float, 8><<<blocks, threads, 0, st>>>(sp);
+  // inputs staged through shared memory when a warp's 4 heads are 32 contiguous
+  // channels of one batch row (H % 4 == 0) and the rows are 16-byte aligned
+  const bool staged = H % 4 == 0 && aligned(P, 16);
+  if (p_dtype == PARARNN_BF16) {
+    if (staged)
+      pararnn_rollout_mhgru_kernel<__nv_bfloat16, 16, true><<<blocks, threads, 0, st>>>(sp);
+    else
+      pararnn_rollout_mhgru_kernel<__nv_bfloat16, 8, false><<<blocks, threads, 0, st>>>(sp);
+  } else {
+    if (staged)
+      pararnn_rollout_mhgru_kernel<float, 16, true><<<blocks, threads, 0, st>>>(sp);
+    else
+      pararnn_rollout_mhgru_kernel<float, 8, false><<<blocks, threads, 0, st>>>(sp);
+  }
   return cudaGetLastError() == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA;
 }
 

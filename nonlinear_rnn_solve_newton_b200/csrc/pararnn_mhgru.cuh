@@ -131,20 +131,6 @@ struct MhParams {
   long long timeout_ns;
 };
 
-// 16-byte asynchronous copy global -> shared; with valid == false it writes
-// zeros and reads nothing.
-__device__ __forceinline__ void cp_async16(unsigned dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-
 // Cell and Jacobian of one head at h (row-major J[i][j] = dh'_i / dh_j).  U is
 // the head's blocks in shared memory (16-byte aligned rows); each row of the
 // three blocks is read once, as float4, for both the product and the Jacobian.

@@ -6,11 +6,17 @@
 //   * the whole rollout with one thread per channel walking t = 1..L in order
 //     -- the "sequential application" the parallel Newton solve is measured
 //     against (ParaRNN abstract; DEER summary), here on the same GPU.
-// The rollout keeps a ring of upcoming steps' inputs in flight (registers) so
-// that memory latency hides behind the per-step dependency chain of the cell.
+// When a warp's 32 threads hold 32 consecutive channels of one batch row (D a
+// multiple of 32), the rollout stages its inputs through shared memory: the
+// warp copies the next R steps' rows of its channels with cp.async into one of
+// two buffers while it applies the cell to the current R steps, and waits for
+// the copy groups one at a time.  Loads kept in registers instead (the
+// fallback for other D) are waited for in batches by the hardware, so in
+// practice each step waits for a memory round trip.
 #pragma once
 
 #include "pararnn_kernel.cuh"
+#include "pararnn_walk.cuh"
 
 namespace pararnn {
 
@@ -108,6 +114,69 @@ __global__ void __launch_bounds__(128) pararnn_rollout_kernel(const SeqParams p)
   }
 }
 
+// One warp's copy of R steps x G gate rows of its 32 channels (one 16-byte
+// chunk per lane and round) into dst[R][G][32]; steps at or past L are zero-filled.
+template <typename PT, int G, int R>
+__device__ __forceinline__ void stage_rows(PT* dst, const PT* src, long long t_first,
+                                           long long L, long long D, int lane) {
+  constexpr int CPR = 32 * (int)sizeof(PT) / 16;  // 16-byte chunks per row
+  constexpr int NCH = R * G * CPR;
+#pragma unroll
+  for (int k = lane; k < NCH; k += 32) {
+    const int s = k / (G * CPR), g = (k / CPR) % G, c = k % CPR;
+    const long long t = t_first + s;
+    const bool valid = t < L;
+    const PT* row = src + ((valid ? t : 0) * G + g) * D;
+    cp_async16(smem_u32(dst + (s * G + g) * 32) + 16u * c,
+               reinterpret_cast<const char*>(row) + 16 * c, valid);
+  }
+  cp_async_commit();
+}
+
+// The rollout above with staged inputs: 4 warps per CTA, each on 32 consecutive
+// channels of one batch row (requires D % 32 == 0 and P 16-byte aligned).
+template <int OP, typename PT, int R>
+__global__ void __launch_bounds__(128) pararnn_rollout_staged_kernel(const SeqParams p) {
+  constexpr int G = OP == kGru ? 3 : 4;
+  __shared__ __align__(16) PT s_in[4][2][R * G * 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= p.B * p.D) return;  // whole warps: B D is a multiple of 32
+  const long long b = i / p.D, d = i - b * p.D;
+  float w[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) w[g] = __ldg(p.w + g * p.D + d);
+  float x[2] = {p.x0a ? p.x0a[i] : 0.0f, 0.0f};
+  if constexpr (OP == kLstm) x[1] = p.x0b ? p.x0b[i] : 0.0f;
+  const PT* P = reinterpret_cast<const PT*>(p.P) + b * p.L * G * p.D + (d - lane);
+  float* o0 = p.out0 + b * p.L * p.D + d;
+  float* o1 = OP == kLstm ? p.out1 + b * p.L * p.D + d : nullptr;
+  PT* buf0 = s_in[warp][0];
+  PT* buf1 = s_in[warp][1];
+  stage_rows<PT, G, R>(buf0, P, 0, p.L, p.D, lane);
+  stage_rows<PT, G, R>(buf1, P, R, p.L, p.D, lane);
+  for (long long t0 = 0, blk = 0; t0 < p.L; t0 += R, ++blk) {
+    PT* buf = (blk & 1) ? buf1 : buf0;
+    cp_async_wait_prior();  // this buffer's group has landed
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < R; ++s) {
+      const long long t = t0 + s;
+      if (t < p.L) {
+        float pin[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) pin[g] = to_f(buf[(s * G + g) * 32 + lane]);
+        cell_apply<OP, PT>(pin, w, x);
+        __stcs(o0 + t * p.D, x[0]);
+        if constexpr (OP == kLstm) __stcs(o1 + t * p.D, x[1]);
+      }
+    }
+    __syncwarp();  // every lane has read this buffer
+    stage_rows<PT, G, R>(buf, P, t0 + 2 * R, p.L, p.D, lane);
+  }
+  cp_async_wait_all();
+}
+
 // Multi-head GRU (dense 8x8 blocks per head of 8 channels) applied in order:
 // 8 lanes per (batch row, head) sequence, lane i = channel i of the head.  Per
 // step the head's state is gathered from the group by shuffles, lane i forms
@@ -123,7 +192,7 @@ struct MhSeqParams {
   long long B, L, H;
 };
 
-template <typename PT, int R>
+template <typename PT, int R, bool STAGED>
 __global__ void __launch_bounds__(64) pararnn_rollout_mhgru_kernel(const MhSeqParams p) {
   const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   const long long seq = gid >> 3;  // (batch row, head); the 8 lanes of a group agree
@@ -144,20 +213,41 @@ __global__ void __launch_bounds__(64) pararnn_rollout_mhgru_kernel(const MhSeqPa
   const PT* P = reinterpret_cast<const PT*>(p.P) + b * p.L * 3 * D + 8 * g + i;
   const long long step = 3 * D;
   float* out = p.h + b * p.L * D + 8 * g + i;
-  float ring[R][3];
+  // staged: this warp's 32 channels (4 heads) through shared memory
+  __shared__ __align__(16) PT s_in[STAGED ? 2 : 1][2][STAGED ? R * 3 * 32 : 1];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const PT* Pw = P - lane;  // staged: the warp's first channel (D % 32 == 0: one batch row)
+  float ring[STAGED ? 1 : R][3];
+  if constexpr (STAGED) {
+    stage_rows<PT, 3, R>(s_in[warp][0], Pw, 0, p.L, D, lane);
+    stage_rows<PT, 3, R>(s_in[warp][1], Pw, R, p.L, D, lane);
+  } else {
 #pragma unroll
-  for (int s = 0; s < R; ++s)
+    for (int s = 0; s < R; ++s)
 #pragma unroll
-    for (int q = 0; q < 3; ++q) ring[s][q] = s < p.L ? to_f(__ldg(P + s * step + q * D)) : 0.0f;
-  for (long long t0 = 0; t0 < p.L; t0 += R) {
+      for (int q = 0; q < 3; ++q) ring[s][q] = s < p.L ? to_f(__ldg(P + s * step + q * D)) : 0.0f;
+  }
+  for (long long t0 = 0, blk = 0; t0 < p.L; t0 += R, ++blk) {
+    PT* buf = s_in[STAGED ? warp : 0][blk & 1];
+    if constexpr (STAGED) {
+      cp_async_wait_prior();
+      __syncwarp();  // every lane's copies of this buffer are visible
+    }
 #pragma unroll
     for (int s = 0; s < R; ++s) {
       const long long t = t0 + s;
       if (t < p.L) {
-        const float pz = ring[s][0], pr = ring[s][1], pc = ring[s][2];
-        if (t + R < p.L) {
+        float pz, pr, pc;
+        if constexpr (STAGED) {
+          pz = to_f(buf[(s * 3 + 0) * 32 + lane]);
+          pr = to_f(buf[(s * 3 + 1) * 32 + lane]);
+          pc = to_f(buf[(s * 3 + 2) * 32 + lane]);
+        } else {
+          pz = ring[s][0], pr = ring[s][1], pc = ring[s][2];
+          if (t + R < p.L) {
 #pragma unroll
-          for (int q = 0; q < 3; ++q) ring[s][q] = to_f(__ldg(P + (t + R) * step + q * D));
+            for (int q = 0; q < 3; ++q) ring[s][q] = to_f(__ldg(P + (t + R) * step + q * D));
+          }
         }
         float az = pz, ar = pr, ac = 0.0f;
 #pragma unroll
@@ -174,7 +264,12 @@ __global__ void __launch_bounds__(64) pararnn_rollout_mhgru_kernel(const MhSeqPa
         __stcs(out + t * D, h);
       }
     }
+    if constexpr (STAGED) {
+      __syncwarp();  // every lane has read this buffer
+      stage_rows<PT, 3, R>(buf, Pw, t0 + 2 * R, p.L, D, lane);
+    }
   }
+  if constexpr (STAGED) cp_async_wait_all();
 }
 
 }  // namespace pararnn

@@ -56,7 +56,7 @@ def test_rollout_gru_matches_oracle(pr, shape):
     assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
 
 
-@pytest.mark.parametrize("shape", [(2, 512, 16), (1, 1, 1), (2, 1200, 33)])
+@pytest.mark.parametrize("shape", [(2, 512, 16), (1, 1, 1), (2, 1200, 33), (2, 700, 64)])
 def test_rollout_lstm_matches_oracle(pr, shape):
     B, L, D = shape
     x = inputs.lstm_inputs(B, L, D, seed=[703, B, L, D], h0_normal=True)
@@ -85,3 +85,21 @@ def test_step_loop_equals_rollout_and_newton(pr):
     loop = hs.permute(1, 0, 2).cpu().numpy()
     assert np.max(np.abs(loop - roll.cpu().numpy())) <= 1e-6
     assert info.converged and np.max(np.abs(newt.cpu().numpy() - loop)) <= 1e-4
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+def test_rollout_bf16_staged_matches_oracle(pr, cell):
+    """bf16 gates with D a multiple of 32 (inputs staged through shared memory)
+    against the oracle's rollout of the rounded gates."""
+    B, L, D = 2, 1000, 96
+    gen = inputs.gru_inputs if cell == "gru" else inputs.lstm_inputs
+    x = gen(B, L, D, seed=[704, B, L, D], bf16=True, h0_normal=True)
+    P16 = torch.from_numpy(x["P_bits"].view(np.int16)).cuda().view(torch.bfloat16)
+    if cell == "gru":
+        h = pr.rollout_gru(P16, dev(x["a"]), dev(x["h0"]))
+        ref = oracle.rollout_gru(x["P"], x["a"], x["h0"])
+    else:
+        _, h = pr.rollout_lstm(P16, dev(x["a"]), dev(x["c0"]), dev(x["h0"]))
+        ref = oracle.rollout_lstm(x["P"], x["a"], x["c0"], x["h0"])[1]
+    torch.cuda.synchronize()
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
