@@ -488,15 +488,17 @@ def time_leg(name, K, W, warm_s, world, rank, device, stream):
     return cs, max_over_ranks(ev[0].elapsed_time(ev[1]) / K, world, device)
 
 
-def scan_summary(sc, ms, world, hbm_peak):
+def scan_summary(sc, ms, world, hbm_peak, peak_kind):
     """The scan leg's line: its 12 algorithmic bytes per channel-step against
-    the measured HBM copy bandwidth and against 8 TB/s."""
+    the HBM copy bandwidth (measured, else the fallback; `hbm_peak_kind` says
+    which) and against 8 TB/s."""
     sbytes = algorithmic_bytes("scan_diag", False, sc.B, sc.L, sc.D)
     sgbs = sbytes / (ms * 1e-3) / 1e9
     st, ssrc = recorded_traffic(sc.name)
     return {"workload": workload_name(sc.name, sc.B, sc.L, sc.D), "ms": ms,
             "channel_steps_per_s": world * sc.N / (ms * 1e-3), "achieved_gbs": sgbs,
-            "algorithmic_bytes": sbytes, "frac_of_measured_hbm": sgbs / hbm_peak,
+            "algorithmic_bytes": sbytes, "frac_of_hbm_peak": sgbs / hbm_peak,
+            "hbm_peak_gbs": hbm_peak, "hbm_peak_kind": peak_kind,
             "frac_of_8tbs": sgbs / 8000.0, "traffic": st, "traffic_source": ssrc}
 
 
@@ -630,7 +632,7 @@ def run_ours(args, world, rank, local):
                "peak_probe": probe, "mufu_ops_per_launch": mufu_ops}
         if alu["frac"] >= hbm_frac:
             roofline = dict(alu)
-            roofline["hbm"] = {k: hbm[k] for k in ("achieved", "peak", "unit", "frac",
+            roofline["hbm"] = {k: hbm[k] for k in ("achieved", "peak", "peak_kind", "unit", "frac",
                                                     "algorithmic_bytes_per_launch")}
         else:
             roofline = dict(hbm)
@@ -649,7 +651,7 @@ def run_ours(args, world, rank, local):
                                   "clock at %.0f MHz, scaled to the timed region's SM clock"
                                   % (probe["per_sm_per_clk"], probe["sm_mhz"])),
                     "peak_probe": probe,
-                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                             "frac": hbm_frac}}
     elif op == "proj_solve":
         ev_iters = evaluated_iterations(passes, cs.max_iters)
@@ -670,7 +672,7 @@ def run_ours(args, world, rank, local):
                             "peak": mufu_peak / 1e12, "unit": "Tops/s (MUFU ex2+rcp)",
                             "frac": mufu_ops / (launch_ms * 1e-3) / mufu_peak,
                             "peak_kind": "measured: ex2+rcp throughput probe"},
-                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                             "frac": hbm_frac, "algorithmic_bytes_per_launch": bytes_launch}}
     elif op == "proj":
         ev_iters = None
@@ -683,7 +685,7 @@ def run_ours(args, world, rank, local):
         roofline = {"bound": "tensor", "achieved": tflops, "peak": tf_peak, "unit": "TFLOP/s",
                     "frac": tflops / tf_peak, "traffic": traffic, "peak_kind": tf_kind,
                     "flops_per_launch": flops,
-                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "hbm": {"achieved": achieved_gbs, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                             "frac": hbm_frac, "algorithmic_bytes_per_launch": bytes_launch}}
     else:
         ev_iters = None
@@ -705,7 +707,7 @@ def run_ours(args, world, rank, local):
     scan_name = SCAN_LEG.get(args.workload)
     if scan_name and not args.no_scan:
         sc, sms = time_leg(scan_name, K, W, args.warmup_seconds, world, rank, device, stream)
-        scan = scan_summary(sc, sms, world, hbm_peak)
+        scan = scan_summary(sc, sms, world, hbm_peak, peak_kind)
         del sc
 
     # ---- the fused layer against the unfused pair (P through HBM) ------------
@@ -760,7 +762,7 @@ def run_ours(args, world, rank, local):
                  "traffic": gtr, "traffic_source": gtsrc}
         del g
         sc, sms = time_leg("scan", K, W, args.warmup_seconds, world, rank, device, stream)
-        extra["scan"] = scan_summary(sc, sms, world, hbm_peak)
+        extra["scan"] = scan_summary(sc, sms, world, hbm_peak, peak_kind)
         del sc
 
     # ---- context: sequential application on the same GPU ---------------------
