@@ -1614,7 +1614,11 @@ namespace {
 #ifndef PARARNN_PS_STAGES
 #define PARARNN_PS_STAGES 5
 #endif
-constexpr int kPsStages = PARARNN_PS_STAGES;
+#ifndef PARARNN_PS_STAGES2
+#define PARARNN_PS_STAGES2 4
+#endif
+constexpr int kPsStages = PARARNN_PS_STAGES;    // one walker group
+constexpr int kPsStages2 = PARARNN_PS_STAGES2;  // two walker groups (two staged chunks)
 
 // W [3 D, K] bf16 viewed as 3 gate blocks of D rows: {K, D, 3}, box {64, 32, 3},
 // 128-byte swizzle (the box lands as 96 consecutive swizzled 128-byte rows).
@@ -1688,13 +1692,17 @@ extern "C" pararnn_status_t pararnn_solve_gru_projected(
   if (B * (long long)pp.ntd >= (1LL << 31) || L / kPsBM >= (1LL << 30))
     return PARARNN_ERR_INVALID_ARGUMENT;
 
-  const void* fn = (const void*)pararnn_projsolve_kernel<kPsStages>;
+  // walker groups: two (two items per CTA at once) unless opts->regime = 1;
+  // measured on B200 two were faster at every K from 256 to 4096
+  const bool two = !(opts && opts->regime == 1);
+  const void* fn = two ? (const void*)pararnn_projsolve_kernel<kPsStages2, 2>
+                       : (const void*)pararnn_projsolve_kernel<kPsStages, 1>;
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
     return PARARNN_ERR_UNSUPPORTED;
   }
-  const size_t smem = ps_smem_bytes<kPsStages>();
+  const size_t smem = two ? ps_smem_bytes<kPsStages2, 2>() : ps_smem_bytes<kPsStages, 1>();
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess) {
     cudaGetLastError();

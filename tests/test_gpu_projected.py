@@ -50,17 +50,22 @@ def run(pr, d, with_bias=True, h0=False, **kw):
 
 
 # (B, L, D, K): one chunk; a ragged last chunk; D not a multiple of 32 and K not
-# a multiple of 64; more work items (batch row x 32 channels) than SMs
+# a multiple of 64; more work items (batch row x 32 channels) than SMs; several
+# rounds of items per CTA with an odd item count per CTA
 SHAPES = [(1, 128, 32, 64), (2, 300, 64, 128), (3, 515, 48, 136), (2, 1000, 96, 256),
-          (8, 256, 1024, 64)]
+          (8, 256, 1024, 64), (7, 130, 2048, 64)]
+
+# walker groups per CTA: one item at a time, two at once
+GROUPS = [1, 2]
 
 
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("with_bias,h0", [(True, False), (False, True)])
-def test_projected_solve_matches_oracle(pr, shape, with_bias, h0):
+@pytest.mark.parametrize("groups", GROUPS)
+def test_projected_solve_matches_oracle(pr, shape, with_bias, h0, groups):
     B, L, D, K = shape
     d = inputs.projected_gru_inputs(B, L, D, K, seed=[730, B, L, D, K], h0_normal=h0)
-    h, info = run(pr, d, with_bias, h0)
+    h, info = run(pr, d, with_bias, h0, opts=pr.Options(regime=groups))
     torch.cuda.synchronize()
     assert info.status == 0 and info.converged
     P = oracle_P(d, B, L, D, with_bias)
@@ -84,13 +89,14 @@ def test_projected_solve_matches_unfused_pair(pr):
     assert float(torch.max(torch.abs(h - h2)).item()) <= 1e-5
 
 
-def test_projected_solve_later_sweeps_recompute(pr):
+@pytest.mark.parametrize("groups", GROUPS)
+def test_projected_solve_later_sweeps_recompute(pr, groups):
     """Two Newton iterations per sweep: the solve needs several sweeps, each of
     which recomputes the projection; same answer as the oracle and as one sweep."""
     B, L, D, K = 2, 700, 64, 128
     d = inputs.projected_gru_inputs(B, L, D, K, seed=732)
-    h1, i1 = run(pr, d)
-    h2, i2 = run(pr, d, opts=pr.Options(iters_first=2, iters_next=1))
+    h1, i1 = run(pr, d, opts=pr.Options(regime=groups))
+    h2, i2 = run(pr, d, opts=pr.Options(iters_first=2, iters_next=1, regime=groups))
     torch.cuda.synchronize()
     assert i2.converged and i2.passes > 1 and i1.passes == 1
     assert i1.iterations == i2.iterations
@@ -100,18 +106,31 @@ def test_projected_solve_later_sweeps_recompute(pr):
 
 
 @pytest.mark.parametrize("max_iters", [0, 1, 2])
-def test_projected_solve_unconverged_is_the_newton_iterate(pr, max_iters):
+@pytest.mark.parametrize("groups", GROUPS)
+def test_projected_solve_unconverged_is_the_newton_iterate(pr, max_iters, groups):
     """Stopped at max_iters, the trajectory is the max_iters-th Newton iterate and
     the residuals rho_0 .. rho_max_iters are the oracle's."""
     B, L, D, K = 2, 400, 64, 128
     d = inputs.projected_gru_inputs(B, L, D, K, seed=733)
-    h, info = run(pr, d, max_iters=max_iters)
+    h, info = run(pr, d, max_iters=max_iters, opts=pr.Options(regime=groups))
     torch.cuda.synchronize()
     assert info.status == 0 and not info.converged and info.iterations == max_iters
     orc = oracle.newton_gru(oracle_P(d, B, L, D), d["a"], tol=1e-4, max_iters=max_iters)
     assert np.max(np.abs(h.cpu().numpy() - orc.h)) <= 1e-5
     for k in range(max_iters + 1):
         assert abs(info.rho[k] - orc.rho[k]) <= 1e-5 * max(1.0, orc.rho[k])
+
+
+def test_projected_solve_groups_agree(pr):
+    """One and two walker groups give the same trajectory and iteration count."""
+    B, L, D, K = 5, 333, 160, 96
+    d = inputs.projected_gru_inputs(B, L, D, K, seed=735, h0_normal=True)
+    h1, i1 = run(pr, d, True, True, opts=pr.Options(regime=1))
+    h2, i2 = run(pr, d, True, True, opts=pr.Options(regime=2))
+    torch.cuda.synchronize()
+    assert i1.converged and i2.converged and i1.iterations == i2.iterations
+    # 8 vs 16 steps per walker thread: the same sums in another order
+    assert float(torch.max(torch.abs(h1 - h2)).item()) <= 1e-5
 
 
 def test_projected_solve_empty(pr):
