@@ -1121,6 +1121,24 @@ static pararnn_status_t seq_common(bool rollout, int op, const void* P, pararnn_
   if (rollout) {
     const int threads = 128;
     const unsigned blocks = (unsigned)((n + threads - 1) / threads);
+    // one channel per batch row: each thread stages its own contiguous inputs
+    const long long G = op == kGru ? 3 : 4;
+    if (D == 1 && aligned(P, 16) && (L * G * (long long)esz) % 16 == 0) {
+      const int t1 = 64;
+      const unsigned b1 = (unsigned)((B + t1 - 1) / t1);
+      if (op == kGru) {
+        if (bf16)
+          pararnn_rollout_seq1_kernel<kGru, __nv_bfloat16, 16><<<b1, t1, 0, st>>>(sp);
+        else
+          pararnn_rollout_seq1_kernel<kGru, float, 16><<<b1, t1, 0, st>>>(sp);
+      } else {
+        if (bf16)
+          pararnn_rollout_seq1_kernel<kLstm, __nv_bfloat16, 8><<<b1, t1, 0, st>>>(sp);
+        else
+          pararnn_rollout_seq1_kernel<kLstm, float, 8><<<b1, t1, 0, st>>>(sp);
+      }
+      return cudaGetLastError() == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA;
+    }
     // inputs staged through shared memory when each warp's channels are one
     // contiguous row segment (D % 32 == 0) and the rows are 16-byte aligned
     if (D % 32 == 0 && aligned(P, 16)) {

@@ -177,6 +177,62 @@ __global__ void __launch_bounds__(128) pararnn_rollout_staged_kernel(const SeqPa
   cp_async_wait_all();
 }
 
+// The rollout for one channel per batch row (D = 1, the DEER shape): a
+// thread's sequence is one contiguous run of L x G inputs, so each thread
+// copies its own next R steps (R G elements, a multiple of 16 bytes) with
+// cp.async into one of two buffers.  Requires P 16-byte aligned and
+// L G sizeof(PT) a multiple of 16.
+template <int OP, typename PT, int R>
+__global__ void __launch_bounds__(64) pararnn_rollout_seq1_kernel(const SeqParams p) {
+  constexpr int G = OP == kGru ? 3 : 4;
+  constexpr int CH = R * G * (int)sizeof(PT) / 16;  // 16-byte chunks per group
+  static_assert((R * G * sizeof(PT)) % 16 == 0, "whole 16-byte chunks");
+  __shared__ __align__(16) PT s_in[64][2][R * G];
+  const long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (b >= p.B) return;
+  float w[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) w[g] = __ldg(p.w + g);
+  float x[2] = {p.x0a ? p.x0a[b] : 0.0f, 0.0f};
+  if constexpr (OP == kLstm) x[1] = p.x0b ? p.x0b[b] : 0.0f;
+  const char* src = reinterpret_cast<const char*>(reinterpret_cast<const PT*>(p.P) + b * p.L * G);
+  const long long nbytes = p.L * G * (long long)sizeof(PT);
+  float* o0 = p.out0 + b * p.L;
+  float* o1 = OP == kLstm ? p.out1 + b * p.L : nullptr;
+  PT* const buf0 = s_in[threadIdx.x][0];
+  PT* const buf1 = s_in[threadIdx.x][1];
+  auto stage = [&](PT* dst, long long t_first) {
+    const long long off = t_first * G * (long long)sizeof(PT);
+#pragma unroll
+    for (int k = 0; k < CH; ++k) {
+      const long long o = off + 16 * k;
+      const bool valid = o < nbytes;  // nbytes is a multiple of 16
+      cp_async16(smem_u32(dst) + 16u * k, src + (valid ? o : 0), valid);
+    }
+    cp_async_commit();
+  };
+  stage(buf0, 0);
+  stage(buf1, R);
+  for (long long t0 = 0, blk = 0; t0 < p.L; t0 += R, ++blk) {
+    PT* cur = (blk & 1) ? buf1 : buf0;
+    cp_async_wait_prior();
+#pragma unroll
+    for (int s = 0; s < R; ++s) {
+      const long long t = t0 + s;
+      if (t < p.L) {
+        float pin[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) pin[g] = to_f(cur[s * G + g]);
+        cell_apply<OP, PT>(pin, w, x);
+        __stcs(o0 + t, x[0]);
+        if constexpr (OP == kLstm) __stcs(o1 + t, x[1]);
+      }
+    }
+    stage(cur, t0 + 2 * R);
+  }
+  cp_async_wait_all();
+}
+
 // Multi-head GRU (dense 8x8 blocks per head of 8 channels) applied in order:
 // 8 lanes per (batch row, head) sequence, lane i = channel i of the head.  Per
 // step the head's state is gathered from the group by shuffles, lane i forms

@@ -103,3 +103,24 @@ def test_rollout_bf16_staged_matches_oracle(pr, cell):
         ref = oracle.rollout_lstm(x["P"], x["a"], x["c0"], x["h0"])[1]
     torch.cuda.synchronize()
     assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
+
+
+@pytest.mark.parametrize("cell,bf16,shape", [("gru", True, (4, 4000, 1)), ("gru", False, (3, 999, 1)),
+                                             ("lstm", False, (3, 999, 1)), ("lstm", True, (2, 1000, 1))])
+def test_rollout_one_channel_staged(pr, cell, bf16, shape):
+    """One channel per batch row (each thread stages its own contiguous inputs)."""
+    B, L, D = shape
+    gen = inputs.gru_inputs if cell == "gru" else inputs.lstm_inputs
+    x = gen(B, L, D, seed=[705, B, L, D], bf16=bf16, h0_normal=True)
+    P = (torch.from_numpy(x["P_bits"].view(np.int16)).cuda().view(torch.bfloat16) if bf16
+         else dev(x["P"]))
+    if cell == "gru":
+        h = pr.rollout_gru(P, dev(x["a"]), dev(x["h0"]))
+        ref = oracle.rollout_gru(x["P"], x["a"], x["h0"])
+    else:
+        c, h = pr.rollout_lstm(P, dev(x["a"]), dev(x["c0"]), dev(x["h0"]))
+        rc, ref = oracle.rollout_lstm(x["P"], x["a"], x["c0"], x["h0"])
+        torch.cuda.synchronize()
+        assert np.max(np.abs(c.cpu().numpy() - rc)) <= 1e-4
+    torch.cuda.synchronize()
+    assert np.max(np.abs(h.cpu().numpy() - ref)) <= 1e-4
