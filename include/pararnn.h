@@ -248,10 +248,11 @@ pararnn_status_t pararnn_step_lstm(const void* P, pararnn_dtype_t p_dtype, const
  * tol, max_iters, workspace or info.  Its time is L times the cell's
  * dependency chain, independent of B * D up to the GPU's thread count.  When D
  * is a multiple of 32 and P 16-byte aligned, each warp stages its channels'
- * upcoming inputs through shared memory; measured on B200 that is about 110 ns
- * per step, so for more than roughly 15 000 channels (B * D) the rollout takes
- * less time than the Newton solve, and for fewer it takes more (768x more at
- * B = 16, D = 1, L = 2^20). */
+ * upcoming inputs through shared memory (with D = 1, each thread its own
+ * contiguous inputs); measured on B200 that is about 110 ns per step, so for
+ * more than roughly 15 000 channels (B * D) the rollout takes less time than
+ * the Newton solve, and for fewer it takes more (422x more at B = 16, D = 1,
+ * L = 2^20). */
 pararnn_status_t pararnn_rollout_gru(const void* P, pararnn_dtype_t p_dtype, const float* a,
                                      const float* h0, float* h, int64_t B, int64_t L, int64_t D,
                                      void* stream);
