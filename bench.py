@@ -302,7 +302,7 @@ def recorded_traffic(workload):
 # workloads: device inputs, one step, host copies for the end-to-end leg
 # ---------------------------------------------------------------------------
 class Case:
-    def __init__(self, name, rank, device, seq_len=None):
+    def __init__(self, name, rank, device, seq_len=None, proj_k=None):
         import torch
 
         import nonlinear_rnn_solve_newton_b200 as pr
@@ -315,6 +315,11 @@ class Case:
             # the sequence-length sweep: the same draws as tests.inputs.workload_inputs(name, L)
             w["L"] = int(seq_len)
             base_seed = [w["seed"], int(seq_len)]
+        if proj_k is not None and "K" in w:
+            # another input width for the projection workloads (its own draws)
+            w["K"] = int(proj_k)
+            base_seed = [base_seed, 7000 + int(proj_k)] if not isinstance(base_seed, list) else \
+                base_seed + [7000 + int(proj_k)]
         self.w = w
         self.op, self.B, self.L, self.D, self.bf16 = w["op"], w["B"], w["L"], w["D"], w["bf16"]
         self.N = self.B * self.L * self.D
@@ -514,7 +519,7 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     maybe_init_pg(world, "nccl")
     pr.load()
-    cs = Case(args.workload, rank, device, args.seq_len)
+    cs = Case(args.workload, rank, device, args.seq_len, args.proj_k)
     op, B, L, D, bf16, N = cs.op, cs.B, cs.L, cs.D, cs.bf16, cs.N
     stream = torch.cuda.current_stream()
 
@@ -1217,6 +1222,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--no-sequential", action="store_true",
                     help="skip the sequential-application context timings")
+    ap.add_argument("--proj-k", type=int, default=None,
+                    help="input width K of the projection workloads (proj, proj_lm, proj_solve)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override L (the sequence-length sweep, e.g. 64 .. 16384 for gru_l)")
     ap.add_argument("--graph", dest="graph", action="store_true", default=None,
